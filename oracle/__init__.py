@@ -1,0 +1,33 @@
+"""Plain CPU oracle of the DeepSeek-V3 / V2-Lite MoE layer forward.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports this package:
+only the tests, the smoke check in the repository's entry module and the
+benchmark's CPU-baseline / reference arm may call it. It shares no code with
+the CUDA library; the two meet only through the seeded inputs of `moe_inputs`.
+
+Every floating-point value is carried in float64, except the router's
+selection decisions, which are taken on float32 scores (the precision of the
+GPU kernel, see `route_from_logits`).
+
+Parity status per function (what pins each one is listed in the tests):
+  e4m3_values / quantize_e4m3 / fp8_quantize_*  pinned (format facts, torch cast)
+  gate_logits                                   pinned (identity gate)
+  route_from_logits                             pinned (brute force, invariants)
+  permute                                       pinned (worked example)
+  swiglu_ffn                                    pinned (closed form SiLU(1))
+  moe_forward                                   pinned (dense brute force,
+                                                combine identities)
+  bias_update / load_cv                         pinned (closed forms)
+"""
+from .moe_oracle import (
+    e4m3_values, quantize_e4m3, dequantize_e4m3, fp8_quantize_blocks,
+    fp8_quantize_rows, gate_logits, selection_scores, route_from_logits,
+    RouteResult, permute, swiglu_ffn, moe_forward, bias_update, load_cv,
+)
+
+__all__ = [
+    "e4m3_values", "quantize_e4m3", "dequantize_e4m3", "fp8_quantize_blocks",
+    "fp8_quantize_rows", "gate_logits", "selection_scores",
+    "route_from_logits", "RouteResult", "permute", "swiglu_ffn",
+    "moe_forward", "bias_update", "load_cv",
+]
