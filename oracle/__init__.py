@@ -10,7 +10,9 @@ selection decisions, which are taken on float32 scores (the precision of the
 GPU kernel, see `route_from_logits`).
 
 Parity status per function (what pins each one is listed in the tests):
-  e4m3_values / quantize_e4m3 / fp8_quantize_*  pinned (format facts, torch cast)
+  e4m3_values / quantize_e4m3 / round_to_e4m3 /
+  fp8_quantize_* / fp8_qdq_*                    pinned (format facts, torch cast,
+                                                the two roundings agree)
   gate_logits                                   pinned (identity gate)
   route_from_logits                             pinned (brute force, invariants)
   permute                                       pinned (worked example)
@@ -20,14 +22,14 @@ Parity status per function (what pins each one is listed in the tests):
   bias_update / load_cv                         pinned (closed forms)
 """
 from .moe_oracle import (
-    e4m3_values, quantize_e4m3, dequantize_e4m3, fp8_quantize_blocks,
-    fp8_quantize_rows, gate_logits, selection_scores, route_from_logits,
+    e4m3_values, quantize_e4m3, dequantize_e4m3, round_to_e4m3, fp8_quantize_blocks,
+    fp8_quantize_rows, fp8_qdq_blocks, fp8_qdq_rows, gate_logits, selection_scores, route_from_logits,
     RouteResult, permute, swiglu_ffn, moe_forward, bias_update, load_cv,
 )
 
 __all__ = [
-    "e4m3_values", "quantize_e4m3", "dequantize_e4m3", "fp8_quantize_blocks",
-    "fp8_quantize_rows", "gate_logits", "selection_scores",
+    "e4m3_values", "quantize_e4m3", "dequantize_e4m3", "round_to_e4m3",
+    "fp8_quantize_blocks", "fp8_quantize_rows", "fp8_qdq_blocks", "fp8_qdq_rows", "gate_logits", "selection_scores",
     "route_from_logits", "RouteResult", "permute", "swiglu_ffn",
     "moe_forward", "bias_update", "load_cv",
 ]

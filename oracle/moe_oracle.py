@@ -83,6 +83,17 @@ def dequantize_e4m3(codes: np.ndarray) -> np.ndarray:
     return e4m3_values()[np.asarray(codes, dtype=np.int64)]
 
 
+def round_to_e4m3(y32: np.ndarray) -> np.ndarray:
+    """The value `quantize_e4m3` picks, computed arithmetically: keep 3
+    mantissa bits (quantum 2^(e-4) for |y| = m * 2^e, m in [0.5, 1), never
+    finer than the subnormal step 2^-9), round half to even, clamp to 448."""
+    y = np.asarray(y32, dtype=np.float32).astype(np.float64)
+    _, e = np.frexp(y)
+    quantum = np.ldexp(1.0, np.maximum(e - 4, -9))
+    r = np.round(y / quantum) * quantum
+    return np.clip(r, -E4M3_MAX, E4M3_MAX)
+
+
 def _scale_of(amax32: np.ndarray) -> np.ndarray:
     amax32 = np.asarray(amax32, dtype=np.float32)
     s = amax32 / np.float32(E4M3_MAX)
@@ -113,6 +124,26 @@ def fp8_quantize_rows(a: np.ndarray, block: int = 128) -> Tuple[np.ndarray, np.n
     scale = _scale_of(amax)
     q = quantize_e4m3(tiles / scale[:, :, None])
     return q.reshape(M, K), scale
+
+
+def fp8_qdq_blocks(w: np.ndarray, block: int = 128) -> np.ndarray:
+    """Dequantised values of `fp8_quantize_blocks(w)` (via `round_to_e4m3`)."""
+    w32 = np.asarray(w, dtype=np.float32)
+    N, K = w32.shape
+    tiles = w32.reshape(N // block, block, K // block, block)
+    scale = _scale_of(np.abs(tiles).max(axis=(1, 3)))
+    v = round_to_e4m3(tiles / scale[:, None, :, None])
+    return (v * scale[:, None, :, None].astype(np.float64)).reshape(N, K)
+
+
+def fp8_qdq_rows(a: np.ndarray, block: int = 128) -> np.ndarray:
+    """Dequantised values of `fp8_quantize_rows(a)` (via `round_to_e4m3`)."""
+    a32 = np.asarray(a, dtype=np.float32)
+    M, K = a32.shape
+    tiles = a32.reshape(M, K // block, block)
+    scale = _scale_of(np.abs(tiles).max(axis=2))
+    v = round_to_e4m3(tiles / scale[:, :, None])
+    return (v * scale[:, :, None].astype(np.float64)).reshape(M, K)
 
 
 def fp8_dequant_blocks(q: np.ndarray, scale: np.ndarray, block: int = 128) -> np.ndarray:
@@ -276,58 +307,66 @@ def swiglu_ffn(x: np.ndarray, w13: np.ndarray, w2: np.ndarray) -> np.ndarray:
     return h @ np.asarray(w2, np.float64).T
 
 
-def _swiglu_fp8(xq, xs, w13, w2):
+def _swiglu_fp8(xd, w13, w2, w2_rows=None):
     """The same expert in E4M3: weights per 128x128 block, activations per
-    1x128 tile (x given pre-quantised), h re-quantised per 1x128."""
-    q13, s13 = fp8_quantize_blocks(w13)
-    q2, s2 = fp8_quantize_blocks(w2)
-    xd = fp8_dequant_rows(xq, xs)
+    1x128 tile (xd = the dequantised activations), h re-quantised per 1x128.
+    `w2_rows` optionally restricts the output to those features (the blocks
+    holding them are quantised exactly as in the whole matrix)."""
     I = w13.shape[0] // 2
-    gu = xd @ fp8_dequant_blocks(q13, s13).T
+    gu = xd @ fp8_qdq_blocks(w13).T
     g, u = gu[:, :I], gu[:, I:]
     h = g * (1.0 / (1.0 + np.exp(-g))) * u
-    hq, hs = fp8_quantize_rows(h.astype(np.float32))
-    return fp8_dequant_rows(hq, hs) @ fp8_dequant_blocks(q2, s2).T
+    hd = fp8_qdq_rows(h.astype(np.float32))
+    if w2_rows is None:
+        return hd @ fp8_qdq_blocks(w2).T
+    blocks = np.unique(np.asarray(w2_rows) // 128)
+    sub = np.concatenate([np.asarray(w2[b * 128:(b + 1) * 128]) for b in blocks])
+    dq = fp8_qdq_blocks(sub)
+    pos = {b: i for i, b in enumerate(blocks)}
+    idx = [pos[r // 128] * 128 + r % 128 for r in w2_rows]
+    return hd @ dq[idx].T
 
 
 def moe_forward(x: np.ndarray, route: RouteResult,
                 expert_weights: Callable[[int], Tuple[np.ndarray, np.ndarray]],
                 shared: Optional[Tuple[np.ndarray, np.ndarray]], fp8: bool = False,
-                return_parts: bool = False):
+                return_parts: bool = False, out_features=None):
     """y_t = shared(x_t) + sum_j w_tj * E_{id_tj}(x_t)  ([MoE-walk] §3.4).
 
     `x` holds the tokens to evaluate (any subset; the layer is per token), and
     `route` their routing. `expert_weights(e)` returns (w13_e, w2_e) for one
-    expert, so the caller can widen one expert at a time.
+    expert, so the caller can widen one expert at a time. `out_features`
+    (optional) limits the output to those hidden features.
     """
     x = np.asarray(x, np.float64)
     T, H = x.shape
     ids = route.ids
     k = ids.shape[1]
-    xq = xs = None
-    if fp8:
-        xq, xs = fp8_quantize_rows(x.astype(np.float32))
-    routed = np.zeros((T, H), dtype=np.float64)
-    per_slot = np.zeros((T, k, H), dtype=np.float64) if return_parts else None
+    xd = fp8_qdq_rows(x.astype(np.float32)) if fp8 else None
+    Hout = H if out_features is None else len(out_features)
+    routed = np.zeros((T, Hout), dtype=np.float64)
+    per_slot = np.zeros((T, k, Hout), dtype=np.float64) if return_parts else None
     for e in np.unique(ids):
         tt, jj = np.nonzero(ids == e)
         w13, w2 = expert_weights(int(e))
         if fp8:
-            out = _swiglu_fp8(xq[tt], xs[tt], np.asarray(w13, np.float32),
-                              np.asarray(w2, np.float32))
+            out = _swiglu_fp8(xd[tt], np.asarray(w13, np.float32), np.asarray(w2, np.float32),
+                              out_features)
         else:
-            out = swiglu_ffn(x[tt], w13, w2)
+            w2s = w2 if out_features is None else np.asarray(w2)[out_features]
+            out = swiglu_ffn(x[tt], w13, w2s)
         contrib = route.weights[tt, jj][:, None] * out
         np.add.at(routed, tt, contrib)
         if return_parts:
             per_slot[tt, jj] = out
-    sh = np.zeros((T, H), dtype=np.float64)
+    sh = np.zeros((T, Hout), dtype=np.float64)
     if shared is not None:
         if fp8:
-            sh = _swiglu_fp8(xq, xs, np.asarray(shared[0], np.float32),
-                             np.asarray(shared[1], np.float32))
+            sh = _swiglu_fp8(xd, np.asarray(shared[0], np.float32),
+                             np.asarray(shared[1], np.float32), out_features)
         else:
-            sh = swiglu_ffn(x, shared[0], shared[1])
+            s2 = shared[1] if out_features is None else np.asarray(shared[1])[out_features]
+            sh = swiglu_ffn(x, shared[0], s2)
     y = routed + sh
     if return_parts:
         return y, routed, sh, per_slot

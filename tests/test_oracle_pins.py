@@ -88,6 +88,23 @@ def test_e4m3_matches_torch_cast_in_range():
     assert np.array_equal(ours, ref)
 
 
+def test_two_e4m3_roundings_agree():
+    # table search over the 256 codes vs arithmetic rounding to 3 mantissa bits
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal(300000) * rng.choice([1e-4, 1e-3, 0.02, 1, 50, 300, 600], 300000)).astype(np.float32)
+    grid = oracle.e4m3_values()[:127]
+    mids = ((grid[1:] + grid[:-1]) / 2).astype(np.float32)   # exact ties
+    x = np.concatenate([x, mids, -mids, np.float32([0.0, -0.0, 448.0, 464.0, 465.0, 1e6])])
+    a = oracle.dequantize_e4m3(oracle.quantize_e4m3(x))
+    b = oracle.round_to_e4m3(x)
+    assert np.array_equal(a, b)
+    w = (rng.standard_normal((256, 256)) * 0.02).astype(np.float32)
+    q, s = oracle.fp8_quantize_blocks(w)
+    assert np.array_equal(O.fp8_dequant_blocks(q, s), oracle.fp8_qdq_blocks(w))
+    qr, sr = oracle.fp8_quantize_rows(w)
+    assert np.array_equal(O.fp8_dequant_rows(qr, sr), oracle.fp8_qdq_rows(w))
+
+
 def test_fp8_block_quant_roundtrip_bound_and_exact_grid():
     rng = np.random.default_rng(1)
     w = (rng.standard_normal((256, 384)) * 0.02).astype(np.float32)
@@ -348,7 +365,11 @@ def test_fp8_expert_matches_torch_cast_formulation():
     w13 = inp.w13.float().numpy()[3]
     w2 = inp.w2.float().numpy()[3]
     xq, xs = oracle.fp8_quantize_rows(x)
-    ours = O._swiglu_fp8(xq, xs, w13, w2)
+    ours = O._swiglu_fp8(O.fp8_dequant_rows(xq, xs), w13, w2)
+    # restricting the output to a few features changes nothing
+    feats = [0, 5, 130, 255]
+    part = O._swiglu_fp8(O.fp8_dequant_rows(xq, xs), w13, w2, feats)
+    np.testing.assert_allclose(part, ours[:, feats], rtol=1e-12, atol=1e-15)
     ref = _torch_fp8_expert(x, w13, w2)
     np.testing.assert_allclose(ours, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max())
     # and quantisation is visible against the unquantised expert
