@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Throughput of the DeepSeek-V3 MoE layer forward on B200 (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole path over one batch of synthetic tokens:
+gate GEMM + routing, permutation, routed SwiGLU experts (two grouped GEMMs),
+the shared expert, combine, and the aux-loss-free bias update. The default
+workload is the V3-shaped layer (T=8192 tokens, H=7168, 256 routed experts
+with I=2048, 1 shared expert, top-8 of 8 groups keeping 4, sigmoid scoring
+with a selection bias, renormalised weights x2.5), bf16 weights and
+activations, fp32 accumulation. Inputs are larger than L2 (22.5 GB of expert
+weights stream through every step), so no L2 flush is done between steps.
+
+N > 1 (launched under torchrun): every rank runs an independent replica on
+its own tokens (weak scaling); the expert counts are summed over ranks before
+the bias step so all replicas keep the same bias.
+
+--impl reference times the CPU oracle (the plain float64 statement of the
+layer) on the host cores, on a bounded sample of tokens per step.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer fwd tokens/s and achieved TFLOP/s vs B200 peak at V3 shape"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "gate_up_swiglu_v3_traffic.txt")
+GEMM_SOURCES = ["grouped_gemm.cu", "common.cuh", "kernels.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="v3")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=16)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def workload_name(cfg):
+    return (f"{cfg.name} MoE layer fwd: T={cfg.T} tokens, H={cfg.H}, {cfg.E} routed experts "
+            f"(I={cfg.I}) + shared (I_s={cfg.I_s}), top-{cfg.k}, n_group={cfg.n_group}/"
+            f"topk_group={cfg.topk_group}, {cfg.scoring}, {cfg.dtype}")
+
+
+def config_block(cfg, world):
+    return {"workload": workload_name(cfg), "T_per_gpu": cfg.T, "global_tokens": cfg.T * world,
+            "H": cfg.H, "E": cfg.E, "I": cfg.I, "I_s": cfg.I_s, "k": cfg.k,
+            "n_group": cfg.n_group, "topk_group": cfg.topk_group, "scoring": cfg.scoring,
+            "norm_topk_prob": cfg.norm_topk_prob, "routed_scaling_factor": cfg.scale,
+            "weights_dtype": cfg.dtype, "parallelism": f"replicas x{world} (token-sharded)",
+            "l2": "inputs larger than L2 (all expert weights stream each step); no flush"}
+
+
+# ------------------------------------------------------------ clock sampling
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.sel = None
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(device_index)
+            self.sel = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        except Exception:
+            self.sel = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.sel:
+            cmd += ["-i", self.sel]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        # samples under load: SM clock above the idle floor
+        load = [s for s in sm if s > 0.3 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
+
+
+# ------------------------------------------------------------ CPU oracle arm
+def oracle_tokens_per_s(cfg, inp, tokens, threads):
+    """Times the float64 oracle on the given tokens: logits, routing, every
+    routed expert they use, the shared expert and the combine."""
+    import numpy as np
+    import torch
+    import oracle
+    toks = torch.as_tensor(tokens, device=inp.x.device)
+    x = inp.x[toks].float().cpu().numpy()
+    gate = inp.gate.float().cpu().numpy()
+    bias = inp.bias.float().cpu().numpy() if inp.bias is not None else None
+    # the experts these tokens use, moved to host memory before the clock starts
+    L0 = (x.astype(np.float64) @ gate.astype(np.float64).T).astype(np.float32)
+    r0 = oracle.route_from_logits(L0, cfg.k, cfg.n_group, cfg.topk_group, cfg.scoring,
+                                  cfg.norm_topk_prob, cfg.scale, bias)
+    experts = {int(e): (inp.w13[int(e)].float().cpu().numpy(), inp.w2[int(e)].float().cpu().numpy())
+               for e in np.unique(r0.ids)}
+    shared = (inp.sw13.float().cpu().numpy(), inp.sw2.float().cpu().numpy()) if inp.sw13 is not None else None
+    t0 = time.perf_counter()
+    L = oracle.gate_logits(x, gate).astype(np.float32)
+    r = oracle.route_from_logits(L, cfg.k, cfg.n_group, cfg.topk_group, cfg.scoring,
+                                 cfg.norm_topk_prob, cfg.scale, bias)
+    missing = [int(e) for e in np.unique(r.ids) if int(e) not in experts]
+    for e in missing:
+        experts[e] = (inp.w13[e].float().cpu().numpy(), inp.w2[e].float().cpu().numpy())
+    oracle.moe_forward(x, r, lambda e: experts[e], shared, fp8=(cfg.dtype == "e4m3"))
+    dt = time.perf_counter() - t0
+    return len(tokens) / dt, dt
+
+
+def host_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+    from moe_inputs import get_config, make_inputs
+    cfg = get_config(args.config)
+    threads = host_threads()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(cfg, device=dev)
+    rng = np.random.default_rng(2024)
+    per_step = 1
+    times, ntok = [], 0
+    for i in range(args.warmup + args.steps):
+        toks = rng.choice(cfg.T, per_step, replace=False)
+        _, dt = oracle_tokens_per_s(cfg, inp, toks, threads)
+        if i >= args.warmup:
+            times.append(dt)
+            ntok += per_step
+    total = sum(times)
+    value = ntok / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / max(1, len(times)), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(cfg, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{per_step} random token(s) of {cfg.T} per step: fp64 logits, "
+                                       "routing, its experts, shared expert, combine"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------ our arm
+def gemm_source_hash():
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        h.update(open(os.path.join(ROOT, "mixture_experts_layer_limited_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the gate/up GEMM from the committed ncu
+    summary, only if the GEMM source has not changed since it was taken."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    kv = {}
+    for line in open(PROFILE_TRAFFIC):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("gemm_source_sha256_16") != gemm_source_hash():
+        return None
+    try:
+        return float(kv["traffic_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+LAUNCHES = {"route": 1, "quantize_x": 1, "permute": 4, "gate_up_routed": 1, "down_routed": 1,
+            "gate_up_shared": 1, "down_shared": 1, "combine": 1, "bias_update": 1}
+
+
+def stage_model(cfg):
+    """Algorithmic FLOPs and bytes of each stage (no padding, no re-reads)."""
+    T, H, E, I, Is, k = cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_s, cfg.k
+    R = T * k
+    ab = 1 if cfg.dtype == "e4m3" else 2
+    return {
+        "route": {"flops": 2.0 * T * H * E, "bytes": T * H * 2 + E * H * 2 + R * 8},
+        "quantize_x": {"flops": 0.0, "bytes": T * H * 2 + T * H + T * (H // 128) * 4},
+        "permute": {"flops": 0.0, "bytes": T * H * ab + R * H * ab + R * 8 + R * 12},
+        "gate_up_routed": {"flops": 2.0 * R * H * 2 * I, "bytes": E * 2 * I * H * ab + R * H * ab + R * I * ab},
+        "down_routed": {"flops": 2.0 * R * I * H, "bytes": E * H * I * ab + R * I * ab + R * H * 2},
+        "gate_up_shared": {"flops": 2.0 * T * H * 2 * Is, "bytes": 2 * Is * H * ab + T * H * ab + T * Is * ab},
+        "down_shared": {"flops": 2.0 * T * Is * H, "bytes": H * Is * ab + T * Is * ab + T * H * 2},
+        "combine": {"flops": 0.0, "bytes": R * H * 2 + T * H * 2 + T * H * 2 + R * 4},
+        "bias_update": {"flops": 0.0, "bytes": E * 12},
+    }
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from moe_inputs import get_config, make_inputs
+    from mixture_experts_layer_limited_b200 import MoELayer, LayerSpec, load_library
+    from mixture_experts_layer_limited_b200 import dist as mdist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    load_library()
+    cfg = get_config(args.config)
+    inp = make_inputs(cfg, device="cuda")
+    if rank > 0:   # same weights, this replica's own tokens
+        g = torch.Generator(device="cuda")
+        g.manual_seed(cfg.seed + 100003 * rank)
+        inp.x = torch.randn(cfg.T, cfg.H, generator=g, device="cuda").to(torch.bfloat16)
+    layer = MoELayer(LayerSpec.from_config(cfg), inp.gate, inp.w13, inp.w2, inp.sw13, inp.sw2,
+                     inp.bias, cfg.T)
+    T_global = cfg.T * world
+    stream = torch.cuda.current_stream()
+    stages = layer.stages(inp.x)
+    names = [n for n, _ in stages] + (["bias_update"] if layer.bias is not None else [])
+
+    def step(marks=None):
+        for i, (_, run) in enumerate(stages):
+            run()
+            if marks is not None:
+                marks[i].record(stream)
+        if layer.bias is not None:
+            mdist.allreduce_counts_(layer.counts)
+            layer.bias_step(T_global, cfg.gamma, load_cv=False)
+            if marks is not None:
+                marks[len(stages)].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0, "device status flagged during warm-up"
+
+    K = args.steps
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in names] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    mdist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)                                   # sampler up before the clock starts
+    start.record(stream)
+    for i in range(K):
+        step(marks[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    mdist.barrier()
+    clk = clocks.stop()
+    ms_local = start.elapsed_time(end)
+    ms = mdist.max_over_ranks(ms_local, device="cuda")
+    status = layer.device_status()
+
+    # per-stage device time from consecutive events on the launching stream
+    per = {n: [] for n in names}
+    for i in range(K):
+        prev = start if i == 0 else marks[i - 1][-1]
+        for j, n in enumerate(names):
+            per[n].append(prev.elapsed_time(marks[i][j]))
+            prev = marks[i][j]
+    avg = {n: sum(v) / len(v) for n, v in per.items()}
+    model = stage_model(cfg)
+    peaks = load_peaks()
+    kernels = {}
+    for n in names:
+        m = model[n]
+        d = {"ms": round(avg[n], 4), "launches": LAUNCHES[n]}
+        if m["flops"]:
+            d["tflops"] = round(m["flops"] / (avg[n] * 1e-3) / 1e12, 1)
+        d["gbs"] = round(m["bytes"] / (avg[n] * 1e-3) / 1e9, 1)
+        kernels[n] = d
+
+    tokens = cfg.T * world * K
+    value = tokens / (ms * 1e-3)
+    flops_step = cfg.flops()
+    dom = "gate_up_routed"
+    achieved = model[dom]["flops"] / (avg[dom] * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"kernel": "grouped_gemm_bf16 (gate/up + SwiGLU, routed experts)", "bound": "tensor",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
+                "peak_note": f"bf16 sustained, {peaks['source']} (MEASURED_PEAKS.json)",
+                "algorithmic_flops_per_launch": model[dom]["flops"],
+                "algorithmic_bytes_per_launch": model[dom]["bytes"]}
+
+    # ---- end to end: host x -> device, forward + bias step, y -> host
+    x_host = inp.x.cpu().pin_memory()
+    y_host = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+    stages_e2e = layer.stages(x_dev)
+
+    def step_e2e():
+        x_dev.copy_(x_host, non_blocking=True)
+        for _, run in stages_e2e:
+            run()
+        if layer.bias is not None:
+            mdist.allreduce_counts_(layer.counts)
+            layer.bias_step(T_global, cfg.gamma, load_cv=False)
+        y_host.copy_(layer.y[:cfg.T], non_blocking=True)
+
+    for _ in range(3):
+        step_e2e()
+    torch.cuda.synchronize()
+    mdist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        step_e2e()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    mdist.barrier()
+    ms_e2e = mdist.max_over_ranks(e0.elapsed_time(e1), device="cuda")
+    e2e = {"value": cfg.T * world * K / (ms_e2e * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2,
+           "path": "MoELayer stages through the C ABI; pinned host x in, pinned host y out"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rng = np.random.default_rng(7)
+        toks = np.sort(rng.choice(cfg.T, args.cpu_sample_tokens, replace=False))
+        rate, dt = oracle_tokens_per_s(cfg, inp, toks, host_threads())
+        cpu = {"value": rate, "unit": "tokens/s", "cores": host_threads(), "kind": "oracle",
+               "sample": f"{len(toks)} random tokens of {cfg.T} ({dt:.1f} s): fp64 logits, routing, "
+                         "their experts, shared expert, combine"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "e4m3",
+                "data": "synthetic (seeded random inputs and weights, V3 shapes)",
+                "config": config_block(cfg, world),
+                "tflops": round(flops_step * world * K / (ms * 1e-3) / 1e12, 1),
+                "tflops_frac_of_measured_sustained": round(flops_step * world * K / (ms * 1e-3) / 1e12 / peak, 4),
+                "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": K * sum(LAUNCHES[n] for n in names), "clocks": clk,
+                "device_status": status}
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

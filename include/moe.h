@@ -1,0 +1,265 @@
+/*
+ * libmoe -- forward pass of a DeepSeek-V3 / DeepSeek-V2-Lite mixture-of-experts
+ * layer on one NVIDIA B200 (sm_100a).
+ *
+ * The layer, as the pages state it:
+ *   [MoE-walk]    zhiyuanblog.org "MoE 混合专家模型推理参数与前向传播详解":
+ *                 §2.1 router, §2.2 stacked expert weights, §2.3 merged shared
+ *                 experts, §3.1 routing, §3.2 token permutation, §3.3 grouped
+ *                 SwiGLU experts and shared experts, §3.4 unpermute + combine.
+ *   [V3-teardown] gsyq.cn "为什么要在本地拆解 DeepSeek-V3 的 MoE 与 MLA":
+ *                 §3 router config (n_group, topk_group, norm_topk_prob,
+ *                 routed_scaling_factor, sigmoid scoring; FP8 128x128 weight
+ *                 blocks, dynamic activations), §4 route() and the load CV.
+ *   [V3-digest]   xxqk.cn DeepSeek V3/R1/Janus-Pro digest, §2.2 aux-loss-free
+ *                 bias and device-limited (group-limited) routing.
+ *   [FP8-infer]   blog.hotdry.top DeepSeek-V3 FP8 inference post, FP8 section
+ *                 (E4M3, 1x128 activation tiles, 128x128 weight blocks).
+ *
+ * Conventions for every call:
+ *   - Tensor pointers are DEVICE pointers to dense row-major arrays, allocated
+ *     and owned by the caller. The library allocates no memory and keeps no
+ *     mutable global state between calls (moe_last_cuda_error aside).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL means the
+ *     legacy default stream). Outputs are valid once the stream reaches it.
+ *   - Arguments are checked on the host before any launch. On a non-OK
+ *     return nothing has been launched or written, except MOE_ERR_CUDA,
+ *     which reports a launch failure (see moe_last_cuda_error).
+ *   - Every device pointer must be 16-byte aligned (MOE_ERR_ALIGNMENT).
+ *   - `dev_status`, where taken, is an optional device int32 (NULL = off).
+ *     Kernels never trap: a bounds check that fails or a bounded wait that
+ *     runs out ORs a code into it (MOE_DEVSTAT_*) and the kernel returns.
+ *     Read it with moe_read_device_status.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef MOE_B200_MOE_H
+#define MOE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#define MOE_ABI_VERSION 1
+
+typedef int32_t moe_status;
+#define MOE_OK                 0
+#define MOE_ERR_INVALID_ARG    1  /* null pointer, bad size, k > E, ...      */
+#define MOE_ERR_UNSUPPORTED    2  /* shape / dtype combination not built      */
+#define MOE_ERR_ALIGNMENT      3  /* a pointer is not 16-byte aligned         */
+#define MOE_ERR_CUDA           4  /* a CUDA launch or driver call failed      */
+#define MOE_ERR_DEVICE_CHECK   5  /* device status: a bounds check failed     */
+#define MOE_ERR_DEVICE_TIMEOUT 6  /* device status: a bounded wait ran out    */
+
+/* bits ORed into *dev_status by kernels */
+#define MOE_DEVSTAT_BAD_EXPERT_ID 0x1 /* a topk id outside [0, E)            */
+#define MOE_DEVSTAT_TIMEOUT       0x2 /* an mbarrier wait exceeded its limit */
+
+typedef int32_t moe_dtype;
+#define MOE_F32  0
+#define MOE_BF16 1
+#define MOE_E4M3 2   /* float8 e4m3 "fn": bias 7, max 448, no inf */
+
+typedef int32_t moe_scoring;
+#define MOE_SOFTMAX 0
+#define MOE_SIGMOID 1
+
+/* ------------------------------------------------------------------------ *
+ * moe_route -- gate projection + scoring + group-limited top-k + weights.
+ * [MoE-walk] §2.1 and §3.1; [V3-teardown] §3-§4 route(); [V3-digest] §2.2.
+ *
+ *   logits = x @ gate^T                       (bf16 inputs, fp32 accumulate)
+ *   scoring  softmax: p = softmax(logits) over all E experts
+ *            sigmoid: s = sigmoid(logits)
+ *   selection score  sel = s + sel_bias (sigmoid), p (softmax with groups or
+ *            a bias), the logit itself (softmax, one group, no bias). The
+ *            sigmoid and softmax are evaluated in double and rounded once to
+ *            float; the bias add is one float add.
+ *   if n_group > 1: experts [g*E/n_group, (g+1)*E/n_group) form group g; a
+ *            group's score is the float sum of its two largest sel; only the
+ *            topk_group best groups stay candidates (ties: lower group index).
+ *   topk_ids = the k best sel among candidates, in slot order sel descending,
+ *            expert index ascending (ties: lower expert index).
+ *   topk_w   = unbiased s (or p) of those experts; if norm_topk_prob they are
+ *            divided by their sum; then multiplied by routed_scaling_factor.
+ *   expert_counts[e] = number of (t, j) with topk_ids[t][j] == e (zeroed by
+ *            the call first).
+ *
+ * Arguments
+ *   p             shapes and routing config (host pointer, read during call).
+ *   x             [T, H] bf16, or NULL: then `logits` is an INPUT [T, E] fp32
+ *                 and routing runs on those logits (no projection).
+ *   gate_w        [E, H] bf16 (ignored when x == NULL).
+ *   sel_bias      [E] fp32 selection-only bias, or NULL (= 0).
+ *   logits        [T, E] fp32: written when x != NULL (may then be NULL to
+ *                 skip writing), read when x == NULL.
+ *   topk_ids      [T, k] int32 out;  topk_w [T, k] fp32 out.
+ *   expert_counts [E] int32 out.
+ * Limits: 1 <= k <= 16, E % 16 == 0, 16 <= E <= 256, E % n_group == 0,
+ *   n_group <= 32, topk_group <= n_group, k <= topk_group * E / n_group,
+ *   H % 64 == 0 when x != NULL. Otherwise MOE_ERR_INVALID_ARG/UNSUPPORTED.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int32_t T, H, E, k;
+    int32_t n_group, topk_group;
+    moe_scoring scoring;
+    int32_t norm_topk_prob;          /* 0 / 1 */
+    float routed_scaling_factor;
+    int32_t* dev_status;             /* optional device status word */
+} moe_route_params;
+
+MOE_API moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_w,
+                     const float* sel_bias, float* logits, int32_t* topk_ids,
+                     float* topk_w, int32_t* expert_counts, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * moe_permute -- expand every token k times and order the copies by expert.
+ * [MoE-walk] §3.2 and its worked example: segment e holds the tokens routed
+ * to expert e in ASCENDING TOKEN ORDER; expert_offsets is
+ * expert_first_token_offset with E + 1 entries (empty experts repeat).
+ *
+ *   expert_offsets [E+1] int32 out, expert_offsets[E] = T*k
+ *   src_token      [T*k] int32 out, row -> token
+ *   slot_to_row    [T*k] int32 out, t*k + j -> row (inv_permuted_idx)
+ *   row_w          [T*k] fp32 out,  topk_w[t][j] at row slot_to_row[t*k+j]
+ *                  (may be NULL, then topk_w may be NULL too)
+ *   x / x_perm     x_dtype MOE_BF16: x [T, H] bf16 -> x_perm [T*k, H] bf16.
+ *                  x_dtype MOE_E4M3: x [T, H] e4m3 codes (moe_quantize_rows)
+ *                  with x_scale [T, H/128] -> x_perm [T*k, H] codes and
+ *                  x_perm_scale [T*k, H/128]. x_perm may be NULL (metadata
+ *                  only).
+ *   workspace      device scratch of moe_permute_workspace_size() bytes.
+ * topk_ids outside [0, E) are counted nowhere and flag
+ * MOE_DEVSTAT_BAD_EXPERT_ID in dev_status (outputs are then undefined).
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_permute_workspace_size(int32_t T, int32_t k, int32_t E, size_t* bytes);
+
+MOE_API moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H,
+                       const int32_t* topk_ids, const float* topk_w,
+                       const void* x, moe_dtype x_dtype, const float* x_scale,
+                       void* x_perm, float* x_perm_scale,
+                       int32_t* expert_offsets, int32_t* src_token,
+                       int32_t* slot_to_row, float* row_w,
+                       void* workspace, size_t workspace_bytes,
+                       int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * moe_grouped_swiglu -- SwiGLU experts over contiguous row segments.
+ * [MoE-walk] §3.3.1 (w13 = [w1; w3], gate = first I outputs, up = last I,
+ * h = SiLU(gate) * up, out = h @ w2^T) and the grouped GEMM of the same
+ * section (one launch for all experts, segmented by expert offsets);
+ * §3.3.2 / §2.3 shared experts (merged into one FFN: call with offsets = NULL).
+ *
+ *   rows      number of activation rows (T*k routed, T shared).
+ *   H         hidden size (K of the first GEMM, N of the second).
+ *   w         weights: w13 [groups, 2I, H], w2 [groups, H, I] (out-major,
+ *             i.e. K contiguous). MOE_E4M3 weights carry fp32 block scales
+ *             w13_scale [groups, 2I/128, H/128], w2_scale [groups, H/128,
+ *             I/128] (moe_quantize_blocks).
+ *   a         [rows, H] activations: bf16, or e4m3 codes with a_scale
+ *             [rows, H/128] when w->dtype == MOE_E4M3.
+ *   offsets   [groups+1] device int32 segment starts (from moe_permute), or
+ *             NULL: one group covering all rows (groups must be 1).
+ *   row_w     [rows] fp32 per-row output weight fused into the epilogue of
+ *             the second GEMM, or NULL (= 1).
+ *   h_ws      [rows, I] intermediate: bf16, or e4m3 codes with h_scale_ws
+ *             [rows, I/128] for MOE_E4M3 (re-quantised per 1x128 tile).
+ *   out       [rows, H] bf16 = row_w * (SiLU(a w1^T) * (a w3^T)) w2^T.
+ * Limits: I % 128 == 0, H % 256 == 0, rows >= 1. E4M3 also needs H % 128
+ * and I % 128. Accumulation is fp32 on the tensor cores; h is rounded to
+ * bf16 (or quantised to e4m3) before the second GEMM.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    const void* w13;
+    const void* w2;
+    const float* w13_scale;   /* E4M3 only, else NULL */
+    const float* w2_scale;    /* E4M3 only, else NULL */
+    moe_dtype dtype;          /* MOE_BF16 or MOE_E4M3 */
+    int32_t groups;
+    int32_t I;
+} moe_ffn_weights;
+
+MOE_API moe_status moe_grouped_swiglu(int32_t rows, int32_t H, const moe_ffn_weights* w,
+                              const void* a, const float* a_scale,
+                              const int32_t* offsets, const float* row_w,
+                              void* h_ws, float* h_scale_ws, void* out,
+                              int32_t* dev_status, void* stream);
+
+/* The two halves of moe_grouped_swiglu, for callers that schedule or time
+ * them separately (same arguments and limits as above):
+ *   moe_gate_up_swiglu: h_ws = SiLU(a w1^T) * (a w3^T)        (w13 only)
+ *   moe_down_proj:      out  = row_w * (h w2^T), h given as  (w2 only)
+ *                       h [rows, I] (+ h_scale [rows, I/128] for E4M3). */
+MOE_API moe_status moe_gate_up_swiglu(int32_t rows, int32_t H, const moe_ffn_weights* w,
+                              const void* a, const float* a_scale,
+                              const int32_t* offsets, void* h_ws, float* h_scale_ws,
+                              int32_t* dev_status, void* stream);
+MOE_API moe_status moe_down_proj(int32_t rows, int32_t H, const moe_ffn_weights* w,
+                         const void* h, const float* h_scale, const int32_t* offsets,
+                         const float* row_w, void* out, int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * moe_combine -- unpermute and weighted combine, [MoE-walk] §3.4:
+ *   y[t] = shared_out[t] + sum_j topk_w[t][j] * expert_out[slot_to_row[t*k+j]]
+ * summed in fp32 in slot order j = 0..k-1, then rounded once to bf16.
+ * expert_out [T*k, H] bf16; slot_to_row [T*k]; topk_w [T, k] fp32 or NULL
+ * (weights already applied, e.g. via row_w in moe_grouped_swiglu);
+ * shared_out [T, H] bf16 or NULL; y [T, H] bf16 out. H % 8 == 0.
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_combine(int32_t T, int32_t k, int32_t H, const void* expert_out,
+                       const int32_t* slot_to_row, const float* topk_w,
+                       const void* shared_out, void* y, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * moe_bias_update -- aux-loss-free load balancing step, [V3-digest] §2.2:
+ * overloaded experts' selection bias goes down, underloaded ones' up:
+ *   bias[e] = bias[e] - gamma * sign(expert_counts[e] * E - T * k)
+ * The sign is taken on exact integers (load vs the mean T*k/E); the update
+ * is one fp32 subtraction. load_cv (optional, [1] fp32 out) receives the
+ * coefficient of variation of the counts, sample std (E-1) / mean
+ * ([V3-teardown] §4 load statistic). E <= 1024.
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_bias_update(int32_t E, int32_t T, int32_t k, const int32_t* expert_counts,
+                           float* bias, float gamma, float* load_cv, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * FP8 E4M3 quantisers ([V3-teardown] §3 infer.toml: weight_block_size
+ * [128, 128], activation_scheme dynamic; [FP8-infer] 1x128 / 128x128 tiles).
+ *   scale = amax / 448 in fp32 (1.0 for an all-zero tile);
+ *   code  = e4m3 round-to-nearest-even, saturating, of v / scale (fp32 div).
+ * moe_quantize_blocks: w [batch, N, K] bf16 -> q [batch, N, K] codes,
+ *   scale [batch, N/128, K/128]. N % 128 == 0, K % 128 == 0.
+ * moe_quantize_rows:   a [M, K] bf16 -> q [M, K] codes, scale [M, K/128].
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_quantize_blocks(int32_t batch, int32_t N, int32_t K, const void* w,
+                               void* q, float* scale, void* stream);
+MOE_API moe_status moe_quantize_rows(int32_t M, int32_t K, const void* a, void* q,
+                             float* scale, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * Status helpers.
+ * moe_read_device_status: copies *dev_status to *out after the work queued
+ *   on `stream` finishes (synchronises that stream) and maps it to a status:
+ *   0 -> MOE_OK, MOE_DEVSTAT_TIMEOUT -> MOE_ERR_DEVICE_TIMEOUT, any other
+ *   nonzero -> MOE_ERR_DEVICE_CHECK.
+ * moe_last_cuda_error: the cudaError_t behind the last MOE_ERR_CUDA on this
+ *   thread (0 if none).
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_read_device_status(const int32_t* dev_status, int32_t* out, void* stream);
+MOE_API int32_t moe_last_cuda_error(void);
+MOE_API const char* moe_status_string(moe_status s);
+MOE_API int32_t moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_MOE_H */

@@ -1,0 +1,315 @@
+// C-ABI entry points of libmoe (declared in include/moe.h): argument checks on
+// the host, TMA tensor-map encoding, kernel launches. No allocation happens
+// here; every buffer belongs to the caller.
+#include <mutex>
+
+#include "kernels.cuh"
+
+
+using namespace moe;
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+moe_status cuda_fail(int32_t code) {
+  g_last_cuda_error = code;
+  return MOE_ERR_CUDA;
+}
+
+moe_status check_launch(cudaError_t e) {
+  if (e != cudaSuccess) return cuda_fail(static_cast<int32_t>(e));
+  return MOE_OK;
+}
+
+bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+template <typename... P>
+bool any_misaligned(P... ps) {
+  return (misaligned(ps) || ...);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime (so the
+// library needs no link-time dependency on libcuda).
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major [outer, inner] matrix; box = 128 bytes of `inner` x box_rows rows,
+// 128-byte swizzle (the layout the tcgen05 smem descriptors expect).
+moe_status make_tmap(CUtensorMap* m, const void* ptr, bool one_byte, uint64_t inner, uint64_t outer,
+                     uint32_t box_rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return cuda_fail(static_cast<int32_t>(cudaErrorNotSupported));
+  const uint64_t esize = one_byte ? 1 : 2;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * esize};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(1000 + static_cast<int32_t>(r));
+  return MOE_OK;
+}
+
+moe_status sm_count(int* n) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return MOE_OK;
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+int32_t moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MOE_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_CHECK: return "device-side bounds check failed";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device-side bounded wait timed out";
+    default: return "unknown status";
+  }
+}
+
+moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_w, const float* sel_bias,
+                     float* logits, int32_t* topk_ids, float* topk_w, int32_t* expert_counts, void* stream) {
+  if (!p || !topk_ids || !topk_w || !expert_counts) return MOE_ERR_INVALID_ARG;
+  if (p->T < 1 || p->k < 1 || p->n_group < 1 || p->topk_group < 1) return MOE_ERR_INVALID_ARG;
+  if (p->scoring != MOE_SOFTMAX && p->scoring != MOE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (p->E < 1 || p->E % p->n_group != 0 || p->topk_group > p->n_group) return MOE_ERR_INVALID_ARG;
+  if (p->k > p->topk_group * (p->E / p->n_group)) return MOE_ERR_INVALID_ARG;
+  if (p->k > 16 || p->E > 256 || p->E < 16 || p->E % 16 != 0 || p->n_group > 32) return MOE_ERR_UNSUPPORTED;
+  if (x) {
+    if (!gate_w || p->H < 64) return MOE_ERR_INVALID_ARG;
+    if (p->H % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  } else if (!logits) {
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (any_misaligned(x, gate_w, sel_bias, logits, topk_ids, topk_w, expert_counts)) return MOE_ERR_ALIGNMENT;
+  cudaStream_t st = as_stream(stream);
+  RouteArgs r{p->T, p->H, p->E, p->k, p->n_group, p->topk_group, p->scoring, p->norm_topk_prob ? 1 : 0,
+              p->routed_scaling_factor, sel_bias, logits, topk_ids, topk_w, expert_counts, p->dev_status};
+  cudaError_t e = cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * p->E, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (x) {
+    CUtensorMap tmX, tmG;
+    moe_status s = make_tmap(&tmX, x, false, p->H, p->T, 128);
+    if (s != MOE_OK) return s;
+    s = make_tmap(&tmG, gate_w, false, p->H, p->E, static_cast<uint32_t>(p->E));
+    if (s != MOE_OK) return s;
+    return check_launch(launch_route_gemm(tmX, tmG, r, st));
+  }
+  return check_launch(launch_route_logits(r, st));
+}
+
+moe_status moe_permute_workspace_size(int32_t T, int32_t k, int32_t E, size_t* bytes) {
+  if (!bytes || T < 1 || k < 1 || E < 1) return MOE_ERR_INVALID_ARG;
+  *bytes = permute_workspace_bytes(T, E);
+  return MOE_OK;
+}
+
+moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t* topk_ids,
+                       const float* topk_w, const void* x, moe_dtype x_dtype, const float* x_scale,
+                       void* x_perm, float* x_perm_scale, int32_t* expert_offsets, int32_t* src_token,
+                       int32_t* slot_to_row, float* row_w, void* workspace, size_t workspace_bytes,
+                       int32_t* dev_status, void* stream) {
+  if (T < 1 || k < 1 || E < 1 || H < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (!topk_ids || !expert_offsets || !src_token || !slot_to_row || !workspace) return MOE_ERR_INVALID_ARG;
+  if (row_w && !topk_w) return MOE_ERR_INVALID_ARG;
+  if (x_perm && !x) return MOE_ERR_INVALID_ARG;
+  if (x_dtype != MOE_BF16 && x_dtype != MOE_E4M3) return MOE_ERR_INVALID_ARG;
+  if (k > 16 || E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * k > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  int row_bytes = 0, nscale = 0;
+  if (x_dtype == MOE_BF16) {
+    if (H % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    row_bytes = 2 * H;
+  } else {
+    if (H % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (x_perm && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
+    row_bytes = H;
+    nscale = H / 128;
+  }
+  if (workspace_bytes < permute_workspace_bytes(T, E)) return MOE_ERR_INVALID_ARG;
+  if (any_misaligned(topk_ids, topk_w, x, x_scale, x_perm, x_perm_scale, expert_offsets, src_token,
+                     slot_to_row, row_w, workspace))
+    return MOE_ERR_ALIGNMENT;
+  return check_launch(launch_permute(T, k, E, row_bytes, topk_ids, topk_w, x, x_dtype == MOE_E4M3 ? x_scale : nullptr,
+                                     nscale, x_perm, x_perm_scale, expert_offsets, src_token, slot_to_row,
+                                     row_w, static_cast<int32_t*>(workspace), dev_status, as_stream(stream)));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shared checks of the grouped SwiGLU calls; `a` is the GEMM's activation
+// operand (x for the first GEMM, h for the second).
+moe_status check_ffn(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a,
+                     const float* a_scale, bool need_w13, bool need_w2) {
+  if (!w || !a) return MOE_ERR_INVALID_ARG;
+  if ((need_w13 && !w->w13) || (need_w2 && !w->w2)) return MOE_ERR_INVALID_ARG;
+  if (rows < 1 || H < 1 || w->I < 1 || w->groups < 1) return MOE_ERR_INVALID_ARG;
+  if (w->dtype != MOE_BF16 && w->dtype != MOE_E4M3) return MOE_ERR_INVALID_ARG;
+  if (H % 256 != 0 || w->I % 128 != 0 || w->groups > 512) return MOE_ERR_UNSUPPORTED;
+  if (w->dtype == MOE_E4M3) {
+    if ((need_w13 && !w->w13_scale) || (need_w2 && !w->w2_scale) || !a_scale) return MOE_ERR_INVALID_ARG;
+    if (H > 8192 || w->I > 8192) return MOE_ERR_UNSUPPORTED;
+  }
+  if (static_cast<long long>(w->groups) * 2 * w->I > 0x7fffffffLL ||
+      static_cast<long long>(w->groups) * H > 0x7fffffffLL)
+    return MOE_ERR_UNSUPPORTED;
+  if (any_misaligned(w->w13, w->w2, w->w13_scale, w->w2_scale, a, a_scale)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+moe_status run_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a,
+                       const float* a_scale, const int32_t* offsets, void* h_ws, float* h_scale_ws,
+                       int32_t* dev_status, cudaStream_t st, int nsm) {
+  const bool fp8 = w->dtype == MOE_E4M3;
+  const int I = w->I;
+  CUtensorMap tmA, tmB;
+  moe_status s = make_tmap(&tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
+  if (s != MOE_OK) return s;
+  s = make_tmap(&tmB, a, fp8, H, rows, 32);
+  if (s != MOE_OK) return s;
+  GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : 256,
+              h_ws, I, nullptr, w->w13_scale, a_scale, h_scale_ws, dev_status};
+  return check_launch(launch_grouped_gemm(fp8, EPI_SWIGLU, tmA, tmB, g1, nsm, st));
+}
+
+moe_status run_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* h, const float* h_scale,
+                    const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status,
+                    cudaStream_t st, int nsm) {
+  const bool fp8 = w->dtype == MOE_E4M3;
+  const int I = w->I;
+  CUtensorMap tmA, tmB;
+  moe_status s = make_tmap(&tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H, 128);
+  if (s != MOE_OK) return s;
+  s = make_tmap(&tmB, h, fp8, I, rows, 32);
+  if (s != MOE_OK) return s;
+  GemmArgs g2{rows, I, w->groups, offsets, H, H / 256, 256, 128, 256, 128, fp8 ? 32 : 256,
+              out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
+  return check_launch(launch_grouped_gemm(fp8, EPI_WEIGHTED, tmA, tmB, g2, nsm, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_gate_up_swiglu(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a,
+                              const float* a_scale, const int32_t* offsets, void* h_ws, float* h_scale_ws,
+                              int32_t* dev_status, void* stream) {
+  moe_status s = check_ffn(rows, H, w, a, a_scale, true, false);
+  if (s != MOE_OK) return s;
+  if (!h_ws || (!offsets && w->groups != 1)) return MOE_ERR_INVALID_ARG;
+  if (w->dtype == MOE_E4M3 && !h_scale_ws) return MOE_ERR_INVALID_ARG;
+  if (any_misaligned(offsets, h_ws, h_scale_ws)) return MOE_ERR_ALIGNMENT;
+  int nsm = 0;
+  if ((s = sm_count(&nsm)) != MOE_OK) return s;
+  return run_gate_up(rows, H, w, a, a_scale, offsets, h_ws, h_scale_ws, dev_status, as_stream(stream), nsm);
+}
+
+moe_status moe_down_proj(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* h, const float* h_scale,
+                         const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status,
+                         void* stream) {
+  moe_status s = check_ffn(rows, H, w, h, h_scale, false, true);
+  if (s != MOE_OK) return s;
+  if (!out || (!offsets && w->groups != 1)) return MOE_ERR_INVALID_ARG;
+  if (any_misaligned(offsets, row_w, out)) return MOE_ERR_ALIGNMENT;
+  int nsm = 0;
+  if ((s = sm_count(&nsm)) != MOE_OK) return s;
+  return run_down(rows, H, w, h, h_scale, offsets, row_w, out, dev_status, as_stream(stream), nsm);
+}
+
+moe_status moe_grouped_swiglu(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a,
+                              const float* a_scale, const int32_t* offsets, const float* row_w,
+                              void* h_ws, float* h_scale_ws, void* out, int32_t* dev_status, void* stream) {
+  moe_status s = check_ffn(rows, H, w, a, a_scale, true, true);
+  if (s != MOE_OK) return s;
+  if (!h_ws || !out || (!offsets && w->groups != 1)) return MOE_ERR_INVALID_ARG;
+  if (w->dtype == MOE_E4M3 && !h_scale_ws) return MOE_ERR_INVALID_ARG;
+  if (any_misaligned(offsets, row_w, h_ws, h_scale_ws, out)) return MOE_ERR_ALIGNMENT;
+  int nsm = 0;
+  if ((s = sm_count(&nsm)) != MOE_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  s = run_gate_up(rows, H, w, a, a_scale, offsets, h_ws, h_scale_ws, dev_status, st, nsm);
+  if (s != MOE_OK) return s;
+  return run_down(rows, H, w, h_ws, h_scale_ws, offsets, row_w, out, dev_status, st, nsm);
+}
+
+moe_status moe_combine(int32_t T, int32_t k, int32_t H, const void* expert_out, const int32_t* slot_to_row,
+                       const float* topk_w, const void* shared_out, void* y, void* stream) {
+  if (T < 1 || k < 1 || H < 1 || !expert_out || !slot_to_row || !y) return MOE_ERR_INVALID_ARG;
+  if (k > 16 || H % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (any_misaligned(expert_out, slot_to_row, topk_w, shared_out, y)) return MOE_ERR_ALIGNMENT;
+  return check_launch(launch_combine(T, k, H, expert_out, slot_to_row, topk_w, shared_out, y, as_stream(stream)));
+}
+
+moe_status moe_bias_update(int32_t E, int32_t T, int32_t k, const int32_t* expert_counts, float* bias,
+                           float gamma, float* load_cv, void* stream) {
+  if (E < 1 || T < 1 || k < 1 || !expert_counts || !bias) return MOE_ERR_INVALID_ARG;
+  if (E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (any_misaligned(expert_counts, bias, load_cv)) return MOE_ERR_ALIGNMENT;
+  return check_launch(launch_bias_update(E, T, k, expert_counts, bias, gamma, load_cv, as_stream(stream)));
+}
+
+moe_status moe_quantize_blocks(int32_t batch, int32_t N, int32_t K, const void* w, void* q, float* scale,
+                               void* stream) {
+  if (batch < 1 || N < 1 || K < 1 || !w || !q || !scale) return MOE_ERR_INVALID_ARG;
+  if (N % 128 != 0 || K % 128 != 0 || batch > 65535 || N / 128 > 65535) return MOE_ERR_UNSUPPORTED;
+  if (any_misaligned(w, q, scale)) return MOE_ERR_ALIGNMENT;
+  return check_launch(launch_quant_blocks(batch, N, K, w, q, scale, as_stream(stream)));
+}
+
+moe_status moe_quantize_rows(int32_t M, int32_t K, const void* a, void* q, float* scale, void* stream) {
+  if (M < 1 || K < 1 || !a || !q || !scale) return MOE_ERR_INVALID_ARG;
+  if (K % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (any_misaligned(a, q, scale)) return MOE_ERR_ALIGNMENT;
+  return check_launch(launch_quant_rows(M, K, a, q, scale, as_stream(stream)));
+}
+
+moe_status moe_read_device_status(const int32_t* dev_status, int32_t* out, void* stream) {
+  if (!dev_status || !out) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *out = v;
+  if (v == 0) return MOE_OK;
+  if (v == MOE_DEVSTAT_TIMEOUT) return MOE_ERR_DEVICE_TIMEOUT;
+  return MOE_ERR_DEVICE_CHECK;
+}
+
+}  // extern "C"

@@ -1,0 +1,540 @@
+// Grouped SwiGLU expert GEMMs on the 5th-generation tensor cores (tcgen05).
+//
+// The layer's experts ("MoE 混合专家模型推理参数与前向传播详解" §3.3.1):
+//   gate_up = x @ w13[e]^T ; h = SiLU(gate_up[:, :I]) * gate_up[:, I:]
+//   out     = h @ w2[e]^T  (times the row's routing weight, §3.4)
+// run for every expert in one launch over the expert-contiguous rows produced
+// by the permutation (§3.2), i.e. a grouped GEMM segmented by expert offsets.
+//
+// Orientation (swap-AB): the weight matrix is the MMA's A operand (M = 128
+// weight rows per tcgen05.mma) and the segment's token rows are the B operand
+// (N = 16..256 tokens, variable per tile). A segment of n rows costs
+// round_up(n, 16) columns, so ragged segment ends waste at most 15 columns,
+// instead of most of a 128-row tile when tokens sit on the M side.
+//
+// Tile = (expert g, weight block mb, token block tb). Each tile holds two
+// 128-row sub-tiles of the weight, accumulated side by side in TMEM:
+//   GEMM1: sub-tile 0 = gate rows [mb*128, +128), sub-tile 1 = up rows
+//          [I + mb*128, +128): the epilogue has gate and up of the same
+//          feature in the same thread and fuses SiLU(gate) * up.
+//   GEMM2: sub-tiles = w2 rows [mb*256, +128) and [mb*256 + 128, +128); the
+//          epilogue multiplies by the routing weight of the row.
+// TMEM: sub-tile s accumulates in columns [s*256, s*256 + N) (fp32).
+//
+// Warp roles (192 threads, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer (A: two 128x64 boxes, B: ceil(N/32) 32x64 boxes
+//               per 64-wide K block, 128-byte swizzle) into an S-stage ring;
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer;
+//   warps 2..5  epilogue: tcgen05.ld (warp w owns TMEM lanes 32*(w%4)..+31),
+//               fused activation / weighting, bf16 stores.
+// The E4M3 variant accumulates each 128-wide K block separately in a TMEM
+// ring and promotes it with the fp32 block scales on the CUDA cores, since
+// the weight scale is per 128x128 block and the activation scale per 1x128.
+#include "kernels.cuh"
+
+namespace moe {
+
+
+
+constexpr int kMaxGroups = 512;
+constexpr int kThreads = 192;
+
+struct TileInfo {
+  int g, mb, row0, n_valid, N;
+};
+
+// Per-CTA copy of the tile schedule: tile_start[g] = first tile of group g.
+struct Sched {
+  int tile_start[kMaxGroups + 1];
+  int seg_start[kMaxGroups + 1];
+};
+
+__device__ __forceinline__ int tiles_of(int n, int bn_max, int n_mblk) {
+  return n <= 0 ? 0 : ((n + bn_max - 1) / bn_max) * n_mblk;
+}
+
+// Warp-cooperative build of the schedule (called by one warp).
+__device__ void build_schedule(Sched& s, const GemmArgs& a, int lane) {
+  int carry = 0;
+  for (int base = 0; base < a.groups; base += 32) {
+    const int g = base + lane;
+    int st = 0, n = 0;
+    if (g < a.groups) {
+      if (a.offsets) {
+        st = a.offsets[g];
+        n = a.offsets[g + 1] - st;
+      } else {
+        st = 0;
+        n = a.rows;
+      }
+    }
+    int t = (g < a.groups) ? tiles_of(n, a.bn_max, a.n_mblk) : 0;
+    int incl = t;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      int v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    if (g < a.groups) {
+      s.tile_start[g] = carry + incl - t;
+      s.seg_start[g] = st;
+    }
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) {
+    s.tile_start[a.groups] = carry;
+    s.seg_start[a.groups] = a.offsets ? a.offsets[a.groups] : a.rows;
+  }
+}
+
+__device__ __forceinline__ TileInfo decode_tile(const Sched& s, const GemmArgs& a, int t) {
+  int lo = 0, hi = a.groups - 1;   // last g with tile_start[g] <= t
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (s.tile_start[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  TileInfo ti;
+  ti.g = lo;
+  const int n = s.seg_start[lo + 1] - s.seg_start[lo];
+  const int ntb = (n + a.bn_max - 1) / a.bn_max;
+  const int bn = ((((n + ntb - 1) / ntb) + 15) / 16) * 16;
+  const int local = t - s.tile_start[lo];
+  const int tb = local / a.n_mblk;
+  ti.mb = local - tb * a.n_mblk;
+  ti.row0 = s.seg_start[lo] + tb * bn;
+  ti.n_valid = min(bn, n - tb * bn);
+  ti.N = ((ti.n_valid + 15) / 16) * 16;
+  return ti;
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+
+// ========================================================================
+// BF16 kernel
+// ========================================================================
+template <int EPI, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
+  constexpr int KB = 64;                           // K elements per stage (128 B)
+  constexpr uint32_t A_SUB_BYTES = 128 * 128;      // one 128-row sub-tile
+  extern __shared__ __align__(1024) uint8_t dsmem[];
+  __shared__ Sched sched;
+  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
+  __shared__ uint64_t tmem_full, tmem_empty, drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int issued_parity[STAGES];
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  const uint32_t b_stage_bytes = static_cast<uint32_t>(a.bn_max) * 128u;
+  const uint32_t stage_bytes = 2 * A_SUB_BYTES + b_stage_bytes;
+  auto sA = [&](int st, int sub) { return smem + st * stage_bytes + sub * A_SUB_BYTES; };
+  auto sB = [&](int st) { return smem + st * stage_bytes + 2 * A_SUB_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+      issued_parity[i] = -1;
+    }
+    mbar_init(&tmem_full, 1);
+    mbar_init(&tmem_empty, 128);
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, 512);
+    tmem_relinquish();
+  }
+  if (warp == 2) build_schedule(sched, a, lane);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int total = sched.tile_start[a.groups];
+  const int nk = a.K / KB;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < total && !abort_flag; t += gridDim.x) {
+        const TileInfo ti = decode_tile(sched, a, t);
+        const int a_row0 = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride;
+        const int a_row1 = a_row0 + a.sub1_off;
+        const int nload = (ti.N + 31) / 32;
+        const uint32_t bytes = 2 * A_SUB_BYTES + static_cast<uint32_t>(nload) * 32u * 128u;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_bar[stage], bytes);
+          tma_load_2d(sA(stage, 0), &tmA, &full_bar[stage], kb * KB, a_row0, pol_w);
+          tma_load_2d(sA(stage, 1), &tmA, &full_bar[stage], kb * KB, a_row1, pol_w);
+          for (int i = 0; i < nload; ++i)
+            tma_load_2d(sB(stage) + i * 4096, &tmB, &full_bar[stage], kb * KB, ti.row0 + 32 * i, pol_x);
+          issued_parity[stage] = static_cast<int>(phase);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      if (abort_flag) {   // let every issued copy land before the CTA exits
+        for (int i = 0; i < STAGES; ++i)
+          if (issued_parity[i] >= 0) mbar_wait_drain(&full_bar[i], static_cast<uint32_t>(issued_parity[i]));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      for (int t = blockIdx.x; t < total && !abort_flag; t += gridDim.x) {
+        const TileInfo ti = decode_tile(sched, a, t);
+        const uint32_t idesc = make_idesc(1u, 128u, static_cast<uint32_t>(ti.N));
+        if (!mbar_wait(&tmem_empty, acc_phase ^ 1u, &abort_flag, a.status)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA(stage, 0)), a1 = smem_u32(sA(stage, 1));
+          const uint32_t b0 = smem_u32(sB(stage));
+#pragma unroll
+          for (int kk = 0; kk < KB / 16; ++kk) {
+            const uint32_t acc = (kb | kk) != 0;
+            const uint64_t bd = sw128_desc(b0 + kk * 32);
+            umma_bf16(tmem_base, sw128_desc(a0 + kk * 32), bd, idesc, acc);
+            umma_bf16(tmem_base + 256, sw128_desc(a1 + kk * 32), bd, idesc, acc);
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tmem_full);
+        acc_phase ^= 1u;
+      }
+      // all issued MMAs must finish before TMEM is released
+      umma_commit(&drain_bar);
+      mbar_wait_drain(&drain_bar, 0);
+    }
+  } else {
+    // epilogue warps 2..5
+    const int q = warp & 3;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    uint32_t acc_phase = 0;
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const TileInfo ti = decode_tile(sched, a, t);
+      if (!mbar_wait(&tmem_full, acc_phase, &abort_flag, a.status)) break;
+      tc_fence_after();
+      const int nchunk = (ti.N + 31) / 32;
+      if (EPI == EPI_SWIGLU) {
+        const int feat = ti.mb * a.feat_stride + 32 * q + lane;
+        for (int c = 0; c < nchunk; ++c) {
+          float g[32], u[32];
+          tmem_ld32(lane_addr + c * 32, g);
+          tmem_ld32(lane_addr + 256 + c * 32, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int tok = c * 32 + j;
+            if (tok < ti.n_valid)
+              out[static_cast<size_t>(ti.row0 + tok) * a.out_ld + feat] = __float2bfloat16_rn(silu(g[j]) * u[j]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int s = 0; s < 2; ++s) {
+          const int feat = ti.mb * a.feat_stride + s * a.feat_sub1 + 32 * q + lane;
+          for (int c = 0; c < nchunk; ++c) {
+            float v[32];
+            tmem_ld32(lane_addr + s * 256 + c * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int tok = c * 32 + j;
+              if (tok < ti.n_valid) {
+                const float w = a.row_w ? __ldg(a.row_w + ti.row0 + tok) : 1.0f;
+                out[static_cast<size_t>(ti.row0 + tok) * a.out_ld + feat] = __float2bfloat16_rn(v[j] * w);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tmem_empty);
+      acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+// ========================================================================
+// E4M3 kernel (block-scaled, promotion on CUDA cores), tokens per tile <= 32
+// ========================================================================
+constexpr int kF8Bn = 32;          // max tokens per tile
+constexpr int kF8Slots = 8;        // TMEM ring of per-K-block partial sums
+constexpr int kF8SlotCols = 2 * kF8Bn;
+constexpr int kF8MaxKb = 64;       // K <= 8192
+
+template <int EPI, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
+  constexpr int KB = 128;                          // K elements per stage (128 B)
+  constexpr uint32_t A_SUB_BYTES = 128 * 128;
+  constexpr uint32_t B_BYTES = kF8Bn * 128;
+  constexpr uint32_t STAGE_BYTES = 2 * A_SUB_BYTES + B_BYTES;
+  extern __shared__ __align__(1024) uint8_t dsmem[];
+  __shared__ Sched sched;
+  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
+  __shared__ uint64_t part_full[kF8Slots], part_empty[kF8Slots];
+  __shared__ uint64_t drain_bar, epi_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int issued_parity[STAGES];
+  __shared__ volatile int abort_flag;
+  __shared__ float bscale_s[kF8Bn * kF8MaxKb];
+  __shared__ float red_s[4][kF8Bn];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  auto sA = [&](int st, int sub) { return smem + st * STAGE_BYTES + sub * A_SUB_BYTES; };
+  auto sB = [&](int st) { return smem + st * STAGE_BYTES + 2 * A_SUB_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+      issued_parity[i] = -1;
+    }
+    for (int i = 0; i < kF8Slots; ++i) {
+      mbar_init(&part_full[i], 1);
+      mbar_init(&part_empty[i], 128);
+    }
+    mbar_init(&drain_bar, 1);
+    mbar_init(&epi_bar, 128);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, 512);
+    tmem_relinquish();
+  }
+  if (warp == 2) build_schedule(sched, a, lane);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int total = sched.tile_start[a.groups];
+  const int nk = a.K / KB;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < total && !abort_flag; t += gridDim.x) {
+        const TileInfo ti = decode_tile(sched, a, t);
+        const int a_row0 = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride;
+        const int a_row1 = a_row0 + a.sub1_off;
+        const uint32_t bytes = 2 * A_SUB_BYTES + B_BYTES;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_bar[stage], bytes);
+          tma_load_2d(sA(stage, 0), &tmA, &full_bar[stage], kb * KB, a_row0, pol_w);
+          tma_load_2d(sA(stage, 1), &tmA, &full_bar[stage], kb * KB, a_row1, pol_w);
+          tma_load_2d(sB(stage), &tmB, &full_bar[stage], kb * KB, ti.row0, pol_x);
+          issued_parity[stage] = static_cast<int>(phase);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      if (abort_flag) {
+        for (int i = 0; i < STAGES; ++i)
+          if (issued_parity[i] >= 0) mbar_wait_drain(&full_bar[i], static_cast<uint32_t>(issued_parity[i]));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t kbg = 0;   // K blocks issued so far (TMEM ring position)
+      for (int t = blockIdx.x; t < total && !abort_flag; t += gridDim.x) {
+        const TileInfo ti = decode_tile(sched, a, t);
+        const uint32_t idesc = make_idesc(0u, 128u, static_cast<uint32_t>(ti.N));
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb, ++kbg) {
+          const uint32_t slot = kbg % kF8Slots;
+          const uint32_t slot_phase = (kbg / kF8Slots) & 1u;
+          if (!mbar_wait(&part_empty[slot], slot_phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem_base + slot * kF8SlotCols;
+          const uint32_t a0 = smem_u32(sA(stage, 0)), a1 = smem_u32(sA(stage, 1));
+          const uint32_t b0 = smem_u32(sB(stage));
+#pragma unroll
+          for (int kk = 0; kk < KB / 32; ++kk) {
+            const uint64_t bd = sw128_desc(b0 + kk * 32);
+            umma_e4m3(d, sw128_desc(a0 + kk * 32), bd, idesc, kk != 0);
+            umma_e4m3(d + kF8Bn, sw128_desc(a1 + kk * 32), bd, idesc, kk != 0);
+          }
+          umma_commit(&empty_bar[stage]);
+          umma_commit(&part_full[slot]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      umma_commit(&drain_bar);
+      mbar_wait_drain(&drain_bar, 0);
+    }
+  } else {
+    const int q = warp & 3;
+    const int et = threadIdx.x - 64;            // 0..127
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    const int nkb_a = a.K / 128;
+    const int a_blk_rows = a.a_rows_per_group / 128;
+    uint32_t kbg = 0, epi_phase = 0;
+    bool ok = true;
+    // Bounded sync of the 128 epilogue threads (an abort ends it, never hangs).
+    auto epi_sync = [&]() -> bool {
+      mbar_arrive(&epi_bar);
+      const bool r = mbar_wait(&epi_bar, epi_phase, &abort_flag, a.status);
+      epi_phase ^= 1u;
+      return r;
+    };
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const TileInfo ti = decode_tile(sched, a, t);
+      // activation scales of this tile's rows -> smem
+      if (!epi_sync()) break;
+      for (int i = et; i < kF8Bn * nk; i += 128) {
+        const int r = i / nk, kb = i - r * nk;
+        bscale_s[r * kF8MaxKb + kb] = (r < ti.n_valid) ? a.b_scale[static_cast<size_t>(ti.row0 + r) * nk + kb] : 0.0f;
+      }
+      if (!epi_sync()) break;
+      const int a_row0 = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride;
+      const int a_row1 = a_row0 + a.sub1_off;
+      const float* as_g = a.a_scale + static_cast<size_t>(ti.g) * a_blk_rows * nkb_a;
+      const float* as0 = as_g + static_cast<size_t>((a_row0 - ti.g * a.a_rows_per_group) / 128) * nkb_a;
+      const float* as1 = as_g + static_cast<size_t>((a_row1 - ti.g * a.a_rows_per_group) / 128) * nkb_a;
+      float acc0[kF8Bn], acc1[kF8Bn];
+#pragma unroll
+      for (int j = 0; j < kF8Bn; ++j) { acc0[j] = 0.f; acc1[j] = 0.f; }
+      for (int kb = 0; kb < nk; ++kb, ++kbg) {
+        const uint32_t slot = kbg % kF8Slots;
+        const uint32_t slot_phase = (kbg / kF8Slots) & 1u;
+        if (!mbar_wait(&part_full[slot], slot_phase, &abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        float v0[32], v1[32];
+        tmem_ld32(lane_addr + slot * kF8SlotCols, v0);
+        tmem_ld32(lane_addr + slot * kF8SlotCols + kF8Bn, v1);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&part_empty[slot]);
+        const float s0 = __ldg(as0 + kb), s1 = __ldg(as1 + kb);
+#pragma unroll
+        for (int j = 0; j < kF8Bn; ++j) {
+          const float sb = bscale_s[j * kF8MaxKb + kb];
+          acc0[j] = fmaf(v0[j], s0 * sb, acc0[j]);
+          acc1[j] = fmaf(v1[j], s1 * sb, acc1[j]);
+        }
+      }
+      if (!ok) break;
+      if (EPI == EPI_SWIGLU) {
+        // h for feature mb*128 + (this thread's TMEM lane), tokens j;
+        // 1x128 quantisation along I (the 128 lanes of the tile)
+        const int feat = ti.mb * a.feat_stride + 32 * q + lane;
+        float h[kF8Bn];
+#pragma unroll
+        for (int j = 0; j < kF8Bn; ++j) {
+          h[j] = silu(acc0[j]) * acc1[j];
+          float m = fabsf(h[j]);
+#pragma unroll
+          for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+          if (lane == 0) red_s[q][j] = m;
+        }
+        if (!epi_sync()) break;
+        uint8_t* outq = reinterpret_cast<uint8_t*>(a.out);
+        const int nsc = a.out_ld / 128;
+#pragma unroll
+        for (int j = 0; j < kF8Bn; ++j) {
+          if (j < ti.n_valid) {
+            const float amax = fmaxf(fmaxf(red_s[0][j], red_s[1][j]), fmaxf(red_s[2][j], red_s[3][j]));
+            const float sc = amax == 0.0f ? 1.0f : amax / 448.0f;
+            outq[static_cast<size_t>(ti.row0 + j) * a.out_ld + feat] = to_e4m3(h[j] / sc);
+            if (et == j) a.out_scale[static_cast<size_t>(ti.row0 + j) * nsc + ti.mb] = sc;
+          }
+        }
+      } else {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+        const int f0 = ti.mb * a.feat_stride + 32 * q + lane;
+        const int f1 = f0 + a.feat_sub1;
+#pragma unroll
+        for (int j = 0; j < kF8Bn; ++j) {
+          if (j < ti.n_valid) {
+            const float w = a.row_w ? __ldg(a.row_w + ti.row0 + j) : 1.0f;
+            const size_t r = static_cast<size_t>(ti.row0 + j) * a.out_ld;
+            out[r + f0] = __float2bfloat16_rn(acc0[j] * w);
+            out[r + f1] = __float2bfloat16_rn(acc1[j] * w);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+// ------------------------------------------------------------------------
+// host-side launch helpers (called from api.cu)
+// ------------------------------------------------------------------------
+size_t gemm_bf16_smem_bytes(int stages, int bn_max) {
+  return static_cast<size_t>(stages) * (2 * 128 * 128 + static_cast<size_t>(bn_max) * 128) + 1024;
+}
+size_t gemm_e4m3_smem_bytes(int stages) {
+  return static_cast<size_t>(stages) * (2 * 128 * 128 + kF8Bn * 128) + 1024;
+}
+
+constexpr int kBf16Stages = 3;
+constexpr int kE4m3Stages = 4;
+
+cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                const GemmArgs& a, int grid, cudaStream_t stream) {
+  if (!e4m3) {
+    const size_t smem = gemm_bf16_smem_bytes(kBf16Stages, a.bn_max);
+    auto kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages>
+                                  : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, smem, stream>>>(tmA, tmB, a);
+  } else {
+    const size_t smem = gemm_e4m3_smem_bytes(kE4m3Stages);
+    auto kern = epi == EPI_SWIGLU ? grouped_gemm_e4m3_kernel<EPI_SWIGLU, kE4m3Stages>
+                                  : grouped_gemm_e4m3_kernel<EPI_WEIGHTED, kE4m3Stages>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, smem, stream>>>(tmA, tmB, a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

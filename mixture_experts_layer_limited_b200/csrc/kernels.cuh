@@ -1,0 +1,62 @@
+// Argument blocks and launchers shared by the kernels and the C-ABI layer.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+struct GemmArgs {
+  int32_t rows;              // activation rows (B operand)
+  int32_t K;                 // reduction length
+  int32_t groups;            // number of segments
+  const int32_t* offsets;    // [groups + 1] or nullptr (one segment)
+  int32_t a_rows_per_group;  // weight rows per group (2I or H)
+  int32_t n_mblk;            // weight blocks per group
+  int32_t mblk_stride;       // weight-row stride between blocks (128 / 256)
+  int32_t sub1_off;          // weight-row offset of sub-tile 1 (I / 128)
+  int32_t feat_stride;       // output-feature stride between blocks (128 / 256)
+  int32_t feat_sub1;         // output-feature offset of sub-tile 1 (0 / 128)
+  int32_t bn_max;            // max tokens per tile (multiple of 32, <= 256)
+  void* out;                 // [rows, out_ld] bf16, or e4m3 codes (GEMM1 FP8)
+  int32_t out_ld;
+  const float* row_w;        // [rows] or nullptr
+  const float* a_scale;      // E4M3: [groups, a_rows_per_group/128, K/128]
+  const float* b_scale;      // E4M3: [rows, K/128]
+  float* out_scale;          // E4M3 GEMM1: [rows, out_ld/128]
+  int32_t* status;
+};
+
+struct RouteArgs {
+  int32_t T, H, E, k, G, g;
+  int32_t scoring, norm;
+  float scale;
+  const float* bias;        // [E] or nullptr
+  float* logits;            // [T, E] (out for the GEMM kernel when non-null, in for the other)
+  int32_t* ids;             // [T, k]
+  float* w;                 // [T, k]
+  int32_t* counts;          // [E], zeroed beforehand
+  int32_t* status;
+};
+
+enum { EPI_SWIGLU = 0, EPI_WEIGHTED = 1 };
+
+cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                const GemmArgs& a, int grid, cudaStream_t stream);
+cudaError_t launch_route_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
+                              cudaStream_t stream);
+cudaError_t launch_route_logits(const RouteArgs& r, cudaStream_t stream);
+size_t permute_workspace_bytes(int T, int E);
+cudaError_t launch_permute(int T, int k, int E, int row_bytes, const int32_t* ids, const float* topk_w,
+                           const void* x, const float* x_scale, int nscale, void* x_perm,
+                           float* x_perm_scale, int32_t* offsets, int32_t* src_token,
+                           int32_t* slot_to_row, float* row_w, int32_t* blockhist, int32_t* status,
+                           cudaStream_t stream);
+cudaError_t launch_combine(int T, int k, int H, const void* eo, const int32_t* slot_to_row,
+                           const float* topk_w, const void* shared, void* y, cudaStream_t stream);
+cudaError_t launch_bias_update(int E, int T, int k, const int32_t* counts, float* bias, float gamma,
+                               float* load_cv, cudaStream_t stream);
+cudaError_t launch_quant_blocks(int batch, int N, int K, const void* w, void* q, float* scale,
+                                cudaStream_t stream);
+cudaError_t launch_quant_rows(int M, int K, const void* a, void* q, float* scale, cudaStream_t stream);
+
+}  // namespace moe

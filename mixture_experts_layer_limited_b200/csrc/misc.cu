@@ -1,0 +1,223 @@
+// Combine, aux-loss-free bias update and E4M3 quantisers.
+#include "kernels.cuh"
+
+namespace moe {
+
+constexpr int kCombKMax = 16;
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 p = __bfloat1622float2(h[i]);
+    f[2 * i] = p.x;
+    f[2 * i + 1] = p.y;
+  }
+}
+
+__device__ __forceinline__ uint4 f32_to_bf16x8(const float (&f)[8]) {
+  uint4 v;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  return v;
+}
+
+// Unpermute + weighted combine ("MoE 混合专家模型推理参数与前向传播详解" §3.4):
+// y[t] = shared[t] + sum_j w[t][j] * expert_out[slot_to_row[t*k+j]], fp32 sum in
+// slot order, one bf16 rounding. One warp per token, 16-byte vectors.
+__global__ void __launch_bounds__(256)
+combine_kernel(int T, int k, int vec_per_row, const uint4* __restrict__ eo,
+               const int32_t* __restrict__ slot_to_row, const float* __restrict__ topk_w,
+               const uint4* __restrict__ shared, uint4* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;                       // warp-uniform
+  const int nrows = T * k;
+  int my_row = lane < k ? slot_to_row[static_cast<size_t>(t) * k + lane] : -1;
+  if (my_row >= nrows) my_row = -1;
+  const float my_w = (lane < k && topk_w) ? topk_w[static_cast<size_t>(t) * k + lane] : 1.0f;
+  int rows[kCombKMax];
+  float ws[kCombKMax];
+#pragma unroll
+  for (int j = 0; j < kCombKMax; ++j) {
+    rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+    ws[j] = __shfl_sync(0xffffffffu, my_w, j);
+  }
+  for (int v = lane; v < vec_per_row; v += 32) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    uint4 raw[kCombKMax];
+#pragma unroll
+    for (int j = 0; j < kCombKMax; ++j)
+      if (j < k && rows[j] >= 0) raw[j] = __ldg(eo + static_cast<size_t>(rows[j]) * vec_per_row + v);
+#pragma unroll
+    for (int j = 0; j < kCombKMax; ++j) {
+      if (j < k && rows[j] >= 0) {
+        float f[8];
+        bf16x8_to_f32(raw[j], f);
+        if (topk_w) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] += ws[j] * f[i];
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] += f[i];
+        }
+      }
+    }
+    if (shared) {
+      float f[8];
+      bf16x8_to_f32(__ldg(shared + static_cast<size_t>(t) * vec_per_row + v), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += f[i];
+    }
+    y[static_cast<size_t>(t) * vec_per_row + v] = f32_to_bf16x8(acc);
+  }
+}
+
+// Aux-loss-free bias step (xxqk.cn digest §2.2): overloaded experts' bias
+// down by gamma, underloaded up, compared with the mean load exactly.
+// Optional load CV = sample std / mean (gsyq.cn teardown §4).
+__global__ void __launch_bounds__(1024)
+bias_update_kernel(int E, int T, int k, const int32_t* __restrict__ counts, float* __restrict__ bias,
+                   float gamma, float* __restrict__ load_cv) {
+  __shared__ double red[32];
+  __shared__ double mean_s;
+  const int e = threadIdx.x;
+  const long long c = e < E ? static_cast<long long>(counts[e]) : 0;
+  if (e < E) {
+    const long long d = c * E - static_cast<long long>(T) * k;
+    const float s = d > 0 ? 1.0f : (d < 0 ? -1.0f : 0.0f);
+    bias[e] = bias[e] - gamma * s;
+  }
+  if (!load_cv) return;                     // block-uniform
+  const int lane = e & 31, warp = e >> 5;
+  double v = static_cast<double>(c);
+  for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (e == 0) {
+    double s = 0.0;
+    for (int w = 0; w < 32; ++w) s += red[w];
+    mean_s = s / E;
+  }
+  __syncthreads();
+  const double dm = e < E ? static_cast<double>(c) - mean_s : 0.0;
+  v = dm * dm;
+  for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (e == 0) {
+    double s = 0.0;
+    for (int w = 0; w < 32; ++w) s += red[w];
+    const double sd = E > 1 ? sqrt(s / (E - 1)) : 0.0;
+    *load_cv = static_cast<float>(mean_s > 0.0 ? sd / mean_s : 0.0);
+  }
+}
+
+// E4M3 weight quantisation per 128x128 block. grid (K/128, N/128, batch),
+// 256 threads: thread i covers row i/2, columns (i%2)*64 .. +64.
+__global__ void __launch_bounds__(256)
+quant_blocks_kernel(const __nv_bfloat16* __restrict__ w, int N, int K, uint8_t* __restrict__ q,
+                    float* __restrict__ scale) {
+  __shared__ float red[8];
+  const int i = threadIdx.x;
+  const size_t b = blockIdx.z;
+  const int r = blockIdx.y * 128 + (i >> 1);
+  const int c0 = blockIdx.x * 128 + (i & 1) * 64;
+  const size_t off = b * static_cast<size_t>(N) * K + static_cast<size_t>(r) * K + c0;
+  const uint4* src = reinterpret_cast<const uint4*>(w + off);
+  float f[64];
+  float amax = 0.0f;
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    float t[8];
+    bf16x8_to_f32(src[v], t);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      f[v * 8 + j] = t[j];
+      amax = fmaxf(amax, fabsf(t[j]));
+    }
+  }
+  for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+  if ((i & 31) == 0) red[i >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int j = 1; j < 8; ++j) amax = fmaxf(amax, red[j]);
+  const float sc = amax == 0.0f ? 1.0f : amax / 448.0f;
+  uint32_t packed[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    packed[j] = static_cast<uint32_t>(to_e4m3(f[4 * j] / sc)) |
+                (static_cast<uint32_t>(to_e4m3(f[4 * j + 1] / sc)) << 8) |
+                (static_cast<uint32_t>(to_e4m3(f[4 * j + 2] / sc)) << 16) |
+                (static_cast<uint32_t>(to_e4m3(f[4 * j + 3] / sc)) << 24);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(q + off);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+  if (i == 0) scale[(b * (N / 128) + blockIdx.y) * (K / 128) + blockIdx.x] = sc;
+}
+
+// E4M3 activation quantisation per 1x128 tile: one warp per tile, 4 values a lane.
+__global__ void __launch_bounds__(256)
+quant_rows_kernel(const __nv_bfloat16* __restrict__ a, int M, int K, uint8_t* __restrict__ q,
+                  float* __restrict__ scale) {
+  const int lane = threadIdx.x & 31;
+  const long long tile = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nkb = K / 128;
+  if (tile >= static_cast<long long>(M) * nkb) return;   // warp-uniform
+  const long long m = tile / nkb;
+  const int kb = static_cast<int>(tile - m * nkb);
+  const size_t off = static_cast<size_t>(m) * K + kb * 128 + lane * 4;
+  const uint2 raw = *reinterpret_cast<const uint2*>(a + off);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  const float2 p0 = __bfloat1622float2(h[0]), p1 = __bfloat1622float2(h[1]);
+  float amax = fmaxf(fmaxf(fabsf(p0.x), fabsf(p0.y)), fmaxf(fabsf(p1.x), fabsf(p1.y)));
+  for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+  const float sc = amax == 0.0f ? 1.0f : amax / 448.0f;
+  const uint32_t packed = static_cast<uint32_t>(to_e4m3(p0.x / sc)) |
+                          (static_cast<uint32_t>(to_e4m3(p0.y / sc)) << 8) |
+                          (static_cast<uint32_t>(to_e4m3(p1.x / sc)) << 16) |
+                          (static_cast<uint32_t>(to_e4m3(p1.y / sc)) << 24);
+  *reinterpret_cast<uint32_t*>(q + off) = packed;
+  if (lane == 0) scale[m * nkb + kb] = sc;
+}
+
+// ------------------------------------------------------------------------
+cudaError_t launch_combine(int T, int k, int H, const void* eo, const int32_t* slot_to_row,
+                           const float* topk_w, const void* shared, void* y, cudaStream_t stream) {
+  const int warps = 8;
+  combine_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
+      T, k, H / 8, reinterpret_cast<const uint4*>(eo), slot_to_row, topk_w,
+      reinterpret_cast<const uint4*>(shared), reinterpret_cast<uint4*>(y));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bias_update(int E, int T, int k, const int32_t* counts, float* bias, float gamma,
+                               float* load_cv, cudaStream_t stream) {
+  bias_update_kernel<<<1, 1024, 0, stream>>>(E, T, k, counts, bias, gamma, load_cv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_blocks(int batch, int N, int K, const void* w, void* q, float* scale,
+                                cudaStream_t stream) {
+  dim3 grid(K / 128, N / 128, batch);
+  quant_blocks_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(w), N, K,
+                                                reinterpret_cast<uint8_t*>(q), scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows(int M, int K, const void* a, void* q, float* scale, cudaStream_t stream) {
+  const long long tiles = static_cast<long long>(M) * (K / 128);
+  const int warps = 8;
+  const long long blocks = (tiles + warps - 1) / warps;
+  quant_rows_kernel<<<static_cast<unsigned>(blocks), warps * 32, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(a), M, K, reinterpret_cast<uint8_t*>(q), scale);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,203 @@
+"""The MoE layer forward as a fixed sequence of libmoe calls.
+
+"MoE 混合专家模型推理参数与前向传播详解" §3 gives the order: routing (§3.1),
+permutation (§3.2), routed experts as one grouped GEMM and the shared experts
+(§3.3), unpermute + combine (§3.4). Between forwards the xxqk.cn digest §2.2
+adds the aux-loss-free bias step. torch only provides the device buffers and
+the stream; there is no host synchronisation inside a forward.
+"""
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import native as N
+
+
+@dataclass
+class LayerSpec:
+    H: int
+    E: int
+    I: int
+    I_s: int
+    k: int
+    n_group: int
+    topk_group: int
+    scoring: str             # "softmax" | "sigmoid"
+    norm_topk_prob: bool
+    scale: float
+    dtype: str = "bf16"      # expert weights / activations: "bf16" | "e4m3"
+
+    @classmethod
+    def from_config(cls, cfg):
+        return cls(cfg.H, cfg.E, cfg.I, cfg.I_s, cfg.k, cfg.n_group, cfg.topk_group,
+                   cfg.scoring, cfg.norm_topk_prob, cfg.scale, cfg.dtype)
+
+
+class MoELayer:
+    """Holds the weights (device tensors) and the per-forward buffers."""
+
+    def __init__(self, spec: LayerSpec, gate: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
+                 sw13: Optional[torch.Tensor], sw2: Optional[torch.Tensor],
+                 bias: Optional[torch.Tensor], T_max: int):
+        self.spec = spec
+        dev = gate.device
+        self.dev = dev
+        self.gate = gate.contiguous()
+        self.bias = bias.contiguous().clone() if bias is not None else None
+        self.fp8 = spec.dtype == "e4m3"
+        H, E, I, I_s, k = spec.H, spec.E, spec.I, spec.I_s, spec.k
+        if self.fp8:
+            # E4M3 weights with 128x128 block scales, quantised once by libmoe
+            self.w13, self.w13_s = self._quant_blocks(w13)
+            self.w2, self.w2_s = self._quant_blocks(w2)
+            if sw13 is not None:
+                self.sw13, self.sw13_s = self._quant_blocks(sw13.unsqueeze(0))
+                self.sw2, self.sw2_s = self._quant_blocks(sw2.unsqueeze(0))
+            else:
+                self.sw13 = self.sw2 = self.sw13_s = self.sw2_s = None
+        else:
+            self.w13, self.w2 = w13.contiguous(), w2.contiguous()
+            self.w13_s = self.w2_s = None
+            self.sw13 = sw13.contiguous() if sw13 is not None else None
+            self.sw2 = sw2.contiguous() if sw2 is not None else None
+            self.sw13_s = self.sw2_s = None
+        self.T_max = T_max
+        R = T_max * k
+        i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
+        act = torch.uint8 if self.fp8 else bf
+        z = lambda *s, dt: torch.empty(*s, dtype=dt, device=dev)
+        self.logits = z(T_max, E, dt=f32)
+        self.ids = z(T_max, k, dt=i32)
+        self.topk_w = z(T_max, k, dt=f32)
+        self.counts = z(E, dt=i32)
+        self.offsets = z(E + 1, dt=i32)
+        self.src_token = z(R, dt=i32)
+        self.slot_to_row = z(R, dt=i32)
+        self.row_w = z(R, dt=f32)
+        ws = N.moe_permute_workspace_size(T_max, k, E)
+        self.ws = z((ws + 15) // 16 * 16, dt=torch.uint8)
+        self.x_perm = z(R, H, dt=act)
+        self.h = z(R, I, dt=act)
+        self.o = z(R, H, dt=bf)
+        self.y = z(T_max, H, dt=bf)
+        self.load_cv = z(1, dt=f32)
+        self.status = torch.zeros(1, dtype=i32, device=dev)
+        if self.fp8:
+            self.xq = z(T_max, H, dt=torch.uint8)
+            self.xs = z(T_max, H // 128, dt=f32)
+            self.x_perm_s = z(R, H // 128, dt=f32)
+            self.h_s = z(R, I // 128, dt=f32)
+            self.sh_h_s = z(T_max, max(I_s, 128) // 128, dt=f32)
+        else:
+            self.xq = self.xs = self.x_perm_s = self.h_s = self.sh_h_s = None
+        if I_s > 0:
+            self.sh_h = z(T_max, I_s, dt=act)
+            self.sh_o = z(T_max, H, dt=bf)
+        else:
+            self.sh_h = self.sh_o = None
+
+    def _quant_blocks(self, w):
+        B, Nr, K = w.shape
+        q = torch.empty(B, Nr, K, dtype=torch.uint8, device=w.device)
+        s = torch.empty(B, Nr // 128, K // 128, dtype=torch.float32, device=w.device)
+        N.moe_quantize_blocks(B, Nr, K, w.contiguous(), q, s)
+        return q, s
+
+    # -------------------------------------------------------------- stages
+    def route(self, x: torch.Tensor, write_logits: bool = False, logits_in: Optional[torch.Tensor] = None):
+        s = self.spec
+        T = (logits_in if logits_in is not None else x).shape[0]
+        N.moe_route(T, s.H, s.E, s.k, s.n_group, s.topk_group,
+                    N.MOE_SIGMOID if s.scoring == "sigmoid" else N.MOE_SOFTMAX,
+                    s.norm_topk_prob, s.scale,
+                    None if logits_in is not None else x,
+                    self.gate, self.bias,
+                    logits_in if logits_in is not None else (self.logits[:T] if write_logits else None),
+                    self.ids[:T], self.topk_w[:T], self.counts, self.status)
+
+    def quantize_x(self, x: torch.Tensor, T: int):
+        """E4M3 layers: x -> 1x128-tile codes + scales (once per token)."""
+        N.moe_quantize_rows(T, self.spec.H, x, self.xq[:T], self.xs[:T])
+
+    def permute(self, x: torch.Tensor, T: int):
+        s = self.spec
+        if self.fp8:
+            src, dt, src_s = self.xq[:T], N.MOE_E4M3, self.xs[:T]
+        else:
+            src, dt, src_s = x, N.MOE_BF16, None
+        R = T * s.k
+        N.moe_permute(T, s.k, s.E, s.H, self.ids[:T], self.topk_w[:T], src, dt, src_s,
+                      self.x_perm[:R], self.x_perm_s[:R] if self.fp8 else None,
+                      self.offsets, self.src_token[:R], self.slot_to_row[:R], self.row_w[:R],
+                      self.ws, self.status)
+
+    def _dt(self):
+        return N.MOE_E4M3 if self.fp8 else N.MOE_BF16
+
+    def experts_gate_up(self, T: int):
+        s = self.spec
+        R = T * s.k
+        N.moe_gate_up_swiglu(R, s.H, self.w13, self._dt(), s.E, s.I, self.x_perm[:R], self.offsets,
+                             self.h[:R], w13_scale=self.w13_s,
+                             a_scale=self.x_perm_s[:R] if self.fp8 else None,
+                             h_scale_ws=self.h_s[:R] if self.fp8 else None, dev_status=self.status)
+
+    def experts_down(self, T: int):
+        s = self.spec
+        R = T * s.k
+        N.moe_down_proj(R, s.H, self.w2, self._dt(), s.E, s.I, self.h[:R], self.offsets,
+                        self.row_w[:R], self.o[:R], w2_scale=self.w2_s,
+                        h_scale=self.h_s[:R] if self.fp8 else None, dev_status=self.status)
+
+    def shared_gate_up(self, x: torch.Tensor, T: int):
+        s = self.spec
+        a = self.xq[:T] if self.fp8 else x
+        N.moe_gate_up_swiglu(T, s.H, self.sw13, self._dt(), 1, s.I_s, a, None, self.sh_h[:T],
+                             w13_scale=self.sw13_s, a_scale=self.xs[:T] if self.fp8 else None,
+                             h_scale_ws=self.sh_h_s[:T] if self.fp8 else None,
+                             dev_status=self.status)
+
+    def shared_down(self, T: int):
+        s = self.spec
+        N.moe_down_proj(T, s.H, self.sw2, self._dt(), 1, s.I_s, self.sh_h[:T], None, None,
+                        self.sh_o[:T], w2_scale=self.sw2_s,
+                        h_scale=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status)
+
+    def combine(self, T: int):
+        s = self.spec
+        N.moe_combine(T, s.k, s.H, self.o[:T * s.k], self.slot_to_row[:T * s.k], None,
+                      self.sh_o[:T] if self.sh_o is not None else None, self.y[:T])
+
+    def stages(self, x: torch.Tensor, write_logits: bool = False):
+        """The forward as named steps, each one or more libmoe launches."""
+        T = x.shape[0]
+        assert T <= self.T_max and x.dtype == torch.bfloat16 and x.is_contiguous()
+        st = [("route", lambda: self.route(x, write_logits))]
+        if self.fp8:
+            st.append(("quantize_x", lambda: self.quantize_x(x, T)))
+        st += [("permute", lambda: self.permute(x, T)),
+               ("gate_up_routed", lambda: self.experts_gate_up(T)),
+               ("down_routed", lambda: self.experts_down(T))]
+        if self.sh_h is not None:
+            st += [("gate_up_shared", lambda: self.shared_gate_up(x, T)),
+                   ("down_shared", lambda: self.shared_down(T))]
+        st.append(("combine", lambda: self.combine(T)))
+        return st
+
+    def forward(self, x: torch.Tensor, write_logits: bool = False) -> torch.Tensor:
+        """y = shared(x) + sum_j w_j E_j(x) for the T rows of x (bf16 [T, H])."""
+        for _, run in self.stages(x, write_logits):
+            run()
+        return self.y[:x.shape[0]]
+
+    def bias_step(self, T: int, gamma: float, load_cv: bool = True):
+        """Aux-loss-free bias update from the last forward's expert counts."""
+        s = self.spec
+        if self.bias is None:
+            raise ValueError("layer has no selection bias")
+        N.moe_bias_update(s.E, T, s.k, self.counts, self.bias, gamma,
+                          self.load_cv if load_cv else None)
+
+    def device_status(self) -> int:
+        return N.moe_read_device_status(self.status)

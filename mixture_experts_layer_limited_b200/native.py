@@ -1,0 +1,198 @@
+"""ctypes binding of libmoe's C ABI (include/moe.h), one function per entry.
+
+Argument marshalling only: torch tensors are passed as raw device pointers on
+torch's current CUDA stream; every step of the layer runs in libmoe's kernels.
+The library is loaded on first use; a missing library is an error, never a
+fallback.
+"""
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from .build import lib_path
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_ALIGNMENT = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_DEVICE_CHECK = 5
+MOE_ERR_DEVICE_TIMEOUT = 6
+MOE_DEVSTAT_BAD_EXPERT_ID = 0x1
+MOE_DEVSTAT_TIMEOUT = 0x2
+MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
+MOE_SOFTMAX, MOE_SIGMOID = 0, 1
+
+EXPORTED = [
+    "moe_route", "moe_permute_workspace_size", "moe_permute", "moe_grouped_swiglu",
+    "moe_gate_up_swiglu", "moe_down_proj",
+    "moe_combine", "moe_bias_update", "moe_quantize_blocks", "moe_quantize_rows",
+    "moe_read_device_status", "moe_last_cuda_error", "moe_status_string", "moe_abi_version",
+]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status} ({detail})")
+
+
+class RouteParams(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
+                ("scoring", ctypes.c_int32), ("norm_topk_prob", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_float), ("dev_status", ctypes.c_void_p)]
+
+
+class FFNWeights(ctypes.Structure):
+    _fields_ = [("w13", ctypes.c_void_p), ("w2", ctypes.c_void_p),
+                ("w13_scale", ctypes.c_void_p), ("w2_scale", ctypes.c_void_p),
+                ("dtype", ctypes.c_int32), ("groups", ctypes.c_int32), ("I", ctypes.c_int32)]
+
+
+_LIB = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Loads libmoe.so (once). Raises if it has not been built."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = path or lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"libmoe not built: {path} is missing "
+                           "(run python -m mixture_experts_layer_limited_b200.build)")
+    lib = ctypes.CDLL(path)
+    sig = {
+        "moe_route": [ctypes.POINTER(RouteParams), _P, _P, _P, _P, _P, _P, _P, _P],
+        "moe_permute_workspace_size": [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
+        "moe_permute": [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
+                        ctypes.c_size_t, _P, _P],
+        "moe_grouped_swiglu": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P, _P, _P],
+        "moe_gate_up_swiglu": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P],
+        "moe_down_proj": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P],
+        "moe_combine": [_I, _I, _I, _P, _P, _P, _P, _P, _P],
+        "moe_bias_update": [_I, _I, _I, _P, _P, ctypes.c_float, _P, _P],
+        "moe_quantize_blocks": [_I, _I, _I, _P, _P, _P, _P],
+        "moe_quantize_rows": [_I, _I, _P, _P, _P, _P],
+        "moe_read_device_status": [_P, ctypes.POINTER(ctypes.c_int32), _P],
+        "moe_last_cuda_error": [],
+        "moe_status_string": [_I],
+        "moe_abi_version": [],
+    }
+    for name, args in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_char_p if name == "moe_status_string" else ctypes.c_int32
+    _LIB = lib
+    return lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmoe takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libmoe takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != MOE_OK:
+        lib = load_library()
+        detail = lib.moe_status_string(status).decode()
+        if status == MOE_ERR_CUDA:
+            detail += f", cuda error {lib.moe_last_cuda_error()}"
+        raise MoEError(fn, status, detail)
+
+
+# ---------------------------------------------------------------- the ABI
+def moe_route(T, H, E, k, n_group, topk_group, scoring, norm_topk_prob, routed_scaling_factor,
+              x, gate_w, sel_bias, logits, topk_ids, topk_w, expert_counts, dev_status=None,
+              stream=None):
+    p = RouteParams(T, H, E, k, n_group, topk_group, scoring, int(bool(norm_topk_prob)),
+                    float(routed_scaling_factor), _ptr(dev_status))
+    _check("moe_route", load_library().moe_route(
+        ctypes.byref(p), _ptr(x), _ptr(gate_w), _ptr(sel_bias), _ptr(logits), _ptr(topk_ids),
+        _ptr(topk_w), _ptr(expert_counts), _stream(stream)))
+
+
+def moe_permute_workspace_size(T, k, E) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_permute_workspace_size",
+           load_library().moe_permute_workspace_size(T, k, E, ctypes.byref(n)))
+    return n.value
+
+
+def moe_permute(T, k, E, H, topk_ids, topk_w, x, x_dtype, x_scale, x_perm, x_perm_scale,
+                expert_offsets, src_token, slot_to_row, row_w, workspace, dev_status=None, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("moe_permute", load_library().moe_permute(
+        T, k, E, H, _ptr(topk_ids), _ptr(topk_w), _ptr(x), x_dtype, _ptr(x_scale), _ptr(x_perm),
+        _ptr(x_perm_scale), _ptr(expert_offsets), _ptr(src_token), _ptr(slot_to_row), _ptr(row_w),
+        _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def moe_grouped_swiglu(rows, H, w13, w2, dtype, groups, I, a, offsets, row_w, h_ws, out,
+                       w13_scale=None, w2_scale=None, a_scale=None, h_scale_ws=None,
+                       dev_status=None, stream=None):
+    w = FFNWeights(_ptr(w13), _ptr(w2), _ptr(w13_scale), _ptr(w2_scale), dtype, groups, I)
+    _check("moe_grouped_swiglu", load_library().moe_grouped_swiglu(
+        rows, H, ctypes.byref(w), _ptr(a), _ptr(a_scale), _ptr(offsets), _ptr(row_w), _ptr(h_ws),
+        _ptr(h_scale_ws), _ptr(out), _ptr(dev_status), _stream(stream)))
+
+
+def moe_gate_up_swiglu(rows, H, w13, dtype, groups, I, a, offsets, h_ws, w13_scale=None,
+                       a_scale=None, h_scale_ws=None, dev_status=None, stream=None):
+    w = FFNWeights(_ptr(w13), None, _ptr(w13_scale), None, dtype, groups, I)
+    _check("moe_gate_up_swiglu", load_library().moe_gate_up_swiglu(
+        rows, H, ctypes.byref(w), _ptr(a), _ptr(a_scale), _ptr(offsets), _ptr(h_ws),
+        _ptr(h_scale_ws), _ptr(dev_status), _stream(stream)))
+
+
+def moe_down_proj(rows, H, w2, dtype, groups, I, h, offsets, row_w, out, w2_scale=None,
+                  h_scale=None, dev_status=None, stream=None):
+    w = FFNWeights(None, _ptr(w2), None, _ptr(w2_scale), dtype, groups, I)
+    _check("moe_down_proj", load_library().moe_down_proj(
+        rows, H, ctypes.byref(w), _ptr(h), _ptr(h_scale), _ptr(offsets), _ptr(row_w), _ptr(out),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_combine(T, k, H, expert_out, slot_to_row, topk_w, shared_out, y, stream=None):
+    _check("moe_combine", load_library().moe_combine(
+        T, k, H, _ptr(expert_out), _ptr(slot_to_row), _ptr(topk_w), _ptr(shared_out), _ptr(y),
+        _stream(stream)))
+
+
+def moe_bias_update(E, T, k, expert_counts, bias, gamma, load_cv=None, stream=None):
+    _check("moe_bias_update", load_library().moe_bias_update(
+        E, T, k, _ptr(expert_counts), _ptr(bias), float(gamma), _ptr(load_cv), _stream(stream)))
+
+
+def moe_quantize_blocks(batch, N, K, w, q, scale, stream=None):
+    _check("moe_quantize_blocks", load_library().moe_quantize_blocks(
+        batch, N, K, _ptr(w), _ptr(q), _ptr(scale), _stream(stream)))
+
+
+def moe_quantize_rows(M, K, a, q, scale, stream=None):
+    _check("moe_quantize_rows", load_library().moe_quantize_rows(
+        M, K, _ptr(a), _ptr(q), _ptr(scale), _stream(stream)))
+
+
+def moe_read_device_status(dev_status, stream=None) -> int:
+    """Synchronises the stream and returns the raw device status word."""
+    out = ctypes.c_int32(0)
+    st = load_library().moe_read_device_status(_ptr(dev_status), ctypes.byref(out), _stream(stream))
+    if st not in (MOE_OK, MOE_ERR_DEVICE_CHECK, MOE_ERR_DEVICE_TIMEOUT):
+        _check("moe_read_device_status", st)
+    return out.value

@@ -1,0 +1,93 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+include/moe.h declares, and rejects bad arguments on the host before any
+launch (nothing here touches a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_limited_b200 import native as N
+from mixture_experts_layer_limited_b200.build import lib_path
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+pytestmark = pytest.mark.skipif(not os.path.exists(lib_path()),
+                                reason="libmoe.so not built (run the package build)")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declarations_match_binding_list():
+    assert declared_functions() == sorted(N.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(lib_path())
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_abi_version_and_status_strings():
+    lib = N.load_library()
+    assert lib.moe_abi_version() == 1
+    assert lib.moe_status_string(0) == b"ok"
+    assert b"invalid" in lib.moe_status_string(N.MOE_ERR_INVALID_ARG)
+    assert lib.moe_status_string(99) == b"unknown status"
+    assert lib.moe_last_cuda_error() == 0
+
+
+def test_workspace_size_is_host_only():
+    assert N.moe_permute_workspace_size(8192, 8, 256) == (8192 // 64) * 256 * 4
+    assert N.moe_permute_workspace_size(65, 8, 16) == 2 * 16 * 4
+    with pytest.raises(N.MoEError):
+        N.moe_permute_workspace_size(0, 8, 256)
+
+
+def _raw(lib, fn, *args):
+    return getattr(lib, fn)(*args)
+
+
+def test_host_validation_rejects_before_launch():
+    lib = N.load_library()
+    P = ctypes.c_void_p
+    fake = P(0x1000)          # never dereferenced: every call below fails validation first
+    odd = P(0x1004)
+    # moe_route: no params / k > E / unsupported E / misaligned pointer
+    assert lib.moe_route(None, fake, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_INVALID_ARG
+    p = N.RouteParams(16, 256, 16, 17, 1, 1, N.MOE_SOFTMAX, 0, 1.0, None)
+    assert lib.moe_route(ctypes.byref(p), fake, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_INVALID_ARG
+    p = N.RouteParams(16, 256, 24, 4, 1, 1, N.MOE_SOFTMAX, 0, 1.0, None)
+    assert lib.moe_route(ctypes.byref(p), fake, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_UNSUPPORTED
+    p = N.RouteParams(16, 256, 256, 8, 8, 4, N.MOE_SIGMOID, 1, 2.5, None)
+    assert lib.moe_route(ctypes.byref(p), odd, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_ALIGNMENT
+    # group limit makes k impossible: 4 groups of 4, keep 1 -> at most 4 candidates
+    p = N.RouteParams(16, 256, 16, 5, 4, 1, N.MOE_SIGMOID, 1, 2.5, None)
+    assert lib.moe_route(ctypes.byref(p), fake, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_INVALID_ARG
+    # moe_permute: missing workspace, too small workspace, unsupported E
+    args = [fake, fake, fake, N.MOE_BF16, None, fake, None, fake, fake, fake, fake]
+    assert lib.moe_permute(64, 4, 16, 256, *args, None, 0, None, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute(64, 4, 16, 256, *args, fake, 4, None, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute(64, 4, 2048, 256, *args, fake, 1 << 20, None, None) == N.MOE_ERR_UNSUPPORTED
+    # moe_grouped_swiglu: H not a multiple of 256, offsets NULL with groups > 1
+    w = N.FFNWeights(fake, fake, None, None, N.MOE_BF16, 4, 128)
+    assert lib.moe_grouped_swiglu(64, 200, ctypes.byref(w), fake, None, fake, None, fake, None, fake,
+                                  None, None) == N.MOE_ERR_UNSUPPORTED
+    assert lib.moe_grouped_swiglu(64, 256, ctypes.byref(w), fake, None, None, None, fake, None, fake,
+                                  None, None) == N.MOE_ERR_INVALID_ARG
+    w8 = N.FFNWeights(fake, fake, None, None, N.MOE_E4M3, 4, 128)
+    assert lib.moe_grouped_swiglu(64, 256, ctypes.byref(w8), fake, None, fake, None, fake, None, fake,
+                                  None, None) == N.MOE_ERR_INVALID_ARG
+    # moe_combine / moe_bias_update / quantisers
+    assert lib.moe_combine(0, 4, 256, fake, fake, None, None, fake, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(8, 4, 252, fake, fake, None, None, fake, None) == N.MOE_ERR_UNSUPPORTED
+    assert lib.moe_bias_update(2048, 8, 4, fake, fake, ctypes.c_float(0.001), None, None) == N.MOE_ERR_UNSUPPORTED
+    assert lib.moe_bias_update(16, 8, 4, None, fake, ctypes.c_float(0.001), None, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_quantize_blocks(1, 100, 128, fake, fake, fake, None) == N.MOE_ERR_UNSUPPORTED
+    assert lib.moe_quantize_rows(4, 128, odd, fake, fake, None) == N.MOE_ERR_ALIGNMENT
+    assert lib.moe_read_device_status(None, None, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_last_cuda_error() == 0

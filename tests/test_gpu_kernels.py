@@ -1,0 +1,330 @@
+"""Per-kernel parity of libmoe against the CPU oracle (needs a B200).
+
+Bit-exact: E4M3 codes and scales, routing ids / counts given identical fp32
+logits, the permutation, the bias trajectory. Floating point: within the
+tolerance each test states."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import moe_oracle as O
+from moe_inputs import get_config, tiny_grouped_config, make_inputs, make_logits
+from mixture_experts_layer_limited_b200 import native as N
+
+from gpu_util import (np64, np32, rel_err, oracle_route, gpu_route, near_tie_mask, uniform_bias,
+                      BF16_TOL, FP8_TOL)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _gen(seed):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    return g
+
+
+# ------------------------------------------------------------------ E4M3
+def test_quantize_blocks_bytes_match_oracle():
+    g = _gen(1)
+    w = (torch.randn(3, 256, 384, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w[1, :128, :128] = 0                     # all-zero block -> scale 1
+    w[2, 5, 7] = 3.0                         # outlier block
+    w[2, 200, 300] = -1e-30                  # tiny negative -> signed zero code
+    q = torch.empty(3, 256, 384, dtype=torch.uint8, device=DEV)
+    s = torch.empty(3, 2, 3, dtype=torch.float32, device=DEV)
+    N.moe_quantize_blocks(3, 256, 384, w, q, s)
+    torch.cuda.synchronize()
+    for b in range(3):
+        qo, so = oracle.fp8_quantize_blocks(np32(w[b]))
+        assert np.array_equal(q[b].cpu().numpy(), qo)
+        assert np.array_equal(s[b].cpu().numpy(), so)
+
+
+def test_quantize_rows_bytes_match_oracle():
+    g = _gen(2)
+    a = (torch.randn(257, 512, generator=g, device=DEV) * 3).to(torch.bfloat16)
+    a[7, 128:256] = 0
+    q = torch.empty(257, 512, dtype=torch.uint8, device=DEV)
+    s = torch.empty(257, 4, dtype=torch.float32, device=DEV)
+    N.moe_quantize_rows(257, 512, a, q, s)
+    qo, so = oracle.fp8_quantize_rows(np32(a))
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy(), so)
+
+
+# ---------------------------------------------------------------- router
+ROUTE_CASES = [("tiny", None), ("tiny_grouped", None), ("v2lite", None), ("v3", None),
+               ("v3", 1000), ("v3_ties", 777), ("v2lite", 1)]
+
+
+def _cfg(name):
+    if name == "tiny_grouped":
+        return tiny_grouped_config()
+    if name == "v3_ties":
+        return get_config("v3")
+    return get_config(name)
+
+
+@pytest.mark.parametrize("name,T", ROUTE_CASES)
+def test_route_from_logits_bit_exact(name, T):
+    cfg = _cfg(name)
+    T = T or cfg.T
+    L = make_logits(cfg, device=DEV, T=T)
+    if name == "v3_ties":
+        L = torch.round(L * 4) / 4           # many exact ties in scores and group scores
+    bias = uniform_bias(cfg.E, cfg.seed + 5) if cfg.scoring == "sigmoid" else None
+    if name == "v3_ties":
+        bias = torch.round(bias * 50) / 50
+    ids, w, counts, _ = gpu_route(cfg, T, bias=bias, logits=L)
+    torch.cuda.synchronize()
+    r = oracle_route(np32(L), cfg, np32(bias) if bias is not None else None)
+    assert np.array_equal(ids.cpu().numpy(), r.ids)
+    assert np.array_equal(counts.cpu().numpy(), r.counts)
+    np.testing.assert_allclose(w.cpu().numpy(), r.weights, rtol=5e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("name,T", [("tiny", None), ("tiny_grouped", None), ("v2lite", None),
+                                    ("v3", None), ("v3", 1000)])
+def test_route_gate_gemm(name, T):
+    cfg = _cfg(name)
+    T = T or cfg.T
+    inp = make_inputs(dataclasses.replace(cfg, T=T), device=DEV, experts=False, shared=False)
+    bias = inp.bias
+    ids, w, counts, L = gpu_route(cfg, T, x=inp.x, gate=inp.gate, bias=bias)
+    torch.cuda.synchronize()
+    L64 = oracle.gate_logits(np64(inp.x), np64(inp.gate))
+    assert rel_err(np64(L), L64) < 1e-5
+    r = oracle_route(L64.astype(np.float32), cfg, np32(bias) if bias is not None else None)
+    flagged = near_tie_mask(r)
+    ids_g = ids.cpu().numpy()
+    mism = np.any(ids_g != r.ids, axis=1)
+    assert not np.any(mism & ~flagged), f"{int(np.sum(mism & ~flagged))} unflagged tokens differ"
+    ok = ~flagged & ~mism
+    np.testing.assert_allclose(w.cpu().numpy()[ok], r.weights[ok], rtol=2e-5, atol=1e-6)
+    assert int(counts.sum()) == T * cfg.k
+    print(f"{name} T={T}: near-tie tokens excluded {int(flagged.sum())}")
+
+
+# --------------------------------------------------------------- permute
+def _ids_from_oracle(T, k, E, seed, skew=0.0):
+    rng = np.random.default_rng(seed)
+    L = rng.standard_normal((T, E)).astype(np.float32)
+    if skew:
+        L[:, :4] += skew
+    r = oracle.route_from_logits(L, k, 1, 1, "softmax", False, 1.0)
+    return r.ids, r.weights.astype(np.float32)
+
+
+@pytest.mark.parametrize("T,k,E,H,skew", [(64, 4, 16, 256, 0.0), (8192, 8, 256, 7168, 0.0),
+                                          (1000, 6, 64, 2048, 0.0), (2000, 8, 256, 512, 3.0),
+                                          (1, 1, 16, 256, 0.0), (3, 16, 16, 128, 0.0)])
+def test_permute_bit_exact(T, k, E, H, skew):
+    ids_np, w_np = _ids_from_oracle(T, k, E, seed=T + E, skew=skew)
+    offsets_o, src_o, s2r_o = oracle.permute(ids_np, E)
+    ids = torch.from_numpy(ids_np).to(DEV)
+    tw = torch.from_numpy(w_np).to(DEV)
+    x = torch.randn(T, H, generator=_gen(3), device=DEV).to(torch.bfloat16)
+    R = T * k
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    src = torch.empty(R, dtype=torch.int32, device=DEV)
+    s2r = torch.empty(R, dtype=torch.int32, device=DEV)
+    roww = torch.empty(R, dtype=torch.float32, device=DEV)
+    xp = torch.empty(R, H, dtype=torch.bfloat16, device=DEV)
+    ws = torch.empty(N.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    N.moe_permute(T, k, E, H, ids, tw, x, N.MOE_BF16, None, xp, None, offsets, src, s2r, roww, ws, status)
+    assert N.moe_read_device_status(status) == 0
+    assert np.array_equal(offsets.cpu().numpy(), offsets_o)
+    assert np.array_equal(src.cpu().numpy(), src_o)
+    assert np.array_equal(s2r.cpu().numpy(), s2r_o)
+    assert np.array_equal(roww.cpu().numpy(), w_np.reshape(-1)[np.argsort(s2r_o)])
+    assert torch.equal(xp, x[torch.from_numpy(src_o).to(DEV)])
+
+
+def test_permute_e4m3_rows_and_scales():
+    T, k, E, H = 300, 8, 64, 512
+    ids_np, w_np = _ids_from_oracle(T, k, E, seed=9)
+    _, src_o, _ = oracle.permute(ids_np, E)
+    xq = torch.randint(0, 255, (T, H), generator=_gen(4), device=DEV, dtype=torch.uint8)
+    xs = torch.rand(T, H // 128, generator=_gen(5), device=DEV)
+    R = T * k
+    out = [torch.empty(E + 1, dtype=torch.int32, device=DEV)] + \
+          [torch.empty(R, dtype=torch.int32, device=DEV) for _ in range(2)]
+    roww = torch.empty(R, dtype=torch.float32, device=DEV)
+    xp = torch.empty(R, H, dtype=torch.uint8, device=DEV)
+    xps = torch.empty(R, H // 128, dtype=torch.float32, device=DEV)
+    ws = torch.empty(N.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device=DEV)
+    N.moe_permute(T, k, E, H, torch.from_numpy(ids_np).to(DEV), torch.from_numpy(w_np).to(DEV),
+                  xq, N.MOE_E4M3, xs, xp, xps, out[0], out[1], out[2], roww, ws)
+    idx = torch.from_numpy(src_o).to(DEV)
+    assert torch.equal(xp, xq[idx])
+    assert torch.equal(xps, xs[idx])
+
+
+def test_permute_flags_out_of_range_ids_without_writing_outside():
+    T, k, E, H = 128, 4, 16, 256
+    ids_np, w_np = _ids_from_oracle(T, k, E, seed=10)
+    ids_np = ids_np.copy()
+    ids_np[5, 2] = 99                         # out of range: counted nowhere, flagged
+    ids_np[77, 0] = -3
+    R = T * k
+    guard = torch.full((R + 64, H), 7, dtype=torch.bfloat16, device=DEV)
+    xp = guard[:R]
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    src = torch.empty(R, dtype=torch.int32, device=DEV)
+    s2r = torch.empty(R, dtype=torch.int32, device=DEV)
+    ws = torch.empty(N.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    x = torch.randn(T, H, generator=_gen(6), device=DEV).to(torch.bfloat16)
+    N.moe_permute(T, k, E, H, torch.from_numpy(ids_np).to(DEV), None, x, N.MOE_BF16, None, xp, None,
+                  offsets, src, s2r, None, ws, status)
+    assert N.moe_read_device_status(status) & N.MOE_DEVSTAT_BAD_EXPERT_ID
+    s2r_np = s2r.cpu().numpy()
+    assert s2r_np[5 * k + 2] == -1 and s2r_np[77 * k + 0] == -1
+    assert torch.all(guard[R:] == 7)         # nothing written past the output
+
+
+# ---------------------------------------------------- grouped SwiGLU GEMM
+def _segments(sizes):
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    return off
+
+
+def _ref_grouped(a, w13, w2, off, row_w):
+    a64, w13_64, w2_64 = np64(a), np64(w13), np64(w2)
+    rw = np32(row_w).astype(np.float64) if row_w is not None else None
+    out = np.zeros((a.shape[0], w2.shape[1]))
+    hs = np.zeros((a.shape[0], w2.shape[2]))
+    I = w2.shape[2]
+    for g in range(len(off) - 1):
+        s, e = off[g], off[g + 1]
+        if e == s:
+            continue
+        gu = a64[s:e] @ w13_64[g].T
+        h = gu[:, :I] / (1 + np.exp(-gu[:, :I])) * gu[:, I:]
+        hs[s:e] = h
+        o = oracle.swiglu_ffn(a64[s:e], w13_64[g], w2_64[g])
+        out[s:e] = o * (rw[s:e, None] if rw is not None else 1.0)
+    return out, hs
+
+
+@pytest.mark.parametrize("H,I,sizes", [
+    (512, 256, [0, 1, 15, 16, 17, 100, 255, 256, 257, 600, 0, 33]),
+    (256, 128, [64]),
+    (7168, 2048, [300, 77]),
+    (2048, 1408, [384, 0, 5, 513]),
+])
+def test_grouped_swiglu_bf16(H, I, sizes):
+    G = len(sizes)
+    off = _segments(sizes)
+    rows = int(off[-1])
+    g = _gen(H + I)
+    a = torch.randn(rows, H, generator=g, device=DEV).to(torch.bfloat16)
+    w13 = (torch.randn(G, 2 * I, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w2 = (torch.randn(G, H, I, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    row_w = torch.rand(rows, generator=g, device=DEV) + 0.5
+    h = torch.empty(rows, I, dtype=torch.bfloat16, device=DEV)
+    out = torch.empty(rows, H, dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    N.moe_grouped_swiglu(rows, H, w13, w2, N.MOE_BF16, G, I, a, torch.from_numpy(off).to(DEV), row_w,
+                         h, out, dev_status=status)
+    assert N.moe_read_device_status(status) == 0
+    ref, href = _ref_grouped(a, w13, w2, off, row_w)
+    eh, eo = rel_err(np64(h), href), rel_err(np64(out), ref)
+    print(f"H={H} I={I}: h err {eh:.2e}, out err {eo:.2e}")
+    assert eh < 1e-2 and eo < BF16_TOL
+
+
+def test_grouped_swiglu_bf16_single_group_no_offsets():
+    rows, H, I = 300, 512, 384
+    g = _gen(77)
+    a = torch.randn(rows, H, generator=g, device=DEV).to(torch.bfloat16)
+    w13 = (torch.randn(1, 2 * I, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w2 = (torch.randn(1, H, I, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    h = torch.empty(rows, I, dtype=torch.bfloat16, device=DEV)
+    out = torch.empty(rows, H, dtype=torch.bfloat16, device=DEV)
+    N.moe_grouped_swiglu(rows, H, w13, w2, N.MOE_BF16, 1, I, a, None, None, h, out)
+    ref, _ = _ref_grouped(a, w13, w2, np.array([0, rows]), None)
+    assert rel_err(np64(out), ref) < BF16_TOL
+
+
+@pytest.mark.parametrize("H,I,sizes", [
+    (512, 256, [0, 1, 8, 31, 32, 33, 70, 16]),
+    (7168, 2048, [9, 3, 40]),
+])
+def test_grouped_swiglu_e4m3(H, I, sizes):
+    G = len(sizes)
+    off = _segments(sizes)
+    rows = int(off[-1])
+    g = _gen(H + I + 1)
+    a = torch.randn(rows, H, generator=g, device=DEV).to(torch.bfloat16)
+    w13 = (torch.randn(G, 2 * I, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w2 = (torch.randn(G, H, I, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    row_w = torch.rand(rows, generator=g, device=DEV) + 0.5
+    q13 = torch.empty(G, 2 * I, H, dtype=torch.uint8, device=DEV)
+    s13 = torch.empty(G, 2 * I // 128, H // 128, dtype=torch.float32, device=DEV)
+    q2 = torch.empty(G, H, I, dtype=torch.uint8, device=DEV)
+    s2 = torch.empty(G, H // 128, I // 128, dtype=torch.float32, device=DEV)
+    N.moe_quantize_blocks(G, 2 * I, H, w13, q13, s13)
+    N.moe_quantize_blocks(G, H, I, w2, q2, s2)
+    aq = torch.empty(rows, H, dtype=torch.uint8, device=DEV)
+    as_ = torch.empty(rows, H // 128, dtype=torch.float32, device=DEV)
+    N.moe_quantize_rows(rows, H, a, aq, as_)
+    h = torch.empty(rows, I, dtype=torch.uint8, device=DEV)
+    hs = torch.empty(rows, I // 128, dtype=torch.float32, device=DEV)
+    out = torch.empty(rows, H, dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    N.moe_grouped_swiglu(rows, H, q13, q2, N.MOE_E4M3, G, I, aq, torch.from_numpy(off).to(DEV), row_w,
+                         h, out, w13_scale=s13, w2_scale=s2, a_scale=as_, h_scale_ws=hs, dev_status=status)
+    assert N.moe_read_device_status(status) == 0
+    a32, rw = np32(a), np32(row_w).astype(np.float64)
+    ref = np.zeros((rows, H))
+    for gi in range(G):
+        s, e = off[gi], off[gi + 1]
+        if e > s:
+            ref[s:e] = O._swiglu_fp8(oracle.fp8_qdq_rows(a32[s:e]), np32(w13[gi]), np32(w2[gi])) * rw[s:e, None]
+    err = rel_err(np64(out), ref)
+    print(f"E4M3 H={H} I={I}: out err {err:.2e}")
+    assert err < FP8_TOL
+
+
+# --------------------------------------------------------------- combine
+@pytest.mark.parametrize("weighted,shared", [(True, True), (False, True), (True, False)])
+def test_combine(weighted, shared):
+    T, k, H = 300, 6, 512
+    g = _gen(8)
+    eo = torch.randn(T * k, H, generator=g, device=DEV).to(torch.bfloat16)
+    perm = torch.randperm(T * k, generator=g, device=DEV).to(torch.int32)
+    tw = torch.rand(T, k, generator=g, device=DEV) if weighted else None
+    sh = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16) if shared else None
+    y = torch.empty(T, H, dtype=torch.bfloat16, device=DEV)
+    N.moe_combine(T, k, H, eo, perm, tw, sh, y)
+    rows = perm.cpu().numpy().reshape(T, k)
+    e64 = np64(eo)
+    w64 = np32(tw).astype(np.float64) if weighted else np.ones((T, k))
+    ref = np.einsum("tj,tjh->th", w64, e64[rows])
+    if shared:
+        ref = ref + np64(sh)
+    assert np.all(np.abs(np64(y) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)
+
+
+# ----------------------------------------------------------- bias update
+def test_bias_update_bit_exact_ten_steps():
+    E, T, k, gamma = 256, 8192, 8, 0.001
+    rng = np.random.default_rng(12)
+    bias_np = (rng.random(E) * 0.1 - 0.05).astype(np.float32)
+    bias = torch.from_numpy(bias_np).to(DEV)
+    cv = torch.empty(1, dtype=torch.float32, device=DEV)
+    for step in range(10):
+        c = rng.multinomial(T * k, np.ones(E) / E).astype(np.int32)
+        if step == 3:
+            c[:] = T * k // E                  # exactly balanced: nothing moves
+        counts = torch.from_numpy(c).to(DEV)
+        N.moe_bias_update(E, T, k, counts, bias, gamma, cv)
+        bias_np = oracle.bias_update(c, bias_np, gamma, T, k)
+        assert np.array_equal(bias.cpu().numpy(), bias_np)
+        assert abs(float(cv.item()) - oracle.load_cv(c)) <= 1e-6 * max(1.0, oracle.load_cv(c))

@@ -1,0 +1,177 @@
+"""End-to-end parity of the MoE layer forward (needs a B200).
+
+Routing is compared id for id on every token whose k-th / (k+1)-th selection
+scores (or g-th / (g+1)-th group scores) are at least 1e-5 apart in the
+oracle; closer tokens are excluded and counted. Outputs are compared as
+max|y - y_oracle| / max|y_oracle| over the compared tokens."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_inputs import get_config, tiny_grouped_config, make_inputs
+from mixture_experts_layer_limited_b200 import MoELayer, LayerSpec
+from mixture_experts_layer_limited_b200 import native as N
+
+from gpu_util import np64, np32, rel_err, oracle_route, near_tie_mask, BF16_TOL, FP8_TOL
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _layer(cfg, inp, T_max=None):
+    return MoELayer(LayerSpec.from_config(cfg), inp.gate, inp.w13, inp.w2, inp.sw13, inp.sw2,
+                    inp.bias, T_max or cfg.T)
+
+
+def _check_permutation_properties(layer, T, k, E):
+    """Properties of the permutation that hold at any size."""
+    ids = layer.ids[:T].cpu().numpy()
+    off = layer.offsets.cpu().numpy()
+    src = layer.src_token[:T * k].cpu().numpy()
+    s2r = layer.slot_to_row[:T * k].cpu().numpy()
+    counts = layer.counts.cpu().numpy()
+    assert off[0] == 0 and off[-1] == T * k and np.all(np.diff(off) >= 0)
+    assert np.array_equal(np.diff(off), counts)
+    assert np.array_equal(np.bincount(ids.ravel(), minlength=E), counts)
+    assert np.array_equal(np.sort(s2r), np.arange(T * k))
+    assert np.array_equal(src[s2r], np.repeat(np.arange(T), k))
+    seg_of_row = np.repeat(np.arange(E), np.diff(off))
+    assert np.array_equal(seg_of_row[s2r], ids.ravel())
+    for e in range(E):                        # ascending tokens inside each segment
+        assert np.all(np.diff(src[off[e]:off[e + 1]]) > 0)
+
+
+def _oracle_tokens(cfg, inp, toks, feats=None, fp8=False):
+    """Oracle routing + output for the given tokens (and features)."""
+    x64 = np64(inp.x[toks])
+    L = oracle.gate_logits(x64, np64(inp.gate)).astype(np.float32)
+    bias = np32(inp.bias) if inp.bias is not None else None
+    r = oracle_route(L, cfg, bias)
+    fidx = None if feats is None else torch.as_tensor(feats, device=DEV)
+
+    def ew(e):
+        w2 = inp.w2[e] if (fidx is None or fp8) else inp.w2[e][fidx]
+        return np32(inp.w13[e]), np32(w2)
+
+    sw2 = inp.sw2 if (fidx is None or fp8) else inp.sw2[fidx]
+    shared = (np32(inp.sw13), np32(sw2)) if inp.sw13 is not None else None
+    y = oracle.moe_forward(x64, r, ew, shared, fp8=fp8, out_features=feats if fp8 else None)
+    return r, y
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_grouped", "v2lite"])
+def test_layer_full_oracle(name):
+    cfg = tiny_grouped_config() if name == "tiny_grouped" else get_config(name)
+    inp = make_inputs(cfg, device=DEV)
+    layer = _layer(cfg, inp)
+    y = layer.forward(inp.x)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    _check_permutation_properties(layer, cfg.T, cfg.k, cfg.E)
+    r, yref = _oracle_tokens(cfg, inp, np.arange(cfg.T))
+    flagged = near_tie_mask(r)
+    mism = np.any(layer.ids[:cfg.T].cpu().numpy() != r.ids, axis=1)
+    assert not np.any(mism & ~flagged)
+    ok = ~flagged & ~mism
+    err = rel_err(np64(y)[ok], yref[ok])
+    print(f"{name}: err {err:.2e}, near-tie tokens excluded {int(flagged.sum())}")
+    assert err < BF16_TOL
+
+
+def test_layer_v3_full_size_sampled():
+    cfg = get_config("v3")
+    inp = make_inputs(cfg, device=DEV)
+    layer = _layer(cfg, inp)
+    y = layer.forward(inp.x)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    _check_permutation_properties(layer, cfg.T, cfg.k, cfg.E)
+    rng = np.random.default_rng(31)
+    toks = np.sort(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 10, replace=False)]))
+    feats = np.sort(rng.choice(cfg.H, 384, replace=False))
+    r, yref = _oracle_tokens(cfg, inp, toks, feats)
+    flagged = near_tie_mask(r)
+    mism = np.any(layer.ids[toks].cpu().numpy() != r.ids, axis=1)
+    assert not np.any(mism & ~flagged)
+    ok = ~flagged & ~mism
+    yg = np64(y[toks][:, torch.as_tensor(feats, device=DEV)])
+    err = rel_err(yg[ok], yref[ok])
+    print(f"v3 T=8192: sampled err {err:.2e}, excluded {int(flagged.sum())}")
+    assert err < BF16_TOL
+
+
+def test_layer_v3_fp8_decode():
+    cfg = get_config("v3_fp8_decode")
+    inp = make_inputs(cfg, device=DEV)
+    layer = _layer(cfg, inp)
+    y = layer.forward(inp.x)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    _check_permutation_properties(layer, cfg.T, cfg.k, cfg.E)
+    # the activation codes the permutation carried are the oracle's bytes
+    qo, so = oracle.fp8_quantize_rows(np32(inp.x))
+    assert np.array_equal(layer.xq[:cfg.T].cpu().numpy(), qo)
+    assert np.array_equal(layer.xs[:cfg.T].cpu().numpy(), so)
+    rng = np.random.default_rng(32)
+    toks = np.sort(rng.choice(cfg.T, 3, replace=False))
+    feats = np.sort(rng.choice(cfg.H, 256, replace=False))
+    r, yref = _oracle_tokens(cfg, inp, toks, feats, fp8=True)
+    flagged = near_tie_mask(r)
+    mism = np.any(layer.ids[toks].cpu().numpy() != r.ids, axis=1)
+    assert not np.any(mism & ~flagged)
+    ok = ~flagged & ~mism
+    yg = np64(y[toks][:, torch.as_tensor(feats, device=DEV)])
+    err = rel_err(yg[ok], yref[ok])
+    print(f"v3 fp8 decode: sampled err {err:.2e}")
+    assert err < FP8_TOL
+
+
+def test_layer_v3_skewed_bias_loop():
+    cfg = get_config("v3_skewed")
+    inp = make_inputs(cfg, device=DEV)
+    layer = _layer(cfg, inp)
+    T, E, k = cfg.T, cfg.E, cfg.k
+    # (a) ten bias steps on identical fp32 logits: routing, counts and the
+    #     bias trajectory must be bit-exact
+    L32 = oracle.gate_logits(np64(inp.x), np64(inp.gate)).astype(np.float32)
+    L_dev = torch.from_numpy(L32).to(DEV)
+    bias_o = np32(inp.bias).copy()
+    cvs = []
+    hot = []
+    for step in range(cfg.bias_steps + 1):
+        layer.route(None, logits_in=L_dev)
+        r = oracle.route_from_logits(L32, k, cfg.n_group, cfg.topk_group, cfg.scoring,
+                                     cfg.norm_topk_prob, cfg.scale, bias_o)
+        ids_g = layer.ids[:T].cpu().numpy()
+        assert np.array_equal(ids_g, r.ids), f"step {step}"
+        assert np.array_equal(layer.counts.cpu().numpy(), r.counts)
+        cvs.append(oracle.load_cv(r.counts))
+        hot.append(float(r.counts[:cfg.skew_experts].sum()) / (T * k))
+        if step == cfg.bias_steps:
+            break
+        layer.bias_step(T, cfg.gamma)
+        torch.cuda.synchronize()
+        bias_o = oracle.bias_update(r.counts, bias_o, cfg.gamma, T, k)
+        assert np.array_equal(layer.bias.cpu().numpy(), bias_o), f"step {step}"
+        assert abs(float(layer.load_cv.item()) - cvs[-1]) < 1e-6
+    print("load CV per step:", " ".join(f"{c:.4f}" for c in cvs))
+    print("share of experts 0-15 per step:", " ".join(f"{h:.3f}" for h in hot))
+    assert cvs[-1] < cvs[0]
+    # (b) a full forward from x at this size, sampled against the oracle
+    y = layer.forward(inp.x)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    _check_permutation_properties(layer, T, k, E)
+    inp.bias = layer.bias.clone()             # the bias the forward used
+    rng = np.random.default_rng(33)
+    toks = np.sort(rng.choice(T, 6, replace=False))
+    feats = np.sort(rng.choice(cfg.H, 256, replace=False))
+    r, yref = _oracle_tokens(cfg, inp, toks, feats)
+    flagged = near_tie_mask(r)
+    mism = np.any(layer.ids[toks].cpu().numpy() != r.ids, axis=1)
+    assert not np.any(mism & ~flagged)
+    ok = ~flagged & ~mism
+    err = rel_err(np64(y[toks][:, torch.as_tensor(feats, device=DEV)])[ok], yref[ok])
+    print(f"v3 skewed: sampled err {err:.2e}")
+    assert err < BF16_TOL
