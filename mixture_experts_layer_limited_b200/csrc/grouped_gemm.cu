@@ -12,7 +12,8 @@
 // round_up(n, 16) columns, so ragged segment ends waste at most 15 columns,
 // instead of most of a 128-row tile when tokens sit on the M side.
 //
-// Tile = (expert g, weight block mb, token block tb). Each tile holds two
+// Tile = (expert g, weight block mb, token block tb), rasterised per segment
+// in chunks of token blocks (token block innermost). Each tile holds two
 // 128-row sub-tiles of the weight, accumulated side by side in TMEM:
 //   GEMM1: sub-tile 0 = gate rows [mb*128, +128), sub-tile 1 = up rows
 //          [I + mb*128, +128): the epilogue has gate and up of the same
@@ -41,7 +42,14 @@ constexpr int kThreads = 192;
 
 struct TileInfo {
   int g, mb, row0, n_valid, N;
+  int ntb;              // token blocks of this segment
 };
+
+// Token blocks per rasterisation chunk: inside a segment, tiles run in chunks
+// of up to kTbChunk token blocks x all weight blocks, token block innermost,
+// so CTAs running side by side share the weight block (HBM once, then L2)
+// and the chunk's token blocks (L2).
+constexpr int kTbChunk = 8;
 
 // Per-CTA copy of the tile schedule: tile_start[g] = first tile of group g.
 struct Sched {
@@ -99,8 +107,13 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, const GemmArgs& 
   const int ntb = (n + a.bn_max - 1) / a.bn_max;
   const int bn = ((((n + ntb - 1) / ntb) + 15) / 16) * 16;
   const int local = t - s.tile_start[lo];
-  const int tb = local / a.n_mblk;
-  ti.mb = local - tb * a.n_mblk;
+  const int chunk_tiles = kTbChunk * a.n_mblk;
+  const int chunk = local / chunk_tiles;
+  const int r = local - chunk * chunk_tiles;
+  const int c_tb = min(kTbChunk, ntb - chunk * kTbChunk);   // token blocks in this chunk
+  ti.mb = r / c_tb;
+  const int tb = chunk * kTbChunk + (r - ti.mb * c_tb);
+  ti.ntb = ntb;
   ti.row0 = s.seg_start[lo] + tb * bn;
   ti.n_valid = min(bn, n - tb * bn);
   ti.N = ((ti.n_valid + 15) / 16) * 16;
@@ -163,7 +176,8 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_once = policy_evict_first();
+      const uint64_t pol_reuse = policy_evict_normal();
       const uint64_t pol_x = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
@@ -172,6 +186,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         const int a_row0 = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride;
         const int a_row1 = a_row0 + a.sub1_off;
         const int nload = (ti.N + 31) / 32;
+        const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;   // re-read by sibling token blocks
         const uint32_t bytes = 2 * A_SUB_BYTES + static_cast<uint32_t>(nload) * 32u * 128u;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
@@ -345,7 +360,8 @@ grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_once = policy_evict_first();
+      const uint64_t pol_reuse = policy_evict_normal();
       const uint64_t pol_x = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
@@ -354,6 +370,7 @@ grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
         const int a_row0 = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride;
         const int a_row1 = a_row0 + a.sub1_off;
         const uint32_t bytes = 2 * A_SUB_BYTES + B_BYTES;
+        const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }

@@ -63,6 +63,12 @@ CONFIGS = {
                            scoring="sigmoid", norm_topk_prob=True, scale=2.5,
                            dtype="bf16", has_bias=True, skew_experts=16,
                            bias_steps=10, gamma=0.001, seed=1005),
+    # V3 shapes and V3's tokens per expert (T*k/E = 256) on 32 experts: the
+    # small case the profiler captures (2.8 GB of weights, larger than L2).
+    "v3_e32": MoEConfig("v3_e32", T=1024, H=7168, E=32, I=2048, I_s=2048, k=8,
+                        n_group=8, topk_group=4, scoring="sigmoid",
+                        norm_topk_prob=True, scale=2.5, dtype="bf16",
+                        has_bias=True, seed=1006),
 }
 
 

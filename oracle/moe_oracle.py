@@ -258,7 +258,8 @@ def route_from_logits(logits32: np.ndarray, k: int, n_group: int, topk_group: in
     ncand = cand.sum(axis=1)
     kth_gap = np.full(T, np.inf)
     more = ncand > k
-    kth_gap[more] = srt[more, k - 1] - srt[more, k]
+    if k < E and more.any():
+        kth_gap[more] = srt[more, k - 1] - srt[more, k]
 
     w = np.take_along_axis(unbiased, ids, axis=1)
     if norm_topk_prob:

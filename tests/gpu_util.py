@@ -54,3 +54,17 @@ def uniform_bias(E, seed, device="cuda"):
     g = torch.Generator(device=device)
     g.manual_seed(seed)
     return torch.rand(E, generator=g, dtype=torch.float32, device=device) * 0.1 - 0.05
+
+
+def routing_mismatch(ids_gpu: np.ndarray, route) -> np.ndarray:
+    """Tokens whose chosen expert SET differs (slot order may flip between
+    two chosen experts whose scores are within float noise; y is the same)."""
+    return np.any(np.sort(ids_gpu, axis=1) != np.sort(route.ids, axis=1), axis=1)
+
+
+def describe_mismatch(ids_gpu, route, tokens):
+    lines = []
+    for t in tokens[:5]:
+        lines.append(f"token {t}: gpu {ids_gpu[t].tolist()} oracle {route.ids[t].tolist()} "
+                     f"kth_gap {route.kth_gap[t]:.3e} group_gap {route.group_gap[t]:.3e}")
+    return "\n".join(lines)

@@ -13,7 +13,8 @@ from moe_inputs import get_config, tiny_grouped_config, make_inputs
 from mixture_experts_layer_limited_b200 import MoELayer, LayerSpec
 from mixture_experts_layer_limited_b200 import native as N
 
-from gpu_util import np64, np32, rel_err, oracle_route, near_tie_mask, BF16_TOL, FP8_TOL
+from gpu_util import (np64, np32, rel_err, oracle_route, near_tie_mask, routing_mismatch,
+                      describe_mismatch, BF16_TOL, FP8_TOL)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -48,15 +49,11 @@ def _oracle_tokens(cfg, inp, toks, feats=None, fp8=False):
     L = oracle.gate_logits(x64, np64(inp.gate)).astype(np.float32)
     bias = np32(inp.bias) if inp.bias is not None else None
     r = oracle_route(L, cfg, bias)
-    fidx = None if feats is None else torch.as_tensor(feats, device=DEV)
-
     def ew(e):
-        w2 = inp.w2[e] if (fidx is None or fp8) else inp.w2[e][fidx]
-        return np32(inp.w13[e]), np32(w2)
+        return np32(inp.w13[e]), np32(inp.w2[e])
 
-    sw2 = inp.sw2 if (fidx is None or fp8) else inp.sw2[fidx]
-    shared = (np32(inp.sw13), np32(sw2)) if inp.sw13 is not None else None
-    y = oracle.moe_forward(x64, r, ew, shared, fp8=fp8, out_features=feats if fp8 else None)
+    shared = (np32(inp.sw13), np32(inp.sw2)) if inp.sw13 is not None else None
+    y = oracle.moe_forward(x64, r, ew, shared, fp8=fp8, out_features=feats)
     return r, y
 
 
@@ -71,8 +68,9 @@ def test_layer_full_oracle(name):
     _check_permutation_properties(layer, cfg.T, cfg.k, cfg.E)
     r, yref = _oracle_tokens(cfg, inp, np.arange(cfg.T))
     flagged = near_tie_mask(r)
-    mism = np.any(layer.ids[:cfg.T].cpu().numpy() != r.ids, axis=1)
-    assert not np.any(mism & ~flagged)
+    ids_g = layer.ids[:cfg.T].cpu().numpy()
+    mism = routing_mismatch(ids_g, r)
+    assert not np.any(mism & ~flagged), describe_mismatch(ids_g, r, np.nonzero(mism & ~flagged)[0])
     ok = ~flagged & ~mism
     err = rel_err(np64(y)[ok], yref[ok])
     print(f"{name}: err {err:.2e}, near-tie tokens excluded {int(flagged.sum())}")
@@ -92,8 +90,9 @@ def test_layer_v3_full_size_sampled():
     feats = np.sort(rng.choice(cfg.H, 384, replace=False))
     r, yref = _oracle_tokens(cfg, inp, toks, feats)
     flagged = near_tie_mask(r)
-    mism = np.any(layer.ids[toks].cpu().numpy() != r.ids, axis=1)
-    assert not np.any(mism & ~flagged)
+    ids_g = layer.ids[toks].cpu().numpy()
+    mism = routing_mismatch(ids_g, r)
+    assert not np.any(mism & ~flagged), describe_mismatch(ids_g, r, np.nonzero(mism & ~flagged)[0])
     ok = ~flagged & ~mism
     yg = np64(y[toks][:, torch.as_tensor(feats, device=DEV)])
     err = rel_err(yg[ok], yref[ok])
@@ -118,8 +117,9 @@ def test_layer_v3_fp8_decode():
     feats = np.sort(rng.choice(cfg.H, 256, replace=False))
     r, yref = _oracle_tokens(cfg, inp, toks, feats, fp8=True)
     flagged = near_tie_mask(r)
-    mism = np.any(layer.ids[toks].cpu().numpy() != r.ids, axis=1)
-    assert not np.any(mism & ~flagged)
+    ids_g = layer.ids[toks].cpu().numpy()
+    mism = routing_mismatch(ids_g, r)
+    assert not np.any(mism & ~flagged), describe_mismatch(ids_g, r, np.nonzero(mism & ~flagged)[0])
     ok = ~flagged & ~mism
     yg = np64(y[toks][:, torch.as_tensor(feats, device=DEV)])
     err = rel_err(yg[ok], yref[ok])
@@ -169,8 +169,9 @@ def test_layer_v3_skewed_bias_loop():
     feats = np.sort(rng.choice(cfg.H, 256, replace=False))
     r, yref = _oracle_tokens(cfg, inp, toks, feats)
     flagged = near_tie_mask(r)
-    mism = np.any(layer.ids[toks].cpu().numpy() != r.ids, axis=1)
-    assert not np.any(mism & ~flagged)
+    ids_g = layer.ids[toks].cpu().numpy()
+    mism = routing_mismatch(ids_g, r)
+    assert not np.any(mism & ~flagged), describe_mismatch(ids_g, r, np.nonzero(mism & ~flagged)[0])
     ok = ~flagged & ~mism
     err = rel_err(np64(y[toks][:, torch.as_tensor(feats, device=DEV)])[ok], yref[ok])
     print(f"v3 skewed: sampled err {err:.2e}")
