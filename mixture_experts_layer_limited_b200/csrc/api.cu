@@ -1,6 +1,7 @@
 // C-ABI entry points of libmoe (declared in include/moe.h): argument checks on
 // the host, TMA tensor-map encoding, kernel launches. No allocation happens
 // here; every buffer belongs to the caller.
+#include <cstdlib>
 #include <mutex>
 
 #include "kernels.cuh"
@@ -78,6 +79,14 @@ moe_status sm_count(int* n) {
 }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// bf16 grouped GEMMs run on CTA pairs (tcgen05 cta_group::2). Setting the
+// environment variable MOE_GEMM_1SM=1 selects the one-CTA kernel instead
+// (same results, for comparison); read at each call.
+bool bf16_on_pairs() {
+  const char* v = std::getenv("MOE_GEMM_1SM");
+  return !(v && v[0] == '1');
+}
 
 }  // namespace
 
@@ -196,13 +205,14 @@ moe_status run_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const 
                        const float* a_scale, const int32_t* offsets, void* h_ws, float* h_scale_ws,
                        int32_t* dev_status, cudaStream_t st, int nsm) {
   const bool fp8 = w->dtype == MOE_E4M3;
+  const bool pair = !fp8 && bf16_on_pairs();   // CTA-pair kernel: 64-row weight, 16-row token boxes
   const int I = w->I;
   CUtensorMap tmA, tmB;
-  moe_status s = make_tmap(&tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
+  moe_status s = make_tmap(&tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, pair ? 64 : 128);
   if (s != MOE_OK) return s;
-  s = make_tmap(&tmB, a, fp8, H, rows, 32);
+  s = make_tmap(&tmB, a, fp8, H, rows, pair ? 16 : 32);
   if (s != MOE_OK) return s;
-  GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : 256,
+  GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : 256, pair ? 64 : 0,
               h_ws, I, nullptr, w->w13_scale, a_scale, h_scale_ws, dev_status};
   return check_launch(launch_grouped_gemm(fp8, EPI_SWIGLU, tmA, tmB, g1, nsm, st));
 }
@@ -211,14 +221,15 @@ moe_status run_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const voi
                     const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status,
                     cudaStream_t st, int nsm) {
   const bool fp8 = w->dtype == MOE_E4M3;
+  const bool pair = !fp8 && bf16_on_pairs();
   const int I = w->I;
   CUtensorMap tmA, tmB;
-  moe_status s = make_tmap(&tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H, 128);
+  moe_status s = make_tmap(&tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H, pair ? 64 : 128);
   if (s != MOE_OK) return s;
-  s = make_tmap(&tmB, h, fp8, I, rows, 32);
+  s = make_tmap(&tmB, h, fp8, I, rows, pair ? 16 : 32);
   if (s != MOE_OK) return s;
-  GemmArgs g2{rows, I, w->groups, offsets, H, H / 256, 256, 128, 256, 128, fp8 ? 32 : 256,
-              out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
+  GemmArgs g2{rows, I, w->groups, offsets, H, H / 256, 256, pair ? 64 : 128, 256, 128, fp8 ? 32 : 256,
+              pair ? 128 : 0, out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
   return check_launch(launch_grouped_gemm(fp8, EPI_WEIGHTED, tmA, tmB, g2, nsm, st));
 }
 

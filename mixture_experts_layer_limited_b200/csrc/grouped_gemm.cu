@@ -296,6 +296,218 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
 }
 
 // ========================================================================
+// BF16 kernel on CTA pairs (tcgen05 cta_group::2), double-buffered TMEM
+// ========================================================================
+// A CTA pair computes a 256 x N tile with one MMA stream issued by the leader
+// (cluster rank 0): each CTA stages its own 128 weight rows and N/2 of the
+// tokens, and holds the 128 x N fp32 accumulator of its rows in its TMEM.
+// Per SM that halves the token traffic of a 1-CTA 256-row tile and leaves
+// TMEM room for two accumulators (2 x 256 columns), so the epilogue of one
+// tile runs while the next tile's MMAs fill the other buffer.
+//   GEMM1: CTA r holds gate rows [f + 64r, +64) in TMEM lanes 0..63 and the
+//          matching up rows in lanes 64..127 (f = mb*128); the epilogue
+//          warps of lanes 64..127 pass the up values through shared memory
+//          to the warps of lanes 0..63, which compute SiLU(gate) * up.
+//   GEMM2: CTA r holds w2 rows [mb*256 + 128r, +128).
+constexpr int k2smStages = 6;
+constexpr int kXStride = 33;               // padded row of the lane exchange buffer
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
+  constexpr int KB = 64;
+  constexpr int STAGES = k2smStages;
+  constexpr uint32_t A_BYTES = 128 * 128;       // this CTA's 128 weight rows x 64 K
+  constexpr uint32_t B_BYTES = 128 * 128;       // up to 128 token rows x 64 K
+  constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  extern __shared__ __align__(1024) uint8_t dsmem[];
+  __shared__ Sched sched;
+  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
+  __shared__ uint64_t tmem_full[2], tmem_empty[2];
+  __shared__ uint64_t drain_bar, epi_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_flag;
+  __shared__ float xbuf[2][64 * kXStride];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(cluster_id_x());
+  const int npairs = static_cast<int>(nclusters_x());
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  auto sA = [&](int st) { return smem + st * STAGE_BYTES; };
+  auto sB = [&](int st) { return smem + st * STAGE_BYTES + A_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tmem_full[b], 1);
+      mbar_init(&tmem_empty[b], 8);               // 4 epilogue warps x 2 CTAs
+    }
+    mbar_init(&drain_bar, 1);
+    mbar_init(&epi_bar, 128);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_2sm(&tmem_base_s, 512);
+    tmem_relinquish_2sm();
+  }
+  if (warp == 2) build_schedule(sched, a, lane);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                 // the peer's barriers exist before any remote signal
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int total = sched.tile_start[a.groups];
+  const int nk = a.K / KB;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_once = policy_evict_first();
+      const uint64_t pol_reuse = policy_evict_normal();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = pair; t < total && !abort_flag; t += npairs) {
+        const TileInfo ti = decode_tile(sched, a, t);
+        const int half = ti.N >> 1;                       // tokens staged by each CTA
+        const int nload = (half + 15) >> 4;               // 16-row boxes
+        const uint32_t tx = 2u * (A_BYTES + static_cast<uint32_t>(nload) * 2048u);
+        const int a_lo = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride + static_cast<int>(rank) * a.cta_stride;
+        const int a_hi = a_lo + a.sub1_off;
+        const int b0 = ti.row0 + static_cast<int>(rank) * half;
+        const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
+          const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
+          tma_load_2d_2sm(sA(stage), &tmA, fb, kb * KB, a_lo, pol_w);
+          tma_load_2d_2sm(sA(stage) + A_BYTES / 2, &tmA, fb, kb * KB, a_hi, pol_w);
+          for (int i = 0; i < nload; ++i)
+            tma_load_2d_2sm(sB(stage) + i * 2048, &tmB, fb, kb * KB, b0 + 16 * i, pol_x);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      if (abort_flag) {   // copies complete on the leader's barrier: give them time to land
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, it = 0;
+      for (int t = pair; t < total && !abort_flag; t += npairs, ++it) {
+        const TileInfo ti = decode_tile(sched, a, t);
+        const uint32_t b = it & 1u, use = it >> 1;
+        if (!mbar_wait(&tmem_empty[b], (use & 1u) ^ 1u, &abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t idesc = make_idesc(1u, 256u, static_cast<uint32_t>(ti.N));
+        const uint32_t d = tmem_base + b * 256u;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA(stage)), b0 = smem_u32(sB(stage));
+#pragma unroll
+          for (int kk = 0; kk < KB / 16; ++kk)
+            umma_bf16_2sm(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (kb | kk) != 0);
+          umma_commit_2sm(&empty_bar[stage], 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_2sm(&tmem_full[b], 0x3);
+      }
+      umma_commit_2sm(&drain_bar, 0x1);             // every MMA done before TMEM is freed
+      mbar_wait_drain(&drain_bar, 0);
+    }
+  } else {
+    const int q = warp & 3;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    const uint32_t empty_addr0 = mapa_shared(smem_u32(&tmem_empty[0]), 0);
+    const uint32_t empty_addr1 = mapa_shared(smem_u32(&tmem_empty[1]), 0);
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+    uint32_t it = 0, epi_phase = 0, xslot = 0;
+    auto epi_sync = [&]() -> bool {
+      mbar_arrive(&epi_bar);
+      const bool r = mbar_wait(&epi_bar, epi_phase, &abort_flag, a.status);
+      epi_phase ^= 1u;
+      return r;
+    };
+    bool ok = true;
+    for (int t = pair; t < total && ok; t += npairs, ++it) {
+      const TileInfo ti = decode_tile(sched, a, t);
+      const uint32_t b = it & 1u, use = it >> 1;
+      if (!mbar_wait(&tmem_full[b], use & 1u, &abort_flag, a.status)) break;
+      tc_fence_after();
+      const uint32_t acc = lane_addr + b * 256u;
+      const int nchunk = (ti.N + 31) / 32;
+      if (EPI == EPI_SWIGLU) {
+        const int feat = ti.mb * 128 + 64 * static_cast<int>(rank) + 32 * q + lane;   // q < 2
+        for (int c = 0; c < nchunk; ++c) {
+          float v[32];
+          tmem_ld32(acc + c * 32, v);
+          tmem_ld_wait();
+          float* xb = xbuf[xslot & 1u];
+          if (q >= 2) {
+            float* row = xb + (32 * (q - 2) + lane) * kXStride;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) row[j] = v[j];
+          }
+          if (!epi_sync()) { ok = false; break; }
+          if (q < 2) {
+            const float* row = xb + (32 * q + lane) * kXStride;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int tok = c * 32 + j;
+              if (tok < ti.n_valid)
+                out[static_cast<size_t>(ti.row0 + tok) * a.out_ld + feat] = __float2bfloat16_rn(silu(v[j]) * row[j]);
+            }
+          }
+          ++xslot;
+        }
+        if (!ok) break;
+      } else {
+        const int feat = ti.mb * 256 + 128 * static_cast<int>(rank) + 32 * q + lane;
+        for (int c = 0; c < nchunk; ++c) {
+          float v[32];
+          tmem_ld32(acc + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int tok = c * 32 + j;
+            if (tok < ti.n_valid) {
+              const float w = a.row_w ? __ldg(a.row_w + ti.row0 + tok) : 1.0f;
+              out[static_cast<size_t>(ti.row0 + tok) * a.out_ld + feat] = __float2bfloat16_rn(v[j] * w);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(b ? empty_addr1 : empty_addr0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                 // the pair is done with each other's memory
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_2sm(tmem_base, 512);
+}
+
+// ========================================================================
 // E4M3 kernel (block-scaled, promotion on CUDA cores), tokens per tile <= 32
 // ========================================================================
 constexpr int kF8Bn = 32;          // max tokens per tile
@@ -527,6 +739,9 @@ grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
 size_t gemm_bf16_smem_bytes(int stages, int bn_max) {
   return static_cast<size_t>(stages) * (2 * 128 * 128 + static_cast<size_t>(bn_max) * 128) + 1024;
 }
+size_t gemm_bf16_2sm_smem_bytes() {
+  return static_cast<size_t>(k2smStages) * (2 * 128 * 128) + 1024;
+}
 size_t gemm_e4m3_smem_bytes(int stages) {
   return static_cast<size_t>(stages) * (2 * 128 * 128 + kF8Bn * 128) + 1024;
 }
@@ -536,7 +751,14 @@ constexpr int kE4m3Stages = 4;
 
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 const GemmArgs& a, int grid, cudaStream_t stream) {
-  if (!e4m3) {
+  if (!e4m3 && a.cta_stride > 0) {
+    const size_t smem = gemm_bf16_2sm_smem_bytes();
+    auto kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_2sm_kernel<EPI_SWIGLU>
+                                  : grouped_gemm_bf16_2sm_kernel<EPI_WEIGHTED>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<grid & ~1, kThreads, smem, stream>>>(tmA, tmB, a);
+  } else if (!e4m3) {
     const size_t smem = gemm_bf16_smem_bytes(kBf16Stages, a.bn_max);
     auto kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages>
                                   : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages>;

@@ -215,13 +215,24 @@ def _ref_grouped(a, w13, w2, off, row_w):
     return out, hs
 
 
+@pytest.fixture(params=["pair", "1sm"])
+def gemm_variant(request, monkeypatch):
+    """bf16 grouped GEMMs: CTA-pair kernel (default) or the one-CTA kernel."""
+    if request.param == "1sm":
+        monkeypatch.setenv("MOE_GEMM_1SM", "1")
+    else:
+        monkeypatch.delenv("MOE_GEMM_1SM", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("H,I,sizes", [
     (512, 256, [0, 1, 15, 16, 17, 100, 255, 256, 257, 600, 0, 33]),
     (256, 128, [64]),
     (7168, 2048, [300, 77]),
     (2048, 1408, [384, 0, 5, 513]),
+    (512, 256, [1200, 2, 8]),
 ])
-def test_grouped_swiglu_bf16(H, I, sizes):
+def test_grouped_swiglu_bf16(H, I, sizes, gemm_variant):
     G = len(sizes)
     off = _segments(sizes)
     rows = int(off[-1])
@@ -238,11 +249,11 @@ def test_grouped_swiglu_bf16(H, I, sizes):
     assert N.moe_read_device_status(status) == 0
     ref, href = _ref_grouped(a, w13, w2, off, row_w)
     eh, eo = rel_err(np64(h), href), rel_err(np64(out), ref)
-    print(f"H={H} I={I}: h err {eh:.2e}, out err {eo:.2e}")
+    print(f"{gemm_variant} H={H} I={I}: h err {eh:.2e}, out err {eo:.2e}")
     assert eh < 1e-2 and eo < BF16_TOL
 
 
-def test_grouped_swiglu_bf16_single_group_no_offsets():
+def test_grouped_swiglu_bf16_single_group_no_offsets(gemm_variant):
     rows, H, I = 300, 512, 384
     g = _gen(77)
     a = torch.randn(rows, H, generator=g, device=DEV).to(torch.bfloat16)
