@@ -152,6 +152,36 @@ MOE_API moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H,
                        int32_t* dev_status, void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * moe_permute_static_ws -- moe_permute without a caller-provided workspace.
+ * The pages have no counterpart: this is a library convenience.
+ *
+ * For callers that cannot allocate device memory where they call the
+ * permutation: code whose device memory all belongs to a framework allocator
+ * and must not be taken around it, code that must not risk the implicit
+ * device synchronisation a cudaMalloc can cause, and plugin interfaces that
+ * hand in only input and output buffers. Arguments, outputs and errors are
+ * those of moe_permute, minus `workspace` / `workspace_bytes`.
+ *
+ * The scratch is a 1 MiB array in the library's own device memory (every GPU
+ * that loads the library holds it until the process exits). It fits
+ * ceil(T / 64) * E <= 262144, e.g. T <= 65536 tokens with E = 256; larger
+ * T, E return MOE_ERR_UNSUPPORTED before anything is launched. No memory is
+ * allocated. The first call on a device looks up the array's address for
+ * that device (cudaGetSymbolAddress), so make that first call before any
+ * stream capture. All calls share the one array: calls whose work overlaps
+ * on the GPU (other streams, other host threads) race and give wrong
+ * results; serialise them. Nothing needs clearing between calls (every call
+ * rewrites the part of the array it reads).
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_permute_static_ws(int32_t T, int32_t k, int32_t E, int32_t H,
+                       const int32_t* topk_ids, const float* topk_w,
+                       const void* x, moe_dtype x_dtype, const float* x_scale,
+                       void* x_perm, float* x_perm_scale,
+                       int32_t* expert_offsets, int32_t* src_token,
+                       int32_t* slot_to_row, float* row_w,
+                       int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * moe_grouped_swiglu -- SwiGLU experts over contiguous row segments.
  * [MoE-walk] §3.3.1 (w13 = [w1; w3], gate = first I outputs, up = last I,
  * h = SiLU(gate) * up, out = h @ w2^T) and the grouped GEMM of the same

@@ -216,3 +216,49 @@ cudaError_t launch_permute(int T, int k, int E, int row_bytes, const int32_t* id
 }
 
 }  // namespace moe
+
+// ------------------------------------------------------------------------
+// moe_permute_static_ws: the permutation with its scratch in this library's
+// own device memory, for callers that cannot allocate (see include/moe.h).
+// ------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr size_t kStaticWsBytes = size_t(1) << 20;      // 1 MiB
+constexpr int kMaxDevices = 64;
+
+// The scratch itself: one copy per device that loads the library. In host
+// code this name is only a stand-in for the symbol; its device address comes
+// from cudaGetSymbolAddress below.
+__device__ __align__(256) int32_t g_permute_static_ws[kStaticWsBytes / sizeof(int32_t)];
+
+std::mutex g_static_ws_mu;
+void* g_static_ws_ptr[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" moe_status moe_permute_static_ws(int32_t T, int32_t k, int32_t E, int32_t H,
+                                            const int32_t* topk_ids, const float* topk_w,
+                                            const void* x, moe_dtype x_dtype, const float* x_scale,
+                                            void* x_perm, float* x_perm_scale, int32_t* expert_offsets,
+                                            int32_t* src_token, int32_t* slot_to_row, float* row_w,
+                                            int32_t* dev_status, void* stream) {
+  if (T < 1 || k < 1 || E < 1) return MOE_ERR_INVALID_ARG;
+  if (moe::permute_workspace_bytes(T, E) > kStaticWsBytes) return MOE_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_ws_mu);
+    if (!g_static_ws_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_permute_static_ws) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+      g_static_ws_ptr[dev] = p;
+    }
+    ws = g_static_ws_ptr[dev];
+  }
+  return moe_permute(T, k, E, H, topk_ids, topk_w, x, x_dtype, x_scale, x_perm, x_perm_scale, expert_offsets,
+                     src_token, slot_to_row, row_w, ws, kStaticWsBytes, dev_status, stream);
+}

@@ -26,7 +26,8 @@ MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
 MOE_SOFTMAX, MOE_SIGMOID = 0, 1
 
 EXPORTED = [
-    "moe_route", "moe_permute_workspace_size", "moe_permute", "moe_grouped_swiglu",
+    "moe_route", "moe_permute_workspace_size", "moe_permute", "moe_permute_static_ws",
+    "moe_grouped_swiglu",
     "moe_gate_up_swiglu", "moe_down_proj",
     "moe_combine", "moe_bias_update", "moe_quantize_blocks", "moe_quantize_rows",
     "moe_read_device_status", "moe_last_cuda_error", "moe_status_string", "moe_abi_version",
@@ -72,6 +73,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_permute_workspace_size": [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
         "moe_permute": [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
                         ctypes.c_size_t, _P, _P],
+        "moe_permute_static_ws": [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P],
         "moe_grouped_swiglu": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P, _P, _P],
         "moe_gate_up_swiglu": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P],
         "moe_down_proj": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P],
