@@ -120,7 +120,9 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, const GemmArgs& 
   return ti;
 }
 
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+// SiLU(g) = g * sigmoid(g). Fast division: for g < -88 the exponential
+// overflows to inf and the quotient is the correct limit (-0).
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // ========================================================================
 // BF16 kernel
