@@ -69,6 +69,18 @@ moe_status make_tmap(CUtensorMap* m, const void* ptr, bool one_byte, uint64_t in
   return MOE_OK;
 }
 
+// Token-row maps of a grouped GEMM: bf16 rows are fetched with 64-, 32- and
+// 16-row boxes; e4m3 rows (at most 32 tokens a tile) with one 32-row box.
+moe_status make_token_tmaps(CUtensorMap* m, const void* ptr, bool fp8, uint64_t K, uint64_t rows) {
+  if (fp8) return make_tmap(&m[0], ptr, true, K, rows, 32);
+  const uint32_t box[3] = {64, 32, 16};
+  for (int i = 0; i < 3; ++i) {
+    moe_status s = make_tmap(&m[i], ptr, false, K, rows, box[i]);
+    if (s != MOE_OK) return s;
+  }
+  return MOE_OK;
+}
+
 moe_status sm_count(int* n) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -80,12 +92,17 @@ moe_status sm_count(int* n) {
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-// bf16 grouped GEMMs run on CTA pairs (tcgen05 cta_group::2). Setting the
-// environment variable MOE_GEMM_1SM=1 selects the one-CTA kernel instead
-// (same results, for comparison); read at each call.
-bool bf16_on_pairs() {
-  const char* v = std::getenv("MOE_GEMM_1SM");
-  return !(v && v[0] == '1');
+// Kernel choice for the bf16 grouped GEMMs, by measurement at the V3 shape:
+// the gate/up GEMM (SwiGLU epilogue) runs on single CTAs, the down GEMM on
+// CTA pairs (tcgen05 cta_group::2, epilogue overlapped with the next tile).
+// MOE_GEMM_1SM=1 puts both on single CTAs, MOE_GEMM_PAIR=1 both on pairs
+// (same results; for comparison). Read at each call.
+bool bf16_on_pairs(bool gate_up) {
+  const char* one = std::getenv("MOE_GEMM_1SM");
+  if (one && one[0] == '1') return false;
+  const char* pr = std::getenv("MOE_GEMM_PAIR");
+  if (pr && pr[0] == '1') return true;
+  return !gate_up;
 }
 
 }  // namespace
@@ -205,12 +222,12 @@ moe_status run_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const 
                        const float* a_scale, const int32_t* offsets, void* h_ws, float* h_scale_ws,
                        int32_t* dev_status, cudaStream_t st, int nsm) {
   const bool fp8 = w->dtype == MOE_E4M3;
-  const bool pair = !fp8 && bf16_on_pairs();   // CTA-pair kernel: 64-row weight, 16-row token boxes
+  const bool pair = !fp8 && bf16_on_pairs(true);
   const int I = w->I;
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB[3];
   moe_status s = make_tmap(&tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, pair ? 64 : 128);
   if (s != MOE_OK) return s;
-  s = make_tmap(&tmB, a, fp8, H, rows, pair ? 16 : 32);
+  s = make_token_tmaps(tmB, a, fp8, H, rows);
   if (s != MOE_OK) return s;
   GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : 256, pair ? 64 : 0,
               h_ws, I, nullptr, w->w13_scale, a_scale, h_scale_ws, dev_status};
@@ -221,12 +238,12 @@ moe_status run_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const voi
                     const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status,
                     cudaStream_t st, int nsm) {
   const bool fp8 = w->dtype == MOE_E4M3;
-  const bool pair = !fp8 && bf16_on_pairs();
+  const bool pair = !fp8 && bf16_on_pairs(false);
   const int I = w->I;
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB[3];
   moe_status s = make_tmap(&tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H, pair ? 64 : 128);
   if (s != MOE_OK) return s;
-  s = make_tmap(&tmB, h, fp8, I, rows, pair ? 16 : 32);
+  s = make_token_tmaps(tmB, h, fp8, I, rows);
   if (s != MOE_OK) return s;
   GemmArgs g2{rows, I, w->groups, offsets, H, H / 256, 256, pair ? 64 : 128, 256, 128, fp8 ? 32 : 256,
               pair ? 128 : 0, out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};

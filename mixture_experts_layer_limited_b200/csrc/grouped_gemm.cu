@@ -120,6 +120,39 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, const GemmArgs& 
   return ti;
 }
 
+// Token rows of one stage are fetched as 64-row boxes, then at most one
+// 32-row and one 16-row box (`rows` is a multiple of 16). Returns rows loaded.
+template <typename LoadFn>
+__device__ __forceinline__ int load_token_rows(int rows, LoadFn&& load) {
+  int off = 0;
+  for (; rows - off >= 64; off += 64) load(0, off);
+  if (rows - off >= 32) { load(1, off); off += 32; }
+  if (rows - off >= 16) { load(2, off); off += 16; }
+  return off;
+}
+
+// Writes NT tokens x 32 features (thread = feature lane, v[j] = token j) to
+// out[(row0 + j) * ld + feat0 + lane] through a per-warp shared tile, so that
+// every global store is a 16-byte vector (4 lanes cover one token's 32
+// features). Tokens j >= n_rows are not written.
+template <int NT>
+__device__ __forceinline__ void store_tile(__nv_bfloat16* stage, const float (&v)[NT], int lane,
+                                           __nv_bfloat16* out, size_t ld, int row0, int n_rows, int feat0) {
+#pragma unroll
+  for (int j = 0; j < NT; ++j) stage[j * 32 + lane] = __float2bfloat16_rn(v[j]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < NT / 8; ++i) {
+    const int t = (lane >> 2) + 8 * i;
+    const int seg = lane & 3;
+    if (t < n_rows) {
+      const uint4 val = *reinterpret_cast<const uint4*>(stage + t * 32 + seg * 8);
+      *reinterpret_cast<uint4*>(out + static_cast<size_t>(row0 + t) * ld + feat0 + seg * 8) = val;
+    }
+  }
+  __syncwarp();
+}
+
 // SiLU(g) = g * sigmoid(g). Fast division: for g < -88 the exponential
 // overflows to inf and the quotient is the correct limit (-0).
 __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
@@ -130,11 +163,14 @@ __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __e
 template <int EPI, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
-                         const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
+                         const __grid_constant__ CUtensorMap tmB64,
+                         const __grid_constant__ CUtensorMap tmB32,
+                         const __grid_constant__ CUtensorMap tmB16, const GemmArgs a) {
   constexpr int KB = 64;                           // K elements per stage (128 B)
   constexpr uint32_t A_SUB_BYTES = 128 * 128;      // one 128-row sub-tile
   extern __shared__ __align__(1024) uint8_t dsmem[];
   __shared__ Sched sched;
+  __shared__ __align__(16) __nv_bfloat16 stage_out[4][32 * 32];
   __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
   __shared__ uint64_t tmem_full, tmem_empty, drain_bar;
   __shared__ uint32_t tmem_base_s;
@@ -162,7 +198,9 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmB64);
+    tma_prefetch_desc(&tmB32);
+    tma_prefetch_desc(&tmB16);
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_s, 512);
@@ -181,23 +219,26 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       const uint64_t pol_once = policy_evict_first();
       const uint64_t pol_reuse = policy_evict_normal();
       const uint64_t pol_x = policy_evict_last();
+      const CUtensorMap* tmB[3] = {&tmB64, &tmB32, &tmB16};
       int stage = 0;
       uint32_t phase = 0;
       for (int t = blockIdx.x; t < total && !abort_flag; t += gridDim.x) {
         const TileInfo ti = decode_tile(sched, a, t);
         const int a_row0 = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride;
         const int a_row1 = a_row0 + a.sub1_off;
-        const int nload = (ti.N + 31) / 32;
         const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;   // re-read by sibling token blocks
-        const uint32_t bytes = 2 * A_SUB_BYTES + static_cast<uint32_t>(nload) * 32u * 128u;
+        const uint32_t bytes = 2 * A_SUB_BYTES + static_cast<uint32_t>(ti.N) * 128u;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
           tma_load_2d(sA(stage, 0), &tmA, &full_bar[stage], kb * KB, a_row0, pol_w);
           tma_load_2d(sA(stage, 1), &tmA, &full_bar[stage], kb * KB, a_row1, pol_w);
-          for (int i = 0; i < nload; ++i)
-            tma_load_2d(sB(stage) + i * 4096, &tmB, &full_bar[stage], kb * KB, ti.row0 + 32 * i, pol_x);
+          uint8_t* bdst = sB(stage);
+          uint64_t* fb = &full_bar[stage];
+          load_token_rows(ti.N, [&](int which, int off) {
+            tma_load_2d(bdst + off * 128, tmB[which], fb, kb * KB, ti.row0 + off, pol_x);
+          });
           issued_parity[stage] = static_cast<int>(phase);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -252,36 +293,32 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       if (!mbar_wait(&tmem_full, acc_phase, &abort_flag, a.status)) break;
       tc_fence_after();
       const int nchunk = (ti.N + 31) / 32;
+      __nv_bfloat16* stg = stage_out[q];
       if (EPI == EPI_SWIGLU) {
-        const int feat = ti.mb * a.feat_stride + 32 * q + lane;
+        const int feat0 = ti.mb * a.feat_stride + 32 * q;          // this warp's 32 features
         for (int c = 0; c < nchunk; ++c) {
           float g[32], u[32];
           tmem_ld32(lane_addr + c * 32, g);
           tmem_ld32(lane_addr + 256 + c * 32, u);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int tok = c * 32 + j;
-            if (tok < ti.n_valid)
-              out[static_cast<size_t>(ti.row0 + tok) * a.out_ld + feat] = __float2bfloat16_rn(silu(g[j]) * u[j]);
-          }
+          for (int j = 0; j < 32; ++j) g[j] = silu(g[j]) * u[j];
+          store_tile<32>(stg, g, lane, out, a.out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
         }
       } else {
 #pragma unroll 1
         for (int s = 0; s < 2; ++s) {
-          const int feat = ti.mb * a.feat_stride + s * a.feat_sub1 + 32 * q + lane;
+          const int feat0 = ti.mb * a.feat_stride + s * a.feat_sub1 + 32 * q;
           for (int c = 0; c < nchunk; ++c) {
             float v[32];
             tmem_ld32(lane_addr + s * 256 + c * 32, v);
             tmem_ld_wait();
+            if (a.row_w) {
+              const float wl = (c * 32 + lane < ti.n_valid) ? __ldg(a.row_w + ti.row0 + c * 32 + lane) : 0.0f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int tok = c * 32 + j;
-              if (tok < ti.n_valid) {
-                const float w = a.row_w ? __ldg(a.row_w + ti.row0 + tok) : 1.0f;
-                out[static_cast<size_t>(ti.row0 + tok) * a.out_ld + feat] = __float2bfloat16_rn(v[j] * w);
-              }
+              for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wl, j);
             }
+            store_tile<32>(stg, v, lane, out, a.out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
           }
         }
       }
@@ -317,7 +354,9 @@ constexpr int kXStride = 33;               // padded row of the lane exchange bu
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
-                             const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
+                             const __grid_constant__ CUtensorMap tmB64,
+                             const __grid_constant__ CUtensorMap tmB32,
+                             const __grid_constant__ CUtensorMap tmB16, const GemmArgs a) {
   constexpr int KB = 64;
   constexpr int STAGES = k2smStages;
   constexpr uint32_t A_BYTES = 128 * 128;       // this CTA's 128 weight rows x 64 K
@@ -331,6 +370,7 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_flag;
   __shared__ float xbuf[2][64 * kXStride];
+  __shared__ __align__(16) __nv_bfloat16 stage_out[4][32 * 32];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -357,7 +397,9 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmB64);
+    tma_prefetch_desc(&tmB32);
+    tma_prefetch_desc(&tmB16);
   }
   if (warp == 1) {
     tmem_alloc_2sm(&tmem_base_s, 512);
@@ -377,13 +419,14 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
       const uint64_t pol_once = policy_evict_first();
       const uint64_t pol_reuse = policy_evict_normal();
       const uint64_t pol_x = policy_evict_last();
+      const CUtensorMap* tmB[3] = {&tmB64, &tmB32, &tmB16};
       int stage = 0;
       uint32_t phase = 0;
       for (int t = pair; t < total && !abort_flag; t += npairs) {
         const TileInfo ti = decode_tile(sched, a, t);
         const int half = ti.N >> 1;                       // tokens staged by each CTA
-        const int nload = (half + 15) >> 4;               // 16-row boxes
-        const uint32_t tx = 2u * (A_BYTES + static_cast<uint32_t>(nload) * 2048u);
+        const int rows = (half + 15) & ~15;               // rows fetched (multiple of 16)
+        const uint32_t tx = 2u * (A_BYTES + static_cast<uint32_t>(rows) * 128u);
         const int a_lo = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride + static_cast<int>(rank) * a.cta_stride;
         const int a_hi = a_lo + a.sub1_off;
         const int b0 = ti.row0 + static_cast<int>(rank) * half;
@@ -395,8 +438,10 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
           tma_load_2d_2sm(sA(stage), &tmA, fb, kb * KB, a_lo, pol_w);
           tma_load_2d_2sm(sA(stage) + A_BYTES / 2, &tmA, fb, kb * KB, a_hi, pol_w);
-          for (int i = 0; i < nload; ++i)
-            tma_load_2d_2sm(sB(stage) + i * 2048, &tmB, fb, kb * KB, b0 + 16 * i, pol_x);
+          uint8_t* bdst = sB(stage);
+          load_token_rows(rows, [&](int which, int off) {
+            tma_load_2d_2sm(bdst + off * 128, tmB[which], fb, kb * KB, b0 + off, pol_x);
+          });
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -455,45 +500,52 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
       tc_fence_after();
       const uint32_t acc = lane_addr + b * 256u;
       const int nchunk = (ti.N + 31) / 32;
+      __nv_bfloat16* stg = stage_out[q];
       if (EPI == EPI_SWIGLU) {
-        const int feat = ti.mb * 128 + 64 * static_cast<int>(rank) + 32 * q + lane;   // q < 2
+        // Lanes 0..63 hold gate, 64..127 up, of the same 64 features. Gate
+        // warps finish tokens 0..15 of each chunk, up warps tokens 16..31:
+        // each hands the other half of its values over through xbuf.
+        const bool gate_warp = q < 2;
+        const int fl = 32 * (q & 1) + lane;                                   // feature within the 64
+        const int feat0 = ti.mb * 128 + 64 * static_cast<int>(rank) + 32 * (q & 1);
         for (int c = 0; c < nchunk; ++c) {
           float v[32];
           tmem_ld32(acc + c * 32, v);
           tmem_ld_wait();
-          float* xb = xbuf[xslot & 1u];
-          if (q >= 2) {
-            float* row = xb + (32 * (q - 2) + lane) * kXStride;
+          float* row = xbuf[xslot & 1u] + fl * kXStride;
+          if (gate_warp) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) row[j] = v[j];
+            for (int j = 16; j < 32; ++j) row[j] = v[j];
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) row[j] = v[j];
           }
           if (!epi_sync()) { ok = false; break; }
-          if (q < 2) {
-            const float* row = xb + (32 * q + lane) * kXStride;
+          float hh[16];
+          if (gate_warp) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int tok = c * 32 + j;
-              if (tok < ti.n_valid)
-                out[static_cast<size_t>(ti.row0 + tok) * a.out_ld + feat] = __float2bfloat16_rn(silu(v[j]) * row[j]);
-            }
+            for (int j = 0; j < 16; ++j) hh[j] = silu(v[j]) * row[j];
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) hh[j] = silu(row[16 + j]) * v[16 + j];
           }
+          const int t0 = c * 32 + (gate_warp ? 0 : 16);
+          store_tile<16>(stg, hh, lane, out, a.out_ld, ti.row0 + t0, ti.n_valid - t0, feat0);
           ++xslot;
         }
         if (!ok) break;
       } else {
-        const int feat = ti.mb * 256 + 128 * static_cast<int>(rank) + 32 * q + lane;
+        const int feat0 = ti.mb * 256 + 128 * static_cast<int>(rank) + 32 * q;
         for (int c = 0; c < nchunk; ++c) {
           float v[32];
           tmem_ld32(acc + c * 32, v);
           tmem_ld_wait();
+          if (a.row_w) {
+            const float wl = (c * 32 + lane < ti.n_valid) ? __ldg(a.row_w + ti.row0 + c * 32 + lane) : 0.0f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int tok = c * 32 + j;
-            if (tok < ti.n_valid) {
-              const float w = a.row_w ? __ldg(a.row_w + ti.row0 + tok) : 1.0f;
-              out[static_cast<size_t>(ti.row0 + tok) * a.out_ld + feat] = __float2bfloat16_rn(v[j] * w);
-            }
+            for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wl, j);
           }
+          store_tile<32>(stg, v, lane, out, a.out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
         }
       }
       tc_fence_before();
@@ -751,7 +803,7 @@ size_t gemm_e4m3_smem_bytes(int stages) {
 constexpr int kBf16Stages = 3;
 constexpr int kE4m3Stages = 4;
 
-cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap* tmB,
                                 const GemmArgs& a, int grid, cudaStream_t stream) {
   if (!e4m3 && a.cta_stride > 0) {
     const size_t smem = gemm_bf16_2sm_smem_bytes();
@@ -759,21 +811,21 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
                                   : grouped_gemm_bf16_2sm_kernel<EPI_WEIGHTED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid & ~1, kThreads, smem, stream>>>(tmA, tmB, a);
+    kern<<<grid & ~1, kThreads, smem, stream>>>(tmA, tmB[0], tmB[1], tmB[2], a);
   } else if (!e4m3) {
     const size_t smem = gemm_bf16_smem_bytes(kBf16Stages, a.bn_max);
     auto kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages>
                                   : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, stream>>>(tmA, tmB, a);
+    kern<<<grid, kThreads, smem, stream>>>(tmA, tmB[0], tmB[1], tmB[2], a);
   } else {
     const size_t smem = gemm_e4m3_smem_bytes(kE4m3Stages);
     auto kern = epi == EPI_SWIGLU ? grouped_gemm_e4m3_kernel<EPI_SWIGLU, kE4m3Stages>
                                   : grouped_gemm_e4m3_kernel<EPI_WEIGHTED, kE4m3Stages>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, stream>>>(tmA, tmB, a);
+    kern<<<grid, kThreads, smem, stream>>>(tmA, tmB[0], a);
   }
   return cudaGetLastError();
 }

@@ -41,7 +41,9 @@ struct RouteArgs {
 
 enum { EPI_SWIGLU = 0, EPI_WEIGHTED = 1 };
 
-cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+// tmB: token-row tensor maps with 64-, 32- and 16-row boxes (bf16), or one
+// 32-row map (e4m3).
+cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap* tmB,
                                 const GemmArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_route_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
                               cudaStream_t stream);

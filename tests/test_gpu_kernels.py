@@ -217,11 +217,10 @@ def _ref_grouped(a, w13, w2, off, row_w):
 
 @pytest.fixture(params=["pair", "1sm"])
 def gemm_variant(request, monkeypatch):
-    """bf16 grouped GEMMs: CTA-pair kernel (default) or the one-CTA kernel."""
-    if request.param == "1sm":
-        monkeypatch.setenv("MOE_GEMM_1SM", "1")
-    else:
-        monkeypatch.delenv("MOE_GEMM_1SM", raising=False)
+    """bf16 grouped GEMMs, both kernels forced: CTA pairs or single CTAs."""
+    monkeypatch.delenv("MOE_GEMM_1SM", raising=False)
+    monkeypatch.delenv("MOE_GEMM_PAIR", raising=False)
+    monkeypatch.setenv("MOE_GEMM_PAIR" if request.param == "pair" else "MOE_GEMM_1SM", "1")
     return request.param
 
 
