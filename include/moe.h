@@ -236,6 +236,23 @@ MOE_API moe_status moe_down_proj(int32_t rows, int32_t H, const moe_ffn_weights*
                          const void* h, const float* h_scale, const int32_t* offsets,
                          const float* row_w, void* out, int32_t* dev_status, void* stream);
 
+/* moe_gate_up_swiglu_gather -- the routed experts' first GEMM with the
+ * permutation fused into its operand fetch ([MoE-walk] §3.2 + §3.3.1): row p
+ * of the expert segments is read directly from x[src_token[p]], so
+ * moe_permute can run with x_perm = NULL (no [T*k, H] copy is written).
+ *   rows      T*k; x [T, H] bf16; src_token [rows] (from moe_permute, each in
+ *             [0, T): indices outside are flagged MOE_DEVSTAT_BAD_EXPERT_ID in
+ *             dev_status and not read); offsets [groups+1] (required);
+ *   h_ws      [rows, I] bf16 = SiLU(x_p w1^T) * (x_p w3^T).
+ * bf16 weights only (MOE_ERR_UNSUPPORTED otherwise); limits as above.
+ * The rows are fetched with 16-byte cp.async by two extra warps; at the V3
+ * shape on B200 this is slower than moe_permute + moe_gate_up_swiglu, whose
+ * token rows arrive as TMA boxes, so use it where memory for x_perm is short. */
+MOE_API moe_status moe_gate_up_swiglu_gather(int32_t rows, int32_t H, const moe_ffn_weights* w,
+                                     const void* x, int32_t T, const int32_t* src_token,
+                                     const int32_t* offsets, void* h_ws,
+                                     int32_t* dev_status, void* stream);
+
 /* ------------------------------------------------------------------------ *
  * moe_combine -- unpermute and weighted combine, [MoE-walk] §3.4:
  *   y[t] = shared_out[t] + sum_j topk_w[t][j] * expert_out[slot_to_row[t*k+j]]

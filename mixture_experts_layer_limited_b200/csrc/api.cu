@@ -267,6 +267,27 @@ moe_status moe_gate_up_swiglu(int32_t rows, int32_t H, const moe_ffn_weights* w,
   return run_gate_up(rows, H, w, a, a_scale, offsets, h_ws, h_scale_ws, dev_status, as_stream(stream), nsm);
 }
 
+moe_status moe_gate_up_swiglu_gather(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* x, int32_t T,
+                                     const int32_t* src_token, const int32_t* offsets, void* h_ws,
+                                     int32_t* dev_status, void* stream) {
+  moe_status s = check_ffn(rows, H, w, x, nullptr, true, false);
+  if (s != MOE_OK) return s;
+  if (w->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (T < 1 || !src_token || !offsets || !h_ws) return MOE_ERR_INVALID_ARG;
+  if (any_misaligned(src_token, offsets, h_ws)) return MOE_ERR_ALIGNMENT;
+  int nsm = 0;
+  if ((s = sm_count(&nsm)) != MOE_OK) return s;
+  const int I = w->I;
+  CUtensorMap tmA, tmB[3];
+  s = make_tmap(&tmA, w->w13, false, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
+  if (s != MOE_OK) return s;
+  s = make_token_tmaps(tmB, x, false, H, T);      // not read: token rows are gathered
+  if (s != MOE_OK) return s;
+  GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, 256, 0,
+              h_ws, I, nullptr, nullptr, nullptr, nullptr, dev_status, x, src_token, T};
+  return check_launch(launch_grouped_gemm(false, EPI_SWIGLU, tmA, tmB, g1, nsm, as_stream(stream)));
+}
+
 moe_status moe_down_proj(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* h, const float* h_scale,
                          const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status,
                          void* stream) {

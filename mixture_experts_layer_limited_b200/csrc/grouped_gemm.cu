@@ -160,8 +160,16 @@ __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __e
 // ========================================================================
 // BF16 kernel
 // ========================================================================
-template <int EPI, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+// GATHER: two more warps (6, 7) fetch the token rows of every stage from
+// a.gather_src at rows a.gather_rows[p] with 16-byte cp.async, writing the
+// same 128-byte-swizzled layout TMA would (16-byte chunk c of row r lands at
+// r * 128 + (c ^ (r % 8)) * 16). Each gather thread arrives on a stage's full
+// barrier once its copies of that stage have landed and been fenced to the
+// async proxy; it keeps one stage of copies in flight ahead of that.
+constexpr int kGatherThreads = 64;
+
+template <int EPI, int STAGES, bool GATHER>
+__global__ void __launch_bounds__(kThreads + (GATHER ? kGatherThreads : 0), 1)
 grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB64,
                          const __grid_constant__ CUtensorMap tmB32,
@@ -186,7 +194,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full_bar[i], 1);
+      mbar_init(&full_bar[i], GATHER ? 1 + kGatherThreads : 1);
       mbar_init(&empty_bar[i], 1);
       issued_parity[i] = -1;
     }
@@ -227,18 +235,20 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         const int a_row0 = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride;
         const int a_row1 = a_row0 + a.sub1_off;
         const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;   // re-read by sibling token blocks
-        const uint32_t bytes = 2 * A_SUB_BYTES + static_cast<uint32_t>(ti.N) * 128u;
+        const uint32_t bytes = 2 * A_SUB_BYTES + (GATHER ? 0u : static_cast<uint32_t>(ti.N) * 128u);
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
           tma_load_2d(sA(stage, 0), &tmA, &full_bar[stage], kb * KB, a_row0, pol_w);
           tma_load_2d(sA(stage, 1), &tmA, &full_bar[stage], kb * KB, a_row1, pol_w);
-          uint8_t* bdst = sB(stage);
-          uint64_t* fb = &full_bar[stage];
-          load_token_rows(ti.N, [&](int which, int off) {
-            tma_load_2d(bdst + off * 128, tmB[which], fb, kb * KB, ti.row0 + off, pol_x);
-          });
+          if (!GATHER) {
+            uint8_t* bdst = sB(stage);
+            uint64_t* fb = &full_bar[stage];
+            load_token_rows(ti.N, [&](int which, int off) {
+              tma_load_2d(bdst + off * 128, tmB[which], fb, kb * KB, ti.row0 + off, pol_x);
+            });
+          }
           issued_parity[stage] = static_cast<int>(phase);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -248,6 +258,48 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int i = 0; i < STAGES; ++i)
           if (issued_parity[i] >= 0) mbar_wait_drain(&full_bar[i], static_cast<uint32_t>(issued_parity[i]));
       }
+    }
+  } else if (GATHER && warp >= 6) {
+    const int gt = threadIdx.x - kThreads;             // 0..63
+    const int chunk = gt & 7;                          // 16-byte chunk of the 128-byte row slice
+    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.gather_src);
+    int stage = 0, pending = -1;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok && !abort_flag; t += gridDim.x) {
+      const TileInfo ti = decode_tile(sched, a, t);
+      int srow[32];                                    // source rows of this thread's token rows
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = (gt >> 3) + 8 * i;
+        int sr = (r < ti.n_valid) ? __ldg(a.gather_rows + ti.row0 + r) : -1;
+        if (sr >= a.gather_src_rows) { flag_status(a.status, MOE_DEVSTAT_BAD_EXPERT_ID); sr = -1; }
+        srow[i] = sr;
+      }
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
+        const uint32_t bbase = smem_u32(sB(stage));
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int r = (gt >> 3) + 8 * i;
+          if (srow[i] >= 0)
+            cp_async_16(bbase + r * 128 + ((chunk ^ (r & 7)) << 4),
+                        src + static_cast<size_t>(srow[i]) * a.K + kb * KB + chunk * 8);
+        }
+        cp_async_commit();
+        if (pending >= 0) {                            // the previous stage has landed
+          cp_async_wait<1>();
+          fence_proxy_async();
+          mbar_arrive(&full_bar[pending]);
+        }
+        pending = stage;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    cp_async_wait<0>();
+    if (pending >= 0 && ok) {
+      fence_proxy_async();
+      mbar_arrive(&full_bar[pending]);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -282,7 +334,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       umma_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0);
     }
-  } else {
+  } else if (warp < 6) {
     // epilogue warps 2..5
     const int q = warp & 3;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
@@ -814,11 +866,14 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
     kern<<<grid & ~1, kThreads, smem, stream>>>(tmA, tmB[0], tmB[1], tmB[2], a);
   } else if (!e4m3) {
     const size_t smem = gemm_bf16_smem_bytes(kBf16Stages, a.bn_max);
-    auto kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages>
-                                  : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages>;
+    const bool gather = a.gather_rows != nullptr;
+    auto kern = gather ? (epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, true>
+                                            : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, true>)
+                       : (epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, false>
+                                            : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, stream>>>(tmA, tmB[0], tmB[1], tmB[2], a);
+    kern<<<grid, kThreads + (gather ? kGatherThreads : 0), smem, stream>>>(tmA, tmB[0], tmB[1], tmB[2], a);
   } else {
     const size_t smem = gemm_e4m3_smem_bytes(kE4m3Stages);
     auto kern = epi == EPI_SWIGLU ? grouped_gemm_e4m3_kernel<EPI_SWIGLU, kE4m3Stages>

@@ -25,6 +25,11 @@ struct GemmArgs {
   const float* b_scale;      // E4M3: [rows, K/128]
   float* out_scale;          // E4M3 GEMM1: [rows, out_ld/128]
   int32_t* status;
+  // Gathered token rows (gate/up GEMM of the routed experts): B row p is
+  // row gather_rows[p] of gather_src [*, K] instead of row p of the B map.
+  const void* gather_src;
+  const int32_t* gather_rows;
+  int32_t gather_src_rows;   // rows of gather_src (indices outside [0, this) are flagged, not read)
 };
 
 struct RouteArgs {

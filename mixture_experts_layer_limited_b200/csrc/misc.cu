@@ -3,8 +3,6 @@
 
 namespace moe {
 
-constexpr int kCombKMax = 16;
-
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
@@ -25,7 +23,10 @@ __device__ __forceinline__ uint4 f32_to_bf16x8(const float (&f)[8]) {
 
 // Unpermute + weighted combine ("MoE 混合专家模型推理参数与前向传播详解" §3.4):
 // y[t] = shared[t] + sum_j w[t][j] * expert_out[slot_to_row[t*k+j]], fp32 sum in
-// slot order, one bf16 rounding. One warp per token, 16-byte vectors.
+// slot order, one bf16 rounding. One warp per token, two 16-byte vectors per
+// lane and step so 2k row loads are in flight. KMAX >= k bounds the rows
+// held in registers.
+template <int KMAX>
 __global__ void __launch_bounds__(256)
 combine_kernel(int T, int k, int vec_per_row, const uint4* __restrict__ eo,
                const int32_t* __restrict__ slot_to_row, const float* __restrict__ topk_w,
@@ -37,42 +38,55 @@ combine_kernel(int T, int k, int vec_per_row, const uint4* __restrict__ eo,
   int my_row = lane < k ? slot_to_row[static_cast<size_t>(t) * k + lane] : -1;
   if (my_row >= nrows) my_row = -1;
   const float my_w = (lane < k && topk_w) ? topk_w[static_cast<size_t>(t) * k + lane] : 1.0f;
-  int rows[kCombKMax];
-  float ws[kCombKMax];
+  int rows[KMAX];
+  float ws[KMAX];
 #pragma unroll
-  for (int j = 0; j < kCombKMax; ++j) {
+  for (int j = 0; j < KMAX; ++j) {
     rows[j] = __shfl_sync(0xffffffffu, my_row, j);
     ws[j] = __shfl_sync(0xffffffffu, my_w, j);
   }
-  for (int v = lane; v < vec_per_row; v += 32) {
-    float acc[8];
+  const uint4* sh = shared ? shared + static_cast<size_t>(t) * vec_per_row : nullptr;
+  uint4* yt = y + static_cast<size_t>(t) * vec_per_row;
+  for (int base = 0; base < vec_per_row; base += 64) {
+    const int v0 = base + lane, v1 = base + 32 + lane;
+    const bool ok0 = v0 < vec_per_row, ok1 = v1 < vec_per_row;
+    uint4 r0[KMAX], r1[KMAX];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    uint4 raw[kCombKMax];
-#pragma unroll
-    for (int j = 0; j < kCombKMax; ++j)
-      if (j < k && rows[j] >= 0) raw[j] = __ldg(eo + static_cast<size_t>(rows[j]) * vec_per_row + v);
-#pragma unroll
-    for (int j = 0; j < kCombKMax; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
       if (j < k && rows[j] >= 0) {
-        float f[8];
-        bf16x8_to_f32(raw[j], f);
-        if (topk_w) {
+        const uint4* src = eo + static_cast<size_t>(rows[j]) * vec_per_row;
+        if (ok0) r0[j] = __ldcs(src + v0);
+        if (ok1) r1[j] = __ldcs(src + v1);
+      }
+    }
+    float a0[8], a1[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] += ws[j] * f[i];
-        } else {
+    for (int i = 0; i < 8; ++i) { a0[i] = 0.0f; a1[i] = 0.0f; }
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] += f[i];
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < k && rows[j] >= 0) {
+        float f0[8], f1[8];
+        bf16x8_to_f32(r0[j], f0);
+        bf16x8_to_f32(r1[j], f1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          a0[i] += ws[j] * f0[i];
+          a1[i] += ws[j] * f1[i];
         }
       }
     }
-    if (shared) {
-      float f[8];
-      bf16x8_to_f32(__ldg(shared + static_cast<size_t>(t) * vec_per_row + v), f);
+    if (sh) {
+      float f0[8], f1[8];
+      if (ok0) bf16x8_to_f32(__ldg(sh + v0), f0);
+      if (ok1) bf16x8_to_f32(__ldg(sh + v1), f1);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += f[i];
+      for (int i = 0; i < 8; ++i) {
+        if (ok0) a0[i] += f0[i];
+        if (ok1) a1[i] += f1[i];
+      }
     }
-    y[static_cast<size_t>(t) * vec_per_row + v] = f32_to_bf16x8(acc);
+    if (ok0) yt[v0] = f32_to_bf16x8(a0);
+    if (ok1) yt[v1] = f32_to_bf16x8(a1);
   }
 }
 
@@ -191,9 +205,13 @@ quant_rows_kernel(const __nv_bfloat16* __restrict__ a, int M, int K, uint8_t* __
 cudaError_t launch_combine(int T, int k, int H, const void* eo, const int32_t* slot_to_row,
                            const float* topk_w, const void* shared, void* y, cudaStream_t stream) {
   const int warps = 8;
-  combine_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
-      T, k, H / 8, reinterpret_cast<const uint4*>(eo), slot_to_row, topk_w,
-      reinterpret_cast<const uint4*>(shared), reinterpret_cast<uint4*>(y));
+  const dim3 grid((T + warps - 1) / warps), block(warps * 32);
+  const uint4* e = reinterpret_cast<const uint4*>(eo);
+  const uint4* sh = reinterpret_cast<const uint4*>(shared);
+  uint4* out = reinterpret_cast<uint4*>(y);
+  if (k <= 4) combine_kernel<4><<<grid, block, 0, stream>>>(T, k, H / 8, e, slot_to_row, topk_w, sh, out);
+  else if (k <= 8) combine_kernel<8><<<grid, block, 0, stream>>>(T, k, H / 8, e, slot_to_row, topk_w, sh, out);
+  else combine_kernel<16><<<grid, block, 0, stream>>>(T, k, H / 8, e, slot_to_row, topk_w, sh, out);
   return cudaGetLastError();
 }
 

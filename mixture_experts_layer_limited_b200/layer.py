@@ -39,8 +39,12 @@ class MoELayer:
 
     def __init__(self, spec: LayerSpec, gate: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
                  sw13: Optional[torch.Tensor], sw2: Optional[torch.Tensor],
-                 bias: Optional[torch.Tensor], T_max: int):
+                 bias: Optional[torch.Tensor], T_max: int, gather: bool = False):
         self.spec = spec
+        # gather=True: bf16 layers read the routed experts' token rows straight
+        # from x (the permutation fused into the first GEMM; no x_perm). At the
+        # V3 shape on B200 the TMA path over x_perm is faster, so it is off.
+        self.gather = gather and spec.dtype != "e4m3"
         dev = gate.device
         self.dev = dev
         self.gate = gate.contiguous()
@@ -77,7 +81,7 @@ class MoELayer:
         self.row_w = z(R, dt=f32)
         ws = N.moe_permute_workspace_size(T_max, k, E)
         self.ws = z((ws + 15) // 16 * 16, dt=torch.uint8)
-        self.x_perm = z(R, H, dt=act)
+        self.x_perm = None if self.gather else z(R, H, dt=act)
         self.h = z(R, I, dt=act)
         self.o = z(R, H, dt=bf)
         self.y = z(T_max, H, dt=bf)
@@ -128,16 +132,20 @@ class MoELayer:
             src, dt, src_s = x, N.MOE_BF16, None
         R = T * s.k
         N.moe_permute(T, s.k, s.E, s.H, self.ids[:T], self.topk_w[:T], src, dt, src_s,
-                      self.x_perm[:R], self.x_perm_s[:R] if self.fp8 else None,
+                      None if self.gather else self.x_perm[:R], self.x_perm_s[:R] if self.fp8 else None,
                       self.offsets, self.src_token[:R], self.slot_to_row[:R], self.row_w[:R],
                       self.ws, self.status)
 
     def _dt(self):
         return N.MOE_E4M3 if self.fp8 else N.MOE_BF16
 
-    def experts_gate_up(self, T: int):
+    def experts_gate_up(self, T: int, x: Optional[torch.Tensor] = None):
         s = self.spec
         R = T * s.k
+        if self.gather:
+            N.moe_gate_up_swiglu_gather(R, s.H, self.w13, s.E, s.I, x, T, self.src_token[:R],
+                                        self.offsets, self.h[:R], dev_status=self.status)
+            return
         N.moe_gate_up_swiglu(R, s.H, self.w13, self._dt(), s.E, s.I, self.x_perm[:R], self.offsets,
                              self.h[:R], w13_scale=self.w13_s,
                              a_scale=self.x_perm_s[:R] if self.fp8 else None,
@@ -177,7 +185,7 @@ class MoELayer:
         if self.fp8:
             st.append(("quantize_x", lambda: self.quantize_x(x, T)))
         st += [("permute", lambda: self.permute(x, T)),
-               ("gate_up_routed", lambda: self.experts_gate_up(T)),
+               ("gate_up_routed", lambda: self.experts_gate_up(T, x)),
                ("down_routed", lambda: self.experts_down(T))]
         if self.sh_h is not None:
             st += [("gate_up_shared", lambda: self.shared_gate_up(x, T)),

@@ -28,7 +28,7 @@ MOE_SOFTMAX, MOE_SIGMOID = 0, 1
 EXPORTED = [
     "moe_route", "moe_permute_workspace_size", "moe_permute", "moe_permute_static_ws",
     "moe_grouped_swiglu",
-    "moe_gate_up_swiglu", "moe_down_proj",
+    "moe_gate_up_swiglu", "moe_gate_up_swiglu_gather", "moe_down_proj",
     "moe_combine", "moe_bias_update", "moe_quantize_blocks", "moe_quantize_rows",
     "moe_read_device_status", "moe_last_cuda_error", "moe_status_string", "moe_abi_version",
 ]
@@ -77,6 +77,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_grouped_swiglu": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P, _P, _P],
         "moe_gate_up_swiglu": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P],
         "moe_down_proj": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P],
+        "moe_gate_up_swiglu_gather": [_I, _I, ctypes.POINTER(FFNWeights), _P, _I, _P, _P, _P, _P, _P],
         "moe_combine": [_I, _I, _I, _P, _P, _P, _P, _P, _P],
         "moe_bias_update": [_I, _I, _I, _P, _P, ctypes.c_float, _P, _P],
         "moe_quantize_blocks": [_I, _I, _I, _P, _P, _P, _P],
@@ -160,6 +161,14 @@ def moe_gate_up_swiglu(rows, H, w13, dtype, groups, I, a, offsets, h_ws, w13_sca
     _check("moe_gate_up_swiglu", load_library().moe_gate_up_swiglu(
         rows, H, ctypes.byref(w), _ptr(a), _ptr(a_scale), _ptr(offsets), _ptr(h_ws),
         _ptr(h_scale_ws), _ptr(dev_status), _stream(stream)))
+
+
+def moe_gate_up_swiglu_gather(rows, H, w13, groups, I, x, T, src_token, offsets, h_ws,
+                              dev_status=None, stream=None):
+    w = FFNWeights(_ptr(w13), None, None, None, MOE_BF16, groups, I)
+    _check("moe_gate_up_swiglu_gather", load_library().moe_gate_up_swiglu_gather(
+        rows, H, ctypes.byref(w), _ptr(x), T, _ptr(src_token), _ptr(offsets), _ptr(h_ws),
+        _ptr(dev_status), _stream(stream)))
 
 
 def moe_down_proj(rows, H, w2, dtype, groups, I, h, offsets, row_w, out, w2_scale=None,

@@ -341,3 +341,47 @@ def test_bias_update_bit_exact_ten_steps():
         bias_np = oracle.bias_update(c, bias_np, gamma, T, k)
         assert np.array_equal(bias.cpu().numpy(), bias_np)
         assert abs(float(cv.item()) - oracle.load_cv(c)) <= 1e-6 * max(1.0, oracle.load_cv(c))
+
+
+# ------------------------------------------- permutation fused into GEMM 1
+def test_gate_up_gather_matches_permuted_copy_and_oracle():
+    T, k, E, H, I = 1500, 6, 16, 512, 256
+    ids_np, w_np = _ids_from_oracle(T, k, E, seed=21)
+    off_np, src_np, _ = oracle.permute(ids_np, E)
+    R = T * k
+    g = _gen(22)
+    x = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
+    w13 = (torch.randn(E, 2 * I, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    src = torch.from_numpy(src_np.astype(np.int32)).to(DEV)
+    off = torch.from_numpy(off_np.astype(np.int32)).to(DEV)
+    xp = x[src.long()].contiguous()
+    h_ref = torch.empty(R, I, dtype=torch.bfloat16, device=DEV)
+    h_gat = torch.empty(R, I, dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    N.moe_gate_up_swiglu(R, H, w13, N.MOE_BF16, E, I, xp, off, h_ref)
+    N.moe_gate_up_swiglu_gather(R, H, w13, E, I, x, T, src, off, h_gat, dev_status=status)
+    assert N.moe_read_device_status(status) == 0
+    assert torch.equal(h_gat, h_ref)             # same tiles, same data: bit-identical
+    x64, w64 = np64(x), np64(w13)
+    href = np.zeros((R, I))
+    for e in range(E):
+        s, t = off_np[e], off_np[e + 1]
+        gu = x64[src_np[s:t]] @ w64[e].T
+        href[s:t] = gu[:, :I] / (1 + np.exp(-gu[:, :I])) * gu[:, I:]
+    assert rel_err(np64(h_gat), href) < 1e-2
+
+
+def test_gate_up_gather_flags_bad_rows():
+    T, k, E, H, I = 200, 4, 16, 256, 128
+    ids_np, _ = _ids_from_oracle(T, k, E, seed=23)
+    off_np, src_np, _ = oracle.permute(ids_np, E)
+    src_np = src_np.astype(np.int32).copy()
+    src_np[7] = T + 5                             # outside x: flagged, never read
+    g = _gen(24)
+    x = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
+    w13 = (torch.randn(E, 2 * I, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    h = torch.empty(T * k, I, dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    N.moe_gate_up_swiglu_gather(T * k, H, w13, E, I, x, T, torch.from_numpy(src_np).to(DEV),
+                                torch.from_numpy(off_np.astype(np.int32)).to(DEV), h, dev_status=status)
+    assert N.moe_read_device_status(status) & N.MOE_DEVSTAT_BAD_EXPERT_ID

@@ -176,3 +176,16 @@ def test_layer_v3_skewed_bias_loop():
     err = rel_err(np64(y[toks][:, torch.as_tensor(feats, device=DEV)])[ok], yref[ok])
     print(f"v3 skewed: sampled err {err:.2e}")
     assert err < BF16_TOL
+
+
+def test_layer_gather_variant_matches_default():
+    """The permutation fused into GEMM 1 gives the same layer output."""
+    cfg = get_config("v2lite", T=1024)
+    inp = make_inputs(cfg, device=DEV)
+    y0 = _layer(cfg, inp).forward(inp.x).clone()
+    lay = MoELayer(LayerSpec.from_config(cfg), inp.gate, inp.w13, inp.w2, inp.sw13, inp.sw2,
+                   inp.bias, cfg.T, gather=True)
+    y1 = lay.forward(inp.x)
+    torch.cuda.synchronize()
+    assert lay.device_status() == 0
+    assert torch.equal(y0, y1)
