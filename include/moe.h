@@ -99,10 +99,13 @@ typedef int32_t moe_scoring;
  *                 and routing runs on those logits (no projection).
  *   gate_w        [E, H] bf16 (ignored when x == NULL).
  *   sel_bias      [E] fp32 selection-only bias, or NULL (= 0).
- *   logits        [T, E] fp32: written when x != NULL (may then be NULL to
- *                 skip writing), read when x == NULL.
+ *   logits        [T, E] fp32, required: written when x != NULL, read when
+ *                 x == NULL.
  *   topk_ids      [T, k] int32 out;  topk_w [T, k] fp32 out.
  *   expert_counts [E] int32 out.
+ * Work: with x, a tcgen05 gate GEMM on CTA pairs (each CTA of a pair sums
+ * half the hidden size; every logit is first half + second half); then one
+ * warp routes each token.
  * Limits: 1 <= k <= 16, E % 16 == 0, 16 <= E <= 256, E % n_group == 0,
  *   n_group <= 32, topk_group <= n_group, k <= topk_group * E / n_group,
  *   H % 64 == 0 when x != NULL. Otherwise MOE_ERR_INVALID_ARG/UNSUPPORTED.

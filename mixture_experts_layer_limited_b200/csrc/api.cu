@@ -128,7 +128,7 @@ const char* moe_status_string(moe_status s) {
 
 moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_w, const float* sel_bias,
                      float* logits, int32_t* topk_ids, float* topk_w, int32_t* expert_counts, void* stream) {
-  if (!p || !topk_ids || !topk_w || !expert_counts) return MOE_ERR_INVALID_ARG;
+  if (!p || !topk_ids || !topk_w || !expert_counts || !logits) return MOE_ERR_INVALID_ARG;
   if (p->T < 1 || p->k < 1 || p->n_group < 1 || p->topk_group < 1) return MOE_ERR_INVALID_ARG;
   if (p->scoring != MOE_SOFTMAX && p->scoring != MOE_SIGMOID) return MOE_ERR_INVALID_ARG;
   if (p->E < 1 || p->E % p->n_group != 0 || p->topk_group > p->n_group) return MOE_ERR_INVALID_ARG;
@@ -137,10 +137,11 @@ moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_
   if (x) {
     if (!gate_w || p->H < 64) return MOE_ERR_INVALID_ARG;
     if (p->H % 64 != 0) return MOE_ERR_UNSUPPORTED;
-  } else if (!logits) {
-    return MOE_ERR_INVALID_ARG;
   }
   if (any_misaligned(x, gate_w, sel_bias, logits, topk_ids, topk_w, expert_counts)) return MOE_ERR_ALIGNMENT;
+  int nsm = 0;
+  moe_status s = sm_count(&nsm);
+  if (s != MOE_OK) return s;
   cudaStream_t st = as_stream(stream);
   RouteArgs r{p->T, p->H, p->E, p->k, p->n_group, p->topk_group, p->scoring, p->norm_topk_prob ? 1 : 0,
               p->routed_scaling_factor, sel_bias, logits, topk_ids, topk_w, expert_counts, p->dev_status};
@@ -148,13 +149,14 @@ moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_
   if (e != cudaSuccess) return cuda_fail(e);
   if (x) {
     CUtensorMap tmX, tmG;
-    moe_status s = make_tmap(&tmX, x, false, p->H, p->T, 128);
+    s = make_tmap(&tmX, x, false, p->H, p->T, 128);
     if (s != MOE_OK) return s;
     s = make_tmap(&tmG, gate_w, false, p->H, p->E, static_cast<uint32_t>(p->E));
     if (s != MOE_OK) return s;
-    return check_launch(launch_route_gemm(tmX, tmG, r, st));
+    s = check_launch(launch_gate_gemm(tmX, tmG, r, st));
+    if (s != MOE_OK) return s;
   }
-  return check_launch(launch_route_logits(r, st));
+  return check_launch(launch_route_tokens(r, nsm, st));
 }
 
 moe_status moe_permute_workspace_size(int32_t T, int32_t k, int32_t E, size_t* bytes) {

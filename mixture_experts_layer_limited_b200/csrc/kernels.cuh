@@ -50,9 +50,9 @@ enum { EPI_SWIGLU = 0, EPI_WEIGHTED = 1 };
 // 32-row map (e4m3).
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap* tmB,
                                 const GemmArgs& a, int grid, cudaStream_t stream);
-cudaError_t launch_route_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
-                              cudaStream_t stream);
-cudaError_t launch_route_logits(const RouteArgs& r, cudaStream_t stream);
+cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
+                             cudaStream_t stream);
+cudaError_t launch_route_tokens(const RouteArgs& r, int num_sms, cudaStream_t stream);
 size_t permute_workspace_bytes(int T, int E);
 cudaError_t launch_permute(int T, int k, int E, int row_bytes, const int32_t* ids, const float* topk_w,
                            const void* x, const float* x_scale, int nscale, void* x_perm,

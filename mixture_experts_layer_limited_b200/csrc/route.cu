@@ -7,158 +7,56 @@
 // top-2, topk_group = 4 kept, top-8 within, renormalise, x routed_scaling_factor);
 // the xxqk.cn digest §2.2 (bias only steers selection; device-limited routing).
 //
-// Kernel 1 (route_gemm_kernel): one CTA per 128 tokens. The gate GEMM runs on
-// tcgen05 (M = 128 tokens, N = E experts, K = H) with TMA-fed operands and an
-// fp32 accumulator of 128 x E in TMEM. Each of the 128 epilogue threads owns
-// one TMEM lane = one token and routes it alone: the E logits are pulled out of
-// TMEM 32 at a time, scored into a per-thread shared-memory column (reusing the
-// operand ring), and the group scores / top-k are kept in registers. No
-// cross-thread communication is needed except the per-CTA expert histogram.
-// Kernel 2 (route_logits_kernel): same routing from fp32 logits in memory.
+// Two kernels:
+//   gate_gemm_pair_kernel  logits = x . gate^T on tcgen05. A cluster of two
+//       CTAs takes 128 tokens: CTA r accumulates over half r of the hidden
+//       size in its own TMEM (M = 128 tokens, N = E, fp32), then the two swap,
+//       through distributed shared memory, the partial sums of the 64 tokens
+//       the other one writes out. Every logit is (first half) + (second half).
+//   route_tokens_kernel  one warp per token: lane l scores experts l, l+32, ...,
+//       groups are scored by the sum of their two best selection scores and
+//       ranked with shuffles, and the top-k is k rounds of a warp arg-max
+//       (larger score first, lower expert index on ties).
 #include "kernels.cuh"
 
 namespace moe {
 
-constexpr int kRouteKMax = 16;
-constexpr int kRouteRows = 128;     // tokens per CTA = scratch column count
-constexpr int kRouteMaxGroups = 32;
-
-
+constexpr int kRouteRows = 128;      // tokens per gate-GEMM tile
+constexpr int kRouteStages = 4;
+constexpr int kEpl = 8;              // experts per lane (E <= 256)
+constexpr int kRouteWarps = 8;       // tokens in flight per routing CTA
 
 // Score -> fp32 as the library states it: sigmoid in double, rounded once.
 __device__ __forceinline__ float sigmoid_rn(float v) {
   return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(v))));
 }
 
-// Routes the token whose scratch column is `col` (expert e at col[e * 128];
-// holds fp32 sigmoid for sigmoid scoring, the raw logit for softmax).
-__device__ void route_token(const float* col, float* gcol, const float* bias_s, float lmax,
-                            double sumexp, const RouteArgs& c, int32_t* ids_out, float* w_out,
-                            int* hist) {
-  const bool sig = c.scoring == MOE_SIGMOID;
-  const bool raw_logit = !sig && c.G == 1 && bias_s == nullptr;
-  auto sel = [&](int e) -> float {
-    const float v = col[e * kRouteRows];
-    if (sig) return bias_s ? v + bias_s[e] : v;
-    if (raw_logit) return v;
-    const float p = static_cast<float>(exp(static_cast<double>(v) - static_cast<double>(lmax)) / sumexp);
-    return bias_s ? p + bias_s[e] : p;
-  };
-  const int gsz = c.E / c.G;
-  uint32_t kept = 0xffffffffu;
-  if (c.G > 1) {
-    for (int gi = 0; gi < c.G; ++gi) {
-      float m1 = -INFINITY, m2 = -INFINITY;
-      for (int e = gi * gsz; e < (gi + 1) * gsz; ++e) {
-        const float v = sel(e);
-        if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
-      }
-      gcol[gi * kRouteRows] = gsz >= 2 ? m1 + m2 : m1;
-    }
-    kept = 0;
-    for (int r = 0; r < c.g; ++r) {
-      float best = -INFINITY;
-      int bi = -1;
-      for (int gi = 0; gi < c.G; ++gi) {
-        if ((kept >> gi) & 1u) continue;
-        const float v = gcol[gi * kRouteRows];
-        if (bi < 0 || v > best) { best = v; bi = gi; }
-      }
-      kept |= 1u << bi;
-    }
-  }
-  float tv[kRouteKMax];
-  int ti[kRouteKMax];
-#pragma unroll
-  for (int s = 0; s < kRouteKMax; ++s) { tv[s] = -INFINITY; ti[s] = 0; }
-  for (int gi = 0; gi < c.G; ++gi) {
-    if (!((kept >> gi) & 1u)) continue;
-    for (int e = gi * gsz; e < (gi + 1) * gsz; ++e) {
-      const float v = sel(e);
-      // insert keeping (value desc, index asc); equal values never displace
-#pragma unroll
-      for (int s = kRouteKMax - 1; s >= 0; --s) {
-        if (s < c.k && v > tv[s]) {
-          if (s > 0 && v > tv[s > 0 ? s - 1 : 0]) {
-            tv[s] = tv[s > 0 ? s - 1 : 0];
-            ti[s] = ti[s > 0 ? s - 1 : 0];
-          } else {
-            tv[s] = v;
-            ti[s] = e;
-          }
-        }
-      }
-    }
-  }
-  float w[kRouteKMax];
-  float sum = 0.0f;
-#pragma unroll
-  for (int s = 0; s < kRouteKMax; ++s) {
-    if (s < c.k) {
-      const float v = col[ti[s] * kRouteRows];
-      w[s] = sig ? v : static_cast<float>(exp(static_cast<double>(v) - static_cast<double>(lmax)) / sumexp);
-      sum += w[s];
-    }
-  }
-#pragma unroll
-  for (int s = 0; s < kRouteKMax; ++s) {
-    if (s < c.k) {
-      float ws = c.norm ? w[s] / sum : w[s];
-      ids_out[s] = ti[s];
-      w_out[s] = ws * c.scale;
-      atomicAdd(&hist[ti[s]], 1);
-    }
-  }
-}
-
-// Per-token scoring pass over an E-wide logit row delivered 32 at a time.
-struct ScorePass {
-  float lmax = -INFINITY;
-  __device__ __forceinline__ void chunk(float* col, const float (&v)[32], int e0, int E, bool sig) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (e0 + j < E) {
-        col[(e0 + j) * kRouteRows] = sig ? sigmoid_rn(v[j]) : v[j];
-        lmax = fmaxf(lmax, v[j]);
-      }
-    }
-  }
-};
-
-__device__ __forceinline__ double softmax_denominator(const float* col, int E, float lmax) {
-  double s = 0.0;
-  for (int e = 0; e < E; ++e) s += exp(static_cast<double>(col[e * kRouteRows]) - static_cast<double>(lmax));
-  return s;
-}
-
-size_t route_scratch_bytes(int E) {
-  return static_cast<size_t>(kRouteRows) * (E + kRouteMaxGroups) * sizeof(float);
-}
-
 // ------------------------------------------------------------------------
-// Kernel 1: fused tcgen05 gate GEMM + routing.
+// Gate GEMM on CTA pairs, split along K.
 // ------------------------------------------------------------------------
-constexpr int kRouteStages = 4;
-
-__global__ void __launch_bounds__(192, 1)
-route_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
-                  const RouteArgs r, uint32_t tmem_cols) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+gate_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
+                      const RouteArgs r, uint32_t tmem_cols) {
   constexpr int KB = 64;
   extern __shared__ __align__(1024) uint8_t dsmem[];
   __shared__ uint64_t full_bar[kRouteStages], empty_bar[kRouteStages];
-  __shared__ uint64_t tmem_full, drain_bar, epi_bar;
+  __shared__ uint64_t tmem_full, drain_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ int issued_parity[kRouteStages];
   __shared__ volatile int abort_flag;
-  __shared__ int hist[256];
-  __shared__ float bias_s[256];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   const uint32_t a_bytes = 128u * 128u;
   const uint32_t b_bytes = static_cast<uint32_t>(r.E) * 128u;
   const uint32_t stage_bytes = a_bytes + b_bytes;
-  const int m0 = blockIdx.x * kRouteRows;
+  const int m0 = static_cast<int>(cluster_id_x()) * kRouteRows;
+  const int nk = r.H / KB;
+  const int nk0 = (nk + 1) / 2;
+  const int kb_begin = rank ? nk0 : 0;
+  const int kb_count = rank ? nk - nk0 : nk0;
+  float* recv = reinterpret_cast<float*>(smem);        // peer partials, after the main loop
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kRouteStages; ++i) {
@@ -168,13 +66,8 @@ route_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     }
     mbar_init(&tmem_full, 1);
     mbar_init(&drain_bar, 1);
-    mbar_init(&epi_bar, 128);
     abort_flag = 0;
     fence_barrier_init();
-  }
-  for (int e = threadIdx.x; e < r.E; e += blockDim.x) {
-    hist[e] = 0;
-    bias_s[e] = r.bias ? r.bias[e] : 0.0f;
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmX);
@@ -188,7 +81,6 @@ route_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
-  const int nk = r.H / KB;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -196,7 +88,8 @@ route_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
       const uint64_t pol_g = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
-      for (int kb = 0; kb < nk; ++kb) {
+      for (int i = 0; i < kb_count; ++i) {
+        const int kb = kb_begin + i;
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, r.status)) break;
         mbar_arrive_expect_tx(&full_bar[stage], stage_bytes);
         uint8_t* st = smem + stage * stage_bytes;
@@ -216,59 +109,79 @@ route_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int kb = 0; kb < nk; ++kb) {
+      for (int i = 0; i < kb_count; ++i) {
         if (!mbar_wait(&full_bar[stage], phase, &abort_flag, r.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a0 = smem_u32(smem + stage * stage_bytes);
         const uint32_t b0 = a0 + a_bytes;
 #pragma unroll
         for (int kk = 0; kk < KB / 16; ++kk)
-          umma_bf16(tmem_base, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (kb | kk) != 0);
+          umma_bf16(tmem_base, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (i | kk) != 0);
         umma_commit(&empty_bar[stage]);
         if (++stage == kRouteStages) { stage = 0; phase ^= 1u; }
       }
-      if (ok) umma_commit(&tmem_full);
+      if (ok && kb_count > 0) umma_commit(&tmem_full);
       umma_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0);
     }
-  } else {
-    const int q = warp & 3;
-    const int row = 32 * q + lane;           // TMEM lane == token row in tile
-    const int tok = m0 + row;
-    bool ok = mbar_wait(&tmem_full, 0, &abort_flag, r.status);
-    if (ok) {
-      tc_fence_after();
-      float* scratch = reinterpret_cast<float*>(smem);   // operand ring is idle now
-      float* col = scratch + row;
-      float* gcol = scratch + static_cast<size_t>(kRouteRows) * r.E + row;
-      const bool sig = r.scoring == MOE_SIGMOID;
-      ScorePass sp;
-      const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-      for (int c = 0; c * 32 < r.E; ++c) {
-        float v[32];
-        tmem_ld32(lane_addr + c * 32, v);
-        tmem_ld_wait();
-        if (tok < r.T) {
-          if (r.logits) {
-            float4* dst = reinterpret_cast<float4*>(r.logits + static_cast<size_t>(tok) * r.E + c * 32);
+  } else if (kb_count > 0) {
+    mbar_wait(&tmem_full, 0, &abort_flag, r.status);   // an abort still reaches the cluster barriers
+    tc_fence_after();
+  }
+  // both CTAs: every MMA has completed (epilogue threads arrive only after
+  // tmem_full), so the operand rings are free for the exchange
+  cluster_sync();
+
+  const int q = warp & 3;
+  const int row = 32 * q + lane;                       // TMEM lane == token row of the tile
+  const bool epi = warp >= 2;
+  const bool mine = (row >> 6) == static_cast<int>(rank);   // CTA r writes rows [64r, 64r + 64)
+  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+  auto partial = [&](int c, float (&v)[32]) {
+    if (kb_count > 0) {
+      tmem_ld32(lane_addr + c * 32, v);
+      tmem_ld_wait();
+    } else {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (c * 32 + 4 * j < r.E) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-          }
-          sp.chunk(col, v, c * 32, r.E, sig);
-        }
+      for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+    }
+  };
+  if (epi && !mine) {                                  // send to the CTA that writes this token
+    const uint32_t dst = mapa_shared(smem_u32(recv), rank ^ 1u) + static_cast<uint32_t>((row & 63) * r.E) * 4u;
+    for (int c = 0; c * 32 < r.E; ++c) {
+      float v[32];
+      partial(c, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (c * 32 + 4 * j < r.E)
+          asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (c * 32 + 4 * j) * 4u),
+                       "f"(v[4 * j]), "f"(v[4 * j + 1]), "f"(v[4 * j + 2]), "f"(v[4 * j + 3])
+                       : "memory");
       }
-      tc_fence_before();
+    }
+  }
+  cluster_sync();                                      // the peer's partials have landed
+
+  if (epi && mine) {
+    const int tok = m0 + row;
+    const float* peer = recv + static_cast<size_t>(row & 63) * r.E;
+    for (int c = 0; c * 32 < r.E; ++c) {
+      float v[32];
+      partial(c, v);
       if (tok < r.T) {
-        const double den = sig ? 1.0 : softmax_denominator(col, r.E, sp.lmax);
-        route_token(col, gcol, r.bias ? bias_s : nullptr, sp.lmax, den, r,
-                    r.ids + static_cast<size_t>(tok) * r.k, r.w + static_cast<size_t>(tok) * r.k, hist);
-      }
-      // bounded sync of the 128 epilogue threads, then flush the histogram
-      mbar_arrive(&epi_bar);
-      if (mbar_wait(&epi_bar, 0, &abort_flag, r.status)) {
-        for (int e = row; e < r.E; e += kRouteRows)
-          if (hist[e]) atomicAdd(r.counts + e, hist[e]);
+        float4* dst = reinterpret_cast<float4*>(r.logits + static_cast<size_t>(tok) * r.E + c * 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (c * 32 + 4 * j < r.E) {
+            float o[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float p = peer[c * 32 + 4 * j + u];
+              o[u] = rank ? p + v[4 * j + u] : v[4 * j + u] + p;      // first half + second half
+            }
+            dst[j] = make_float4(o[0], o[1], o[2], o[3]);
+          }
+        }
       }
     }
   }
@@ -280,67 +193,155 @@ route_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 }
 
 // ------------------------------------------------------------------------
-// Kernel 2: routing from fp32 logits already in memory.
+// Routing, one warp per token.
 // ------------------------------------------------------------------------
-__global__ void __launch_bounds__(kRouteRows)
-route_logits_kernel(const RouteArgs r) {
-  extern __shared__ __align__(16) float scratch_dyn[];
+// (ov, oe) beats (v, e): larger score, or equal score and lower expert index.
+__device__ __forceinline__ bool beats(float v, int e, float ov, int oe) {
+  return ov > v || (ov == v && oe < e);
+}
+
+__global__ void __launch_bounds__(kRouteWarps * 32)
+route_tokens_kernel(const RouteArgs r) {
   __shared__ int hist[256];
   __shared__ float bias_s[256];
-  const int row = threadIdx.x;
-  const int tok = blockIdx.x * kRouteRows + row;
-  for (int e = row; e < r.E; e += kRouteRows) {
+  __shared__ float sel_s[kRouteWarps][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < r.E; e += blockDim.x) {
     hist[e] = 0;
     bias_s[e] = r.bias ? r.bias[e] : 0.0f;
   }
   __syncthreads();
-  float* col = scratch_dyn + row;
-  float* gcol = scratch_dyn + static_cast<size_t>(kRouteRows) * r.E + row;
   const bool sig = r.scoring == MOE_SIGMOID;
-  if (tok < r.T) {
-    ScorePass sp;
-    const float4* src = reinterpret_cast<const float4*>(r.logits + static_cast<size_t>(tok) * r.E);
-    for (int c = 0; c * 32 < r.E; ++c) {
-      float v[32];
+  const bool has_bias = r.bias != nullptr;
+  const bool raw_logit = !sig && r.G == 1 && !has_bias;     // softmax, one group: select on logits
+  const int gsz = r.E / r.G;
+  float* my_sel = sel_s[warp];
+
+  for (int tok = blockIdx.x * kRouteWarps + warp; tok < r.T; tok += gridDim.x * kRouteWarps) {
+    const float* L = r.logits + static_cast<size_t>(tok) * r.E;
+    float lg[kEpl], sel[kEpl], unb[kEpl];
+    float lmax = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float4 f = (c * 32 + 4 * j < r.E) ? src[c * 8 + j] : make_float4(0.f, 0.f, 0.f, 0.f);
-        v[4 * j] = f.x; v[4 * j + 1] = f.y; v[4 * j + 2] = f.z; v[4 * j + 3] = f.w;
-      }
-      sp.chunk(col, v, c * 32, r.E, sig);
+    for (int i = 0; i < kEpl; ++i) {
+      const int e = lane + 32 * i;
+      lg[i] = e < r.E ? L[e] : -INFINITY;
+      lmax = fmaxf(lmax, lg[i]);
     }
-    const double den = sig ? 1.0 : softmax_denominator(col, r.E, sp.lmax);
-    route_token(col, gcol, r.bias ? bias_s : nullptr, sp.lmax, den, r,
-                r.ids + static_cast<size_t>(tok) * r.k, r.w + static_cast<size_t>(tok) * r.k, hist);
+    double den = 1.0;
+    if (!sig) {
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, d));
+      double sum = 0.0;
+#pragma unroll
+      for (int i = 0; i < kEpl; ++i)
+        if (lane + 32 * i < r.E) sum += exp(static_cast<double>(lg[i]) - static_cast<double>(lmax));
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
+      den = sum;
+    }
+#pragma unroll
+    for (int i = 0; i < kEpl; ++i) {
+      const int e = lane + 32 * i;
+      if (e < r.E) {
+        const float u = sig ? sigmoid_rn(lg[i])
+                            : static_cast<float>(exp(static_cast<double>(lg[i]) - static_cast<double>(lmax)) / den);
+        unb[i] = u;
+        sel[i] = raw_logit ? lg[i] : (has_bias ? u + bias_s[e] : u);
+      } else {
+        unb[i] = 0.0f;
+        sel[i] = -INFINITY;
+      }
+    }
+    if (r.G > 1) {
+      // group score = fp32 sum of the group's two largest selection scores
+#pragma unroll
+      for (int i = 0; i < kEpl; ++i)
+        if (lane + 32 * i < r.E) my_sel[lane + 32 * i] = sel[i];
+      __syncwarp();
+      float gs = -INFINITY;
+      if (lane < r.G) {
+        float m1 = -INFINITY, m2 = -INFINITY;
+        for (int e = lane * gsz; e < (lane + 1) * gsz; ++e) {
+          const float v = my_sel[e];
+          if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
+        }
+        gs = gsz >= 2 ? m1 + m2 : m1;
+      }
+      __syncwarp();
+      // keep the topk_group best groups (lower group index first on ties)
+      int rank_g = 0;
+      for (int j = 0; j < r.G; ++j) {
+        const float o = __shfl_sync(0xffffffffu, gs, j);
+        rank_g += (o > gs || (o == gs && j < lane)) ? 1 : 0;
+      }
+      const uint32_t kept = __ballot_sync(0xffffffffu, lane < r.G && rank_g < r.g);
+#pragma unroll
+      for (int i = 0; i < kEpl; ++i) {
+        const int e = lane + 32 * i;
+        if (e < r.E && !((kept >> (e / gsz)) & 1u)) sel[i] = -INFINITY;
+      }
+    }
+    // top-k: k rounds of a warp arg-max
+    uint32_t taken = 0;
+    int my_id = 0;
+    float my_w = 0.0f;
+    for (int j = 0; j < r.k; ++j) {
+      float v = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < kEpl; ++i) {
+        const int e = lane + 32 * i;
+        if (e < r.E && !((taken >> i) & 1u) && beats(v, be, sel[i], e)) { v = sel[i]; be = e; }
+      }
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, v, d);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, d);
+        if (beats(v, be, ov, oe)) { v = ov; be = oe; }
+      }
+      const int owner = be & 31, slot = be >> 5;
+      float u = 0.0f;
+#pragma unroll
+      for (int i = 0; i < kEpl; ++i)
+        if (i == slot) u = unb[i];
+      u = __shfl_sync(0xffffffffu, u, owner);
+      if (lane == owner) taken |= 1u << slot;
+      if (lane == j) { my_id = be; my_w = u; }
+    }
+    float sum = 0.0f;
+    for (int j = 0; j < r.k; ++j) sum += __shfl_sync(0xffffffffu, my_w, j);
+    if (lane < r.k) {
+      const float w = (r.norm ? my_w / sum : my_w) * r.scale;
+      r.ids[static_cast<size_t>(tok) * r.k + lane] = my_id;
+      r.w[static_cast<size_t>(tok) * r.k + lane] = w;
+      atomicAdd(&hist[my_id], 1);
+    }
   }
   __syncthreads();
-  for (int e = row; e < r.E; e += kRouteRows)
+  for (int e = threadIdx.x; e < r.E; e += blockDim.x)
     if (hist[e]) atomicAdd(r.counts + e, hist[e]);
 }
 
 // ------------------------------------------------------------------------
-cudaError_t launch_route_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
-                              cudaStream_t stream) {
+cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
+                             cudaStream_t stream) {
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(r.E)) cols <<= 1;
   const size_t ring = static_cast<size_t>(kRouteStages) * (128 * 128 + static_cast<size_t>(r.E) * 128);
-  const size_t scratch = route_scratch_bytes(r.E);
-  const size_t smem = (ring > scratch ? ring : scratch) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(route_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t recv = static_cast<size_t>(64) * r.E * sizeof(float);
+  const size_t smem = (ring > recv ? ring : recv) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(gate_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int grid = (r.T + kRouteRows - 1) / kRouteRows;
-  route_gemm_kernel<<<grid, 192, smem, stream>>>(tmX, tmG, r, cols);
+  const int tiles = (r.T + kRouteRows - 1) / kRouteRows;
+  gate_gemm_pair_kernel<<<2 * tiles, 192, smem, stream>>>(tmX, tmG, r, cols);
   return cudaGetLastError();
 }
 
-cudaError_t launch_route_logits(const RouteArgs& r, cudaStream_t stream) {
-  const size_t smem = route_scratch_bytes(r.E);
-  cudaError_t e = cudaFuncSetAttribute(route_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  const int grid = (r.T + kRouteRows - 1) / kRouteRows;
-  route_logits_kernel<<<grid, kRouteRows, smem, stream>>>(r);
+cudaError_t launch_route_tokens(const RouteArgs& r, int num_sms, cudaStream_t stream) {
+  const int need = (r.T + kRouteWarps - 1) / kRouteWarps;
+  const int grid = need < 8 * num_sms ? need : 8 * num_sms;
+  route_tokens_kernel<<<grid, kRouteWarps * 32, 0, stream>>>(r);
   return cudaGetLastError();
 }
 

@@ -117,7 +117,7 @@ class MoELayer:
                     s.norm_topk_prob, s.scale,
                     None if logits_in is not None else x,
                     self.gate, self.bias,
-                    logits_in if logits_in is not None else (self.logits[:T] if write_logits else None),
+                    logits_in if logits_in is not None else self.logits[:T],
                     self.ids[:T], self.topk_w[:T], self.counts, self.status)
 
     def quantize_x(self, x: torch.Tensor, T: int):

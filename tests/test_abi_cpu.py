@@ -60,14 +60,17 @@ def test_host_validation_rejects_before_launch():
     # moe_route: no params / k > E / unsupported E / misaligned pointer
     assert lib.moe_route(None, fake, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_INVALID_ARG
     p = N.RouteParams(16, 256, 16, 17, 1, 1, N.MOE_SOFTMAX, 0, 1.0, None)
-    assert lib.moe_route(ctypes.byref(p), fake, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(ctypes.byref(p), fake, fake, None, fake, fake, fake, fake, None) == N.MOE_ERR_INVALID_ARG
     p = N.RouteParams(16, 256, 24, 4, 1, 1, N.MOE_SOFTMAX, 0, 1.0, None)
-    assert lib.moe_route(ctypes.byref(p), fake, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_UNSUPPORTED
+    assert lib.moe_route(ctypes.byref(p), fake, fake, None, fake, fake, fake, fake, None) == N.MOE_ERR_UNSUPPORTED
     p = N.RouteParams(16, 256, 256, 8, 8, 4, N.MOE_SIGMOID, 1, 2.5, None)
-    assert lib.moe_route(ctypes.byref(p), odd, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_ALIGNMENT
+    assert lib.moe_route(ctypes.byref(p), odd, fake, None, fake, fake, fake, fake, None) == N.MOE_ERR_ALIGNMENT
+    # logits are required (the gate GEMM writes them, routing reads them)
+    p = N.RouteParams(16, 256, 16, 4, 1, 1, N.MOE_SOFTMAX, 0, 1.0, None)
+    assert lib.moe_route(ctypes.byref(p), fake, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_INVALID_ARG
     # group limit makes k impossible: 4 groups of 4, keep 1 -> at most 4 candidates
     p = N.RouteParams(16, 256, 16, 5, 4, 1, N.MOE_SIGMOID, 1, 2.5, None)
-    assert lib.moe_route(ctypes.byref(p), fake, fake, None, None, fake, fake, fake, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(ctypes.byref(p), fake, fake, None, fake, fake, fake, fake, None) == N.MOE_ERR_INVALID_ARG
     # moe_permute: missing workspace, too small workspace, unsupported E
     args = [fake, fake, fake, N.MOE_BF16, None, fake, None, fake, fake, fake, fake]
     assert lib.moe_permute(64, 4, 16, 256, *args, None, 0, None, None) == N.MOE_ERR_INVALID_ARG

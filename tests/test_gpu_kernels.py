@@ -88,7 +88,7 @@ def test_route_from_logits_bit_exact(name, T):
 
 
 @pytest.mark.parametrize("name,T", [("tiny", None), ("tiny_grouped", None), ("v2lite", None),
-                                    ("v3", None), ("v3", 1000)])
+                                    ("v3", None), ("v3", 1000), ("v3", 1), ("v2lite", 129)])
 def test_route_gate_gemm(name, T):
     cfg = _cfg(name)
     T = T or cfg.T
@@ -97,7 +97,9 @@ def test_route_gate_gemm(name, T):
     ids, w, counts, L = gpu_route(cfg, T, x=inp.x, gate=inp.gate, bias=bias)
     torch.cuda.synchronize()
     L64 = oracle.gate_logits(np64(inp.x), np64(inp.gate))
-    assert rel_err(np64(L), L64) < 1e-5
+    # fp32 accumulation of H bf16 products on the tensor cores: ~sqrt(H) * 2^-24 of
+    # the partial sums; a layout or index mistake is O(1)
+    assert rel_err(np64(L), L64) < 3e-5
     r = oracle_route(L64.astype(np.float32), cfg, np32(bias) if bias is not None else None)
     flagged = near_tie_mask(r)
     ids_g = ids.cpu().numpy()
