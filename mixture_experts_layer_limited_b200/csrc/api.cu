@@ -97,12 +97,25 @@ cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 // CTA pairs (tcgen05 cta_group::2, epilogue overlapped with the next tile).
 // MOE_GEMM_1SM=1 puts both on single CTAs, MOE_GEMM_PAIR=1 both on pairs
 // (same results; for comparison). Read at each call.
-bool bf16_on_pairs(bool gate_up) {
-  const char* one = std::getenv("MOE_GEMM_1SM");
-  if (one && one[0] == '1') return false;
-  const char* pr = std::getenv("MOE_GEMM_PAIR");
-  if (pr && pr[0] == '1') return true;
-  return !gate_up;
+bool env_on(const char* name) {
+  const char* v = std::getenv(name);
+  return v && v[0] == '1';
+}
+// Kernel choice per bf16 GEMM (measured at the V3 shape on B200): both run on
+// single CTAs. Gate/up keeps 256-token tiles with one TMEM accumulator (the
+// 128-token tiles two accumulators need halve the reuse of each weight tile);
+// the down projection, whose epilogue stores twice the features, uses two
+// accumulators so the epilogue of one tile overlaps the MMAs of the next.
+// MOE_GEMM_PAIR=1 / MOE_GEMM_1SM=1 force CTA pairs / single CTAs for both;
+// MOE_GEMM_DB=1 / MOE_GEMM_SB=1 force two / one accumulators on single CTAs.
+bool bf16_on_pairs() {
+  if (env_on("MOE_GEMM_1SM")) return false;
+  return env_on("MOE_GEMM_PAIR");
+}
+int one_cta_buffers(bool gate_up) {
+  if (env_on("MOE_GEMM_DB")) return 2;
+  if (env_on("MOE_GEMM_SB")) return 1;
+  return gate_up ? 1 : 2;
 }
 
 }  // namespace
@@ -224,15 +237,16 @@ moe_status run_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const 
                        const float* a_scale, const int32_t* offsets, void* h_ws, float* h_scale_ws,
                        int32_t* dev_status, cudaStream_t st, int nsm) {
   const bool fp8 = w->dtype == MOE_E4M3;
-  const bool pair = !fp8 && bf16_on_pairs(true);
+  const bool pair = !fp8 && bf16_on_pairs();
   const int I = w->I;
   CUtensorMap tmA, tmB[3];
   moe_status s = make_tmap(&tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, pair ? 64 : 128);
   if (s != MOE_OK) return s;
   s = make_token_tmaps(tmB, a, fp8, H, rows);
   if (s != MOE_OK) return s;
-  GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : 256, pair ? 64 : 0,
-              h_ws, I, nullptr, w->w13_scale, a_scale, h_scale_ws, dev_status};
+  const int nb = (fp8 || pair) ? 1 : one_cta_buffers(true);
+  GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : (nb == 2 ? 128 : 256),
+              pair ? 64 : 0, nb, 0, h_ws, I, nullptr, w->w13_scale, a_scale, h_scale_ws, dev_status};
   return check_launch(launch_grouped_gemm(fp8, EPI_SWIGLU, tmA, tmB, g1, nsm, st));
 }
 
@@ -240,15 +254,17 @@ moe_status run_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const voi
                     const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status,
                     cudaStream_t st, int nsm) {
   const bool fp8 = w->dtype == MOE_E4M3;
-  const bool pair = !fp8 && bf16_on_pairs(false);
+  const bool pair = !fp8 && bf16_on_pairs();
   const int I = w->I;
   CUtensorMap tmA, tmB[3];
-  moe_status s = make_tmap(&tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H, pair ? 64 : 128);
+  moe_status s = make_tmap(&tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H, 128);
   if (s != MOE_OK) return s;
   s = make_token_tmaps(tmB, h, fp8, I, rows);
   if (s != MOE_OK) return s;
-  GemmArgs g2{rows, I, w->groups, offsets, H, H / 256, 256, pair ? 64 : 128, 256, 128, fp8 ? 32 : 256,
-              pair ? 128 : 0, out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
+  const int nb = (fp8 || pair) ? 1 : one_cta_buffers(false);
+  GemmArgs g2{rows, I, w->groups, offsets, H, H / 256, 256, pair ? 64 : 128, 256, 128,
+              fp8 ? 32 : (nb == 2 ? 128 : 256), pair ? 128 : 0, nb, pair ? 1 : 0,
+              out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
   return check_launch(launch_grouped_gemm(fp8, EPI_WEIGHTED, tmA, tmB, g2, nsm, st));
 }
 
@@ -285,7 +301,7 @@ moe_status moe_gate_up_swiglu_gather(int32_t rows, int32_t H, const moe_ffn_weig
   if (s != MOE_OK) return s;
   s = make_token_tmaps(tmB, x, false, H, T);      // not read: token rows are gathered
   if (s != MOE_OK) return s;
-  GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, 256, 0,
+  GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, 256, 0, 1, 0,
               h_ws, I, nullptr, nullptr, nullptr, nullptr, dev_status, x, src_token, T};
   return check_launch(launch_grouped_gemm(false, EPI_SWIGLU, tmA, tmB, g1, nsm, as_stream(stream)));
 }

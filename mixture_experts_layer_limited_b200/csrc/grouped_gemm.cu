@@ -180,7 +180,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   __shared__ Sched sched;
   __shared__ __align__(16) __nv_bfloat16 stage_out[4][32 * 32];
   __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
-  __shared__ uint64_t tmem_full, tmem_empty, drain_bar;
+  __shared__ uint64_t tmem_full[2], tmem_empty[2], drain_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ int issued_parity[STAGES];
   __shared__ volatile int abort_flag;
@@ -188,6 +188,10 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   const uint32_t b_stage_bytes = static_cast<uint32_t>(a.bn_max) * 128u;
+  // TMEM: nbuf accumulators of two sub-tiles; sub-tile s of buffer b starts at
+  // column b * 2 * sub_cols + s * sub_cols
+  const int nbuf = a.nbuf == 2 ? 2 : 1;
+  const uint32_t sub_cols = nbuf == 2 ? 128u : 256u;
   const uint32_t stage_bytes = 2 * A_SUB_BYTES + b_stage_bytes;
   auto sA = [&](int st, int sub) { return smem + st * stage_bytes + sub * A_SUB_BYTES; };
   auto sB = [&](int st) { return smem + st * stage_bytes + 2 * A_SUB_BYTES; };
@@ -198,8 +202,10 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       mbar_init(&empty_bar[i], 1);
       issued_parity[i] = -1;
     }
-    mbar_init(&tmem_full, 1);
-    mbar_init(&tmem_empty, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tmem_full[b], 1);
+      mbar_init(&tmem_empty[b], 128);
+    }
     mbar_init(&drain_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
@@ -304,11 +310,13 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   } else if (warp == 1) {
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      for (int t = blockIdx.x; t < total && !abort_flag; t += gridDim.x) {
+      uint32_t phase = 0, it = 0;
+      for (int t = blockIdx.x; t < total && !abort_flag; t += gridDim.x, ++it) {
         const TileInfo ti = decode_tile(sched, a, t);
         const uint32_t idesc = make_idesc(1u, 128u, static_cast<uint32_t>(ti.N));
-        if (!mbar_wait(&tmem_empty, acc_phase ^ 1u, &abort_flag, a.status)) break;
+        const uint32_t bi = nbuf == 2 ? (it & 1u) : 0u, use = nbuf == 2 ? (it >> 1) : it;
+        const uint32_t d0 = tmem_base + bi * 2u * sub_cols;
+        if (!mbar_wait(&tmem_empty[bi], (use & 1u) ^ 1u, &abort_flag, a.status)) break;
         tc_fence_after();
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
@@ -320,15 +328,14 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
           for (int kk = 0; kk < KB / 16; ++kk) {
             const uint32_t acc = (kb | kk) != 0;
             const uint64_t bd = sw128_desc(b0 + kk * 32);
-            umma_bf16(tmem_base, sw128_desc(a0 + kk * 32), bd, idesc, acc);
-            umma_bf16(tmem_base + 256, sw128_desc(a1 + kk * 32), bd, idesc, acc);
+            umma_bf16(d0, sw128_desc(a0 + kk * 32), bd, idesc, acc);
+            umma_bf16(d0 + sub_cols, sw128_desc(a1 + kk * 32), bd, idesc, acc);
           }
           umma_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tmem_full);
-        acc_phase ^= 1u;
+        umma_commit(&tmem_full[bi]);
       }
       // all issued MMAs must finish before TMEM is released
       umma_commit(&drain_bar);
@@ -338,20 +345,22 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     // epilogue warps 2..5
     const int q = warp & 3;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-    uint32_t acc_phase = 0;
+    uint32_t it = 0;
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       const TileInfo ti = decode_tile(sched, a, t);
-      if (!mbar_wait(&tmem_full, acc_phase, &abort_flag, a.status)) break;
+      const uint32_t bi = nbuf == 2 ? (it & 1u) : 0u, use = nbuf == 2 ? (it >> 1) : it;
+      if (!mbar_wait(&tmem_full[bi], use & 1u, &abort_flag, a.status)) break;
       tc_fence_after();
+      const uint32_t acc_addr = lane_addr + bi * 2u * sub_cols;
       const int nchunk = (ti.N + 31) / 32;
       __nv_bfloat16* stg = stage_out[q];
       if (EPI == EPI_SWIGLU) {
         const int feat0 = ti.mb * a.feat_stride + 32 * q;          // this warp's 32 features
         for (int c = 0; c < nchunk; ++c) {
           float g[32], u[32];
-          tmem_ld32(lane_addr + c * 32, g);
-          tmem_ld32(lane_addr + 256 + c * 32, u);
+          tmem_ld32(acc_addr + c * 32, g);
+          tmem_ld32(acc_addr + sub_cols + c * 32, u);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) g[j] = silu(g[j]) * u[j];
@@ -363,7 +372,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
           const int feat0 = ti.mb * a.feat_stride + s * a.feat_sub1 + 32 * q;
           for (int c = 0; c < nchunk; ++c) {
             float v[32];
-            tmem_ld32(lane_addr + s * 256 + c * 32, v);
+            tmem_ld32(acc_addr + s * sub_cols + c * 32, v);
             tmem_ld_wait();
             if (a.row_w) {
               const float wl = (c * 32 + lane < ti.n_valid) ? __ldg(a.row_w + ti.row0 + c * 32 + lane) : 0.0f;
@@ -375,8 +384,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         }
       }
       tc_fence_before();
-      mbar_arrive(&tmem_empty);
-      acc_phase ^= 1u;
+      mbar_arrive(&tmem_empty[bi]);
     }
   }
 
@@ -489,7 +497,7 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
           const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
           tma_load_2d_2sm(sA(stage), &tmA, fb, kb * KB, a_lo, pol_w);
-          tma_load_2d_2sm(sA(stage) + A_BYTES / 2, &tmA, fb, kb * KB, a_hi, pol_w);
+          if (!a.a_box128) tma_load_2d_2sm(sA(stage) + A_BYTES / 2, &tmA, fb, kb * KB, a_hi, pol_w);
           uint8_t* bdst = sB(stage);
           load_token_rows(rows, [&](int which, int off) {
             tma_load_2d_2sm(bdst + off * 128, tmB[which], fb, kb * KB, b0 + off, pol_x);
@@ -853,6 +861,7 @@ size_t gemm_e4m3_smem_bytes(int stages) {
 }
 
 constexpr int kBf16Stages = 3;
+constexpr int kBf16StagesDb = 4;
 constexpr int kE4m3Stages = 4;
 
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap* tmB,
@@ -865,9 +874,13 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
     if (e != cudaSuccess) return e;
     kern<<<grid & ~1, kThreads, smem, stream>>>(tmA, tmB[0], tmB[1], tmB[2], a);
   } else if (!e4m3) {
-    const size_t smem = gemm_bf16_smem_bytes(kBf16Stages, a.bn_max);
     const bool gather = a.gather_rows != nullptr;
-    auto kern = gather ? (epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, true>
+    // two accumulators hold <= 128-token tiles: 48 KB stages, four of them
+    const bool db = a.nbuf == 2 && !gather;
+    const size_t smem = gemm_bf16_smem_bytes(db ? kBf16StagesDb : kBf16Stages, a.bn_max);
+    auto kern = db ? (epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16StagesDb, false>
+                                        : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16StagesDb, false>)
+              : gather ? (epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, true>
                                             : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, true>)
                        : (epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, false>
                                             : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, false>);

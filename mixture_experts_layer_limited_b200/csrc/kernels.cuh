@@ -18,6 +18,8 @@ struct GemmArgs {
   int32_t feat_sub1;         // output-feature offset of sub-tile 1 (0 / 128)
   int32_t bn_max;            // max tokens per tile (multiple of 32, <= 256)
   int32_t cta_stride;        // CTA-pair kernel: weight-row offset of the second CTA (0 = 1-CTA kernel)
+  int32_t nbuf;              // 1-CTA kernel: TMEM accumulators (2 needs bn_max <= 128)
+  int32_t a_box128;          // CTA-pair kernel: a CTA's 128 weight rows are one 128-row box
   void* out;                 // [rows, out_ld] bf16, or e4m3 codes (GEMM1 FP8)
   int32_t out_ld;
   const float* row_w;        // [rows] or nullptr

@@ -217,12 +217,17 @@ def _ref_grouped(a, w13, w2, off, row_w):
     return out, hs
 
 
-@pytest.fixture(params=["pair", "1sm"])
+@pytest.fixture(params=["pair", "1sm-sb", "1sm-db"])
 def gemm_variant(request, monkeypatch):
-    """bf16 grouped GEMMs, both kernels forced: CTA pairs or single CTAs."""
-    monkeypatch.delenv("MOE_GEMM_1SM", raising=False)
-    monkeypatch.delenv("MOE_GEMM_PAIR", raising=False)
-    monkeypatch.setenv("MOE_GEMM_PAIR" if request.param == "pair" else "MOE_GEMM_1SM", "1")
+    """bf16 grouped GEMMs, each kernel forced: CTA pairs, single CTAs with one
+    TMEM accumulator, or single CTAs with two."""
+    for var in ("MOE_GEMM_1SM", "MOE_GEMM_PAIR", "MOE_GEMM_DB", "MOE_GEMM_SB"):
+        monkeypatch.delenv(var, raising=False)
+    if request.param == "pair":
+        monkeypatch.setenv("MOE_GEMM_PAIR", "1")
+    else:
+        monkeypatch.setenv("MOE_GEMM_1SM", "1")
+        monkeypatch.setenv("MOE_GEMM_DB" if request.param == "1sm-db" else "MOE_GEMM_SB", "1")
     return request.param
 
 
