@@ -69,13 +69,13 @@ moe_status make_tmap(CUtensorMap* m, const void* ptr, bool one_byte, uint64_t in
   return MOE_OK;
 }
 
-// Token-row maps of a grouped GEMM: bf16 rows are fetched with 64-, 32- and
-// 16-row boxes; e4m3 rows (at most 32 tokens a tile) with one 32-row box.
-moe_status make_token_tmaps(CUtensorMap* m, const void* ptr, bool fp8, uint64_t K, uint64_t rows) {
-  if (fp8) return make_tmap(&m[0], ptr, true, K, rows, 32);
-  const uint32_t box[3] = {64, 32, 16};
-  for (int i = 0; i < 3; ++i) {
-    moe_status s = make_tmap(&m[i], ptr, false, K, rows, box[i]);
+// Token-row maps of a grouped GEMM: bf16 rows are fetched with 256-, 128-,
+// 64-, 32- and 16-row boxes; e4m3 rows (at most 32 tokens a tile) with one
+// 32-row box.
+moe_status make_token_tmaps(TokenMaps* m, const void* ptr, bool fp8, uint64_t K, uint64_t rows) {
+  if (fp8) return make_tmap(&m->box[0], ptr, true, K, rows, 32);
+  for (int i = 0; i < kTokBoxes; ++i) {
+    moe_status s = make_tmap(&m->box[i], ptr, false, K, rows, 256u >> i);
     if (s != MOE_OK) return s;
   }
   return MOE_OK;
@@ -239,10 +239,11 @@ moe_status run_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const 
   const bool fp8 = w->dtype == MOE_E4M3;
   const bool pair = !fp8 && bf16_on_pairs();
   const int I = w->I;
-  CUtensorMap tmA, tmB[3];
+  CUtensorMap tmA;
+  TokenMaps tmB;
   moe_status s = make_tmap(&tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, pair ? 64 : 128);
   if (s != MOE_OK) return s;
-  s = make_token_tmaps(tmB, a, fp8, H, rows);
+  s = make_token_tmaps(&tmB, a, fp8, H, rows);
   if (s != MOE_OK) return s;
   const int nb = (fp8 || pair) ? 1 : one_cta_buffers(true);
   GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : (nb == 2 ? 128 : 256),
@@ -256,14 +257,18 @@ moe_status run_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const voi
   const bool fp8 = w->dtype == MOE_E4M3;
   const bool pair = !fp8 && bf16_on_pairs();
   const int I = w->I;
-  CUtensorMap tmA, tmB[3];
-  moe_status s = make_tmap(&tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H, 128);
+  CUtensorMap tmA;
+  TokenMaps tmB;
+  // the single-CTA bf16 kernel reads its 256 contiguous w2 rows as one box
+  const bool one_box = !fp8;
+  moe_status s = make_tmap(&tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H,
+                           (fp8 || pair) ? 128 : 256);
   if (s != MOE_OK) return s;
-  s = make_token_tmaps(tmB, h, fp8, I, rows);
+  s = make_token_tmaps(&tmB, h, fp8, I, rows);
   if (s != MOE_OK) return s;
   const int nb = (fp8 || pair) ? 1 : one_cta_buffers(false);
   GemmArgs g2{rows, I, w->groups, offsets, H, H / 256, 256, pair ? 64 : 128, 256, 128,
-              fp8 ? 32 : (nb == 2 ? 128 : 256), pair ? 128 : 0, nb, pair ? 1 : 0,
+              fp8 ? 32 : (nb == 2 ? 128 : 256), pair ? 128 : 0, nb, one_box ? 1 : 0,
               out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
   return check_launch(launch_grouped_gemm(fp8, EPI_WEIGHTED, tmA, tmB, g2, nsm, st));
 }
@@ -296,10 +301,11 @@ moe_status moe_gate_up_swiglu_gather(int32_t rows, int32_t H, const moe_ffn_weig
   int nsm = 0;
   if ((s = sm_count(&nsm)) != MOE_OK) return s;
   const int I = w->I;
-  CUtensorMap tmA, tmB[3];
+  CUtensorMap tmA;
+  TokenMaps tmB;
   s = make_tmap(&tmA, w->w13, false, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
   if (s != MOE_OK) return s;
-  s = make_token_tmaps(tmB, x, false, H, T);      // not read: token rows are gathered
+  s = make_token_tmaps(&tmB, x, false, H, T);      // not read: token rows are gathered
   if (s != MOE_OK) return s;
   GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, 256, 0, 1, 0,
               h_ws, I, nullptr, nullptr, nullptr, nullptr, dev_status, x, src_token, T};

@@ -120,14 +120,17 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, const GemmArgs& 
   return ti;
 }
 
-// Token rows of one stage are fetched as 64-row boxes, then at most one
-// 32-row and one 16-row box (`rows` is a multiple of 16). Returns rows loaded.
+// Token rows of one stage (a multiple of 16, at most 256) are fetched with at
+// most one box of each size 256, 128, 64, 32, 16: the binary digits of
+// rows / 16. Returns rows loaded.
 template <typename LoadFn>
 __device__ __forceinline__ int load_token_rows(int rows, LoadFn&& load) {
   int off = 0;
-  for (; rows - off >= 64; off += 64) load(0, off);
-  if (rows - off >= 32) { load(1, off); off += 32; }
-  if (rows - off >= 16) { load(2, off); off += 16; }
+#pragma unroll
+  for (int i = 0; i < kTokBoxes; ++i) {
+    const int box = 256 >> i;
+    if (rows - off >= box) { load(i, off); off += box; }
+  }
   return off;
 }
 
@@ -171,9 +174,7 @@ constexpr int kGatherThreads = 64;
 template <int EPI, int STAGES, bool GATHER>
 __global__ void __launch_bounds__(kThreads + (GATHER ? kGatherThreads : 0), 1)
 grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
-                         const __grid_constant__ CUtensorMap tmB64,
-                         const __grid_constant__ CUtensorMap tmB32,
-                         const __grid_constant__ CUtensorMap tmB16, const GemmArgs a) {
+                         const __grid_constant__ TokenMaps tmB, const GemmArgs a) {
   constexpr int KB = 64;                           // K elements per stage (128 B)
   constexpr uint32_t A_SUB_BYTES = 128 * 128;      // one 128-row sub-tile
   extern __shared__ __align__(1024) uint8_t dsmem[];
@@ -212,9 +213,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB64);
-    tma_prefetch_desc(&tmB32);
-    tma_prefetch_desc(&tmB16);
+    for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&tmB.box[i]);
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_s, 512);
@@ -233,7 +232,6 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       const uint64_t pol_once = policy_evict_first();
       const uint64_t pol_reuse = policy_evict_normal();
       const uint64_t pol_x = policy_evict_last();
-      const CUtensorMap* tmB[3] = {&tmB64, &tmB32, &tmB16};
       int stage = 0;
       uint32_t phase = 0;
       for (int t = blockIdx.x; t < total && !abort_flag; t += gridDim.x) {
@@ -247,12 +245,12 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
           tma_load_2d(sA(stage, 0), &tmA, &full_bar[stage], kb * KB, a_row0, pol_w);
-          tma_load_2d(sA(stage, 1), &tmA, &full_bar[stage], kb * KB, a_row1, pol_w);
+          if (!a.a_one_box) tma_load_2d(sA(stage, 1), &tmA, &full_bar[stage], kb * KB, a_row1, pol_w);
           if (!GATHER) {
             uint8_t* bdst = sB(stage);
             uint64_t* fb = &full_bar[stage];
             load_token_rows(ti.N, [&](int which, int off) {
-              tma_load_2d(bdst + off * 128, tmB[which], fb, kb * KB, ti.row0 + off, pol_x);
+              tma_load_2d(bdst + off * 128, &tmB.box[which], fb, kb * KB, ti.row0 + off, pol_x);
             });
           }
           issued_parity[stage] = static_cast<int>(phase);
@@ -414,9 +412,7 @@ constexpr int kXStride = 33;               // padded row of the lane exchange bu
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
-                             const __grid_constant__ CUtensorMap tmB64,
-                             const __grid_constant__ CUtensorMap tmB32,
-                             const __grid_constant__ CUtensorMap tmB16, const GemmArgs a) {
+                             const __grid_constant__ TokenMaps tmB, const GemmArgs a) {
   constexpr int KB = 64;
   constexpr int STAGES = k2smStages;
   constexpr uint32_t A_BYTES = 128 * 128;       // this CTA's 128 weight rows x 64 K
@@ -457,9 +453,7 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB64);
-    tma_prefetch_desc(&tmB32);
-    tma_prefetch_desc(&tmB16);
+    for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&tmB.box[i]);
   }
   if (warp == 1) {
     tmem_alloc_2sm(&tmem_base_s, 512);
@@ -479,7 +473,6 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
       const uint64_t pol_once = policy_evict_first();
       const uint64_t pol_reuse = policy_evict_normal();
       const uint64_t pol_x = policy_evict_last();
-      const CUtensorMap* tmB[3] = {&tmB64, &tmB32, &tmB16};
       int stage = 0;
       uint32_t phase = 0;
       for (int t = pair; t < total && !abort_flag; t += npairs) {
@@ -497,10 +490,10 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
           const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
           tma_load_2d_2sm(sA(stage), &tmA, fb, kb * KB, a_lo, pol_w);
-          if (!a.a_box128) tma_load_2d_2sm(sA(stage) + A_BYTES / 2, &tmA, fb, kb * KB, a_hi, pol_w);
+          if (!a.a_one_box) tma_load_2d_2sm(sA(stage) + A_BYTES / 2, &tmA, fb, kb * KB, a_hi, pol_w);
           uint8_t* bdst = sB(stage);
           load_token_rows(rows, [&](int which, int off) {
-            tma_load_2d_2sm(bdst + off * 128, tmB[which], fb, kb * KB, b0 + off, pol_x);
+            tma_load_2d_2sm(bdst + off * 128, &tmB.box[which], fb, kb * KB, b0 + off, pol_x);
           });
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -864,7 +857,7 @@ constexpr int kBf16Stages = 3;
 constexpr int kBf16StagesDb = 4;
 constexpr int kE4m3Stages = 4;
 
-cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap* tmB,
+cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const TokenMaps& tmB,
                                 const GemmArgs& a, int grid, cudaStream_t stream) {
   if (!e4m3 && a.cta_stride > 0) {
     const size_t smem = gemm_bf16_2sm_smem_bytes();
@@ -872,7 +865,7 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
                                   : grouped_gemm_bf16_2sm_kernel<EPI_WEIGHTED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid & ~1, kThreads, smem, stream>>>(tmA, tmB[0], tmB[1], tmB[2], a);
+    kern<<<grid & ~1, kThreads, smem, stream>>>(tmA, tmB, a);
   } else if (!e4m3) {
     const bool gather = a.gather_rows != nullptr;
     // two accumulators hold <= 128-token tiles: 48 KB stages, four of them
@@ -886,14 +879,14 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
                                             : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads + (gather ? kGatherThreads : 0), smem, stream>>>(tmA, tmB[0], tmB[1], tmB[2], a);
+    kern<<<grid, kThreads + (gather ? kGatherThreads : 0), smem, stream>>>(tmA, tmB, a);
   } else {
     const size_t smem = gemm_e4m3_smem_bytes(kE4m3Stages);
     auto kern = epi == EPI_SWIGLU ? grouped_gemm_e4m3_kernel<EPI_SWIGLU, kE4m3Stages>
                                   : grouped_gemm_e4m3_kernel<EPI_WEIGHTED, kE4m3Stages>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, stream>>>(tmA, tmB[0], a);
+    kern<<<grid, kThreads, smem, stream>>>(tmA, tmB.box[0], a);
   }
   return cudaGetLastError();
 }

@@ -19,7 +19,7 @@ struct GemmArgs {
   int32_t bn_max;            // max tokens per tile (multiple of 32, <= 256)
   int32_t cta_stride;        // CTA-pair kernel: weight-row offset of the second CTA (0 = 1-CTA kernel)
   int32_t nbuf;              // 1-CTA kernel: TMEM accumulators (2 needs bn_max <= 128)
-  int32_t a_box128;          // CTA-pair kernel: a CTA's 128 weight rows are one 128-row box
+  int32_t a_one_box;         // a CTA's weight rows are contiguous: one TMA box (256 rows, pair: 128)
   void* out;                 // [rows, out_ld] bf16, or e4m3 codes (GEMM1 FP8)
   int32_t out_ld;
   const float* row_w;        // [rows] or nullptr
@@ -50,7 +50,14 @@ enum { EPI_SWIGLU = 0, EPI_WEIGHTED = 1 };
 
 // tmB: token-row tensor maps with 64-, 32- and 16-row boxes (bf16), or one
 // 32-row map (e4m3).
-cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const CUtensorMap* tmB,
+// Token-row tensor maps: bf16 boxes of 256, 128, 64, 32 and 16 rows (a tile's
+// rows are fetched with the fewest boxes); e4m3 uses box[0] of 32 rows.
+constexpr int kTokBoxes = 5;
+struct TokenMaps {
+  CUtensorMap box[kTokBoxes];
+};
+
+cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const TokenMaps& tmB,
                                 const GemmArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
                              cudaStream_t stream);
