@@ -20,16 +20,18 @@ Parity status per function (what pins each one is listed in the tests):
   moe_forward                                   pinned (dense brute force,
                                                 combine identities)
   bias_update / load_cv                         pinned (closed forms)
+  seq_aux_loss                                  pinned (closed forms: balanced,
+                                                collapsed, disjoint, per-sequence)
 """
 from .moe_oracle import (
     e4m3_values, quantize_e4m3, dequantize_e4m3, round_to_e4m3, fp8_quantize_blocks,
     fp8_quantize_rows, fp8_qdq_blocks, fp8_qdq_rows, gate_logits, selection_scores, route_from_logits,
-    RouteResult, permute, swiglu_ffn, moe_forward, bias_update, load_cv,
+    RouteResult, permute, swiglu_ffn, moe_forward, bias_update, load_cv, seq_aux_loss,
 )
 
 __all__ = [
     "e4m3_values", "quantize_e4m3", "dequantize_e4m3", "round_to_e4m3",
     "fp8_quantize_blocks", "fp8_quantize_rows", "fp8_qdq_blocks", "fp8_qdq_rows", "gate_logits", "selection_scores",
     "route_from_logits", "RouteResult", "permute", "swiglu_ffn",
-    "moe_forward", "bias_update", "load_cv",
+    "moe_forward", "bias_update", "load_cv", "seq_aux_loss",
 ]

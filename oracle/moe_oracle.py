@@ -14,6 +14,8 @@ Pages followed (cited by title and section):
                  bias and device-limited routing).
   [FP8-infer]    blog.hotdry.top DeepSeek-V3 FP8 inference post, "FP8 混合精度"
                  section (E4M3, 1x128 activation / 128x128 weight tiles).
+  [MoE-walk §6.2] the same zhiyuanblog.org page, "辅助损失（训练时）": the
+                 sequence-level auxiliary balance loss (seq_aux, alpha 0.001).
 
 Readings taken where the pages are silent or disagree:
   * The selection bias only decides which experts are chosen; the weights
@@ -30,6 +32,13 @@ Readings taken where the pages are silent or disagree:
     round-to-nearest-even, saturating, of x / scale computed in fp32.
   * Bias step: b_e <- b_e - gamma * sign(c_e * E - T * k), the sign taken on
     exact integers, the subtraction rounded once in fp32.
+  * Sequence-level aux loss: the T tokens form T / seq_len sequences of
+    seq_len consecutive tokens. An expert's load is its share of the
+    sequence's seq_len * k assignments; its importance is the mean over the
+    sequence's tokens of the token's score for it, normalised over all E
+    experts (the softmax probability; for sigmoid scoring sigma / sum of
+    sigma). Per sequence: E * sum_e load_e * importance_e (1 when both are
+    uniform); the value is alpha times the mean over sequences.
 """
 from dataclasses import dataclass
 from typing import Callable, Optional, Tuple
@@ -396,3 +405,35 @@ def load_cv(counts: np.ndarray) -> float:
     mean = c.sum() / E
     var = ((c - mean) ** 2).sum() / (E - 1)
     return float(np.sqrt(var) / mean)
+
+
+# --------------------------------------------------------------------------
+# Sequence-level auxiliary balance loss ([MoE-walk §6.2]; seq_aux and
+# aux_loss_alpha also appear in [V3-teardown] §3 moe_router.json).
+# --------------------------------------------------------------------------
+def seq_aux_loss(logits32: np.ndarray, ids: np.ndarray, E: int, k: int, scoring: str,
+                 seq_len: int, alpha: float) -> float:
+    """alpha * mean over sequences of E * sum_e f_e * P_e, where f_e is the
+    fraction of the sequence's seq_len * k assignments that go to expert e
+    and P_e the mean of the tokens' normalised scores for e. Forward value
+    only; fp64 throughout."""
+    L = np.asarray(logits32, dtype=np.float32).astype(np.float64)
+    ids = np.asarray(ids, dtype=np.int64)
+    T = L.shape[0]
+    if seq_len <= 0 or T % seq_len:
+        raise ValueError("seq_len must divide T")
+    if scoring == "softmax":
+        z = np.exp(L - L.max(axis=1, keepdims=True))
+    elif scoring == "sigmoid":
+        z = 1.0 / (1.0 + np.exp(-L))
+    else:
+        raise ValueError(scoring)
+    p = z / z.sum(axis=1, keepdims=True)          # per-token scores summing to 1
+    total = 0.0
+    n_seq = T // seq_len
+    for b in range(n_seq):
+        rows = slice(b * seq_len, (b + 1) * seq_len)
+        f = np.bincount(ids[rows].ravel(), minlength=E).astype(np.float64) / (seq_len * k)
+        P = p[rows].mean(axis=0)
+        total += E * float(np.dot(f, P))
+    return alpha * total / n_seq

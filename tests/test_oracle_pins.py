@@ -421,3 +421,58 @@ def test_v2lite_parameter_counts():
     assert round(per_expert / 1e6, 2) == 8.65
     active = cfg.flops() / cfg.T / 2
     assert round(active / 1e6, 1) == 69.3
+
+
+# ------------------------------------- sequence-level aux loss (closed forms)
+# "MoE 混合专家模型推理参数与前向传播详解" §6.2: aux = E * sum_e load_e * importance_e,
+# added to the loss times aux_loss_alpha = 0.001.
+def _round_robin_ids(T, k, E):
+    return (np.arange(T)[:, None] * k + np.arange(k)[None, :]) % E
+
+
+@pytest.mark.parametrize("scoring", ["softmax", "sigmoid"])
+def test_seq_aux_loss_is_one_when_balanced(scoring):
+    T, E, k = 64, 16, 4
+    L = np.zeros((T, E), np.float32)                 # every score equal: importance 1/E
+    ids = _round_robin_ids(T, k, E)                  # every expert gets T*k/E assignments
+    assert oracle.seq_aux_loss(L, ids, E, k, scoring, T, 1.0) == pytest.approx(1.0, rel=1e-14)
+    assert oracle.seq_aux_loss(L, ids, E, k, scoring, T, 0.001) == pytest.approx(0.001, rel=1e-14)
+
+
+def test_seq_aux_loss_collapsed_routing_is_E_over_k():
+    T, E, k = 64, 16, 4
+    L = np.full((T, E), -1e4, np.float32)
+    L[:, :k] = 0.0                                   # softmax mass 1/k on experts 0..k-1, 0 elsewhere
+    ids = np.tile(np.arange(k), (T, 1))
+    assert oracle.seq_aux_loss(L, ids, E, k, "softmax", T, 1.0) == pytest.approx(E / k, rel=1e-14)
+    # the same loads against scores that sit on other experts: no overlap, zero loss
+    L2 = np.full((T, E), -1e4, np.float32)
+    L2[:, k:2 * k] = 0.0
+    assert oracle.seq_aux_loss(L2, ids, E, k, "softmax", T, 1.0) == 0.0
+
+
+def test_seq_aux_loss_is_per_sequence():
+    T, E, k = 64, 16, 4
+    L = np.full((T, E), -1e4, np.float32)
+    ids = np.zeros((T, k), np.int64)
+    L[:32, 0:4] = 0.0
+    ids[:32] = np.arange(0, 4)
+    L[32:, 4:8] = 0.0
+    ids[32:] = np.arange(4, 8)
+    # two sequences, each collapsed on its own four experts: E/k each
+    assert oracle.seq_aux_loss(L, ids, E, k, "softmax", 32, 1.0) == pytest.approx(4.0, rel=1e-14)
+    # one sequence: loads and importances spread over eight experts, 16 * 8 / 64
+    assert oracle.seq_aux_loss(L, ids, E, k, "softmax", 64, 1.0) == pytest.approx(2.0, rel=1e-14)
+
+
+@pytest.mark.parametrize("scoring,row0", [("softmax", [np.log(3.0), 0.0]),
+                                          ("sigmoid", [np.log(3.0), -np.log(3.0)])])
+def test_seq_aux_loss_two_token_hand_example(scoring, row0):
+    # token 0 scores (3/4, 1/4) in both scorings (sigmoid(ln 3) = 3/4 and the two
+    # sigmoids sum to 1), token 1 scores (1/2, 1/2): importance (5/8, 3/8)
+    L = np.array([row0, [0.0, 0.0]], np.float32)
+    both_on_0 = np.array([[0], [0]])
+    split = np.array([[0], [1]])
+    assert oracle.seq_aux_loss(L, both_on_0, 2, 1, scoring, 2, 1.0) == pytest.approx(1.25, rel=1e-6)
+    assert oracle.seq_aux_loss(L, split, 2, 1, scoring, 2, 1.0) == pytest.approx(1.0, rel=1e-6)
+    assert oracle.seq_aux_loss(L, np.array([[1], [1]]), 2, 1, scoring, 2, 1.0) == pytest.approx(0.75, rel=1e-6)
