@@ -281,6 +281,31 @@ MOE_API moe_status moe_bias_update(int32_t E, int32_t T, int32_t k, const int32_
                            float* bias, float gamma, float* load_cv, void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * moe_aux_loss -- sequence-level auxiliary balance loss, forward value only,
+ * [MoE-walk] §6.2 (seq_aux, aux_loss_alpha = 0.001 for V2-Lite):
+ *   the T tokens form T / seq_len sequences of seq_len consecutive tokens;
+ *   per sequence   E * sum_e f_e * P_e   with
+ *     f_e = #{(t, j) in the sequence : topk_ids[t][j] == e} / (seq_len * k)
+ *     P_e = mean over the sequence's tokens of the token's score for e,
+ *           normalised over all E experts (softmax probability, or the
+ *           sigmoid divided by the sum of the E sigmoids);
+ *   aux_out[0] = alpha * (mean over the sequences), fp32.
+ * The value is 1 * alpha when loads and scores are uniform.
+ *   logits    [T, E] fp32 (e.g. as written by moe_route); topk_ids [T, k]
+ *   scoring   MOE_SOFTMAX or MOE_SIGMOID
+ *   seq_len   divides T (seq_len = T: the batch is one sequence)
+ *   workspace device scratch of moe_aux_loss_workspace_size() bytes, 8-byte
+ *             aligned. E <= 256.
+ * Scores are evaluated and summed in fp64; partial sums are combined in a
+ * fixed order, so the result does not vary from run to run. topk_ids outside
+ * [0, E) are not counted and flag MOE_DEVSTAT_BAD_EXPERT_ID in dev_status.
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_aux_loss_workspace_size(int32_t T, int32_t E, int32_t seq_len, size_t* bytes);
+MOE_API moe_status moe_aux_loss(int32_t T, int32_t E, int32_t k, int32_t seq_len, int32_t scoring,
+                        const float* logits, const int32_t* topk_ids, float alpha, float* aux_out,
+                        void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * FP8 E4M3 quantisers ([V3-teardown] §3 infer.toml: weight_block_size
  * [128, 128], activation_scheme dynamic; [FP8-infer] 1x128 / 128x128 tiles).
  *   scale = amax / 448 in fp32 (1.0 for an all-zero tile);

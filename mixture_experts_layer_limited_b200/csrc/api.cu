@@ -356,6 +356,27 @@ moe_status moe_bias_update(int32_t E, int32_t T, int32_t k, const int32_t* exper
   return check_launch(launch_bias_update(E, T, k, expert_counts, bias, gamma, load_cv, as_stream(stream)));
 }
 
+moe_status moe_aux_loss_workspace_size(int32_t T, int32_t E, int32_t seq_len, size_t* bytes) {
+  if (!bytes || T < 1 || E < 1 || seq_len < 1 || T % seq_len != 0) return MOE_ERR_INVALID_ARG;
+  *bytes = aux_loss_workspace_bytes(T, E, seq_len);
+  return MOE_OK;
+}
+
+moe_status moe_aux_loss(int32_t T, int32_t E, int32_t k, int32_t seq_len, int32_t scoring, const float* logits,
+                        const int32_t* topk_ids, float alpha, float* aux_out, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (T < 1 || E < 1 || k < 1 || k > E || seq_len < 1 || T % seq_len != 0) return MOE_ERR_INVALID_ARG;
+  if (scoring != MOE_SOFTMAX && scoring != MOE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (!logits || !topk_ids || !aux_out || !workspace) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < aux_loss_workspace_bytes(T, E, seq_len)) return MOE_ERR_INVALID_ARG;
+  if (E > 256) return MOE_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(workspace) % 8 != 0 || reinterpret_cast<uintptr_t>(logits) % 4 != 0 ||
+      reinterpret_cast<uintptr_t>(topk_ids) % 4 != 0 || reinterpret_cast<uintptr_t>(aux_out) % 4 != 0)
+    return MOE_ERR_ALIGNMENT;
+  return check_launch(launch_aux_loss(T, E, k, seq_len, scoring, logits, topk_ids, alpha, aux_out, workspace,
+                                      dev_status, as_stream(stream)));
+}
+
 moe_status moe_quantize_blocks(int32_t batch, int32_t N, int32_t K, const void* w, void* q, float* scale,
                                void* stream) {
   if (batch < 1 || N < 1 || K < 1 || !w || !q || !scale) return MOE_ERR_INVALID_ARG;

@@ -70,6 +70,15 @@ cudaError_t launch_permute(int T, int k, int E, int row_bytes, const int32_t* id
                            cudaStream_t stream);
 cudaError_t launch_combine(int T, int k, int H, const void* eo, const int32_t* slot_to_row,
                            const float* topk_w, const void* shared, void* y, cudaStream_t stream);
+constexpr int kAuxChunk = 128;   // tokens per aux-loss partial
+constexpr int kAuxWarps = 8;
+inline size_t aux_loss_workspace_bytes(int T, int E, int seq_len) {
+  const size_t chunks = static_cast<size_t>(T / seq_len) * ((seq_len + kAuxChunk - 1) / kAuxChunk);
+  return chunks * E * (sizeof(double) + sizeof(int32_t));
+}
+cudaError_t launch_aux_loss(int T, int E, int k, int seq_len, int scoring, const float* logits,
+                            const int32_t* ids, float alpha, float* out, void* ws, int32_t* status,
+                            cudaStream_t stream);
 cudaError_t launch_bias_update(int E, int T, int k, const int32_t* counts, float* bias, float gamma,
                                float* load_cv, cudaStream_t stream);
 cudaError_t launch_quant_blocks(int batch, int N, int K, const void* w, void* q, float* scale,

@@ -131,6 +131,106 @@ bias_update_kernel(int E, int T, int k, const int32_t* __restrict__ counts, floa
   }
 }
 
+// ------------------------------------------------------------------------
+// Sequence-level auxiliary balance loss ("MoE 混合专家模型推理参数与前向传播详解"
+// §6.2): per sequence E * sum_e f_e * P_e, f_e = the expert's share of the
+// sequence's seq_len * k assignments, P_e = mean normalised score.
+// Pass 1, one CTA per chunk of <= kAuxChunk tokens inside one sequence: warp w
+// takes tokens w, w + 8, ...; lane l keeps the fp64 score sums of experts
+// l, l + 32, ...; the eight warps' sums are added in warp order and the chunk's
+// sums and assignment counts go to the workspace.
+// Pass 2, one CTA: per expert, chunks in order, sum_b count_be * P_be; then a
+// fixed tree over experts. Deterministic for given inputs.
+// ------------------------------------------------------------------------
+__global__ void __launch_bounds__(kAuxWarps * 32)
+aux_chunk_kernel(int T, int E, int k, int seq_len, int scoring, const float* __restrict__ logits,
+                 const int32_t* __restrict__ ids, double* __restrict__ psum, int32_t* __restrict__ cnt,
+                 int32_t* status) {
+  __shared__ double part[kAuxWarps][256];
+  __shared__ int hist[256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cps = (seq_len + kAuxChunk - 1) / kAuxChunk;          // chunks per sequence
+  const int seq = blockIdx.x / cps, c = blockIdx.x % cps;
+  const int t0 = seq * seq_len + c * kAuxChunk;
+  const int t1 = min(t0 + kAuxChunk, (seq + 1) * seq_len);
+  for (int e = threadIdx.x; e < 256; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  double acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+  for (int t = t0 + warp; t < t1; t += kAuxWarps) {
+    const float* L = logits + static_cast<size_t>(t) * E;
+    double z[8];
+    double m = -INFINITY;
+    if (scoring == MOE_SOFTMAX) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i < E) m = fmax(m, static_cast<double>(L[lane + 32 * i]));
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, d));
+    }
+    double sum = 0.0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      z[i] = 0.0;
+      if (e < E) {
+        const double l = static_cast<double>(L[e]);
+        z[i] = scoring == MOE_SOFTMAX ? exp(l - m) : 1.0 / (1.0 + exp(-l));
+      }
+      sum += z[i];
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += z[i] / sum;
+    if (lane < k) {
+      const int e = ids[static_cast<size_t>(t) * k + lane];
+      if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+      else flag_status(status, MOE_DEVSTAT_BAD_EXPERT_ID);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) part[warp][lane + 32 * i] = acc[i];
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    double v = 0.0;
+    for (int w = 0; w < kAuxWarps; ++w) v += part[w][e];
+    psum[static_cast<size_t>(blockIdx.x) * E + e] = v;
+    cnt[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
+  }
+}
+
+__global__ void __launch_bounds__(256)
+aux_reduce_kernel(int E, int k, int seq_len, int n_seq, int cps, float alpha, const double* __restrict__ psum,
+                  const int32_t* __restrict__ cnt, float* __restrict__ out) {
+  __shared__ double red[256];
+  const int e = threadIdx.x;
+  double v = 0.0;
+  if (e < E) {
+    for (int b = 0; b < n_seq; ++b) {
+      double p = 0.0;
+      long long n = 0;
+      for (int c = 0; c < cps; ++c) {
+        const size_t i = (static_cast<size_t>(b) * cps + c) * E + e;
+        p += psum[i];
+        n += cnt[i];
+      }
+      v += static_cast<double>(n) * p;
+    }
+  }
+  red[e] = v;
+  __syncthreads();
+  for (int s = 128; s > 0; s >>= 1) {
+    if (e < s) red[e] += red[e + s];
+    __syncthreads();
+  }
+  if (e == 0) {
+    const double S = static_cast<double>(seq_len);
+    *out = static_cast<float>(static_cast<double>(alpha) * E * red[0] / (static_cast<double>(n_seq) * S * S * k));
+  }
+}
+
 // E4M3 weight quantisation per 128x128 block. grid (K/128, N/128, batch),
 // 256 threads: thread i covers row i/2, columns (i%2)*64 .. +64.
 __global__ void __launch_bounds__(256)
@@ -218,6 +318,22 @@ cudaError_t launch_combine(int T, int k, int H, const void* eo, const int32_t* s
 cudaError_t launch_bias_update(int E, int T, int k, const int32_t* counts, float* bias, float gamma,
                                float* load_cv, cudaStream_t stream) {
   bias_update_kernel<<<1, 1024, 0, stream>>>(E, T, k, counts, bias, gamma, load_cv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_aux_loss(int T, int E, int k, int seq_len, int scoring, const float* logits,
+                            const int32_t* ids, float alpha, float* out, void* ws, int32_t* status,
+                            cudaStream_t stream) {
+  const int n_seq = T / seq_len;
+  const int cps = (seq_len + kAuxChunk - 1) / kAuxChunk;
+  const long long chunks = static_cast<long long>(n_seq) * cps;
+  double* psum = reinterpret_cast<double*>(ws);
+  int32_t* cnt = reinterpret_cast<int32_t*>(psum + chunks * E);
+  aux_chunk_kernel<<<static_cast<unsigned>(chunks), kAuxWarps * 32, 0, stream>>>(
+      T, E, k, seq_len, scoring, logits, ids, psum, cnt, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  aux_reduce_kernel<<<1, 256, 0, stream>>>(E, k, seq_len, n_seq, cps, alpha, psum, cnt, out);
   return cudaGetLastError();
 }
 

@@ -207,5 +207,18 @@ class MoELayer:
         N.moe_bias_update(s.E, T, s.k, self.counts, self.bias, gamma,
                           self.load_cv if load_cv else None)
 
+    def aux_loss(self, T: int, seq_len: Optional[int] = None, alpha: float = 0.001) -> torch.Tensor:
+        """Sequence-level auxiliary balance loss of the last forward ("MoE 混合
+        专家模型推理参数与前向传播详解" §6.2), from its logits and expert ids;
+        a [1] fp32 device tensor, alpha * mean over sequences of seq_len
+        tokens (default: the T tokens as one sequence)."""
+        s = self.spec
+        seq_len = T if seq_len is None else seq_len
+        ws = torch.empty(N.moe_aux_loss_workspace_size(T, s.E, seq_len), dtype=torch.uint8, device=self.dev)
+        out = torch.empty(1, dtype=torch.float32, device=self.dev)
+        N.moe_aux_loss(T, s.E, s.k, seq_len, N.MOE_SIGMOID if s.scoring == "sigmoid" else N.MOE_SOFTMAX,
+                       self.logits[:T], self.ids[:T], alpha, out, ws, self.status)
+        return out
+
     def device_status(self) -> int:
         return N.moe_read_device_status(self.status)

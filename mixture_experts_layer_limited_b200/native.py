@@ -29,7 +29,8 @@ EXPORTED = [
     "moe_route", "moe_permute_workspace_size", "moe_permute", "moe_permute_static_ws",
     "moe_grouped_swiglu",
     "moe_gate_up_swiglu", "moe_gate_up_swiglu_gather", "moe_down_proj",
-    "moe_combine", "moe_bias_update", "moe_quantize_blocks", "moe_quantize_rows",
+    "moe_combine", "moe_bias_update", "moe_aux_loss_workspace_size", "moe_aux_loss",
+    "moe_quantize_blocks", "moe_quantize_rows",
     "moe_read_device_status", "moe_last_cuda_error", "moe_status_string", "moe_abi_version",
 ]
 
@@ -80,6 +81,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_gate_up_swiglu_gather": [_I, _I, ctypes.POINTER(FFNWeights), _P, _I, _P, _P, _P, _P, _P],
         "moe_combine": [_I, _I, _I, _P, _P, _P, _P, _P, _P],
         "moe_bias_update": [_I, _I, _I, _P, _P, ctypes.c_float, _P, _P],
+        "moe_aux_loss_workspace_size": [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
+        "moe_aux_loss": [_I, _I, _I, _I, _I, _P, _P, ctypes.c_float, _P, _P, ctypes.c_size_t, _P, _P],
         "moe_quantize_blocks": [_I, _I, _I, _P, _P, _P, _P],
         "moe_quantize_rows": [_I, _I, _P, _P, _P, _P],
         "moe_read_device_status": [_P, ctypes.POINTER(ctypes.c_int32), _P],
@@ -188,6 +191,21 @@ def moe_combine(T, k, H, expert_out, slot_to_row, topk_w, shared_out, y, stream=
 def moe_bias_update(E, T, k, expert_counts, bias, gamma, load_cv=None, stream=None):
     _check("moe_bias_update", load_library().moe_bias_update(
         E, T, k, _ptr(expert_counts), _ptr(bias), float(gamma), _ptr(load_cv), _stream(stream)))
+
+
+def moe_aux_loss_workspace_size(T, E, seq_len) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_aux_loss_workspace_size",
+           load_library().moe_aux_loss_workspace_size(T, E, seq_len, ctypes.byref(n)))
+    return n.value
+
+
+def moe_aux_loss(T, E, k, seq_len, scoring, logits, topk_ids, alpha, aux_out, workspace,
+                 dev_status=None, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("moe_aux_loss", load_library().moe_aux_loss(
+        T, E, k, seq_len, scoring, _ptr(logits), _ptr(topk_ids), float(alpha), _ptr(aux_out),
+        _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
 
 
 def moe_quantize_blocks(batch, N, K, w, q, scale, stream=None):

@@ -90,6 +90,18 @@ def test_host_validation_rejects_before_launch():
     assert lib.moe_combine(8, 4, 252, fake, fake, None, None, fake, None) == N.MOE_ERR_UNSUPPORTED
     assert lib.moe_bias_update(2048, 8, 4, fake, fake, ctypes.c_float(0.001), None, None) == N.MOE_ERR_UNSUPPORTED
     assert lib.moe_bias_update(16, 8, 4, None, fake, ctypes.c_float(0.001), None, None) == N.MOE_ERR_INVALID_ARG
+    # moe_aux_loss: seq_len must divide T, workspace too small, E beyond 256, scoring
+    assert N.moe_aux_loss_workspace_size(256, 16, 128) == 2 * 16 * 12
+    with pytest.raises(N.MoEError):
+        N.moe_aux_loss_workspace_size(100, 16, 30)
+    assert lib.moe_aux_loss(100, 16, 4, 30, N.MOE_SOFTMAX, fake, fake, ctypes.c_float(1.0), fake, fake,
+                            1 << 20, None, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_aux_loss(256, 16, 4, 128, N.MOE_SOFTMAX, fake, fake, ctypes.c_float(1.0), fake, fake,
+                            16, None, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_aux_loss(256, 512, 4, 256, N.MOE_SIGMOID, fake, fake, ctypes.c_float(1.0), fake, fake,
+                            1 << 20, None, None) == N.MOE_ERR_UNSUPPORTED
+    assert lib.moe_aux_loss(256, 16, 4, 256, 7, fake, fake, ctypes.c_float(1.0), fake, fake,
+                            1 << 20, None, None) == N.MOE_ERR_INVALID_ARG
     assert lib.moe_quantize_blocks(1, 100, 128, fake, fake, fake, None) == N.MOE_ERR_UNSUPPORTED
     assert lib.moe_quantize_rows(4, 128, odd, fake, fake, None) == N.MOE_ERR_ALIGNMENT
     assert lib.moe_read_device_status(None, None, None) == N.MOE_ERR_INVALID_ARG
