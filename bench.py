@@ -45,6 +45,9 @@ def parse_args():
     ap.add_argument("--config", default="v3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=16)
+    ap.add_argument("--routing-sweep", action="store_true",
+                    help="instead of the throughput line: load CV, aux loss and router time for "
+                         "topk_group 8/4/2/1 of 8 groups on the V3 and skewed inputs (one line each)")
     return ap.parse_args()
 
 
@@ -406,8 +409,59 @@ def run_ours(args):
     return 0
 
 
+def run_routing_sweep(args):
+    """The group-limit experiment of the V3 teardown page (§4: lowering
+    topk_group from 4 to 2 concentrates load, 8 removes the limit): for each
+    topk_group, one routing pass of the V3 and of the skewed inputs through
+    moe_route, then the load CV (moe_bias_update with gamma 0 leaves the bias
+    as it is) and the sequence-level aux loss, and the router's device time."""
+    import torch
+    from moe_inputs import get_config, make_inputs
+    from mixture_experts_layer_limited_b200 import native as N
+    N.load_library()
+    dev = "cuda"
+    for name in ("v3", "v3_skewed"):
+        cfg = get_config(name)
+        inp = make_inputs(cfg, device=dev, experts=False, shared=False)
+        T, E, k = cfg.T, cfg.E, cfg.k
+        f32, i32 = torch.float32, torch.int32
+        logits = torch.empty(T, E, dtype=f32, device=dev)
+        ids = torch.empty(T, k, dtype=i32, device=dev)
+        w = torch.empty(T, k, dtype=f32, device=dev)
+        counts = torch.empty(E, dtype=i32, device=dev)
+        cv = torch.empty(1, dtype=f32, device=dev)
+        aux = torch.empty(1, dtype=f32, device=dev)
+        bias = inp.bias.clone()
+        ws = torch.empty(N.moe_aux_loss_workspace_size(T, E, T), dtype=torch.uint8, device=dev)
+        for g in (8, 4, 2, 1):
+            def route():
+                N.moe_route(T, cfg.H, E, k, cfg.n_group, g, N.MOE_SIGMOID, cfg.norm_topk_prob, cfg.scale,
+                            inp.x, inp.gate, bias, logits, ids, w, counts)
+            for _ in range(3):
+                route()
+            reps = 20
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for _ in range(reps):
+                route()
+            t1.record()
+            N.moe_bias_update(E, T, k, counts, bias, 0.0, cv)
+            N.moe_aux_loss(T, E, k, T, N.MOE_SIGMOID, logits, ids, 0.001, aux, ws)
+            torch.cuda.synchronize()
+            c = counts.cpu()
+            print(json.dumps({"sweep": "topk_group", "workload": name, "T": T, "E": E, "k": k,
+                              "n_group": cfg.n_group, "topk_group": g, "load_cv": round(cv.item(), 5),
+                              "max_load_over_mean": round(int(c.max()) * E / (T * k), 3),
+                              "hot_0_15_share": round(int(c[:16].sum()) / (T * k), 4),
+                              "aux_loss": float(f"{aux.item():.6g}"),
+                              "route_ms": round(t0.elapsed_time(t1) / reps, 4)}))
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.routing_sweep:
+        return run_routing_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -87,6 +87,30 @@ def test_route_from_logits_bit_exact(name, T):
     np.testing.assert_allclose(w.cpu().numpy(), r.weights, rtol=5e-6, atol=1e-7)
 
 
+@pytest.mark.parametrize("topk_group", [1, 2, 4, 8])
+def test_route_topk_group_sweep_bit_exact_with_load_cv(topk_group):
+    """The group-limit sweep at the V3 shape (8 groups): ids and counts
+    bit-exact for every topk_group, and the load CV of moe_bias_update (gamma
+    0: the bias stays) equal to the oracle's from the same integer counts."""
+    cfg = dataclasses.replace(get_config("v3"), topk_group=topk_group)
+    L = make_logits(cfg, device=DEV)
+    bias = uniform_bias(cfg.E, cfg.seed + 5)
+    ids, w, counts, _ = gpu_route(cfg, cfg.T, bias=bias, logits=L)
+    cv = torch.empty(1, dtype=torch.float32, device=DEV)
+    b = bias.clone()
+    N.moe_bias_update(cfg.E, cfg.T, cfg.k, counts, b, 0.0, cv)
+    torch.cuda.synchronize()
+    r = oracle_route(np32(L), cfg, np32(bias))
+    assert np.array_equal(ids.cpu().numpy(), r.ids)
+    assert np.array_equal(counts.cpu().numpy(), r.counts)
+    assert torch.equal(b, bias)
+    ref_cv = oracle.load_cv(r.counts)
+    print(f"topk_group={topk_group}: load CV {cv.item():.5f} (oracle {ref_cv:.5f})")
+    assert cv.item() == pytest.approx(ref_cv, rel=1e-6)
+    groups_used = (r.ids // (cfg.E // cfg.n_group))
+    assert max(len(set(row)) for row in groups_used.tolist()) <= topk_group
+
+
 @pytest.mark.parametrize("name,T", [("tiny", None), ("tiny_grouped", None), ("v2lite", None),
                                     ("v3", None), ("v3", 1000), ("v3", 1), ("v2lite", 129)])
 def test_route_gate_gemm(name, T):
