@@ -243,7 +243,7 @@ def stage_model(cfg):
     R = T * k
     ab = 1 if cfg.dtype == "e4m3" else 2
     return {
-        "route": {"flops": 2.0 * T * H * E, "bytes": T * H * 2 + E * H * 2 + R * 8},
+        "route": {"flops": 2.0 * T * H * E, "bytes": T * H * 2 + E * H * 2 + T * E * 4 + R * 8},
         "quantize_x": {"flops": 0.0, "bytes": T * H * 2 + T * H + T * (H // 128) * 4},
         "permute": {"flops": 0.0, "bytes": T * H * ab + R * H * ab + R * 8 + R * 12},
         "gate_up_routed": {"flops": 2.0 * R * H * 2 * I, "bytes": E * 2 * I * H * ab + R * H * ab + R * I * ab},
