@@ -215,9 +215,10 @@ def gemm_source_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
+def profiled_traffic(stage):
     """DRAM bytes per launch of the gate/up GEMM from the committed ncu
-    summary, only if the GEMM source has not changed since it was taken."""
+    summary, only if it was taken of this stage's launch and the GEMM source
+    has not changed since."""
     if not os.path.exists(PROFILE_TRAFFIC):
         return None
     kv = {}
@@ -225,7 +226,7 @@ def profiled_traffic():
         if ":" in line:
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
-    if kv.get("gemm_source_sha256_16") != gemm_source_hash():
+    if kv.get("gemm_source_sha256_16") != gemm_source_hash() or kv.get("stage") != stage:
         return None
     try:
         return float(kv["traffic_bytes_per_launch_full_size"])
@@ -234,7 +235,15 @@ def profiled_traffic():
 
 
 LAUNCHES = {"route": 2, "quantize_x": 1, "permute": 4, "gate_up_routed": 1, "down_routed": 1,
-            "gate_up_shared": 1, "down_shared": 1, "combine": 1, "bias_update": 1}
+            "gate_up_shared": 1, "down_shared": 1, "gate_up": 1, "down": 1, "combine": 1, "bias_update": 1}
+
+
+def launches_of(name, cfg):
+    """Kernel launches of one stage (the fused routed + shared GEMM stages run
+    as two launches for E4M3 layers)."""
+    if name in ("gate_up", "down") and cfg.dtype == "e4m3":
+        return 2
+    return LAUNCHES[name]
 
 
 def stage_model(cfg):
@@ -242,7 +251,7 @@ def stage_model(cfg):
     T, H, E, I, Is, k = cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_s, cfg.k
     R = T * k
     ab = 1 if cfg.dtype == "e4m3" else 2
-    return {
+    m = {
         "route": {"flops": 2.0 * T * H * E, "bytes": T * H * 2 + E * H * 2 + T * E * 4 + R * 8},
         "quantize_x": {"flops": 0.0, "bytes": T * H * 2 + T * H + T * (H // 128) * 4},
         "permute": {"flops": 0.0, "bytes": T * H * ab + R * H * ab + R * 8 + R * 12},
@@ -253,6 +262,10 @@ def stage_model(cfg):
         "combine": {"flops": 0.0, "bytes": R * H * 2 + T * H * 2 + T * H * 2 + R * 4},
         "bias_update": {"flops": 0.0, "bytes": E * 12},
     }
+    # routed + shared expert in one launch per GEMM
+    for fused, parts in (("gate_up", ("gate_up_routed", "gate_up_shared")), ("down", ("down_routed", "down_shared"))):
+        m[fused] = {key: sum(m[p][key] for p in parts) for key in ("flops", "bytes")}
+    return m
 
 
 def run_ours(args):
@@ -333,7 +346,7 @@ def run_ours(args):
     kernels = {}
     for n in names:
         m = model[n]
-        d = {"ms": round(avg[n], 4), "launches": LAUNCHES[n]}
+        d = {"ms": round(avg[n], 4), "launches": launches_of(n, cfg)}
         if m["flops"]:
             d["tflops"] = round(m["flops"] / (avg[n] * 1e-3) / 1e12, 1)
         d["gbs"] = round(m["bytes"] / (avg[n] * 1e-3) / 1e9, 1)
@@ -342,12 +355,13 @@ def run_ours(args):
     tokens = cfg.T * world * K
     value = tokens / (ms * 1e-3)
     flops_step = cfg.flops()
-    dom = "gate_up_routed"
+    dom = "gate_up" if "gate_up" in avg else "gate_up_routed"
     achieved = model[dom]["flops"] / (avg[dom] * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
-    roofline = {"kernel": "grouped_gemm_bf16 (gate/up + SwiGLU, routed experts)", "bound": "tensor",
+    what = "routed experts + shared expert, one launch" if dom == "gate_up" else "routed experts"
+    roofline = {"kernel": f"grouped_gemm_bf16 (gate/up + SwiGLU, {what})", "bound": "tensor",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(dom),
                 "peak_note": f"bf16 sustained, {peaks['source']} (MEASURED_PEAKS.json)",
                 "algorithmic_flops_per_launch": model[dom]["flops"],
                 "algorithmic_bytes_per_launch": model[dom]["bytes"]}
@@ -401,7 +415,7 @@ def run_ours(args):
                 "tflops": round(flops_step * world * K / (ms * 1e-3) / 1e12, 1),
                 "tflops_frac_of_measured_sustained": round(flops_step * world * K / (ms * 1e-3) / 1e12 / peak, 4),
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": K * sum(LAUNCHES[n] for n in names), "clocks": clk,
+                "gpu_launches": K * sum(launches_of(n, cfg) for n in names), "clocks": clk,
                 "device_status": status}
         print(json.dumps(line))
     if world > 1:

@@ -239,6 +239,35 @@ MOE_API moe_status moe_down_proj(int32_t rows, int32_t H, const moe_ffn_weights*
                          const void* h, const float* h_scale, const int32_t* offsets,
                          const float* row_w, void* out, int32_t* dev_status, void* stream);
 
+/* The routed experts and the shared expert in one launch per GEMM ([MoE-walk]
+ * §3.3: the routed experts as one grouped GEMM, the merged shared expert as
+ * one more group of all T rows), so the shared expert's tiles and the routed
+ * experts' ragged tiles share the persistent CTAs instead of each launch
+ * ending on its own partly idle last wave:
+ *   moe_gate_up_swiglu_with_shared: h_ws = SwiGLU of (a, w13) per segment
+ *       of offsets, and sh_h_ws = SwiGLU of (sh_a, sw13);
+ *   moe_down_proj_with_shared: out = row_w * (h w2^T) per segment, and
+ *       sh_out = sh_h sw2^T (weight 1).
+ * w: routed weights (groups = E), sw: shared weights (groups must be 1, same
+ * dtype; its I may differ from w's). rows / sh_rows: T*k / T. Other
+ * arguments, limits and errors as moe_gate_up_swiglu / moe_down_proj; E4M3
+ * scales as there (sh_a_scale / sh_h_scale for the shared rows). bf16 layers
+ * run as one launch; E4M3 layers (and MOE_GEMM_PAIR=1) as two launches of the
+ * same calls in this order. */
+MOE_API moe_status moe_gate_up_swiglu_with_shared(int32_t rows, int32_t H, const moe_ffn_weights* w,
+                              const void* a, const float* a_scale, const int32_t* offsets,
+                              void* h_ws, float* h_scale_ws,
+                              int32_t sh_rows, const moe_ffn_weights* sw,
+                              const void* sh_a, const float* sh_a_scale,
+                              void* sh_h_ws, float* sh_h_scale_ws,
+                              int32_t* dev_status, void* stream);
+MOE_API moe_status moe_down_proj_with_shared(int32_t rows, int32_t H, const moe_ffn_weights* w,
+                              const void* h, const float* h_scale, const int32_t* offsets,
+                              const float* row_w, void* out,
+                              int32_t sh_rows, const moe_ffn_weights* sw,
+                              const void* sh_h, const float* sh_h_scale, void* sh_out,
+                              int32_t* dev_status, void* stream);
+
 /* moe_gate_up_swiglu_gather -- the routed experts' first GEMM with the
  * permutation fused into its operand fetch ([MoE-walk] §3.2 + §3.3.1): row p
  * of the expert segments is read directly from x[src_token[p]], so

@@ -233,45 +233,80 @@ moe_status check_ffn(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
   return MOE_OK;
 }
 
-moe_status run_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a,
-                       const float* a_scale, const int32_t* offsets, void* h_ws, float* h_scale_ws,
-                       int32_t* dev_status, cudaStream_t st, int nsm) {
+// Tensor maps and kernel arguments of one grouped GEMM.
+struct GemmPlan {
+  CUtensorMap tmA;
+  TokenMaps tmB;
+  GemmArgs g;
+  bool fp8;
+};
+
+moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a, const float* a_scale,
+                        const int32_t* offsets, void* h_ws, float* h_scale_ws, int32_t* dev_status, GemmPlan* p) {
   const bool fp8 = w->dtype == MOE_E4M3;
   const bool pair = !fp8 && bf16_on_pairs();
   const int I = w->I;
-  CUtensorMap tmA;
-  TokenMaps tmB;
-  moe_status s = make_tmap(&tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, pair ? 64 : 128);
+  moe_status s = make_tmap(&p->tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, pair ? 64 : 128);
   if (s != MOE_OK) return s;
-  s = make_token_tmaps(&tmB, a, fp8, H, rows);
+  s = make_token_tmaps(&p->tmB, a, fp8, H, rows);
   if (s != MOE_OK) return s;
   const int nb = (fp8 || pair) ? 1 : one_cta_buffers(true);
-  GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : (nb == 2 ? 128 : 256),
-              pair ? 64 : 0, nb, 0, h_ws, I, nullptr, w->w13_scale, a_scale, h_scale_ws, dev_status};
-  return check_launch(launch_grouped_gemm(fp8, EPI_SWIGLU, tmA, tmB, g1, nsm, st));
+  p->g = GemmArgs{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : (nb == 2 ? 128 : 256),
+                  pair ? 64 : 0, nb, 0, h_ws, I, nullptr, w->w13_scale, a_scale, h_scale_ws, dev_status};
+  p->fp8 = fp8;
+  return MOE_OK;
+}
+
+moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* h, const float* h_scale,
+                     const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status, GemmPlan* p) {
+  const bool fp8 = w->dtype == MOE_E4M3;
+  const bool pair = !fp8 && bf16_on_pairs();
+  const int I = w->I;
+  // the single-CTA bf16 kernel reads its 256 contiguous w2 rows as one box
+  const bool one_box = !fp8;
+  moe_status s = make_tmap(&p->tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H,
+                           (fp8 || pair) ? 128 : 256);
+  if (s != MOE_OK) return s;
+  s = make_token_tmaps(&p->tmB, h, fp8, I, rows);
+  if (s != MOE_OK) return s;
+  const int nb = (fp8 || pair) ? 1 : one_cta_buffers(false);
+  p->g = GemmArgs{rows, I, w->groups, offsets, H, H / 256, 256, pair ? 64 : 128, 256, 128,
+                  fp8 ? 32 : (nb == 2 ? 128 : 256), pair ? 128 : 0, nb, one_box ? 1 : 0,
+                  out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
+  p->fp8 = fp8;
+  return MOE_OK;
+}
+
+moe_status launch_plan(const GemmPlan& p, int epi, cudaStream_t st, int nsm, const GemmPlan* second = nullptr) {
+  // one launch needs the same kernel form for both: single-CTA bf16, same tile shape
+  const bool one = second && !p.fp8 && !second->fp8 && p.g.cta_stride == 0 && second->g.cta_stride == 0 &&
+                   p.g.bn_max == second->g.bn_max && p.g.nbuf == second->g.nbuf;
+  if (second && !one) {
+    moe_status s = check_launch(launch_grouped_gemm(p.fp8, epi, p.tmA, p.tmB, p.g, nsm, st));
+    return s != MOE_OK ? s : check_launch(launch_grouped_gemm(second->fp8, epi, second->tmA, second->tmB,
+                                                              second->g, nsm, st));
+  }
+  if (!second) return check_launch(launch_grouped_gemm(p.fp8, epi, p.tmA, p.tmB, p.g, nsm, st));
+  const SecondProblem two{second->tmA, second->tmB, second->g};
+  return check_launch(launch_grouped_gemm(p.fp8, epi, p.tmA, p.tmB, p.g, nsm, st, &two));
+}
+
+moe_status run_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a,
+                       const float* a_scale, const int32_t* offsets, void* h_ws, float* h_scale_ws,
+                       int32_t* dev_status, cudaStream_t st, int nsm) {
+  GemmPlan p;
+  moe_status s = plan_gate_up(rows, H, w, a, a_scale, offsets, h_ws, h_scale_ws, dev_status, &p);
+  return s != MOE_OK ? s : launch_plan(p, EPI_SWIGLU, st, nsm);
 }
 
 moe_status run_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* h, const float* h_scale,
                     const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status,
                     cudaStream_t st, int nsm) {
-  const bool fp8 = w->dtype == MOE_E4M3;
-  const bool pair = !fp8 && bf16_on_pairs();
-  const int I = w->I;
-  CUtensorMap tmA;
-  TokenMaps tmB;
-  // the single-CTA bf16 kernel reads its 256 contiguous w2 rows as one box
-  const bool one_box = !fp8;
-  moe_status s = make_tmap(&tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H,
-                           (fp8 || pair) ? 128 : 256);
-  if (s != MOE_OK) return s;
-  s = make_token_tmaps(&tmB, h, fp8, I, rows);
-  if (s != MOE_OK) return s;
-  const int nb = (fp8 || pair) ? 1 : one_cta_buffers(false);
-  GemmArgs g2{rows, I, w->groups, offsets, H, H / 256, 256, pair ? 64 : 128, 256, 128,
-              fp8 ? 32 : (nb == 2 ? 128 : 256), pair ? 128 : 0, nb, one_box ? 1 : 0,
-              out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
-  return check_launch(launch_grouped_gemm(fp8, EPI_WEIGHTED, tmA, tmB, g2, nsm, st));
+  GemmPlan p;
+  moe_status s = plan_down(rows, H, w, h, h_scale, offsets, row_w, out, dev_status, &p);
+  return s != MOE_OK ? s : launch_plan(p, EPI_WEIGHTED, st, nsm);
 }
+
 
 }  // namespace
 
@@ -338,6 +373,51 @@ moe_status moe_grouped_swiglu(int32_t rows, int32_t H, const moe_ffn_weights* w,
   s = run_gate_up(rows, H, w, a, a_scale, offsets, h_ws, h_scale_ws, dev_status, st, nsm);
   if (s != MOE_OK) return s;
   return run_down(rows, H, w, h_ws, h_scale_ws, offsets, row_w, out, dev_status, st, nsm);
+}
+
+moe_status moe_gate_up_swiglu_with_shared(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a,
+                                          const float* a_scale, const int32_t* offsets, void* h_ws,
+                                          float* h_scale_ws, int32_t sh_rows, const moe_ffn_weights* sw,
+                                          const void* sh_a, const float* sh_a_scale, void* sh_h_ws,
+                                          float* sh_h_scale_ws, int32_t* dev_status, void* stream) {
+  moe_status s = check_ffn(rows, H, w, a, a_scale, true, false);
+  if (s != MOE_OK) return s;
+  if ((s = check_ffn(sh_rows, H, sw, sh_a, sh_a_scale, true, false)) != MOE_OK) return s;
+  if (!offsets || !h_ws || !sh_h_ws || sw->groups != 1 || sw->dtype != w->dtype) return MOE_ERR_INVALID_ARG;
+  if (w->dtype == MOE_E4M3 && (!h_scale_ws || !sh_h_scale_ws)) return MOE_ERR_INVALID_ARG;
+  if (any_misaligned(offsets, h_ws, h_scale_ws, sh_h_ws, sh_h_scale_ws)) return MOE_ERR_ALIGNMENT;
+  int nsm = 0;
+  if ((s = sm_count(&nsm)) != MOE_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  GemmPlan p, q;
+  if ((s = plan_gate_up(rows, H, w, a, a_scale, offsets, h_ws, h_scale_ws, dev_status, &p)) != MOE_OK) return s;
+  if ((s = plan_gate_up(sh_rows, H, sw, sh_a, sh_a_scale, nullptr, sh_h_ws, sh_h_scale_ws, dev_status, &q)) !=
+      MOE_OK)
+    return s;
+  if (!env_on("MOE_SHARED_APART")) return launch_plan(p, EPI_SWIGLU, st, nsm, &q);
+  if ((s = launch_plan(p, EPI_SWIGLU, st, nsm)) != MOE_OK) return s;
+  return launch_plan(q, EPI_SWIGLU, st, nsm);
+}
+
+moe_status moe_down_proj_with_shared(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* h,
+                                     const float* h_scale, const int32_t* offsets, const float* row_w, void* out,
+                                     int32_t sh_rows, const moe_ffn_weights* sw, const void* sh_h,
+                                     const float* sh_h_scale, void* sh_out, int32_t* dev_status, void* stream) {
+  moe_status s = check_ffn(rows, H, w, h, h_scale, false, true);
+  if (s != MOE_OK) return s;
+  if ((s = check_ffn(sh_rows, H, sw, sh_h, sh_h_scale, false, true)) != MOE_OK) return s;
+  if (!offsets || !out || !sh_out || sw->groups != 1 || sw->dtype != w->dtype) return MOE_ERR_INVALID_ARG;
+  if (any_misaligned(offsets, row_w, out, sh_out)) return MOE_ERR_ALIGNMENT;
+  int nsm = 0;
+  if ((s = sm_count(&nsm)) != MOE_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  GemmPlan p, q;
+  if ((s = plan_down(rows, H, w, h, h_scale, offsets, row_w, out, dev_status, &p)) != MOE_OK) return s;
+  if ((s = plan_down(sh_rows, H, sw, sh_h, sh_h_scale, nullptr, nullptr, sh_out, dev_status, &q)) != MOE_OK)
+    return s;
+  if (!env_on("MOE_SHARED_APART")) return launch_plan(p, EPI_WEIGHTED, st, nsm, &q);
+  if ((s = launch_plan(p, EPI_WEIGHTED, st, nsm)) != MOE_OK) return s;
+  return launch_plan(q, EPI_WEIGHTED, st, nsm);
 }
 
 moe_status moe_combine(int32_t T, int32_t k, int32_t H, const void* expert_out, const int32_t* slot_to_row,

@@ -95,18 +95,12 @@ __device__ void build_schedule(Sched& s, const GemmArgs& a, int lane) {
   }
 }
 
-__device__ __forceinline__ TileInfo decode_tile(const Sched& s, const GemmArgs& a, int t) {
-  int lo = 0, hi = a.groups - 1;   // last g with tile_start[g] <= t
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (s.tile_start[mid] <= t) lo = mid; else hi = mid - 1;
-  }
+// Tile `local` of a segment of n rows starting at row seg0 (group g).
+__device__ __forceinline__ TileInfo decode_in_segment(const GemmArgs& a, int g, int seg0, int n, int local) {
   TileInfo ti;
-  ti.g = lo;
-  const int n = s.seg_start[lo + 1] - s.seg_start[lo];
+  ti.g = g;
   const int ntb = (n + a.bn_max - 1) / a.bn_max;
   const int bn = ((((n + ntb - 1) / ntb) + 15) / 16) * 16;
-  const int local = t - s.tile_start[lo];
   const int chunk_tiles = kTbChunk * a.n_mblk;
   const int chunk = local / chunk_tiles;
   const int r = local - chunk * chunk_tiles;
@@ -114,10 +108,20 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, const GemmArgs& 
   ti.mb = r / c_tb;
   const int tb = chunk * kTbChunk + (r - ti.mb * c_tb);
   ti.ntb = ntb;
-  ti.row0 = s.seg_start[lo] + tb * bn;
+  ti.row0 = seg0 + tb * bn;
   ti.n_valid = min(bn, n - tb * bn);
   ti.N = ((ti.n_valid + 15) / 16) * 16;
   return ti;
+}
+
+__device__ __forceinline__ TileInfo decode_tile(const Sched& s, const GemmArgs& a, int t) {
+  int lo = 0, hi = a.groups - 1;   // last g with tile_start[g] <= t
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (s.tile_start[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  return decode_in_segment(a, lo, s.seg_start[lo], s.seg_start[lo + 1] - s.seg_start[lo],
+                           t - s.tile_start[lo]);
 }
 
 // Token rows of one stage (a multiple of 16, at most 256) are fetched with at
@@ -171,10 +175,15 @@ __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __e
 // async proxy; it keeps one stage of copies in flight ahead of that.
 constexpr int kGatherThreads = 64;
 
-template <int EPI, int STAGES, bool GATHER>
+// TWO: a second single-group problem a2 (the shared expert: its own weights
+// tmA2, token rows tmB2 and output) runs in the same launch. Its tiles come
+// first in the tile order, so the routed experts' ragged tiles fill the tail.
+template <int EPI, int STAGES, bool GATHER, bool TWO>
 __global__ void __launch_bounds__(kThreads + (GATHER ? kGatherThreads : 0), 1)
 grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
-                         const __grid_constant__ TokenMaps tmB, const GemmArgs a) {
+                         const __grid_constant__ TokenMaps tmB, const GemmArgs a,
+                         const __grid_constant__ CUtensorMap tmA2,
+                         const __grid_constant__ TokenMaps tmB2, const GemmArgs a2) {
   constexpr int KB = 64;                           // K elements per stage (128 B)
   constexpr uint32_t A_SUB_BYTES = 128 * 128;      // one 128-row sub-tile
   extern __shared__ __align__(1024) uint8_t dsmem[];
@@ -214,6 +223,10 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&tmB.box[i]);
+    if (TWO) {
+      tma_prefetch_desc(&tmA2);
+      for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&tmB2.box[i]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_s, 512);
@@ -224,8 +237,8 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
-  const int total = sched.tile_start[a.groups];
-  const int nk = a.K / KB;
+  const int total2 = TWO ? tiles_of(a2.rows, a.bn_max, a2.n_mblk) : 0;
+  const int total = total2 + sched.tile_start[a.groups];
 
   if (warp == 0) {
     if (lane == 0) {
@@ -235,22 +248,27 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       int stage = 0;
       uint32_t phase = 0;
       for (int t = blockIdx.x; t < total && !abort_flag; t += gridDim.x) {
-        const TileInfo ti = decode_tile(sched, a, t);
-        const int a_row0 = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride;
-        const int a_row1 = a_row0 + a.sub1_off;
+        const bool sh = TWO && t < total2;
+        const TileInfo ti = sh ? decode_in_segment(a2, 0, 0, a2.rows, t) : decode_tile(sched, a, t - total2);
+        const int nk = (sh ? a2.K : a.K) / KB;
+        const CUtensorMap* mA = sh ? &tmA2 : &tmA;
+        const TokenMaps* mB = sh ? &tmB2 : &tmB;
+        const int a_row0 = sh ? ti.mb * a2.mblk_stride : ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride;
+        const int a_row1 = a_row0 + (sh ? a2.sub1_off : a.sub1_off);
+        const bool one_box = sh ? a2.a_one_box != 0 : a.a_one_box != 0;
         const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;   // re-read by sibling token blocks
         const uint32_t bytes = 2 * A_SUB_BYTES + (GATHER ? 0u : static_cast<uint32_t>(ti.N) * 128u);
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
-          tma_load_2d(sA(stage, 0), &tmA, &full_bar[stage], kb * KB, a_row0, pol_w);
-          if (!a.a_one_box) tma_load_2d(sA(stage, 1), &tmA, &full_bar[stage], kb * KB, a_row1, pol_w);
+          tma_load_2d(sA(stage, 0), mA, &full_bar[stage], kb * KB, a_row0, pol_w);
+          if (!one_box) tma_load_2d(sA(stage, 1), mA, &full_bar[stage], kb * KB, a_row1, pol_w);
           if (!GATHER) {
             uint8_t* bdst = sB(stage);
             uint64_t* fb = &full_bar[stage];
             load_token_rows(ti.N, [&](int which, int off) {
-              tma_load_2d(bdst + off * 128, &tmB.box[which], fb, kb * KB, ti.row0 + off, pol_x);
+              tma_load_2d(bdst + off * 128, &mB->box[which], fb, kb * KB, ti.row0 + off, pol_x);
             });
           }
           issued_parity[stage] = static_cast<int>(phase);
@@ -267,6 +285,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     const int gt = threadIdx.x - kThreads;             // 0..63
     const int chunk = gt & 7;                          // 16-byte chunk of the 128-byte row slice
     const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.gather_src);
+    const int nk = a.K / KB;                          // (no second problem with GATHER)
     int stage = 0, pending = -1;
     uint32_t phase = 0;
     bool ok = true;
@@ -310,7 +329,9 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       int stage = 0;
       uint32_t phase = 0, it = 0;
       for (int t = blockIdx.x; t < total && !abort_flag; t += gridDim.x, ++it) {
-        const TileInfo ti = decode_tile(sched, a, t);
+        const bool sh = TWO && t < total2;
+        const TileInfo ti = sh ? decode_in_segment(a2, 0, 0, a2.rows, t) : decode_tile(sched, a, t - total2);
+        const int nk = (sh ? a2.K : a.K) / KB;
         const uint32_t idesc = make_idesc(1u, 128u, static_cast<uint32_t>(ti.N));
         const uint32_t bi = nbuf == 2 ? (it & 1u) : 0u, use = nbuf == 2 ? (it >> 1) : it;
         const uint32_t d0 = tmem_base + bi * 2u * sub_cols;
@@ -344,9 +365,14 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     const int q = warp & 3;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
     uint32_t it = 0;
-    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile(sched, a, t);
+      const bool sh = TWO && t < total2;
+      const TileInfo ti = sh ? decode_in_segment(a2, 0, 0, a2.rows, t) : decode_tile(sched, a, t - total2);
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(sh ? a2.out : a.out);
+      const size_t out_ld = sh ? a2.out_ld : a.out_ld;
+      const int feat_stride = sh ? a2.feat_stride : a.feat_stride;
+      const int feat_sub1 = sh ? a2.feat_sub1 : a.feat_sub1;
+      const float* row_w = sh ? a2.row_w : a.row_w;
       const uint32_t bi = nbuf == 2 ? (it & 1u) : 0u, use = nbuf == 2 ? (it >> 1) : it;
       if (!mbar_wait(&tmem_full[bi], use & 1u, &abort_flag, a.status)) break;
       tc_fence_after();
@@ -354,7 +380,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       const int nchunk = (ti.N + 31) / 32;
       __nv_bfloat16* stg = stage_out[q];
       if (EPI == EPI_SWIGLU) {
-        const int feat0 = ti.mb * a.feat_stride + 32 * q;          // this warp's 32 features
+        const int feat0 = ti.mb * feat_stride + 32 * q;            // this warp's 32 features
         for (int c = 0; c < nchunk; ++c) {
           float g[32], u[32];
           tmem_ld32(acc_addr + c * 32, g);
@@ -362,22 +388,22 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) g[j] = silu(g[j]) * u[j];
-          store_tile<32>(stg, g, lane, out, a.out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
+          store_tile<32>(stg, g, lane, out, out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
         }
       } else {
 #pragma unroll 1
         for (int s = 0; s < 2; ++s) {
-          const int feat0 = ti.mb * a.feat_stride + s * a.feat_sub1 + 32 * q;
+          const int feat0 = ti.mb * feat_stride + s * feat_sub1 + 32 * q;
           for (int c = 0; c < nchunk; ++c) {
             float v[32];
             tmem_ld32(acc_addr + s * sub_cols + c * 32, v);
             tmem_ld_wait();
-            if (a.row_w) {
-              const float wl = (c * 32 + lane < ti.n_valid) ? __ldg(a.row_w + ti.row0 + c * 32 + lane) : 0.0f;
+            if (row_w) {
+              const float wl = (c * 32 + lane < ti.n_valid) ? __ldg(row_w + ti.row0 + c * 32 + lane) : 0.0f;
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wl, j);
             }
-            store_tile<32>(stg, v, lane, out, a.out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
+            store_tile<32>(stg, v, lane, out, out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
           }
         }
       }
@@ -857,8 +883,16 @@ constexpr int kBf16Stages = 3;
 constexpr int kBf16StagesDb = 4;
 constexpr int kE4m3Stages = 4;
 
+using Bf16Kernel = void (*)(CUtensorMap, TokenMaps, GemmArgs, CUtensorMap, TokenMaps, GemmArgs);
+
+// The single-CTA bf16 kernel in its four forms: stages x (one problem | two).
+template <int EPI, int STAGES>
+Bf16Kernel bf16_kernel(bool two) {
+  return two ? grouped_gemm_bf16_kernel<EPI, STAGES, false, true> : grouped_gemm_bf16_kernel<EPI, STAGES, false, false>;
+}
+
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const TokenMaps& tmB,
-                                const GemmArgs& a, int grid, cudaStream_t stream) {
+                                const GemmArgs& a, int grid, cudaStream_t stream, const SecondProblem* two) {
   if (!e4m3 && a.cta_stride > 0) {
     const size_t smem = gemm_bf16_2sm_smem_bytes();
     auto kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_2sm_kernel<EPI_SWIGLU>
@@ -871,15 +905,23 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
     // two accumulators hold <= 128-token tiles: 48 KB stages, four of them
     const bool db = a.nbuf == 2 && !gather;
     const size_t smem = gemm_bf16_smem_bytes(db ? kBf16StagesDb : kBf16Stages, a.bn_max);
-    auto kern = db ? (epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16StagesDb, false>
-                                        : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16StagesDb, false>)
-              : gather ? (epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, true>
-                                            : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, true>)
-                       : (epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, false>
-                                            : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, false>);
+    const bool pair2 = two != nullptr && !gather;
+    Bf16Kernel kern;
+    if (gather)
+      kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, true, false>
+                               : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, true, false>;
+    else if (db)
+      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16StagesDb>(pair2)
+                               : bf16_kernel<EPI_WEIGHTED, kBf16StagesDb>(pair2);
+    else
+      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16Stages>(pair2)
+                               : bf16_kernel<EPI_WEIGHTED, kBf16Stages>(pair2);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads + (gather ? kGatherThreads : 0), smem, stream>>>(tmA, tmB, a);
+    if (pair2)
+      kern<<<grid, kThreads, smem, stream>>>(tmA, tmB, a, two->tmA, two->tmB, two->a);
+    else
+      kern<<<grid, kThreads + (gather ? kGatherThreads : 0), smem, stream>>>(tmA, tmB, a, tmA, tmB, a);
   } else {
     const size_t smem = gemm_e4m3_smem_bytes(kE4m3Stages);
     auto kern = epi == EPI_SWIGLU ? grouped_gemm_e4m3_kernel<EPI_SWIGLU, kE4m3Stages>

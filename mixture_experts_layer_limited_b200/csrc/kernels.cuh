@@ -57,8 +57,15 @@ struct TokenMaps {
   CUtensorMap box[kTokBoxes];
 };
 
+// A second single-group problem for the same launch (bf16, single-CTA kernel).
+struct SecondProblem {
+  CUtensorMap tmA;
+  TokenMaps tmB;
+  GemmArgs a;
+};
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const TokenMaps& tmB,
-                                const GemmArgs& a, int grid, cudaStream_t stream);
+                                const GemmArgs& a, int grid, cudaStream_t stream,
+                                const SecondProblem* two = nullptr);
 cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
                              cudaStream_t stream);
 cudaError_t launch_route_tokens(const RouteArgs& r, int num_sms, cudaStream_t stream);

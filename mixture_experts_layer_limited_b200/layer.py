@@ -39,12 +39,15 @@ class MoELayer:
 
     def __init__(self, spec: LayerSpec, gate: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
                  sw13: Optional[torch.Tensor], sw2: Optional[torch.Tensor],
-                 bias: Optional[torch.Tensor], T_max: int, gather: bool = False):
+                 bias: Optional[torch.Tensor], T_max: int, gather: bool = False,
+                 fuse_shared: bool = True):
         self.spec = spec
         # gather=True: bf16 layers read the routed experts' token rows straight
         # from x (the permutation fused into the first GEMM; no x_perm). At the
         # V3 shape on B200 the TMA path over x_perm is faster, so it is off.
         self.gather = gather and spec.dtype != "e4m3"
+        # fuse_shared: the shared expert's GEMMs share the routed experts' launches
+        self.fuse_shared = fuse_shared
         dev = gate.device
         self.dev = dev
         self.gate = gate.contiguous()
@@ -172,6 +175,28 @@ class MoELayer:
                         self.sh_o[:T], w2_scale=self.sw2_s,
                         h_scale=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status)
 
+    def gate_up_with_shared(self, x: torch.Tensor, T: int):
+        """Routed experts' and shared expert's first GEMM in one launch."""
+        s = self.spec
+        R = T * s.k
+        N.moe_gate_up_swiglu_with_shared(
+            R, s.H, self.w13, self._dt(), s.E, s.I, self.x_perm[:R], self.offsets, self.h[:R],
+            T, self.sw13, s.I_s, self.xq[:T] if self.fp8 else x, self.sh_h[:T],
+            w13_scale=self.w13_s, a_scale=self.x_perm_s[:R] if self.fp8 else None,
+            h_scale_ws=self.h_s[:R] if self.fp8 else None, sw13_scale=self.sw13_s,
+            sh_a_scale=self.xs[:T] if self.fp8 else None,
+            sh_h_scale_ws=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status)
+
+    def down_with_shared(self, T: int):
+        """Routed experts' and shared expert's second GEMM in one launch."""
+        s = self.spec
+        R = T * s.k
+        N.moe_down_proj_with_shared(
+            R, s.H, self.w2, self._dt(), s.E, s.I, self.h[:R], self.offsets, self.row_w[:R], self.o[:R],
+            T, self.sw2, s.I_s, self.sh_h[:T], self.sh_o[:T], w2_scale=self.w2_s,
+            h_scale=self.h_s[:R] if self.fp8 else None, sw2_scale=self.sw2_s,
+            sh_h_scale=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status)
+
     def combine(self, T: int):
         s = self.spec
         N.moe_combine(T, s.k, s.H, self.o[:T * s.k], self.slot_to_row[:T * s.k], None,
@@ -184,12 +209,17 @@ class MoELayer:
         st = [("route", lambda: self.route(x, write_logits))]
         if self.fp8:
             st.append(("quantize_x", lambda: self.quantize_x(x, T)))
-        st += [("permute", lambda: self.permute(x, T)),
-               ("gate_up_routed", lambda: self.experts_gate_up(T, x)),
-               ("down_routed", lambda: self.experts_down(T))]
-        if self.sh_h is not None:
-            st += [("gate_up_shared", lambda: self.shared_gate_up(x, T)),
-                   ("down_shared", lambda: self.shared_down(T))]
+        st.append(("permute", lambda: self.permute(x, T)))
+        if self.sh_h is not None and self.fuse_shared and not self.gather:
+            # routed + shared expert in one launch per GEMM
+            st += [("gate_up", lambda: self.gate_up_with_shared(x, T)),
+                   ("down", lambda: self.down_with_shared(T))]
+        else:
+            st += [("gate_up_routed", lambda: self.experts_gate_up(T, x)),
+                   ("down_routed", lambda: self.experts_down(T))]
+            if self.sh_h is not None:
+                st += [("gate_up_shared", lambda: self.shared_gate_up(x, T)),
+                       ("down_shared", lambda: self.shared_down(T))]
         st.append(("combine", lambda: self.combine(T)))
         return st
 

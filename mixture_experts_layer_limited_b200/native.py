@@ -29,6 +29,7 @@ EXPORTED = [
     "moe_route", "moe_permute_workspace_size", "moe_permute", "moe_permute_static_ws",
     "moe_grouped_swiglu",
     "moe_gate_up_swiglu", "moe_gate_up_swiglu_gather", "moe_down_proj",
+    "moe_gate_up_swiglu_with_shared", "moe_down_proj_with_shared",
     "moe_combine", "moe_bias_update", "moe_aux_loss_workspace_size", "moe_aux_loss",
     "moe_quantize_blocks", "moe_quantize_rows",
     "moe_read_device_status", "moe_last_cuda_error", "moe_status_string", "moe_abi_version",
@@ -79,6 +80,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_gate_up_swiglu": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P],
         "moe_down_proj": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P],
         "moe_gate_up_swiglu_gather": [_I, _I, ctypes.POINTER(FFNWeights), _P, _I, _P, _P, _P, _P, _P],
+        "moe_gate_up_swiglu_with_shared": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P,
+                                           _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P],
+        "moe_down_proj_with_shared": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P,
+                                      _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P],
         "moe_combine": [_I, _I, _I, _P, _P, _P, _P, _P, _P],
         "moe_bias_update": [_I, _I, _I, _P, _P, ctypes.c_float, _P, _P],
         "moe_aux_loss_workspace_size": [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
@@ -179,6 +184,29 @@ def moe_down_proj(rows, H, w2, dtype, groups, I, h, offsets, row_w, out, w2_scal
     w = FFNWeights(None, _ptr(w2), None, _ptr(w2_scale), dtype, groups, I)
     _check("moe_down_proj", load_library().moe_down_proj(
         rows, H, ctypes.byref(w), _ptr(h), _ptr(h_scale), _ptr(offsets), _ptr(row_w), _ptr(out),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_gate_up_swiglu_with_shared(rows, H, w13, dtype, groups, I, a, offsets, h_ws,
+                                   sh_rows, sw13, I_s, sh_a, sh_h_ws, w13_scale=None, a_scale=None,
+                                   h_scale_ws=None, sw13_scale=None, sh_a_scale=None, sh_h_scale_ws=None,
+                                   dev_status=None, stream=None):
+    w = FFNWeights(_ptr(w13), None, _ptr(w13_scale), None, dtype, groups, I)
+    sw = FFNWeights(_ptr(sw13), None, _ptr(sw13_scale), None, dtype, 1, I_s)
+    _check("moe_gate_up_swiglu_with_shared", load_library().moe_gate_up_swiglu_with_shared(
+        rows, H, ctypes.byref(w), _ptr(a), _ptr(a_scale), _ptr(offsets), _ptr(h_ws), _ptr(h_scale_ws),
+        sh_rows, ctypes.byref(sw), _ptr(sh_a), _ptr(sh_a_scale), _ptr(sh_h_ws), _ptr(sh_h_scale_ws),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_down_proj_with_shared(rows, H, w2, dtype, groups, I, h, offsets, row_w, out,
+                              sh_rows, sw2, I_s, sh_h, sh_out, w2_scale=None, h_scale=None,
+                              sw2_scale=None, sh_h_scale=None, dev_status=None, stream=None):
+    w = FFNWeights(None, _ptr(w2), None, _ptr(w2_scale), dtype, groups, I)
+    sw = FFNWeights(None, _ptr(sw2), None, _ptr(sw2_scale), dtype, 1, I_s)
+    _check("moe_down_proj_with_shared", load_library().moe_down_proj_with_shared(
+        rows, H, ctypes.byref(w), _ptr(h), _ptr(h_scale), _ptr(offsets), _ptr(row_w), _ptr(out),
+        sh_rows, ctypes.byref(sw), _ptr(sh_h), _ptr(sh_h_scale), _ptr(sh_out),
         _ptr(dev_status), _stream(stream)))
 
 

@@ -283,6 +283,50 @@ def test_grouped_swiglu_bf16(H, I, sizes, gemm_variant):
     assert eh < 1e-2 and eo < BF16_TOL
 
 
+@pytest.mark.parametrize("H,I,I_s,sizes,T", [
+    (512, 256, 384, [0, 17, 300, 5, 256, 0, 129], 300),
+    (7168, 2048, 2048, [300, 77, 512, 1], 1000),
+    (2048, 1408, 2816, [384, 0, 5, 513], 129),
+])
+def test_routed_and_shared_in_one_launch(H, I, I_s, sizes, T, gemm_variant):
+    """moe_*_with_shared: the routed segments and a shared FFN of T rows (its
+    own I_s, weight 1) in one launch per GEMM. Every output tile is computed as
+    in the separate launches, so the results must be bit-identical to them,
+    and within the bf16 tolerance of the oracle."""
+    G = len(sizes)
+    off = _segments(sizes)
+    R = int(off[-1])
+    g = _gen(H + I + I_s + T)
+    xp = torch.randn(R, H, generator=g, device=DEV).to(torch.bfloat16)
+    x = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
+    w13 = (torch.randn(G, 2 * I, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w2 = (torch.randn(G, H, I, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    sw13 = (torch.randn(1, 2 * I_s, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    sw2 = (torch.randn(1, H, I_s, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    row_w = torch.rand(R, generator=g, device=DEV) + 0.5
+    offd = torch.from_numpy(off).to(DEV)
+    e = lambda *shape: torch.empty(*shape, dtype=torch.bfloat16, device=DEV)
+    h, sh_h, o, sh_o = e(R, I), e(T, I_s), e(R, H), e(T, H)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    N.moe_gate_up_swiglu_with_shared(R, H, w13, N.MOE_BF16, G, I, xp, offd, h, T, sw13, I_s, x, sh_h,
+                                     dev_status=status)
+    N.moe_down_proj_with_shared(R, H, w2, N.MOE_BF16, G, I, h, offd, row_w, o, T, sw2, I_s, sh_h, sh_o,
+                                dev_status=status)
+    h2, sh_h2, o2, sh_o2 = e(R, I), e(T, I_s), e(R, H), e(T, H)
+    N.moe_gate_up_swiglu(R, H, w13, N.MOE_BF16, G, I, xp, offd, h2)
+    N.moe_gate_up_swiglu(T, H, sw13, N.MOE_BF16, 1, I_s, x, None, sh_h2)
+    N.moe_down_proj(R, H, w2, N.MOE_BF16, G, I, h2, offd, row_w, o2)
+    N.moe_down_proj(T, H, sw2, N.MOE_BF16, 1, I_s, sh_h2, None, None, sh_o2)
+    assert N.moe_read_device_status(status) == 0
+    for got, sep, name in ((h, h2, "h"), (sh_h, sh_h2, "shared h"), (o, o2, "out"), (sh_o, sh_o2, "shared out")):
+        assert torch.equal(got, sep), f"{gemm_variant}: {name} differs from the separate launches"
+    ref, href = _ref_grouped(xp, w13, w2, off, row_w)
+    sref, shref = _ref_grouped(x, sw13, sw2, np.array([0, T], np.int32), None)
+    errs = [rel_err(np64(h), href), rel_err(np64(o), ref), rel_err(np64(sh_h), shref), rel_err(np64(sh_o), sref)]
+    print(f"{gemm_variant} H={H} I={I} I_s={I_s}: errors {[f'{v:.2e}' for v in errs]}")
+    assert errs[0] < 1e-2 and errs[2] < 1e-2 and errs[1] < BF16_TOL and errs[3] < BF16_TOL
+
+
 def test_grouped_swiglu_bf16_single_group_no_offsets(gemm_variant):
     rows, H, I = 300, 512, 384
     g = _gen(77)

@@ -189,3 +189,20 @@ def test_layer_gather_variant_matches_default():
     torch.cuda.synchronize()
     assert lay.device_status() == 0
     assert torch.equal(y0, y1)
+
+
+@pytest.mark.parametrize("name", ["v2lite", "v3"])
+def test_layer_shared_expert_in_routed_launches_matches_separate(name):
+    """The shared expert run inside the routed experts' launches (the default)
+    gives the same layer output as its own launches, bit for bit."""
+    cfg = get_config(name, T=1024)
+    inp = make_inputs(cfg, device=DEV)
+    fused = _layer(cfg, inp)
+    assert fused.fuse_shared
+    y0 = fused.forward(inp.x).clone()
+    apart = MoELayer(LayerSpec.from_config(cfg), inp.gate, inp.w13, inp.w2, inp.sw13, inp.sw2,
+                     inp.bias, cfg.T, fuse_shared=False)
+    y1 = apart.forward(inp.x)
+    torch.cuda.synchronize()
+    assert fused.device_status() == 0 and apart.device_status() == 0
+    assert torch.equal(y0, y1)
