@@ -365,6 +365,15 @@ def run_ours(args):
                 "peak_note": f"bf16 sustained, {peaks['source']} (MEASURED_PEAKS.json)",
                 "algorithmic_flops_per_launch": model[dom]["flops"],
                 "algorithmic_bytes_per_launch": model[dom]["bytes"]}
+    if cfg.dtype == "e4m3":
+        # E4M3 decode: every expert's weights stream once for a few tokens each
+        gbs = model[dom]["bytes"] / (avg[dom] * 1e-3) / 1e9
+        roofline = {"kernel": f"grouped_gemm_e4m3 (gate/up + SwiGLU, {what})", "bound": "hbm",
+                    "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                    "peak_note": f"HBM copy, {peaks['source']} (MEASURED_PEAKS.json)",
+                    "algorithmic_flops_per_launch": model[dom]["flops"],
+                    "algorithmic_bytes_per_launch": model[dom]["bytes"]}
 
     # ---- end to end: host x -> device, forward + bias step, y -> host
     x_host = inp.x.cpu().pin_memory()
