@@ -274,7 +274,7 @@ def run_ours(args):
     import torch.distributed as dist
     from datetime import timedelta
     from moe_inputs import get_config, make_inputs
-    from mixture_experts_layer_limited_b200 import MoELayer, LayerSpec, load_library
+    from mixture_experts_layer_limited_b200 import MoELayer, LayerSpec, HostPipeline, load_library
     from mixture_experts_layer_limited_b200 import dist as mdist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -375,36 +375,38 @@ def run_ours(args):
                     "algorithmic_flops_per_launch": model[dom]["flops"],
                     "algorithmic_bytes_per_launch": model[dom]["bytes"]}
 
-    # ---- end to end: host x -> device, forward + bias step, y -> host
-    x_host = inp.x.cpu().pin_memory()
-    y_host = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(inp.x)
-    stages_e2e = layer.stages(x_dev)
+    # ---- end to end: host x -> device, forward + bias step, y -> host. Each
+    # step copies its batch in from pinned host memory and its output back out;
+    # HostPipeline overlaps those copies with the neighbouring steps' compute.
+    g = torch.Generator(device="cuda")
+    g.manual_seed(cfg.seed + 4242 + rank)
+    x_hosts = [inp.x.cpu().pin_memory(),
+               torch.randn(cfg.T, cfg.H, generator=g, device="cuda").to(torch.bfloat16).cpu().pin_memory()]
+    y_hosts = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    pipe = HostPipeline(layer, cfg.T)
 
-    def step_e2e():
-        x_dev.copy_(x_host, non_blocking=True)
-        for _, run in stages_e2e:
-            run()
+    def bias_after(_i):
         if layer.bias is not None:
             mdist.allreduce_counts_(layer.counts)
             layer.bias_step(T_global, cfg.gamma, load_cv=False)
-        y_host.copy_(layer.y[:cfg.T], non_blocking=True)
 
-    for _ in range(3):
-        step_e2e()
+    def run_e2e(n):
+        pipe.run([x_hosts[i % 2] for i in range(n)], [y_hosts[i % 2] for i in range(n)], bias_after)
+
+    run_e2e(3)
     torch.cuda.synchronize()
     mdist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(K):
-        step_e2e()
+    run_e2e(K)
     e1.record(stream)
     torch.cuda.synchronize()
     mdist.barrier()
     ms_e2e = mdist.max_over_ranks(e0.elapsed_time(e1), device="cuda")
     e2e = {"value": cfg.T * world * K / (ms_e2e * 1e-3), "unit": "tokens/s",
            "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2,
-           "path": "MoELayer stages through the C ABI; pinned host x in, pinned host y out"}
+           "path": "HostPipeline over MoELayer (C ABI): per step pinned host x in and y out, "
+                   "copies on two streams overlapped with the neighbouring steps"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -206,3 +206,37 @@ def test_layer_shared_expert_in_routed_launches_matches_separate(name):
     torch.cuda.synchronize()
     assert fused.device_status() == 0 and apart.device_status() == 0
     assert torch.equal(y0, y1)
+
+
+@pytest.mark.parametrize("name", ["v2lite", "v3"])
+def test_host_pipeline_matches_one_forward_at_a_time(name):
+    """HostPipeline overlaps each batch's copies with its neighbours' compute;
+    every output must equal the plain forward of that batch, bit for bit,
+    also with a bias step between forwards."""
+    from mixture_experts_layer_limited_b200 import HostPipeline
+    cfg = get_config(name, T=1024)
+    inp = make_inputs(cfg, device=DEV)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(77)
+    xs = [torch.randn(cfg.T, cfg.H, generator=g, device=DEV).to(torch.bfloat16) for _ in range(5)]
+    with_bias = inp.bias is not None
+
+    ref_layer = _layer(cfg, inp)
+    refs = []
+    for x in xs:
+        refs.append(ref_layer.forward(x).clone())
+        if with_bias:
+            ref_layer.bias_step(cfg.T, cfg.gamma, load_cv=False)
+
+    layer = _layer(cfg, inp)
+    pipe = HostPipeline(layer, cfg.T)
+    x_host = [x.cpu().pin_memory() for x in xs]
+    y_host = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory() for _ in xs]
+    step = (lambda i: layer.bias_step(cfg.T, cfg.gamma, load_cv=False)) if with_bias else None
+    pipe.run(x_host, y_host, step)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    for i, (y, r) in enumerate(zip(y_host, refs)):
+        assert torch.equal(y, r.cpu()), f"batch {i} differs"
+    if with_bias:
+        assert torch.equal(layer.bias, ref_layer.bias)
