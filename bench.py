@@ -234,7 +234,7 @@ def profiled_traffic(stage):
         return None
 
 
-LAUNCHES = {"route": 2, "quantize_x": 1, "permute": 4, "gate_up_routed": 1, "down_routed": 1,
+LAUNCHES = {"route": 2, "quantize_x": 1, "permute": 3, "gate_up_routed": 1, "down_routed": 1,
             "gate_up_shared": 1, "down_shared": 1, "gate_up": 1, "down": 1, "combine": 1, "bias_update": 1}
 
 

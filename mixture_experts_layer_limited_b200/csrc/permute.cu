@@ -5,16 +5,13 @@
 // example there orders each expert's segment by ascending token index and
 // gives expert_first_token_offset as the segment boundaries. That is a stable
 // counting sort of the T*k (token, slot) pairs keyed by expert, done here in
-// four launches:
+// three launches:
 //   1. perm_hist  : per block of kTokBlock tokens, an expert histogram;
 //   2. perm_scan  : expert offsets (exclusive scan of the totals) and, per
 //                   block, the first row of each expert's part of the segment;
-//   3. perm_rank  : per block, one warp walks the slots in token order and
-//                   gives each its row (warp match on equal experts ranks the
-//                   32 slots of a step at once);
-//   4. perm_copy  : one warp per token reads the token's row once and writes
-//                   it to its k rows with 16-byte vector loads and stores
-//                   (fp8 rows also carry their 1x128 scales).
+//   3. perm_place : one warp per token ranks its slots among the earlier
+//                   slots of its block (ballots), writes the metadata, reads
+//                   the token's row once and writes it to its k rows.
 #include "kernels.cuh"
 
 namespace moe {
@@ -104,58 +101,70 @@ perm_scan_kernel(int32_t* __restrict__ blockhist, int nb, int E, int total,
   }
 }
 
-// One warp per block of kTokBlock tokens.
-__global__ void __launch_bounds__(32)
-perm_rank_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T, int k,
-                 int E, const int32_t* __restrict__ blockbase, int32_t* __restrict__ slot_to_row,
-                 int32_t* __restrict__ src_token, float* __restrict__ row_w) {
-  extern __shared__ int cnt[];
-  const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) cnt[e] = blockbase[static_cast<size_t>(blockIdx.x) * E + e];
-  __syncwarp();
-  const int s0 = blockIdx.x * kTokBlock * k;
-  const int s1 = min(T, (blockIdx.x + 1) * kTokBlock) * k;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = s0; base < s1; base += 32) {
-    const int s = base + lane;
-    int e = -1;
-    if (s < s1) {
-      e = ids[s];
-      if (e < 0 || e >= E) e = -2 - lane;   // unique key: never grouped, never counted
-    } else {
-      e = -2 - lane;
-    }
-    const unsigned grp = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(grp & lt_mask);
-    const bool valid = e >= 0;
-    const int base_row = valid ? cnt[e] : 0;
-    __syncwarp();
-    if (valid && lane == 31 - __clz(grp)) cnt[e] = base_row + __popc(grp);
-    __syncwarp();
-    if (valid) {
-      const int r = base_row + rank;
-      slot_to_row[s] = r;
-      src_token[r] = s / k;
-      if (row_w) row_w[r] = topk_w[s];
-    } else if (s < s1) {
-      slot_to_row[s] = -1;                   // id out of range (flagged by perm_hist)
-    }
-  }
-}
-
-// One warp per token: x[t] -> x_perm[slot_to_row[t*k + j]] for j < k.
+// One warp per token t: its rows, then the copies.
+//   row of slot (t, j) = first row of (block of t, expert e) from perm_scan
+//                        + the number of earlier slots of the block with expert e
+// (token order, then slot order: the stable counting sort). The warp counts
+// the earlier slots 32 at a time with one ballot per slot of t, writes
+// slot_to_row / src_token / row_w, reads the token's row once and writes it
+// to its k rows with 16-byte vector loads and stores (fp8 rows also carry
+// their 1x128 scales). Slots with ids outside [0, E) get row -1 (flagged by
+// perm_hist) and are not written.
 constexpr int kPermKMax = 16;
 
 __global__ void __launch_bounds__(256)
-perm_copy_kernel(const uint4* __restrict__ x, int T, int k, int vec_per_row,
-                 const int32_t* __restrict__ slot_to_row, uint4* __restrict__ x_perm,
-                 const float* __restrict__ x_scale, float* __restrict__ x_perm_scale, int nscale) {
+perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T, int k, int E,
+                  const int32_t* __restrict__ blockbase, int32_t* __restrict__ slot_to_row,
+                  int32_t* __restrict__ src_token, float* __restrict__ row_w,
+                  const uint4* __restrict__ x, int vec_per_row, uint4* __restrict__ x_perm,
+                  const float* __restrict__ x_scale, float* __restrict__ x_perm_scale, int nscale) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;                                  // warp-uniform
   const int nrows = T * k;
-  int my_row = lane < k ? slot_to_row[static_cast<size_t>(t) * k + lane] : -1;
-  if (my_row >= nrows) my_row = -1;                   // never write outside x_perm
+  const int b = t / kTokBlock;
+  const size_t s_me = static_cast<size_t>(t) * k;
+  int my_e = -1;
+  if (lane < k) {
+    my_e = ids[s_me + lane];
+    if (my_e < 0 || my_e >= E) my_e = -1;
+  }
+  // earlier slots of the block with my expert
+  int cnt = 0;
+  const size_t s_blk = static_cast<size_t>(b) * kTokBlock * k;
+  for (size_t base = s_blk; base < s_me; base += 32) {  // same trip count on every lane
+    const size_t s = base + lane;
+    const int e = s < s_me ? ids[s] : -1;
+#pragma unroll
+    for (int j = 0; j < kPermKMax; ++j) {
+      if (j < k) {
+        const int ej = __shfl_sync(0xffffffffu, my_e, j);
+        const int c = __popc(__ballot_sync(0xffffffffu, ej >= 0 && e == ej));
+        if (lane == j) cnt += c;
+      }
+    }
+  }
+  // earlier slots of this token with the same expert (repeated ids)
+#pragma unroll
+  for (int j = 0; j < kPermKMax; ++j) {
+    if (j < k) {
+      const int ej = __shfl_sync(0xffffffffu, my_e, j);
+      if (j < lane && ej == my_e) ++cnt;
+    }
+  }
+  int my_row = -1;
+  if (lane < k && my_e >= 0) {
+    my_row = blockbase[static_cast<size_t>(b) * E + my_e] + cnt;
+    if (my_row >= nrows) my_row = -1;                 // never write outside the rows
+  }
+  if (lane < k) {
+    slot_to_row[s_me + lane] = my_row;
+    if (my_row >= 0) {
+      src_token[my_row] = t;
+      if (row_w) row_w[my_row] = topk_w[s_me + lane];
+    }
+  }
+  if (!x_perm) return;                                 // metadata only
   int rows[kPermKMax];
 #pragma unroll
   for (int j = 0; j < kPermKMax; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
@@ -204,14 +213,10 @@ cudaError_t launch_permute(int T, int k, int E, int row_bytes, const int32_t* id
   const int parts = 1024 / E;
   const size_t scan_smem = (static_cast<size_t>(parts) * E + E + 32) * sizeof(int);
   perm_scan_kernel<<<1, 1024, scan_smem, stream>>>(blockhist, nb, E, T * k, offsets);
-  perm_rank_kernel<<<nb, 32, E * sizeof(int), stream>>>(ids, topk_w, T, k, E, blockhist, slot_to_row,
-                                                       src_token, row_w);
-  if (x_perm) {
-    const int warps = 8;
-    perm_copy_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
-        reinterpret_cast<const uint4*>(x), T, k, row_bytes / 16, slot_to_row,
-        reinterpret_cast<uint4*>(x_perm), x_scale, x_perm_scale, nscale);
-  }
+  const int warps = 8;
+  perm_place_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
+      ids, topk_w, T, k, E, blockhist, slot_to_row, src_token, row_w, reinterpret_cast<const uint4*>(x),
+      row_bytes / 16, reinterpret_cast<uint4*>(x_perm), x_scale, x_perm_scale, nscale);
   return cudaGetLastError();
 }
 
