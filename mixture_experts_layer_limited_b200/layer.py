@@ -229,6 +229,29 @@ class MoELayer:
             run()
         return self.y[:x.shape[0]]
 
+    def capture(self, x: torch.Tensor, bias_gamma: Optional[float] = None):
+        """Records the forward on the rows of x (and, with bias_gamma, the
+        bias step after it) as one CUDA graph; returns the function that
+        replays it on the current stream. The graph keeps x's and the layer's
+        buffers: refill x in place between replays. Every launch of the
+        forward is one node, so a replay costs one launch on the host."""
+        T = x.shape[0]
+        stages = self.stages(x)
+        side = torch.cuda.Stream(device=self.dev)
+        side.wait_stream(torch.cuda.current_stream(self.dev))
+        with torch.cuda.stream(side):                   # first run outside the capture
+            for _, run in stages:
+                run()
+        torch.cuda.current_stream(self.dev).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _, run in stages:
+                run()
+            if bias_gamma is not None:
+                self.bias_step(T, bias_gamma, load_cv=False)
+        self._graphs = getattr(self, "_graphs", []) + [graph]   # kept alive with the layer
+        return graph.replay
+
     def bias_step(self, T: int, gamma: float, load_cv: bool = True):
         """Aux-loss-free bias update from the last forward's expert counts."""
         s = self.spec

@@ -240,3 +240,93 @@ def test_host_pipeline_matches_one_forward_at_a_time(name):
         assert torch.equal(y, r.cpu()), f"batch {i} differs"
     if with_bias:
         assert torch.equal(layer.bias, ref_layer.bias)
+
+
+def _run_from_logits(layer, x, L):
+    """The forward with routing taken from the given fp32 logits."""
+    T = x.shape[0]
+    layer.route(x, logits_in=L)
+    for name, run in layer.stages(x)[1:]:
+        run()
+    return layer.y[:T]
+
+
+@pytest.mark.parametrize("name", ["v2lite", "v3"])
+def test_layer_collapsed_routing(name):
+    """Degenerate load: every token picks the same k experts (the other
+    experts get no rows at all; the k segments hold T rows each, several
+    token blocks). Through the permutation, both grouped GEMMs and combine."""
+    cfg = get_config(name, T=512 if name == "v2lite" else 256)
+    inp = make_inputs(cfg, device=DEV)
+    layer = _layer(cfg, inp)
+    L = torch.full((cfg.T, cfg.E), -8.0, dtype=torch.float32, device=DEV)
+    hot = torch.arange(cfg.k, device=DEV)                 # inside the first group
+    L[:, hot] = 8.0 + torch.arange(cfg.k, device=DEV, dtype=torch.float32) * 0.25
+    y = _run_from_logits(layer, inp.x, L)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    counts = layer.counts.cpu().numpy()
+    assert sorted(np.nonzero(counts)[0].tolist()) == sorted(hot.cpu().tolist())
+    assert np.all(counts[hot.cpu().numpy()] == cfg.T)
+    _check_permutation_properties(layer, cfg.T, cfg.k, cfg.E)
+    bias = np32(inp.bias) if inp.bias is not None else None
+    r = oracle_route(np32(L), cfg, bias)
+    assert np.array_equal(layer.ids[:cfg.T].cpu().numpy(), r.ids)
+    rng = np.random.default_rng(5)
+    feats = np.sort(rng.choice(cfg.H, 256, replace=False))
+    ew = lambda e: (np32(inp.w13[e]), np32(inp.w2[e]))
+    shared = (np32(inp.sw13), np32(inp.sw2)) if inp.sw13 is not None else None
+    yref = oracle.moe_forward(np64(inp.x), r, ew, shared, out_features=feats)
+    err = rel_err(np64(y[:, torch.as_tensor(feats, device=DEV)]), yref)
+    print(f"{name} collapsed routing: err {err:.2e}")
+    assert err < BF16_TOL
+
+
+@pytest.mark.parametrize("name", ["tiny", "v3"])
+def test_layer_single_token(name):
+    """T = 1: every routed segment has one row or none."""
+    cfg = get_config(name, T=1)
+    inp = make_inputs(cfg, device=DEV)
+    layer = _layer(cfg, inp)
+    y = layer.forward(inp.x)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    _check_permutation_properties(layer, 1, cfg.k, cfg.E)
+    r, yref = _oracle_tokens(cfg, inp, np.arange(1))
+    assert not (near_tie_mask(r)[0]) and np.array_equal(np.sort(layer.ids[:1].cpu().numpy()), np.sort(r.ids))
+    err = rel_err(np64(y), yref)
+    print(f"{name} T=1: err {err:.2e}")
+    assert err < BF16_TOL
+
+
+@pytest.mark.parametrize("name", ["tiny", "v3"])
+def test_layer_cuda_graph_replay_matches_eager(name):
+    """The forward (+ bias step) captured as one CUDA graph gives the eager
+    results, bit for bit, over several replays with new inputs."""
+    cfg = get_config(name, T=64 if name == "tiny" else 1024)
+    inp = make_inputs(cfg, device=DEV)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(3)
+    xs = [torch.randn(cfg.T, cfg.H, generator=g, device=DEV).to(torch.bfloat16) for _ in range(3)]
+    gamma = cfg.gamma if inp.bias is not None else None
+    eager = _layer(cfg, inp)
+    refs = []
+    for x in xs:
+        refs.append(eager.forward(x).clone())
+        if gamma is not None:
+            eager.bias_step(cfg.T, gamma, load_cv=False)
+    layer = _layer(cfg, inp)
+    x_in = torch.empty_like(xs[0])
+    x_in.copy_(xs[0])
+    replay = layer.capture(x_in, gamma)
+    # capture ran the forward once outside the graph (no bias step): start over
+    if gamma is not None:
+        layer.bias.copy_(inp.bias)
+    for x, r in zip(xs, refs):
+        x_in.copy_(x)
+        replay()
+        torch.cuda.synchronize()
+        assert torch.equal(layer.y[:cfg.T], r)
+    assert layer.device_status() == 0
+    if gamma is not None:
+        assert torch.equal(layer.bias, eager.bias)
