@@ -50,9 +50,16 @@ perm_scan_kernel(int32_t* __restrict__ blockhist, int nb, int E, int total,
   const bool active = part < parts;
   const int per = (nb + parts - 1) / parts;
   const int b0 = min(nb, part * per), b1 = min(nb, b0 + per);
+  constexpr int kChunk = 16;                        // independent loads in flight per thread
   if (active) {
     int s = 0;
-    for (int b = b0; b < b1; ++b) s += blockhist[static_cast<size_t>(b) * E + e];
+    for (int c = b0; c < b1; c += kChunk) {
+      int v[kChunk];
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i) v[i] = c + i < b1 ? blockhist[static_cast<size_t>(c + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i) s += v[i];
+    }
     part_sum[part * E + e] = s;
   }
   __syncthreads();
@@ -92,11 +99,15 @@ perm_scan_kernel(int32_t* __restrict__ blockhist, int nb, int E, int total,
   if (active) {
     int run = tot[e];
     for (int p = 0; p < part; ++p) run += part_sum[p * E + e];
-    for (int b = b0; b < b1; ++b) {
-      const size_t i = static_cast<size_t>(b) * E + e;
-      const int c = blockhist[i];
-      blockhist[i] = run;
-      run += c;
+    for (int c = b0; c < b1; c += kChunk) {
+      int v[kChunk];
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i) v[i] = c + i < b1 ? blockhist[static_cast<size_t>(c + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i) {
+        if (c + i < b1) blockhist[static_cast<size_t>(c + i) * E + e] = run;
+        run += v[i];
+      }
     }
   }
 }
@@ -183,7 +194,7 @@ perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ top
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int v = base + u * 32 + lane;
-          if (v < vec_per_row) dst[v] = val[u];
+          if (v < vec_per_row) __stcs(dst + v, val[u]);        // streamed: x_perm is far larger than L2
         }
       }
     }
