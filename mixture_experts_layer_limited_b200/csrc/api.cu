@@ -108,9 +108,9 @@ bool env_on(const char* name) {
 // accumulators so the epilogue of one tile overlaps the MMAs of the next.
 // MOE_GEMM_PAIR=1 / MOE_GEMM_1SM=1 force CTA pairs / single CTAs for both;
 // MOE_GEMM_DB=1 / MOE_GEMM_SB=1 force two / one accumulators on single CTAs.
-bool bf16_on_pairs() {
+bool bf16_on_pairs(bool gate_up) {
   if (env_on("MOE_GEMM_1SM")) return false;
-  return env_on("MOE_GEMM_PAIR");
+  return env_on("MOE_GEMM_PAIR") || (!gate_up && env_on("MOE_GEMM_PAIR_DOWN"));
 }
 int one_cta_buffers(bool gate_up) {
   if (env_on("MOE_GEMM_DB")) return 2;
@@ -244,7 +244,7 @@ struct GemmPlan {
 moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a, const float* a_scale,
                         const int32_t* offsets, void* h_ws, float* h_scale_ws, int32_t* dev_status, GemmPlan* p) {
   const bool fp8 = w->dtype == MOE_E4M3;
-  const bool pair = !fp8 && bf16_on_pairs();
+  const bool pair = !fp8 && bf16_on_pairs(true);
   const int I = w->I;
   moe_status s = make_tmap(&p->tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, pair ? 64 : 128);
   if (s != MOE_OK) return s;
@@ -260,7 +260,7 @@ moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const
 moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* h, const float* h_scale,
                      const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status, GemmPlan* p) {
   const bool fp8 = w->dtype == MOE_E4M3;
-  const bool pair = !fp8 && bf16_on_pairs();
+  const bool pair = !fp8 && bf16_on_pairs(false);
   const int I = w->I;
   // the single-CTA bf16 kernel reads its 256 contiguous w2 rows as one box
   const bool one_box = !fp8;

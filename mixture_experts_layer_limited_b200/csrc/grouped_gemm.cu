@@ -432,7 +432,8 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
 //          warps of lanes 64..127 pass the up values through shared memory
 //          to the warps of lanes 0..63, which compute SiLU(gate) * up.
 //   GEMM2: CTA r holds w2 rows [mb*256 + 128r, +128).
-constexpr int k2smStages = 6;
+constexpr int k2smStages = 3;
+constexpr int k2smChunks = 2;              // 64-K chunks per stage: 128 K, 64 KB a stage per CTA
 constexpr int kXStride = 33;               // padded row of the lane exchange buffer
 
 template <int EPI>
@@ -440,10 +441,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ TokenMaps tmB, const GemmArgs a) {
   constexpr int KB = 64;
+  constexpr int KC = k2smChunks;
   constexpr int STAGES = k2smStages;
   constexpr uint32_t A_BYTES = 128 * 128;       // this CTA's 128 weight rows x 64 K
   constexpr uint32_t B_BYTES = 128 * 128;       // up to 128 token rows x 64 K
-  constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t CHUNK_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t STAGE_BYTES = KC * CHUNK_BYTES;
   extern __shared__ __align__(1024) uint8_t dsmem[];
   __shared__ Sched sched;
   __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
@@ -460,8 +463,8 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
   const int pair = static_cast<int>(cluster_id_x());
   const int npairs = static_cast<int>(nclusters_x());
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
-  auto sA = [&](int st) { return smem + st * STAGE_BYTES; };
-  auto sB = [&](int st) { return smem + st * STAGE_BYTES + A_BYTES; };
+  auto sA = [&](int st, int c) { return smem + st * STAGE_BYTES + c * CHUNK_BYTES; };
+  auto sB = [&](int st, int c) { return smem + st * STAGE_BYTES + c * CHUNK_BYTES + A_BYTES; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -505,22 +508,26 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
         const TileInfo ti = decode_tile(sched, a, t);
         const int half = ti.N >> 1;                       // tokens staged by each CTA
         const int rows = (half + 15) & ~15;               // rows fetched (multiple of 16)
-        const uint32_t tx = 2u * (A_BYTES + static_cast<uint32_t>(rows) * 128u);
+        const uint32_t tx = 2u * KC * (A_BYTES + static_cast<uint32_t>(rows) * 128u);
         const int a_lo = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride + static_cast<int>(rank) * a.cta_stride;
         const int a_hi = a_lo + a.sub1_off;
         const int b0 = ti.row0 + static_cast<int>(rank) * half;
         const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int ks = 0; ks < nk / KC; ++ks) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
           const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
-          tma_load_2d_2sm(sA(stage), &tmA, fb, kb * KB, a_lo, pol_w);
-          if (!a.a_one_box) tma_load_2d_2sm(sA(stage) + A_BYTES / 2, &tmA, fb, kb * KB, a_hi, pol_w);
-          uint8_t* bdst = sB(stage);
-          load_token_rows(rows, [&](int which, int off) {
-            tma_load_2d_2sm(bdst + off * 128, &tmB.box[which], fb, kb * KB, b0 + off, pol_x);
-          });
+#pragma unroll
+          for (int c = 0; c < KC; ++c) {
+            const int kb = ks * KC + c;
+            tma_load_2d_2sm(sA(stage, c), &tmA, fb, kb * KB, a_lo, pol_w);
+            if (!a.a_one_box) tma_load_2d_2sm(sA(stage, c) + A_BYTES / 2, &tmA, fb, kb * KB, a_hi, pol_w);
+            uint8_t* bdst = sB(stage, c);
+            load_token_rows(rows, [&](int which, int off) {
+              tma_load_2d_2sm(bdst + off * 128, &tmB.box[which], fb, kb * KB, b0 + off, pol_x);
+            });
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -542,13 +549,16 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t idesc = make_idesc(1u, 256u, static_cast<uint32_t>(ti.N));
         const uint32_t d = tmem_base + b * 256u;
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int ks = 0; ks < nk / KC; ++ks) {
           if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA(stage)), b0 = smem_u32(sB(stage));
 #pragma unroll
-          for (int kk = 0; kk < KB / 16; ++kk)
-            umma_bf16_2sm(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (kb | kk) != 0);
+          for (int c = 0; c < KC; ++c) {
+            const uint32_t a0 = smem_u32(sA(stage, c)), b0 = smem_u32(sB(stage, c));
+#pragma unroll
+            for (int kk = 0; kk < KB / 16; ++kk)
+              umma_bf16_2sm(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (ks | c | kk) != 0);
+          }
           umma_commit_2sm(&empty_bar[stage], 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -873,7 +883,7 @@ size_t gemm_bf16_smem_bytes(int stages, int bn_max) {
   return static_cast<size_t>(stages) * (2 * 128 * 128 + static_cast<size_t>(bn_max) * 128) + 1024;
 }
 size_t gemm_bf16_2sm_smem_bytes() {
-  return static_cast<size_t>(k2smStages) * (2 * 128 * 128) + 1024;
+  return static_cast<size_t>(k2smStages) * k2smChunks * (2 * 128 * 128) + 1024;
 }
 size_t gemm_e4m3_smem_bytes(int stages) {
   return static_cast<size_t>(stages) * (2 * 128 * 128 + kF8Bn * 128) + 1024;
