@@ -273,6 +273,9 @@ moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
   p->g = GemmArgs{rows, I, w->groups, offsets, H, H / 256, 256, pair ? 64 : 128, 256, 128,
                   fp8 ? 32 : (nb == 2 ? 128 : 256), pair ? 128 : 0, nb, one_box ? 1 : 0,
                   out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
+  // two accumulators on single CTAs: stages of 128 K (2 x 96 KB), measured a
+  // little faster than 4 x 48 KB stages of 64 K; MOE_DOWN_K64=1 keeps 64 K
+  p->g.kc = (!fp8 && !pair && nb == 2 && !env_on("MOE_DOWN_K64")) ? 2 : 1;
   p->fp8 = fp8;
   return MOE_OK;
 }
@@ -280,7 +283,7 @@ moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
 moe_status launch_plan(const GemmPlan& p, int epi, cudaStream_t st, int nsm, const GemmPlan* second = nullptr) {
   // one launch needs the same kernel form for both: single-CTA bf16, same tile shape
   const bool one = second && !p.fp8 && !second->fp8 && p.g.cta_stride == 0 && second->g.cta_stride == 0 &&
-                   p.g.bn_max == second->g.bn_max && p.g.nbuf == second->g.nbuf;
+                   p.g.bn_max == second->g.bn_max && p.g.nbuf == second->g.nbuf && p.g.kc == second->g.kc;
   if (second && !one) {
     moe_status s = check_launch(launch_grouped_gemm(p.fp8, epi, p.tmA, p.tmB, p.g, nsm, st));
     return s != MOE_OK ? s : check_launch(launch_grouped_gemm(second->fp8, epi, second->tmA, second->tmB,

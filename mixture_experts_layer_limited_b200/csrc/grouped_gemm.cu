@@ -178,7 +178,7 @@ constexpr int kGatherThreads = 64;
 // TWO: a second single-group problem a2 (the shared expert: its own weights
 // tmA2, token rows tmB2 and output) runs in the same launch. Its tiles come
 // first in the tile order, so the routed experts' ragged tiles fill the tail.
-template <int EPI, int STAGES, bool GATHER, bool TWO>
+template <int EPI, int STAGES, bool GATHER, bool TWO, int KC = 1>
 __global__ void __launch_bounds__(kThreads + (GATHER ? kGatherThreads : 0), 1)
 grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ TokenMaps tmB, const GemmArgs a,
@@ -202,9 +202,11 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   // column b * 2 * sub_cols + s * sub_cols
   const int nbuf = a.nbuf == 2 ? 2 : 1;
   const uint32_t sub_cols = nbuf == 2 ? 128u : 256u;
-  const uint32_t stage_bytes = 2 * A_SUB_BYTES + b_stage_bytes;
-  auto sA = [&](int st, int sub) { return smem + st * stage_bytes + sub * A_SUB_BYTES; };
-  auto sB = [&](int st) { return smem + st * stage_bytes + 2 * A_SUB_BYTES; };
+  // a stage holds KC chunks of 64 K, each [A sub-tile 0][A sub-tile 1][B rows]
+  const uint32_t chunk_bytes = 2 * A_SUB_BYTES + b_stage_bytes;
+  const uint32_t stage_bytes = KC * chunk_bytes;
+  auto sA = [&](int st, int sub, int c = 0) { return smem + st * stage_bytes + c * chunk_bytes + sub * A_SUB_BYTES; };
+  auto sB = [&](int st, int c = 0) { return smem + st * stage_bytes + c * chunk_bytes + 2 * A_SUB_BYTES; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -257,19 +259,23 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         const int a_row1 = a_row0 + (sh ? a2.sub1_off : a.sub1_off);
         const bool one_box = sh ? a2.a_one_box != 0 : a.a_one_box != 0;
         const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;   // re-read by sibling token blocks
-        const uint32_t bytes = 2 * A_SUB_BYTES + (GATHER ? 0u : static_cast<uint32_t>(ti.N) * 128u);
+        const uint32_t bytes = KC * (2 * A_SUB_BYTES + (GATHER ? 0u : static_cast<uint32_t>(ti.N) * 128u));
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int ks = 0; ks < nk / KC; ++ks) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
-          tma_load_2d(sA(stage, 0), mA, &full_bar[stage], kb * KB, a_row0, pol_w);
-          if (!one_box) tma_load_2d(sA(stage, 1), mA, &full_bar[stage], kb * KB, a_row1, pol_w);
-          if (!GATHER) {
-            uint8_t* bdst = sB(stage);
-            uint64_t* fb = &full_bar[stage];
-            load_token_rows(ti.N, [&](int which, int off) {
-              tma_load_2d(bdst + off * 128, &mB->box[which], fb, kb * KB, ti.row0 + off, pol_x);
-            });
+#pragma unroll
+          for (int c = 0; c < KC; ++c) {
+            const int kb = ks * KC + c;
+            tma_load_2d(sA(stage, 0, c), mA, &full_bar[stage], kb * KB, a_row0, pol_w);
+            if (!one_box) tma_load_2d(sA(stage, 1, c), mA, &full_bar[stage], kb * KB, a_row1, pol_w);
+            if (!GATHER) {
+              uint8_t* bdst = sB(stage, c);
+              uint64_t* fb = &full_bar[stage];
+              load_token_rows(ti.N, [&](int which, int off) {
+                tma_load_2d(bdst + off * 128, &mB->box[which], fb, kb * KB, ti.row0 + off, pol_x);
+              });
+            }
           }
           issued_parity[stage] = static_cast<int>(phase);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -338,17 +344,20 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         if (!mbar_wait(&tmem_empty[bi], (use & 1u) ^ 1u, &abort_flag, a.status)) break;
         tc_fence_after();
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int ks = 0; ks < nk / KC; ++ks) {
           if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA(stage, 0)), a1 = smem_u32(sA(stage, 1));
-          const uint32_t b0 = smem_u32(sB(stage));
 #pragma unroll
-          for (int kk = 0; kk < KB / 16; ++kk) {
-            const uint32_t acc = (kb | kk) != 0;
-            const uint64_t bd = sw128_desc(b0 + kk * 32);
-            umma_bf16(d0, sw128_desc(a0 + kk * 32), bd, idesc, acc);
-            umma_bf16(d0 + sub_cols, sw128_desc(a1 + kk * 32), bd, idesc, acc);
+          for (int c = 0; c < KC; ++c) {
+            const uint32_t a0 = smem_u32(sA(stage, 0, c)), a1 = smem_u32(sA(stage, 1, c));
+            const uint32_t b0 = smem_u32(sB(stage, c));
+#pragma unroll
+            for (int kk = 0; kk < KB / 16; ++kk) {
+              const uint32_t acc = (ks | c | kk) != 0;
+              const uint64_t bd = sw128_desc(b0 + kk * 32);
+              umma_bf16(d0, sw128_desc(a0 + kk * 32), bd, idesc, acc);
+              umma_bf16(d0 + sub_cols, sw128_desc(a1 + kk * 32), bd, idesc, acc);
+            }
           }
           umma_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -891,13 +900,18 @@ size_t gemm_e4m3_smem_bytes(int stages) {
 
 constexpr int kBf16Stages = 3;
 constexpr int kBf16StagesDb = 4;
+constexpr int kBf16StagesK128 = 1;        // 128 K per stage (two 64-K chunks)
+constexpr int kBf16StagesDbK128 = 2;
 constexpr int kE4m3Stages = 4;
 
 using Bf16Kernel = void (*)(CUtensorMap, TokenMaps, GemmArgs, CUtensorMap, TokenMaps, GemmArgs);
 
-// The single-CTA bf16 kernel in its four forms: stages x (one problem | two).
-template <int EPI, int STAGES>
-Bf16Kernel bf16_kernel(bool two) {
+// The single-CTA bf16 kernel: (one problem | two) x (64 | 128 K per stage).
+template <int EPI, int STAGES, int STAGES_K128>
+Bf16Kernel bf16_kernel(bool two, bool k128) {
+  if (k128)
+    return two ? grouped_gemm_bf16_kernel<EPI, STAGES_K128, false, true, 2>
+               : grouped_gemm_bf16_kernel<EPI, STAGES_K128, false, false, 2>;
   return two ? grouped_gemm_bf16_kernel<EPI, STAGES, false, true> : grouped_gemm_bf16_kernel<EPI, STAGES, false, false>;
 }
 
@@ -914,18 +928,20 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
     const bool gather = a.gather_rows != nullptr;
     // two accumulators hold <= 128-token tiles: 48 KB stages, four of them
     const bool db = a.nbuf == 2 && !gather;
-    const size_t smem = gemm_bf16_smem_bytes(db ? kBf16StagesDb : kBf16Stages, a.bn_max);
+    const bool k128 = a.kc == 2 && !gather;
+    const int stages = k128 ? (db ? kBf16StagesDbK128 : kBf16StagesK128) : (db ? kBf16StagesDb : kBf16Stages);
+    const size_t smem = gemm_bf16_smem_bytes(stages, a.bn_max) * (k128 ? 2 : 1) - (k128 ? 1024 : 0);
     const bool pair2 = two != nullptr && !gather;
     Bf16Kernel kern;
     if (gather)
       kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, true, false>
                                : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, true, false>;
     else if (db)
-      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16StagesDb>(pair2)
-                               : bf16_kernel<EPI_WEIGHTED, kBf16StagesDb>(pair2);
+      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128)
+                               : bf16_kernel<EPI_WEIGHTED, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128);
     else
-      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16Stages>(pair2)
-                               : bf16_kernel<EPI_WEIGHTED, kBf16Stages>(pair2);
+      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16Stages, kBf16StagesK128>(pair2, k128)
+                               : bf16_kernel<EPI_WEIGHTED, kBf16Stages, kBf16StagesK128>(pair2, k128);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     if (pair2)

@@ -32,6 +32,7 @@ struct GemmArgs {
   const void* gather_src;
   const int32_t* gather_rows;
   int32_t gather_src_rows;   // rows of gather_src (indices outside [0, this) are flagged, not read)
+  int32_t kc;                // 1-CTA bf16 kernel: 64-K chunks per pipeline stage (1 or 2)
 };
 
 struct RouteArgs {
