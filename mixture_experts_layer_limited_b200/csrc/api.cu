@@ -253,6 +253,8 @@ moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const
   const int nb = (fp8 || pair) ? 1 : one_cta_buffers(true);
   p->g = GemmArgs{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : (nb == 2 ? 128 : 256),
                   pair ? 64 : 0, nb, 0, h_ws, I, nullptr, w->w13_scale, a_scale, h_scale_ws, dev_status};
+  // with two accumulators (128-token tiles) the stages carry 128 K, as for down
+  p->g.kc = (!fp8 && !pair && nb == 2 && !env_on("MOE_DOWN_K64")) ? 2 : 1;
   p->fp8 = fp8;
   return MOE_OK;
 }
