@@ -20,22 +20,26 @@
 //          feature in the same thread and fuses SiLU(gate) * up.
 //   GEMM2: sub-tiles = w2 rows [mb*256, +128) and [mb*256 + 128, +128); the
 //          epilogue multiplies by the routing weight of the row.
-// TMEM: sub-tile s accumulates in columns [s*256, s*256 + N) (fp32).
+// TMEM (512 fp32 columns): one accumulator pair of up to 256 tokens (GEMM1),
+// or two pairs of up to 128 tokens (GEMM2), so that the epilogue of one tile
+// runs while the MMAs of the next fill the other pair.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over tiles):
-//   warp 0      TMA producer (A: two 128x64 boxes, B: ceil(N/32) 32x64 boxes
-//               per 64-wide K block, 128-byte swizzle) into an S-stage ring;
+//   warp 0      TMA producer (A: the weight rows, B: the tile's token rows in
+//               boxes of 256/128/64/32/16 rows, 128-byte swizzle) into a ring
+//               of stages of one or two 64-K chunks;
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer;
 //   warps 2..5  epilogue: tcgen05.ld (warp w owns TMEM lanes 32*(w%4)..+31),
 //               fused activation / weighting, bf16 stores.
+// A launch may carry a second, single-group problem (the shared expert) whose
+// tiles come first in the tile order.
 // The E4M3 variant accumulates each 128-wide K block separately in a TMEM
 // ring and promotes it with the fp32 block scales on the CUDA cores, since
 // the weight scale is per 128x128 block and the activation scale per 1x128.
+// A CTA-pair variant (tcgen05 cta_group::2) is kept as an option.
 #include "kernels.cuh"
 
 namespace moe {
-
-
 
 constexpr int kMaxGroups = 512;
 constexpr int kThreads = 192;
