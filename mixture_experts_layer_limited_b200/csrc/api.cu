@@ -102,12 +102,16 @@ bool env_on(const char* name) {
   return v && v[0] == '1';
 }
 // Kernel choice per bf16 GEMM (measured at the V3 shape on B200): both run on
-// single CTAs. Gate/up keeps 256-token tiles with one TMEM accumulator (the
-// 128-token tiles two accumulators need halve the reuse of each weight tile);
-// the down projection, whose epilogue stores twice the features, uses two
-// accumulators so the epilogue of one tile overlaps the MMAs of the next.
-// MOE_GEMM_PAIR=1 / MOE_GEMM_1SM=1 force CTA pairs / single CTAs for both;
-// MOE_GEMM_DB=1 / MOE_GEMM_SB=1 force two / one accumulators on single CTAs.
+// single CTAs with 256-token tiles and one TMEM accumulator pair (two pairs
+// of 128-token tiles would overlap the epilogue with the next tile's MMAs but
+// halve the reuse of each weight tile). The down projection's epilogue stores
+// twice the features of gate/up's, so it runs on 8 epilogue warps (two per
+// TMEM lane quarter), gate/up on 4.
+// Switches, for comparisons: MOE_GEMM_PAIR=1 / MOE_GEMM_1SM=1 force CTA pairs
+// / single CTAs for both GEMMs, MOE_GEMM_PAIR_DOWN=1 pairs for down only;
+// MOE_GEMM_DB=1 / MOE_GEMM_SB=1 force two / one accumulator pairs for both,
+// MOE_DOWN_DB=1 two for down only; MOE_EPI8=1 / MOE_EPI4=1 force 8 / 4
+// epilogue warps for both.
 bool bf16_on_pairs(bool gate_up) {
   if (env_on("MOE_GEMM_1SM")) return false;
   return env_on("MOE_GEMM_PAIR") || (!gate_up && env_on("MOE_GEMM_PAIR_DOWN"));
@@ -115,7 +119,12 @@ bool bf16_on_pairs(bool gate_up) {
 int one_cta_buffers(bool gate_up) {
   if (env_on("MOE_GEMM_DB")) return 2;
   if (env_on("MOE_GEMM_SB")) return 1;
-  return gate_up ? 1 : 2;
+  return (!gate_up && env_on("MOE_DOWN_DB")) ? 2 : 1;
+}
+int epilogue_warps(bool gate_up) {
+  if (env_on("MOE_EPI8")) return 8;
+  if (env_on("MOE_EPI4")) return 4;
+  return gate_up ? 4 : 8;
 }
 
 }  // namespace
@@ -255,6 +264,7 @@ moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const
                   pair ? 64 : 0, nb, 0, h_ws, I, nullptr, w->w13_scale, a_scale, h_scale_ws, dev_status};
   // with two accumulators (128-token tiles) the stages carry 128 K, as for down
   p->g.kc = (!fp8 && !pair && nb == 2 && !env_on("MOE_DOWN_K64")) ? 2 : 1;
+  p->g.epi_warps = epilogue_warps(true);
   p->fp8 = fp8;
   return MOE_OK;
 }
@@ -278,14 +288,17 @@ moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
   // two accumulators on single CTAs: stages of 128 K (2 x 96 KB), measured a
   // little faster than 4 x 48 KB stages of 64 K; MOE_DOWN_K64=1 keeps 64 K
   p->g.kc = (!fp8 && !pair && nb == 2 && !env_on("MOE_DOWN_K64")) ? 2 : 1;
+  p->g.epi_warps = epilogue_warps(false);
   p->fp8 = fp8;
   return MOE_OK;
 }
 
 moe_status launch_plan(const GemmPlan& p, int epi, cudaStream_t st, int nsm, const GemmPlan* second = nullptr) {
+
   // one launch needs the same kernel form for both: single-CTA bf16, same tile shape
   const bool one = second && !p.fp8 && !second->fp8 && p.g.cta_stride == 0 && second->g.cta_stride == 0 &&
-                   p.g.bn_max == second->g.bn_max && p.g.nbuf == second->g.nbuf && p.g.kc == second->g.kc;
+                   p.g.bn_max == second->g.bn_max && p.g.nbuf == second->g.nbuf && p.g.kc == second->g.kc &&
+                   p.g.epi_warps == second->g.epi_warps;
   if (second && !one) {
     moe_status s = check_launch(launch_grouped_gemm(p.fp8, epi, p.tmA, p.tmB, p.g, nsm, st));
     return s != MOE_OK ? s : check_launch(launch_grouped_gemm(second->fp8, epi, second->tmA, second->tmB,

@@ -182,8 +182,8 @@ constexpr int kGatherThreads = 64;
 // TWO: a second single-group problem a2 (the shared expert: its own weights
 // tmA2, token rows tmB2 and output) runs in the same launch. Its tiles come
 // first in the tile order, so the routed experts' ragged tiles fill the tail.
-template <int EPI, int STAGES, bool GATHER, bool TWO, int KC = 1>
-__global__ void __launch_bounds__(kThreads + (GATHER ? kGatherThreads : 0), 1)
+template <int EPI, int STAGES, bool GATHER, bool TWO, int KC = 1, int EPIW = 4>
+__global__ void __launch_bounds__(64 + 32 * EPIW + (GATHER ? kGatherThreads : 0), 1)
 grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ TokenMaps tmB, const GemmArgs a,
                          const __grid_constant__ CUtensorMap tmA2,
@@ -192,7 +192,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   constexpr uint32_t A_SUB_BYTES = 128 * 128;      // one 128-row sub-tile
   extern __shared__ __align__(1024) uint8_t dsmem[];
   __shared__ Sched sched;
-  __shared__ __align__(16) __nv_bfloat16 stage_out[4][32 * 32];
+  __shared__ __align__(16) __nv_bfloat16 stage_out[EPIW][32 * 32];
   __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
   __shared__ uint64_t tmem_full[2], tmem_empty[2], drain_bar;
   __shared__ uint32_t tmem_base_s;
@@ -220,7 +220,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tmem_full[b], 1);
-      mbar_init(&tmem_empty[b], 128);
+      mbar_init(&tmem_empty[b], 32 * EPIW);
     }
     mbar_init(&drain_bar, 1);
     abort_flag = 0;
@@ -291,8 +291,8 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
           if (issued_parity[i] >= 0) mbar_wait_drain(&full_bar[i], static_cast<uint32_t>(issued_parity[i]));
       }
     }
-  } else if (GATHER && warp >= 6) {
-    const int gt = threadIdx.x - kThreads;             // 0..63
+  } else if (GATHER && warp >= 2 + EPIW) {
+    const int gt = threadIdx.x - (64 + 32 * EPIW);    // 0..63
     const int chunk = gt & 7;                          // 16-byte chunk of the 128-byte row slice
     const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.gather_src);
     const int nk = a.K / KB;                          // (no second problem with GATHER)
@@ -373,9 +373,11 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       umma_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0);
     }
-  } else if (warp < 6) {
-    // epilogue warps 2..5
+  } else if (warp < 2 + EPIW) {
+    // epilogue warps 2 .. 1+EPIW: warp w reads TMEM lanes 32*(w%4)..+31; with
+    // 8 warps, two share each lane quarter and take alternate 32-token chunks
     const int q = warp & 3;
+    const int c0 = (warp - 2) / 4, cstep = EPIW / 4;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
     uint32_t it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
@@ -391,10 +393,10 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       tc_fence_after();
       const uint32_t acc_addr = lane_addr + bi * 2u * sub_cols;
       const int nchunk = (ti.N + 31) / 32;
-      __nv_bfloat16* stg = stage_out[q];
+      __nv_bfloat16* stg = stage_out[warp - 2];
       if (EPI == EPI_SWIGLU) {
         const int feat0 = ti.mb * feat_stride + 32 * q;            // this warp's 32 features
-        for (int c = 0; c < nchunk; ++c) {
+        for (int c = c0; c < nchunk; c += cstep) {
           float g[32], u[32];
           tmem_ld32(acc_addr + c * 32, g);
           tmem_ld32(acc_addr + sub_cols + c * 32, u);
@@ -407,7 +409,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll 1
         for (int s = 0; s < 2; ++s) {
           const int feat0 = ti.mb * feat_stride + s * feat_sub1 + 32 * q;
-          for (int c = 0; c < nchunk; ++c) {
+          for (int c = c0; c < nchunk; c += cstep) {
             float v[32];
             tmem_ld32(acc_addr + s * sub_cols + c * 32, v);
             tmem_ld_wait();
@@ -910,13 +912,20 @@ constexpr int kE4m3Stages = 4;
 
 using Bf16Kernel = void (*)(CUtensorMap, TokenMaps, GemmArgs, CUtensorMap, TokenMaps, GemmArgs);
 
-// The single-CTA bf16 kernel: (one problem | two) x (64 | 128 K per stage).
-template <int EPI, int STAGES, int STAGES_K128>
-Bf16Kernel bf16_kernel(bool two, bool k128) {
+// The single-CTA bf16 kernel: (one problem | two) x (64 | 128 K per stage)
+// x (4 | 8 epilogue warps).
+template <int EPI, int STAGES, int STAGES_K128, int EPIW>
+Bf16Kernel bf16_kernel_w(bool two, bool k128) {
   if (k128)
-    return two ? grouped_gemm_bf16_kernel<EPI, STAGES_K128, false, true, 2>
-               : grouped_gemm_bf16_kernel<EPI, STAGES_K128, false, false, 2>;
-  return two ? grouped_gemm_bf16_kernel<EPI, STAGES, false, true> : grouped_gemm_bf16_kernel<EPI, STAGES, false, false>;
+    return two ? grouped_gemm_bf16_kernel<EPI, STAGES_K128, false, true, 2, EPIW>
+               : grouped_gemm_bf16_kernel<EPI, STAGES_K128, false, false, 2, EPIW>;
+  return two ? grouped_gemm_bf16_kernel<EPI, STAGES, false, true, 1, EPIW>
+             : grouped_gemm_bf16_kernel<EPI, STAGES, false, false, 1, EPIW>;
+}
+template <int EPI, int STAGES, int STAGES_K128>
+Bf16Kernel bf16_kernel(bool two, bool k128, bool epi8) {
+  return epi8 ? bf16_kernel_w<EPI, STAGES, STAGES_K128, 8>(two, k128)
+              : bf16_kernel_w<EPI, STAGES, STAGES_K128, 4>(two, k128);
 }
 
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const TokenMaps& tmB,
@@ -933,6 +942,8 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
     // two accumulators hold <= 128-token tiles: 48 KB stages, four of them
     const bool db = a.nbuf == 2 && !gather;
     const bool k128 = a.kc == 2 && !gather;
+    const bool epi8 = a.epi_warps == 8 && !gather;
+    const int threads = 64 + 32 * (epi8 ? 8 : 4) + (gather ? kGatherThreads : 0);
     const int stages = k128 ? (db ? kBf16StagesDbK128 : kBf16StagesK128) : (db ? kBf16StagesDb : kBf16Stages);
     const size_t smem = gemm_bf16_smem_bytes(stages, a.bn_max) * (k128 ? 2 : 1) - (k128 ? 1024 : 0);
     const bool pair2 = two != nullptr && !gather;
@@ -941,17 +952,17 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
       kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, true, false>
                                : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, true, false>;
     else if (db)
-      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128)
-                               : bf16_kernel<EPI_WEIGHTED, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128);
+      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128, epi8)
+                               : bf16_kernel<EPI_WEIGHTED, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128, epi8);
     else
-      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16Stages, kBf16StagesK128>(pair2, k128)
-                               : bf16_kernel<EPI_WEIGHTED, kBf16Stages, kBf16StagesK128>(pair2, k128);
+      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16Stages, kBf16StagesK128>(pair2, k128, epi8)
+                               : bf16_kernel<EPI_WEIGHTED, kBf16Stages, kBf16StagesK128>(pair2, k128, epi8);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     if (pair2)
-      kern<<<grid, kThreads, smem, stream>>>(tmA, tmB, a, two->tmA, two->tmB, two->a);
+      kern<<<grid, threads, smem, stream>>>(tmA, tmB, a, two->tmA, two->tmB, two->a);
     else
-      kern<<<grid, kThreads + (gather ? kGatherThreads : 0), smem, stream>>>(tmA, tmB, a, tmA, tmB, a);
+      kern<<<grid, threads, smem, stream>>>(tmA, tmB, a, tmA, tmB, a);
   } else {
     const size_t smem = gemm_e4m3_smem_bytes(kE4m3Stages);
     auto kern = epi == EPI_SWIGLU ? grouped_gemm_e4m3_kernel<EPI_SWIGLU, kE4m3Stages>

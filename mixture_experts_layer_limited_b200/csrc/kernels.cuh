@@ -33,6 +33,7 @@ struct GemmArgs {
   const int32_t* gather_rows;
   int32_t gather_src_rows;   // rows of gather_src (indices outside [0, this) are flagged, not read)
   int32_t kc;                // 1-CTA bf16 kernel: 64-K chunks per pipeline stage (1 or 2)
+  int32_t epi_warps;         // 1-CTA bf16 kernel: epilogue warps (4, or 8: two per TMEM lane quarter)
 };
 
 struct RouteArgs {

@@ -241,21 +241,27 @@ def _ref_grouped(a, w13, w2, off, row_w):
     return out, hs
 
 
-@pytest.fixture(params=["pair", "1sm-sb", "1sm-db", "1sm-db-k64"])
+@pytest.fixture(params=["pair", "1sm-sb", "1sm-sb-epi4", "1sm-sb-epi8", "1sm-db", "1sm-db-k64"])
 def gemm_variant(request, monkeypatch):
-    """bf16 grouped GEMMs, each kernel forced: CTA pairs, single CTAs with one
-    TMEM accumulator, or single CTAs with two (the down GEMM's stages of 128 K,
-    or of 64 K for k64)."""
-    for var in ("MOE_GEMM_1SM", "MOE_GEMM_PAIR", "MOE_GEMM_DB", "MOE_GEMM_SB", "MOE_DOWN_K64"):
+    """bf16 grouped GEMMs, each kernel forced: CTA pairs, or single CTAs with
+    one TMEM accumulator pair (epilogue warps per GEMM, or 4 / 8 for both) or
+    with two (stages of 128 K, or of 64 K for k64)."""
+    for var in ("MOE_GEMM_1SM", "MOE_GEMM_PAIR", "MOE_GEMM_DB", "MOE_GEMM_SB", "MOE_DOWN_K64",
+                "MOE_DOWN_DB", "MOE_EPI4", "MOE_EPI8"):
         monkeypatch.delenv(var, raising=False)
-    if request.param == "pair":
+    v = request.param
+    if v == "pair":
         monkeypatch.setenv("MOE_GEMM_PAIR", "1")
     else:
         monkeypatch.setenv("MOE_GEMM_1SM", "1")
-        monkeypatch.setenv("MOE_GEMM_DB" if request.param.startswith("1sm-db") else "MOE_GEMM_SB", "1")
-        if request.param.endswith("k64"):
+        monkeypatch.setenv("MOE_GEMM_DB" if v.startswith("1sm-db") else "MOE_GEMM_SB", "1")
+        if v.endswith("k64"):
             monkeypatch.setenv("MOE_DOWN_K64", "1")
-    return request.param
+        if v.endswith("epi4"):
+            monkeypatch.setenv("MOE_EPI4", "1")
+        if v.endswith("epi8"):
+            monkeypatch.setenv("MOE_EPI8", "1")
+    return v
 
 
 @pytest.mark.parametrize("H,I,sizes", [
