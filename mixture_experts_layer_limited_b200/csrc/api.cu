@@ -105,7 +105,7 @@ bool env_on(const char* name) {
 // single CTAs with 256-token tiles and one TMEM accumulator pair (two pairs
 // of 128-token tiles would overlap the epilogue with the next tile's MMAs but
 // halve the reuse of each weight tile). The down projection's epilogue stores
-// twice the features of gate/up's, so it runs on 8 epilogue warps (two per
+// twice the features of gate/up's, so it runs on 12 epilogue warps (three per
 // TMEM lane quarter), gate/up on 4.
 // Switches, for comparisons: MOE_GEMM_PAIR=1 / MOE_GEMM_1SM=1 force CTA pairs
 // / single CTAs for both GEMMs, MOE_GEMM_PAIR_DOWN=1 pairs for down only;
@@ -124,7 +124,7 @@ int one_cta_buffers(bool gate_up) {
 int epilogue_warps(bool gate_up) {
   if (env_on("MOE_EPI8")) return 8;
   if (env_on("MOE_EPI4")) return 4;
-  return gate_up ? 4 : 8;
+  return gate_up ? 4 : 12;
 }
 
 }  // namespace

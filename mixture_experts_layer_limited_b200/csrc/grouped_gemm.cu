@@ -375,7 +375,8 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     }
   } else if (warp < 2 + EPIW) {
     // epilogue warps 2 .. 1+EPIW: warp w reads TMEM lanes 32*(w%4)..+31; with
-    // 8 warps, two share each lane quarter and take alternate 32-token chunks
+    // 8 or 12 warps, two or three share each lane quarter and take turns on
+    // its 32-token chunks
     const int q = warp & 3;
     const int c0 = (warp - 2) / 4, cstep = EPIW / 4;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
@@ -913,7 +914,7 @@ constexpr int kE4m3Stages = 4;
 using Bf16Kernel = void (*)(CUtensorMap, TokenMaps, GemmArgs, CUtensorMap, TokenMaps, GemmArgs);
 
 // The single-CTA bf16 kernel: (one problem | two) x (64 | 128 K per stage)
-// x (4 | 8 epilogue warps).
+// x (4 | 8 | 12 epilogue warps).
 template <int EPI, int STAGES, int STAGES_K128, int EPIW>
 Bf16Kernel bf16_kernel_w(bool two, bool k128) {
   if (k128)
@@ -923,9 +924,10 @@ Bf16Kernel bf16_kernel_w(bool two, bool k128) {
              : grouped_gemm_bf16_kernel<EPI, STAGES, false, false, 1, EPIW>;
 }
 template <int EPI, int STAGES, int STAGES_K128>
-Bf16Kernel bf16_kernel(bool two, bool k128, bool epi8) {
-  return epi8 ? bf16_kernel_w<EPI, STAGES, STAGES_K128, 8>(two, k128)
-              : bf16_kernel_w<EPI, STAGES, STAGES_K128, 4>(two, k128);
+Bf16Kernel bf16_kernel(bool two, bool k128, int epi_warps) {
+  if (epi_warps == 12) return bf16_kernel_w<EPI, STAGES, STAGES_K128, 12>(two, k128);
+  return epi_warps == 8 ? bf16_kernel_w<EPI, STAGES, STAGES_K128, 8>(two, k128)
+                        : bf16_kernel_w<EPI, STAGES, STAGES_K128, 4>(two, k128);
 }
 
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const TokenMaps& tmB,
@@ -942,8 +944,8 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
     // two accumulators hold <= 128-token tiles: 48 KB stages, four of them
     const bool db = a.nbuf == 2 && !gather;
     const bool k128 = a.kc == 2 && !gather;
-    const bool epi8 = a.epi_warps == 8 && !gather;
-    const int threads = 64 + 32 * (epi8 ? 8 : 4) + (gather ? kGatherThreads : 0);
+    const int epiw = gather ? 4 : (a.epi_warps == 8 || a.epi_warps == 12 ? a.epi_warps : 4);
+    const int threads = 64 + 32 * epiw + (gather ? kGatherThreads : 0);
     const int stages = k128 ? (db ? kBf16StagesDbK128 : kBf16StagesK128) : (db ? kBf16StagesDb : kBf16Stages);
     const size_t smem = gemm_bf16_smem_bytes(stages, a.bn_max) * (k128 ? 2 : 1) - (k128 ? 1024 : 0);
     const bool pair2 = two != nullptr && !gather;
@@ -952,11 +954,11 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
       kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, true, false>
                                : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, true, false>;
     else if (db)
-      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128, epi8)
-                               : bf16_kernel<EPI_WEIGHTED, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128, epi8);
+      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128, epiw)
+                               : bf16_kernel<EPI_WEIGHTED, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128, epiw);
     else
-      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16Stages, kBf16StagesK128>(pair2, k128, epi8)
-                               : bf16_kernel<EPI_WEIGHTED, kBf16Stages, kBf16StagesK128>(pair2, k128, epi8);
+      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16Stages, kBf16StagesK128>(pair2, k128, epiw)
+                               : bf16_kernel<EPI_WEIGHTED, kBf16Stages, kBf16StagesK128>(pair2, k128, epiw);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     if (pair2)

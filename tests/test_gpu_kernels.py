@@ -244,7 +244,8 @@ def _ref_grouped(a, w13, w2, off, row_w):
 @pytest.fixture(params=["pair", "1sm-sb", "1sm-sb-epi4", "1sm-sb-epi8", "1sm-db", "1sm-db-k64"])
 def gemm_variant(request, monkeypatch):
     """bf16 grouped GEMMs, each kernel forced: CTA pairs, or single CTAs with
-    one TMEM accumulator pair (epilogue warps per GEMM, or 4 / 8 for both) or
+    one TMEM accumulator pair (epilogue warps per GEMM: 4 gate/up, 12 down; or
+    4 / 8 for both) or
     with two (stages of 128 K, or of 64 K for k64)."""
     for var in ("MOE_GEMM_1SM", "MOE_GEMM_PAIR", "MOE_GEMM_DB", "MOE_GEMM_SB", "MOE_DOWN_K64",
                 "MOE_DOWN_DB", "MOE_EPI4", "MOE_EPI8"):
