@@ -330,3 +330,29 @@ def test_layer_cuda_graph_replay_matches_eager(name):
     assert layer.device_status() == 0
     if gamma is not None:
         assert torch.equal(layer.bias, eager.bias)
+
+
+def test_layer_v3_largest_batch_sampled():
+    """T = 65536 tokens (524288 routed rows, 7.5 GB of permuted activations):
+    the permutation's invariants on every row and sampled outputs against
+    the oracle."""
+    cfg = get_config("v3", T=65536)
+    inp = make_inputs(cfg, device=DEV)
+    layer = _layer(cfg, inp)
+    y = layer.forward(inp.x)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    _check_permutation_properties(layer, cfg.T, cfg.k, cfg.E)
+    rng = np.random.default_rng(65536)
+    toks = np.sort(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 4, replace=False)]))
+    feats = np.sort(rng.choice(cfg.H, 256, replace=False))
+    r, yref = _oracle_tokens(cfg, inp, toks, feats)
+    flagged = near_tie_mask(r)
+    ids_g = layer.ids[toks].cpu().numpy()
+    mism = routing_mismatch(ids_g, r)
+    assert not np.any(mism & ~flagged), describe_mismatch(ids_g, r, np.nonzero(mism & ~flagged)[0])
+    ok = ~flagged & ~mism
+    yg = np64(y[toks][:, torch.as_tensor(feats, device=DEV)])
+    err = rel_err(yg[ok], yref[ok])
+    print(f"v3 T=65536: sampled err {err:.2e}, excluded {int(flagged.sum())}")
+    assert err < BF16_TOL
