@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--config", default="v3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=16)
+    ap.add_argument("--fuse-combine", action="store_true",
+                    help="run the combine inside the down GEMM (atomic fp32 scatter-add) instead of after it")
     ap.add_argument("--routing-sweep", action="store_true",
                     help="instead of the throughput line: load CV, aux loss and router time for "
                          "topk_group 8/4/2/1 of 8 groups on the V3 and skewed inputs (one line each)")
@@ -235,7 +237,8 @@ def profiled_traffic(stage):
 
 
 LAUNCHES = {"route": 2, "quantize_x": 1, "permute": 3, "gate_up_routed": 1, "down_routed": 1,
-            "gate_up_shared": 1, "down_shared": 1, "gate_up": 1, "down": 1, "combine": 1, "bias_update": 1}
+            "gate_up_shared": 1, "down_shared": 1, "gate_up": 1, "down": 1, "combine": 1, "bias_update": 1,
+            "down_combine": 2}
 
 
 def launches_of(name, cfg):
@@ -265,6 +268,9 @@ def stage_model(cfg):
     # routed + shared expert in one launch per GEMM
     for fused, parts in (("gate_up", ("gate_up_routed", "gate_up_shared")), ("down", ("down_routed", "down_shared"))):
         m[fused] = {key: sum(m[p][key] for p in parts) for key in ("flops", "bytes")}
+    # down GEMMs with the combine in the epilogue: weights and h in, y out
+    m["down_combine"] = {"flops": m["down"]["flops"],
+                         "bytes": E * H * I * ab + R * I * ab + H * Is * ab + T * Is * ab + T * H * 2}
     return m
 
 
@@ -292,7 +298,7 @@ def run_ours(args):
         g.manual_seed(cfg.seed + 100003 * rank)
         inp.x = torch.randn(cfg.T, cfg.H, generator=g, device="cuda").to(torch.bfloat16)
     layer = MoELayer(LayerSpec.from_config(cfg), inp.gate, inp.w13, inp.w2, inp.sw13, inp.sw2,
-                     inp.bias, cfg.T)
+                     inp.bias, cfg.T, fuse_combine=args.fuse_combine)
     T_global = cfg.T * world
     stream = torch.cuda.current_stream()
     stages = layer.stages(inp.x)
@@ -437,7 +443,8 @@ def run_ours(args):
                 "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "e4m3",
                 "data": f"synthetic (seeded random inputs and weights, {cfg.name} shapes)",
-                "config": config_block(cfg, world),
+                "config": dict(config_block(cfg, world),
+                               **({"combine": "inside the down GEMM (atomic fp32 adds)"} if args.fuse_combine else {})),
                 "tflops": round(flops_step * world * K / (ms * 1e-3) / 1e12, 1),
                 "tflops_frac_of_measured_sustained": round(flops_step * world * K / (ms * 1e-3) / 1e12 / peak, 4),
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,

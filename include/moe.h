@@ -268,6 +268,24 @@ MOE_API moe_status moe_down_proj_with_shared(int32_t rows, int32_t H, const moe_
                               const void* sh_h, const float* sh_h_scale, void* sh_out,
                               int32_t* dev_status, void* stream);
 
+/* moe_down_proj_combine -- the second GEMM with the combine fused into its
+ * epilogue ([MoE-walk] §3.3.1 + §3.4): every routed row's weighted output
+ * row_w[r] * (h[r] w2[e]^T) is added in fp32 straight into the row of its token
+ * src_token[r] of acc_ws, the shared expert's output (sw, sh_h: optional) into
+ * its own token's row, and y = bf16(acc_ws) at the end; no [rows, H]
+ * intermediate and no separate combine.
+ *   rows = T*k; h [rows, I] bf16; offsets, row_w, src_token from moe_permute;
+ *   sw / sh_h: shared expert (groups 1) and its h [T, I_s], or NULL / NULL;
+ *   acc_ws [T, H] fp32 device scratch (zeroed by the call); y [T, H] bf16.
+ * bf16 only. The adds are atomic, so their order, and the last bits of y,
+ * can differ from run to run; y agrees with moe_down_proj + moe_combine to
+ * the rounding of o to bf16 that it skips. */
+MOE_API moe_status moe_down_proj_combine(int32_t rows, int32_t T, int32_t H, const moe_ffn_weights* w,
+                                 const void* h, const int32_t* offsets, const float* row_w,
+                                 const int32_t* src_token, const moe_ffn_weights* sw,
+                                 const void* sh_h, float* acc_ws, void* y,
+                                 int32_t* dev_status, void* stream);
+
 /* moe_gate_up_swiglu_gather -- the routed experts' first GEMM with the
  * permutation fused into its operand fetch ([MoE-walk] §3.2 + §3.3.1): row p
  * of the expert segments is read directly from x[src_token[p]], so

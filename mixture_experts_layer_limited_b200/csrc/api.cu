@@ -270,9 +270,11 @@ moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const
 }
 
 moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* h, const float* h_scale,
-                     const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status, GemmPlan* p) {
+                     const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status, GemmPlan* p,
+                     bool scatter = false) {
   const bool fp8 = w->dtype == MOE_E4M3;
-  const bool pair = !fp8 && bf16_on_pairs(false);
+  // the scatter form (combine fused in) runs on single CTAs, one accumulator pair
+  const bool pair = !fp8 && !scatter && bf16_on_pairs(false);
   const int I = w->I;
   // the single-CTA bf16 kernel reads its 256 contiguous w2 rows as one box
   const bool one_box = !fp8;
@@ -281,7 +283,7 @@ moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
   if (s != MOE_OK) return s;
   s = make_token_tmaps(&p->tmB, h, fp8, I, rows);
   if (s != MOE_OK) return s;
-  const int nb = (fp8 || pair) ? 1 : one_cta_buffers(false);
+  const int nb = (fp8 || pair || scatter) ? 1 : one_cta_buffers(false);
   p->g = GemmArgs{rows, I, w->groups, offsets, H, H / 256, 256, pair ? 64 : 128, 256, 128,
                   fp8 ? 32 : (nb == 2 ? 128 : 256), pair ? 128 : 0, nb, one_box ? 1 : 0,
                   out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
@@ -436,6 +438,38 @@ moe_status moe_down_proj_with_shared(int32_t rows, int32_t H, const moe_ffn_weig
   if (!env_on("MOE_SHARED_APART")) return launch_plan(p, EPI_WEIGHTED, st, nsm, &q);
   if ((s = launch_plan(p, EPI_WEIGHTED, st, nsm)) != MOE_OK) return s;
   return launch_plan(q, EPI_WEIGHTED, st, nsm);
+}
+
+moe_status moe_down_proj_combine(int32_t rows, int32_t T, int32_t H, const moe_ffn_weights* w, const void* h,
+                                 const int32_t* offsets, const float* row_w, const int32_t* src_token,
+                                 const moe_ffn_weights* sw, const void* sh_h, float* acc_ws, void* y,
+                                 int32_t* dev_status, void* stream) {
+  moe_status s = check_ffn(rows, H, w, h, nullptr, false, true);
+  if (s != MOE_OK) return s;
+  if (w->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (T < 1 || !offsets || !row_w || !src_token || !acc_ws || !y) return MOE_ERR_INVALID_ARG;
+  if (sw) {
+    if ((s = check_ffn(T, H, sw, sh_h, nullptr, false, true)) != MOE_OK) return s;
+    if (sw->groups != 1 || sw->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  }
+  if (any_misaligned(offsets, row_w, src_token, acc_ws, y)) return MOE_ERR_ALIGNMENT;
+  int nsm = 0;
+  if ((s = sm_count(&nsm)) != MOE_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e = cudaMemsetAsync(acc_ws, 0, static_cast<size_t>(T) * H * sizeof(float), st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  // the scatter runs on the single-CTA kernel: one accumulator pair, 256 tokens
+  GemmPlan p, q;
+  if ((s = plan_down(rows, H, w, h, nullptr, offsets, row_w, acc_ws, dev_status, &p, true)) != MOE_OK) return s;
+  p.g.scatter_tok = src_token;
+  p.g.scatter_T = T;
+  if (sw) {
+    if ((s = plan_down(T, H, sw, sh_h, nullptr, nullptr, nullptr, acc_ws, dev_status, &q, true)) != MOE_OK) return s;
+    q.g.scatter_tok = nullptr;
+    q.g.scatter_T = T;
+  }
+  if ((s = launch_plan(p, EPI_SCATTER, st, nsm, sw ? &q : nullptr)) != MOE_OK) return s;
+  return check_launch(launch_cast_rows(T, H, acc_ws, y, st));
 }
 
 moe_status moe_combine(int32_t T, int32_t k, int32_t H, const void* expert_out, const int32_t* slot_to_row,

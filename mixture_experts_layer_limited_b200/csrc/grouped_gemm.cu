@@ -419,7 +419,22 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wl, j);
             }
-            store_tile<32>(stg, v, lane, out, out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
+            if (EPI == EPI_SCATTER) {
+              // row -> token (routed rows through src_token, shared rows are tokens)
+              const int32_t* src = sh ? a2.scatter_tok : a.scatter_tok;
+              const int ntok = sh ? a2.scatter_T : a.scatter_T;
+              const int r = ti.row0 + c * 32 + lane;
+              int tok = c * 32 + lane < ti.n_valid ? (src ? __ldg(src + r) : r) : -1;
+              if (tok >= ntok) { flag_status(a.status, MOE_DEVSTAT_BAD_EXPERT_ID); tok = -1; }
+              float* acc_out = reinterpret_cast<float*>(sh ? a2.out : a.out);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int tj = __shfl_sync(0xffffffffu, tok, j);
+                if (tj >= 0) atomicAdd(acc_out + static_cast<size_t>(tj) * out_ld + feat0 + lane, v[j]);
+              }
+            } else {
+              store_tile<32>(stg, v, lane, out, out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
+            }
           }
         }
       }
@@ -953,6 +968,8 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
     if (gather)
       kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, true, false>
                                : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, true, false>;
+    else if (epi == EPI_SCATTER)
+      kern = bf16_kernel<EPI_SCATTER, kBf16Stages, kBf16StagesK128>(pair2, false, epiw);
     else if (db)
       kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128, epiw)
                                : bf16_kernel<EPI_WEIGHTED, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128, epiw);

@@ -33,7 +33,11 @@ struct GemmArgs {
   const int32_t* gather_rows;
   int32_t gather_src_rows;   // rows of gather_src (indices outside [0, this) are flagged, not read)
   int32_t kc;                // 1-CTA bf16 kernel: 64-K chunks per pipeline stage (1 or 2)
-  int32_t epi_warps;         // 1-CTA bf16 kernel: epilogue warps (4, or 8: two per TMEM lane quarter)
+  int32_t epi_warps;         // 1-CTA bf16 kernel: epilogue warps (4, 8 or 12)
+  // EPI_SCATTER: token of each row ([rows], NULL: the row is the token) and the
+  // number of tokens (rows of the fp32 accumulator `out`)
+  const int32_t* scatter_tok;
+  int32_t scatter_T;
 };
 
 struct RouteArgs {
@@ -48,7 +52,9 @@ struct RouteArgs {
   int32_t* status;
 };
 
-enum { EPI_SWIGLU = 0, EPI_WEIGHTED = 1 };
+// EPI_SCATTER: GEMM2 with the combine fused in: the weighted fp32 rows are
+// added atomically into a [tokens, H] fp32 accumulator at their token.
+enum { EPI_SWIGLU = 0, EPI_WEIGHTED = 1, EPI_SCATTER = 2 };
 
 // tmB: token-row tensor maps with 64-, 32- and 16-row boxes (bf16), or one
 // 32-row map (e4m3).
@@ -88,6 +94,7 @@ inline size_t aux_loss_workspace_bytes(int T, int E, int seq_len) {
 cudaError_t launch_aux_loss(int T, int E, int k, int seq_len, int scoring, const float* logits,
                             const int32_t* ids, float alpha, float* out, void* ws, int32_t* status,
                             cudaStream_t stream);
+cudaError_t launch_cast_rows(int T, int H, const float* acc, void* y, cudaStream_t stream);
 cudaError_t launch_bias_update(int E, int T, int k, const int32_t* counts, float* bias, float gamma,
                                float* load_cv, cudaStream_t stream);
 cudaError_t launch_quant_blocks(int batch, int N, int K, const void* w, void* q, float* scale,

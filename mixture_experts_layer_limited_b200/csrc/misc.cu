@@ -315,6 +315,32 @@ cudaError_t launch_combine(int T, int k, int H, const void* eo, const int32_t* s
   return cudaGetLastError();
 }
 
+// y[t] = bf16(acc[t]) for the fp32 accumulator of the combine fused into the
+// down GEMM; 8 elements (32 B in, 16 B out) per thread, streamed.
+__global__ void __launch_bounds__(256)
+cast_rows_kernel(const float4* __restrict__ acc, uint4* __restrict__ y, size_t n8) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 a = __ldcs(acc + 2 * i), b = __ldcs(acc + 2 * i + 1);
+    __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
+    __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+    uint4 o;
+    o.x = *reinterpret_cast<uint32_t*>(&p0);
+    o.y = *reinterpret_cast<uint32_t*>(&p1);
+    o.z = *reinterpret_cast<uint32_t*>(&p2);
+    o.w = *reinterpret_cast<uint32_t*>(&p3);
+    y[i] = o;
+  }
+}
+
+cudaError_t launch_cast_rows(int T, int H, const float* acc, void* y, cudaStream_t stream) {
+  const size_t n8 = static_cast<size_t>(T) * H / 8;
+  const size_t blocks = (n8 + 255) / 256;
+  cast_rows_kernel<<<static_cast<unsigned>(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(acc), reinterpret_cast<uint4*>(y), n8);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bias_update(int E, int T, int k, const int32_t* counts, float* bias, float gamma,
                                float* load_cv, cudaStream_t stream) {
   bias_update_kernel<<<1, 1024, 0, stream>>>(E, T, k, counts, bias, gamma, load_cv);

@@ -40,7 +40,7 @@ class MoELayer:
     def __init__(self, spec: LayerSpec, gate: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
                  sw13: Optional[torch.Tensor], sw2: Optional[torch.Tensor],
                  bias: Optional[torch.Tensor], T_max: int, gather: bool = False,
-                 fuse_shared: bool = True):
+                 fuse_shared: bool = True, fuse_combine: bool = False):
         self.spec = spec
         # gather=True: bf16 layers read the routed experts' token rows straight
         # from x (the permutation fused into the first GEMM; no x_perm). At the
@@ -48,6 +48,9 @@ class MoELayer:
         self.gather = gather and spec.dtype != "e4m3"
         # fuse_shared: the shared expert's GEMMs share the routed experts' launches
         self.fuse_shared = fuse_shared
+        # fuse_combine: the combine runs inside the down GEMM (atomic fp32 adds
+        # into a [T, H] accumulator); measured slower at the V3 shape, so off
+        self.fuse_combine = fuse_combine and spec.dtype != "e4m3"
         dev = gate.device
         self.dev = dev
         self.gate = gate.contiguous()
@@ -89,6 +92,7 @@ class MoELayer:
         self.o = z(R, H, dt=bf)
         self.y = z(T_max, H, dt=bf)
         self.load_cv = z(1, dt=f32)
+        self.y_acc = z(T_max, H, dt=f32) if self.fuse_combine else None
         self.status = torch.zeros(1, dtype=i32, device=dev)
         if self.fp8:
             self.xq = z(T_max, H, dt=torch.uint8)
@@ -197,6 +201,15 @@ class MoELayer:
             h_scale=self.h_s[:R] if self.fp8 else None, sw2_scale=self.sw2_s,
             sh_h_scale=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status)
 
+    def down_with_combine(self, T: int):
+        """The routed and shared down GEMMs with the combine in their epilogue."""
+        s = self.spec
+        R = T * s.k
+        N.moe_down_proj_combine(R, T, s.H, self.w2, s.E, s.I, self.h[:R], self.offsets, self.row_w[:R],
+                                self.src_token[:R], self.sw2, s.I_s,
+                                self.sh_h[:T] if self.sh_h is not None else None,
+                                self.y_acc[:T], self.y[:T], dev_status=self.status)
+
     def combine(self, T: int):
         s = self.spec
         N.moe_combine(T, s.k, s.H, self.o[:T * s.k], self.slot_to_row[:T * s.k], None,
@@ -210,6 +223,15 @@ class MoELayer:
         if self.fp8:
             st.append(("quantize_x", lambda: self.quantize_x(x, T)))
         st.append(("permute", lambda: self.permute(x, T)))
+        if self.fuse_combine:
+            if self.sh_h is not None and not self.gather:
+                st.append(("gate_up", lambda: self.gate_up_with_shared(x, T)))
+            else:
+                st.append(("gate_up_routed", lambda: self.experts_gate_up(T, x)))
+                if self.sh_h is not None:
+                    st.append(("gate_up_shared", lambda: self.shared_gate_up(x, T)))
+            st.append(("down_combine", lambda: self.down_with_combine(T)))
+            return st
         if self.sh_h is not None and self.fuse_shared and not self.gather:
             # routed + shared expert in one launch per GEMM
             st += [("gate_up", lambda: self.gate_up_with_shared(x, T)),

@@ -29,7 +29,7 @@ EXPORTED = [
     "moe_route", "moe_permute_workspace_size", "moe_permute", "moe_permute_static_ws",
     "moe_grouped_swiglu",
     "moe_gate_up_swiglu", "moe_gate_up_swiglu_gather", "moe_down_proj",
-    "moe_gate_up_swiglu_with_shared", "moe_down_proj_with_shared",
+    "moe_gate_up_swiglu_with_shared", "moe_down_proj_with_shared", "moe_down_proj_combine",
     "moe_combine", "moe_bias_update", "moe_aux_loss_workspace_size", "moe_aux_loss",
     "moe_quantize_blocks", "moe_quantize_rows",
     "moe_read_device_status", "moe_last_cuda_error", "moe_status_string", "moe_abi_version",
@@ -84,6 +84,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
                                            _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P],
         "moe_down_proj_with_shared": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P,
                                       _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P],
+        "moe_down_proj_combine": [_I, _I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P,
+                                  ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P],
         "moe_combine": [_I, _I, _I, _P, _P, _P, _P, _P, _P],
         "moe_bias_update": [_I, _I, _I, _P, _P, ctypes.c_float, _P, _P],
         "moe_aux_loss_workspace_size": [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
@@ -207,6 +209,16 @@ def moe_down_proj_with_shared(rows, H, w2, dtype, groups, I, h, offsets, row_w, 
     _check("moe_down_proj_with_shared", load_library().moe_down_proj_with_shared(
         rows, H, ctypes.byref(w), _ptr(h), _ptr(h_scale), _ptr(offsets), _ptr(row_w), _ptr(out),
         sh_rows, ctypes.byref(sw), _ptr(sh_h), _ptr(sh_h_scale), _ptr(sh_out),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_down_proj_combine(rows, T, H, w2, groups, I, h, offsets, row_w, src_token, sw2, I_s, sh_h,
+                          acc_ws, y, dev_status=None, stream=None):
+    w = FFNWeights(None, _ptr(w2), None, None, MOE_BF16, groups, I)
+    sw = FFNWeights(None, _ptr(sw2), None, None, MOE_BF16, 1, I_s) if sw2 is not None else None
+    _check("moe_down_proj_combine", load_library().moe_down_proj_combine(
+        rows, T, H, ctypes.byref(w), _ptr(h), _ptr(offsets), _ptr(row_w), _ptr(src_token),
+        ctypes.byref(sw) if sw is not None else None, _ptr(sh_h), _ptr(acc_ws), _ptr(y),
         _ptr(dev_status), _stream(stream)))
 
 

@@ -17,8 +17,9 @@ import torch
 
 from .layer import MoELayer
 
-# stages that read the forward's input x
+# stages that read the forward's input x, and the stage that writes its output y
 _READS_X = ("route", "quantize_x", "permute", "gate_up", "gate_up_routed", "gate_up_shared")
+_WRITES_Y = ("combine", "down_combine")
 
 
 class HostPipeline:
@@ -58,7 +59,7 @@ class HostPipeline:
             self.x_loaded[b].record(self.h2d)
             compute.wait_event(self.x_loaded[b])
             for j, (name, fn) in enumerate(self.stages[b]):
-                if name == "combine":
+                if name in _WRITES_Y:
                     compute.wait_event(self.y_free)        # the previous output has left y
                 fn()
                 if j == self.last_x_reader[b]:

@@ -356,3 +356,30 @@ def test_layer_v3_largest_batch_sampled():
     err = rel_err(yg[ok], yref[ok])
     print(f"v3 T=65536: sampled err {err:.2e}, excluded {int(flagged.sum())}")
     assert err < BF16_TOL
+
+
+@pytest.mark.parametrize("name", ["tiny", "v2lite", "v3"])
+def test_layer_combine_fused_into_down_gemm(name):
+    """The combine inside the down GEMM (fp32 atomic adds at each row's token)
+    against the oracle, and close to the default path, which rounds each
+    expert's output to bf16 before the combine."""
+    cfg = get_config(name) if name != "v3" else get_config("v3", T=2048)
+    inp = make_inputs(cfg, device=DEV)
+    y_ref_path = _layer(cfg, inp).forward(inp.x).clone()
+    lay = MoELayer(LayerSpec.from_config(cfg), inp.gate, inp.w13, inp.w2, inp.sw13, inp.sw2,
+                   inp.bias, cfg.T, fuse_combine=True)
+    assert [n for n, _ in lay.stages(inp.x)][-1] == "down_combine"
+    y = lay.forward(inp.x)
+    torch.cuda.synchronize()
+    assert lay.device_status() == 0
+    diff = rel_err(np64(y), np64(y_ref_path))
+    rng = np.random.default_rng(8)
+    toks = np.arange(cfg.T) if cfg.T <= 4096 and name != "v3" else np.sort(rng.choice(cfg.T, 8, replace=False))
+    feats = None if name != "v3" else np.sort(rng.choice(cfg.H, 256, replace=False))
+    r, yref = _oracle_tokens(cfg, inp, toks, feats)
+    flagged = near_tie_mask(r)
+    ok = ~flagged & ~routing_mismatch(lay.ids[toks].cpu().numpy(), r)
+    yg = np64(y[toks]) if feats is None else np64(y[toks][:, torch.as_tensor(feats, device=DEV)])
+    err = rel_err(yg[ok], yref[ok])
+    print(f"{name} fused combine: err {err:.2e}, vs default path {diff:.2e}")
+    assert err < BF16_TOL and diff < 1e-2
