@@ -85,6 +85,20 @@ def test_host_validation_rejects_before_launch():
     w8 = N.FFNWeights(fake, fake, None, None, N.MOE_E4M3, 4, 128)
     assert lib.moe_grouped_swiglu(64, 256, ctypes.byref(w8), fake, None, fake, None, fake, None, fake,
                                   None, None) == N.MOE_ERR_INVALID_ARG
+    # moe_down_proj_combine: T, the token map, the shared expert's groups, H, alignment, E4M3
+    w2 = N.FFNWeights(None, fake, None, None, N.MOE_BF16, 4, 128)
+    sw2 = N.FFNWeights(None, fake, None, None, N.MOE_BF16, 2, 128)
+    w2e = N.FFNWeights(None, fake, None, None, N.MOE_E4M3, 4, 128)
+    def dpc(T, H, w, src, sw, y):
+        return lib.moe_down_proj_combine(64, T, H, ctypes.byref(w), fake, fake, fake, src,
+                                         ctypes.byref(sw) if sw is not None else None, fake, fake, y,
+                                         None, None)
+    assert dpc(0, 256, w2, fake, None, fake) == N.MOE_ERR_INVALID_ARG
+    assert dpc(16, 256, w2, None, None, fake) == N.MOE_ERR_INVALID_ARG
+    assert dpc(16, 256, w2, fake, sw2, fake) == N.MOE_ERR_INVALID_ARG
+    assert dpc(16, 200, w2, fake, None, fake) == N.MOE_ERR_UNSUPPORTED
+    assert dpc(16, 256, w2, fake, None, odd) == N.MOE_ERR_ALIGNMENT
+    assert dpc(16, 256, w2e, fake, None, fake) != N.MOE_OK
     # moe_combine / moe_bias_update / quantisers
     assert lib.moe_combine(0, 4, 256, fake, fake, None, None, fake, None) == N.MOE_ERR_INVALID_ARG
     assert lib.moe_combine(8, 4, 252, fake, fake, None, None, fake, None) == N.MOE_ERR_UNSUPPORTED
