@@ -355,7 +355,8 @@ def run_ours(args):
         d = {"ms": round(avg[n], 4), "launches": launches_of(n, cfg)}
         if m["flops"]:
             d["tflops"] = round(m["flops"] / (avg[n] * 1e-3) / 1e12, 1)
-        d["gbs"] = round(m["bytes"] / (avg[n] * 1e-3) / 1e9, 1)
+        if m["bytes"] and avg[n] > 0:
+            d["gbs"] = round(m["bytes"] / (avg[n] * 1e-3) / 1e9, 1)
         kernels[n] = d
 
     tokens = cfg.T * world * K

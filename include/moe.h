@@ -124,6 +124,21 @@ MOE_API moe_status moe_route(const moe_route_params* p, const void* x, const voi
                      float* topk_w, int32_t* expert_counts, void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * moe_gate_logits -- the gate projection of moe_route alone.
+ * [MoE-walk] §2.1: router_logits = hidden_states @ gate.weight^T.
+ *
+ *   logits [T, E] fp32 out = x [T, H] bf16 @ gate_w [E, H] bf16 ^T, computed
+ *   exactly as moe_route computes them (same kernel, same summation order).
+ * Followed by moe_route with x = NULL on the same logits it is moe_route in
+ * two calls, so that other work (another stream's launch) can be ordered
+ * between the projection and the routing.
+ * Limits: H % 64 == 0, H >= 64, E % 16 == 0, 16 <= E <= 256.
+ * dev_status: optional device status word (bounded waits report into it).
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_gate_logits(int32_t T, int32_t H, int32_t E, const void* x, const void* gate_w,
+                                   float* logits, int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * moe_permute -- expand every token k times and order the copies by expert.
  * [MoE-walk] §3.2 and its worked example: segment e holds the tokens routed
  * to expert e in ASCENDING TOKEN ORDER; expert_offsets is

@@ -148,6 +148,30 @@ const char* moe_status_string(moe_status s) {
   }
 }
 
+// logits = x @ gate^T on the CTA-pair gate GEMM (r carries T, H, E, logits, status)
+moe_status gate_gemm(const RouteArgs& r, const void* x, const void* gate_w, cudaStream_t st) {
+  CUtensorMap tmX, tmG;
+  moe_status s = make_tmap(&tmX, x, false, r.H, r.T, 128);
+  if (s != MOE_OK) return s;
+  s = make_tmap(&tmG, gate_w, false, r.H, r.E, static_cast<uint32_t>(r.E));
+  if (s != MOE_OK) return s;
+  return check_launch(launch_gate_gemm(tmX, tmG, r, st));
+}
+
+moe_status moe_gate_logits(int32_t T, int32_t H, int32_t E, const void* x, const void* gate_w, float* logits,
+                           int32_t* dev_status, void* stream) {
+  if (T < 1 || H < 64 || !x || !gate_w || !logits) return MOE_ERR_INVALID_ARG;
+  if (H % 64 != 0 || E > 256 || E < 16 || E % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (any_misaligned(x, gate_w, logits)) return MOE_ERR_ALIGNMENT;
+  RouteArgs r{};
+  r.T = T;
+  r.H = H;
+  r.E = E;
+  r.logits = logits;
+  r.status = dev_status;
+  return gate_gemm(r, x, gate_w, as_stream(stream));
+}
+
 moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_w, const float* sel_bias,
                      float* logits, int32_t* topk_ids, float* topk_w, int32_t* expert_counts, void* stream) {
   if (!p || !topk_ids || !topk_w || !expert_counts || !logits) return MOE_ERR_INVALID_ARG;
@@ -169,15 +193,7 @@ moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_
               p->routed_scaling_factor, sel_bias, logits, topk_ids, topk_w, expert_counts, p->dev_status};
   cudaError_t e = cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * p->E, st);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (x) {
-    CUtensorMap tmX, tmG;
-    s = make_tmap(&tmX, x, false, p->H, p->T, 128);
-    if (s != MOE_OK) return s;
-    s = make_tmap(&tmG, gate_w, false, p->H, p->E, static_cast<uint32_t>(p->E));
-    if (s != MOE_OK) return s;
-    s = check_launch(launch_gate_gemm(tmX, tmG, r, st));
-    if (s != MOE_OK) return s;
-  }
+  if (x && (s = gate_gemm(r, x, gate_w, st)) != MOE_OK) return s;
   return check_launch(launch_route_tokens(r, nsm, st));
 }
 

@@ -123,7 +123,7 @@ perm_scan_kernel(int32_t* __restrict__ blockhist, int nb, int E, int total,
 // perm_hist) and are not written.
 constexpr int kPermKMax = 16;
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
 perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T, int k, int E,
                   const int32_t* __restrict__ blockbase, int32_t* __restrict__ slot_to_row,
                   int32_t* __restrict__ src_token, float* __restrict__ row_w,
@@ -176,9 +176,6 @@ perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ top
     }
   }
   if (!x_perm) return;                                 // metadata only
-  int rows[kPermKMax];
-#pragma unroll
-  for (int j = 0; j < kPermKMax; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
   const uint4* src = x + static_cast<size_t>(t) * vec_per_row;
   for (int base = 0; base < vec_per_row; base += 128) {   // same trip count on every lane
     uint4 val[4];
@@ -189,8 +186,10 @@ perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ top
     }
 #pragma unroll
     for (int j = 0; j < kPermKMax; ++j) {
-      if (j < k && rows[j] >= 0) {
-        uint4* dst = x_perm + static_cast<size_t>(rows[j]) * vec_per_row;
+      if (j >= k) break;                                  // warp-uniform
+      const int row = __shfl_sync(0xffffffffu, my_row, j);   // the row of slot j (lane j holds it)
+      if (row >= 0) {
+        uint4* dst = x_perm + static_cast<size_t>(row) * vec_per_row;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int v = base + u * 32 + lane;
@@ -200,11 +199,11 @@ perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ top
     }
   }
   if (x_scale) {
-    for (int i = lane; i < nscale; i += 32) {
-      const float sc = x_scale[static_cast<size_t>(t) * nscale + i];
-#pragma unroll
-      for (int j = 0; j < kPermKMax; ++j)
-        if (j < k && rows[j] >= 0) x_perm_scale[static_cast<size_t>(rows[j]) * nscale + i] = sc;
+    for (int j = 0; j < k; ++j) {
+      const int row = __shfl_sync(0xffffffffu, my_row, j);
+      if (row < 0) continue;                              // warp-uniform
+      for (int i = lane; i < nscale; i += 32)
+        x_perm_scale[static_cast<size_t>(row) * nscale + i] = x_scale[static_cast<size_t>(t) * nscale + i];
     }
   }
 }

@@ -26,7 +26,7 @@ MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
 MOE_SOFTMAX, MOE_SIGMOID = 0, 1
 
 EXPORTED = [
-    "moe_route", "moe_permute_workspace_size", "moe_permute", "moe_permute_static_ws",
+    "moe_route", "moe_gate_logits", "moe_permute_workspace_size", "moe_permute", "moe_permute_static_ws",
     "moe_grouped_swiglu",
     "moe_gate_up_swiglu", "moe_gate_up_swiglu_gather", "moe_down_proj",
     "moe_gate_up_swiglu_with_shared", "moe_down_proj_with_shared", "moe_down_proj_combine",
@@ -72,6 +72,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     sig = {
         "moe_route": [ctypes.POINTER(RouteParams), _P, _P, _P, _P, _P, _P, _P, _P],
+        "moe_gate_logits": [_I, _I, _I, _P, _P, _P, _P, _P],
         "moe_permute_workspace_size": [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
         "moe_permute": [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
                         ctypes.c_size_t, _P, _P],
@@ -138,6 +139,11 @@ def moe_route(T, H, E, k, n_group, topk_group, scoring, norm_topk_prob, routed_s
     _check("moe_route", load_library().moe_route(
         ctypes.byref(p), _ptr(x), _ptr(gate_w), _ptr(sel_bias), _ptr(logits), _ptr(topk_ids),
         _ptr(topk_w), _ptr(expert_counts), _stream(stream)))
+
+
+def moe_gate_logits(T, H, E, x, gate_w, logits, dev_status=None, stream=None):
+    _check("moe_gate_logits", load_library().moe_gate_logits(
+        T, H, E, _ptr(x), _ptr(gate_w), _ptr(logits), _ptr(dev_status), _stream(stream)))
 
 
 def moe_permute_workspace_size(T, k, E) -> int:

@@ -71,6 +71,12 @@ def test_host_validation_rejects_before_launch():
     # group limit makes k impossible: 4 groups of 4, keep 1 -> at most 4 candidates
     p = N.RouteParams(16, 256, 16, 5, 4, 1, N.MOE_SIGMOID, 1, 2.5, None)
     assert lib.moe_route(ctypes.byref(p), fake, fake, None, fake, fake, fake, fake, None) == N.MOE_ERR_INVALID_ARG
+    # moe_gate_logits: T, H not a multiple of 64, E beyond 256, misaligned logits
+    assert lib.moe_gate_logits(0, 256, 16, fake, fake, fake, None, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_gate_logits(8, 200, 16, fake, fake, fake, None, None) == N.MOE_ERR_UNSUPPORTED
+    assert lib.moe_gate_logits(8, 256, 512, fake, fake, fake, None, None) == N.MOE_ERR_UNSUPPORTED
+    assert lib.moe_gate_logits(8, 256, 16, fake, None, fake, None, None) == N.MOE_ERR_INVALID_ARG
+    assert lib.moe_gate_logits(8, 256, 16, fake, fake, odd, None, None) == N.MOE_ERR_ALIGNMENT
     # moe_permute: missing workspace, too small workspace, unsupported E
     args = [fake, fake, fake, N.MOE_BF16, None, fake, None, fake, fake, fake, fake]
     assert lib.moe_permute(64, 4, 16, 256, *args, None, 0, None, None) == N.MOE_ERR_INVALID_ARG

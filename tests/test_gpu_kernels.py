@@ -138,6 +138,22 @@ def test_route_gate_gemm(name, T):
     print(f"{name} T={T}: near-tie tokens excluded {int(flagged.sum())}")
 
 
+@pytest.mark.parametrize("name,T", [("tiny", None), ("v3", None), ("v3", 1000)])
+def test_gate_logits_then_route_equals_route(name, T):
+    """moe_gate_logits followed by moe_route on those logits (x = NULL) is
+    moe_route in two calls: logits, ids, weights and counts bit for bit."""
+    cfg = _cfg(name)
+    T = T or cfg.T
+    inp = make_inputs(dataclasses.replace(cfg, T=T), device=DEV, experts=False, shared=False)
+    ids0, w0, c0, L0 = gpu_route(cfg, T, x=inp.x, gate=inp.gate, bias=inp.bias)
+    L1 = torch.full_like(L0, float("nan"))
+    N.moe_gate_logits(T, cfg.H, cfg.E, inp.x, inp.gate, L1)
+    ids1, w1, c1, _ = gpu_route(cfg, T, bias=inp.bias, logits=L1)
+    torch.cuda.synchronize()
+    assert torch.equal(L0, L1)
+    assert torch.equal(ids0, ids1) and torch.equal(w0, w1) and torch.equal(c0, c1)
+
+
 # --------------------------------------------------------------- permute
 def _ids_from_oracle(T, k, E, seed, skew=0.0):
     rng = np.random.default_rng(seed)
