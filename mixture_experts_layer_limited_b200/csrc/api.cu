@@ -111,7 +111,13 @@ bool env_on(const char* name) {
 // / single CTAs for both GEMMs, MOE_GEMM_PAIR_DOWN=1 pairs for down only;
 // MOE_GEMM_DB=1 / MOE_GEMM_SB=1 force two / one accumulator pairs for both,
 // MOE_DOWN_DB=1 two for down only; MOE_EPI8=1 / MOE_EPI4=1 force 8 / 4
-// epilogue warps for both.
+// epilogue warps for both; MOE_GEMM_WIDE=1 runs both on CTA pairs with two
+// weight sub-tiles per CTA where the shape allows (gate/up: I % 256 == 0,
+// down: H % 512 == 0).
+bool wide_pairs(bool gate_up, int I, int H) {
+  if (env_on("MOE_GEMM_1SM") || !env_on("MOE_GEMM_WIDE")) return false;
+  return gate_up ? I % 256 == 0 : H % 512 == 0;
+}
 bool bf16_on_pairs(bool gate_up) {
   if (env_on("MOE_GEMM_1SM")) return false;
   return env_on("MOE_GEMM_PAIR") || (!gate_up && env_on("MOE_GEMM_PAIR_DOWN"));
@@ -271,6 +277,19 @@ moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const
   const bool fp8 = w->dtype == MOE_E4M3;
   const bool pair = !fp8 && bf16_on_pairs(true);
   const int I = w->I;
+  if (!fp8 && wide_pairs(true, I, H)) {
+    moe_status s = make_tmap(&p->tmA, w->w13, false, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
+    if (s != MOE_OK) return s;
+    if ((s = make_token_tmaps(&p->tmB, a, false, H, rows)) != MOE_OK) return s;
+    // pair tile: 256 features; CTA r: gate rows [mb*256 + 128r, +128) and their up rows
+    p->g = GemmArgs{rows, H, w->groups, offsets, 2 * I, I / 256, 256, I, 256, 0, 256, 128, 1, 0,
+                    h_ws, I, nullptr, nullptr, nullptr, nullptr, dev_status};
+    p->g.kc = env_on("MOE_WIDE_K128") ? 2 : 1;   // 2 stages of 128 K instead of 4 of 64 K
+    p->g.epi_warps = epilogue_warps(true);
+    p->g.wide = 1;
+    p->fp8 = false;
+    return MOE_OK;
+  }
   moe_status s = make_tmap(&p->tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, pair ? 64 : 128);
   if (s != MOE_OK) return s;
   s = make_token_tmaps(&p->tmB, a, fp8, H, rows);
@@ -292,6 +311,19 @@ moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
   // the scatter form (combine fused in) runs on single CTAs, one accumulator pair
   const bool pair = !fp8 && !scatter && bf16_on_pairs(false);
   const int I = w->I;
+  if (!fp8 && !scatter && wide_pairs(false, I, H)) {
+    moe_status s = make_tmap(&p->tmA, w->w2, false, I, static_cast<uint64_t>(w->groups) * H, 128);
+    if (s != MOE_OK) return s;
+    if ((s = make_token_tmaps(&p->tmB, h, false, I, rows)) != MOE_OK) return s;
+    // pair tile: 512 output features; CTA r sub-tile s: w2 rows [mb*512 + 256s + 128r, +128)
+    p->g = GemmArgs{rows, I, w->groups, offsets, H, H / 512, 512, 256, 512, 256, 256, 128, 1, 0,
+                    out, H, row_w, nullptr, nullptr, nullptr, dev_status};
+    p->g.kc = env_on("MOE_WIDE_K128") ? 2 : 1;   // 2 stages of 128 K instead of 4 of 64 K
+    p->g.epi_warps = epilogue_warps(false);
+    p->g.wide = 1;
+    p->fp8 = false;
+    return MOE_OK;
+  }
   // the single-CTA bf16 kernel reads its 256 contiguous w2 rows as one box
   const bool one_box = !fp8;
   moe_status s = make_tmap(&p->tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H,
@@ -314,7 +346,10 @@ moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
 moe_status launch_plan(const GemmPlan& p, int epi, cudaStream_t st, int nsm, const GemmPlan* second = nullptr) {
 
   // one launch needs the same kernel form for both: single-CTA bf16, same tile shape
-  const bool one = second && !p.fp8 && !second->fp8 && p.g.cta_stride == 0 && second->g.cta_stride == 0 &&
+  // (or both on wide CTA pairs)
+  const bool same_form = (p.g.cta_stride == 0 && second && second->g.cta_stride == 0) ||
+                         (p.g.wide && second && second->g.wide);
+  const bool one = second && !p.fp8 && !second->fp8 && same_form &&
                    p.g.bn_max == second->g.bn_max && p.g.nbuf == second->g.nbuf && p.g.kc == second->g.kc &&
                    p.g.epi_warps == second->g.epi_warps;
   if (second && !one) {

@@ -36,7 +36,8 @@
 // The E4M3 variant accumulates each 128-wide K block separately in a TMEM
 // ring and promotes it with the fp32 block scales on the CUDA cores, since
 // the weight scale is per 128x128 block and the activation scale per 1x128.
-// A CTA-pair variant (tcgen05 cta_group::2) is kept as an option.
+// Two CTA-pair variants (tcgen05 cta_group::2: one or two weight sub-tiles
+// per CTA) are kept as options; at the V3 shape both are slower.
 #include "kernels.cuh"
 
 namespace moe {
@@ -682,6 +683,224 @@ grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
 }
 
 // ========================================================================
+// BF16 kernel on CTA pairs, two weight sub-tiles per CTA ("wide" pairs)
+// ========================================================================
+// A CTA pair computes a 512 x N tile: two tcgen05 cta_group::2 MMA streams
+// (M = 256 each) share the pair's token rows. Each CTA stages two 128-row
+// weight sub-tiles and N/2 of the tokens and holds 2 x 128 x N fp32 in its
+// TMEM (512 columns, one accumulator pair, as the single-CTA kernel). Per SM
+// and per 64 K that is 48 KB staged for the same 1024 MMA cycles the
+// single-CTA kernel stages 64 KB for (its 256 tokens are read by both CTAs
+// there), so four stages fit where that kernel holds three.
+//   GEMM1: CTA r sub-tile 0 = gate rows [mb*256 + 128r, +128), sub-tile 1 =
+//          the up rows of the same features: SiLU(gate) * up in-thread.
+//   GEMM2: CTA r sub-tile s = w2 rows [mb*512 + 256s + 128r, +128).
+// TWO: a second single-group problem (the shared expert) whose tiles come
+// first, as in the single-CTA kernel.
+constexpr int kWideStages = 4;           // of 64 K (KC = 1), or 2 of 128 K (KC = 2)
+
+template <int EPI, bool TWO, int EPIW, int KC>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * EPIW, 1)
+grouped_gemm_bf16_2sm_wide_kernel(const __grid_constant__ CUtensorMap tmA,
+                                  const __grid_constant__ TokenMaps tmB, const GemmArgs a,
+                                  const __grid_constant__ CUtensorMap tmA2,
+                                  const __grid_constant__ TokenMaps tmB2, const GemmArgs a2) {
+  constexpr int KB = 64;
+  constexpr int STAGES = kWideStages / KC;
+  constexpr uint32_t A_SUB = 128 * 128;         // one 128-row weight sub-tile x 64 K
+  constexpr uint32_t B_BYTES = 128 * 128;       // up to 128 token rows x 64 K
+  constexpr uint32_t CHUNK_BYTES = 2 * A_SUB + B_BYTES;
+  constexpr uint32_t STAGE_BYTES = KC * CHUNK_BYTES;
+  extern __shared__ __align__(1024) uint8_t dsmem[];
+  __shared__ Sched sched;
+  __shared__ __align__(16) __nv_bfloat16 stage_out[EPIW][32 * 32];
+  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
+  __shared__ uint64_t tmem_full, tmem_empty, drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(cluster_id_x());
+  const int npairs = static_cast<int>(nclusters_x());
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  auto sA = [&](int st, int sub, int c) { return smem + st * STAGE_BYTES + c * CHUNK_BYTES + sub * A_SUB; };
+  auto sB = [&](int st, int c) { return smem + st * STAGE_BYTES + c * CHUNK_BYTES + 2 * A_SUB; };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    mbar_init(&tmem_full, 1);
+    mbar_init(&tmem_empty, 2 * EPIW);             // every epilogue warp of both CTAs
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&tmB.box[i]);
+    if (TWO) {
+      tma_prefetch_desc(&tmA2);
+      for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&tmB2.box[i]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_2sm(&tmem_base_s, 512);
+    tmem_relinquish_2sm();
+  }
+  if (warp == 2) build_schedule(sched, a, lane);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                 // the peer's barriers exist before any remote signal
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int total2 = TWO ? tiles_of(a2.rows, a.bn_max, a2.n_mblk) : 0;
+  const int total = total2 + sched.tile_start[a.groups];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_once = policy_evict_first();
+      const uint64_t pol_reuse = policy_evict_normal();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = pair; t < total && !abort_flag; t += npairs) {
+        const bool sh = TWO && t < total2;
+        const GemmArgs& g = sh ? a2 : a;
+        const TileInfo ti = sh ? decode_in_segment(a2, 0, 0, a2.rows, t) : decode_tile(sched, a, t - total2);
+        const CUtensorMap* mA = sh ? &tmA2 : &tmA;
+        const TokenMaps* mB = sh ? &tmB2 : &tmB;
+        const int nk = g.K / KB;
+        const int half = ti.N >> 1;                       // tokens staged by each CTA
+        const int rows = (half + 15) & ~15;               // rows fetched (multiple of 16)
+        const uint32_t tx = 2u * KC * (2u * A_SUB + static_cast<uint32_t>(rows) * 128u);
+        const int a_lo = ti.g * g.a_rows_per_group + ti.mb * g.mblk_stride + static_cast<int>(rank) * g.cta_stride;
+        const int a_hi = a_lo + g.sub1_off;
+        const int b0 = ti.row0 + static_cast<int>(rank) * half;
+        const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;   // re-read by sibling token blocks
+        bool ok = true;
+        for (int ks = 0; ks < nk / KC; ++ks) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
+          const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
+#pragma unroll
+          for (int c = 0; c < KC; ++c) {
+            const int kb = ks * KC + c;
+            tma_load_2d_2sm(sA(stage, 0, c), mA, fb, kb * KB, a_lo, pol_w);
+            tma_load_2d_2sm(sA(stage, 1, c), mA, fb, kb * KB, a_hi, pol_w);
+            uint8_t* bdst = sB(stage, c);
+            load_token_rows(rows, [&](int which, int off) {
+              tma_load_2d_2sm(bdst + off * 128, &mB->box[which], fb, kb * KB, b0 + off, pol_x);
+            });
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      if (abort_flag) {   // copies complete on the leader's barrier: give them time to land
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, it = 0;
+      for (int t = pair; t < total && !abort_flag; t += npairs, ++it) {
+        const bool sh = TWO && t < total2;
+        const TileInfo ti = sh ? decode_in_segment(a2, 0, 0, a2.rows, t) : decode_tile(sched, a, t - total2);
+        const int nk = (sh ? a2.K : a.K) / KB;
+        if (!mbar_wait(&tmem_empty, (it & 1u) ^ 1u, &abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t idesc = make_idesc(1u, 256u, static_cast<uint32_t>(ti.N));
+        bool ok = true;
+        for (int ks = 0; ks < nk / KC; ++ks) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < KC; ++c) {
+            const uint32_t a0 = smem_u32(sA(stage, 0, c)), a1 = smem_u32(sA(stage, 1, c));
+            const uint32_t b0 = smem_u32(sB(stage, c));
+#pragma unroll
+            for (int kk = 0; kk < KB / 16; ++kk) {
+              const uint32_t acc = (ks | c | kk) != 0;
+              const uint64_t bd = sw128_desc(b0 + kk * 32);
+              umma_bf16_2sm(tmem_base, sw128_desc(a0 + kk * 32), bd, idesc, acc);
+              umma_bf16_2sm(tmem_base + 256u, sw128_desc(a1 + kk * 32), bd, idesc, acc);
+            }
+          }
+          umma_commit_2sm(&empty_bar[stage], 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_2sm(&tmem_full, 0x3);
+      }
+      umma_commit_2sm(&drain_bar, 0x1);             // every MMA done before TMEM is freed
+      mbar_wait_drain(&drain_bar, 0);
+    }
+  } else {
+    // epilogue warps 2 .. 1+EPIW: warp w reads TMEM lanes 32*(w%4)..+31 of
+    // both sub-tiles; with 8 or 12 warps, two or three share each lane
+    // quarter and take turns on its 32-token chunks
+    const int q = warp & 3;
+    const int c0 = (warp - 2) / 4, cstep = EPIW / 4;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    const uint32_t empty_addr = mapa_shared(smem_u32(&tmem_empty), 0);
+    __nv_bfloat16* stg = stage_out[warp - 2];
+    uint32_t it = 0;
+    for (int t = pair; t < total; t += npairs, ++it) {
+      const bool sh = TWO && t < total2;
+      const GemmArgs& g = sh ? a2 : a;
+      const TileInfo ti = sh ? decode_in_segment(a2, 0, 0, a2.rows, t) : decode_tile(sched, a, t - total2);
+      if (!mbar_wait(&tmem_full, it & 1u, &abort_flag, a.status)) break;
+      tc_fence_after();
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out);
+      const int nchunk = (ti.N + 31) / 32;
+      const int fbase = ti.mb * g.feat_stride + 128 * static_cast<int>(rank) + 32 * q;
+      if (EPI == EPI_SWIGLU) {
+        for (int c = c0; c < nchunk; c += cstep) {
+          float gt[32], up[32];
+          tmem_ld32(lane_addr + c * 32, gt);
+          tmem_ld32(lane_addr + 256u + c * 32, up);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) gt[j] = silu(gt[j]) * up[j];
+          store_tile<32>(stg, gt, lane, out, g.out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, fbase);
+        }
+      } else {
+#pragma unroll 1
+        for (int s = 0; s < 2; ++s) {
+          for (int c = c0; c < nchunk; c += cstep) {
+            float v[32];
+            tmem_ld32(lane_addr + s * 256u + c * 32, v);
+            tmem_ld_wait();
+            if (g.row_w) {
+              const float wl = (c * 32 + lane < ti.n_valid) ? __ldg(g.row_w + ti.row0 + c * 32 + lane) : 0.0f;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wl, j);
+            }
+            store_tile<32>(stg, v, lane, out, g.out_ld, ti.row0 + c * 32, ti.n_valid - c * 32,
+                           fbase + s * g.feat_sub1);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(empty_addr);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                 // the pair is done with each other's memory
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_2sm(tmem_base, 512);
+}
+
+// ========================================================================
 // E4M3 kernel (block-scaled, promotion on CUDA cores), tokens per tile <= 32
 // ========================================================================
 constexpr int kF8Bn = 32;          // max tokens per tile
@@ -916,6 +1135,9 @@ size_t gemm_bf16_smem_bytes(int stages, int bn_max) {
 size_t gemm_bf16_2sm_smem_bytes() {
   return static_cast<size_t>(k2smStages) * k2smChunks * (2 * 128 * 128) + 1024;
 }
+size_t gemm_bf16_2sm_wide_smem_bytes() {
+  return static_cast<size_t>(kWideStages) * (3 * 128 * 128) + 1024;
+}
 size_t gemm_e4m3_smem_bytes(int stages) {
   return static_cast<size_t>(stages) * (2 * 128 * 128 + kF8Bn * 128) + 1024;
 }
@@ -945,9 +1167,35 @@ Bf16Kernel bf16_kernel(bool two, bool k128, int epi_warps) {
                         : bf16_kernel_w<EPI, STAGES, STAGES_K128, 4>(two, k128);
 }
 
+template <int EPI, bool TWO, int KC>
+Bf16Kernel wide_kernel_k(int epi_warps) {
+  if (epi_warps == 12) return grouped_gemm_bf16_2sm_wide_kernel<EPI, TWO, 12, KC>;
+  return epi_warps == 8 ? grouped_gemm_bf16_2sm_wide_kernel<EPI, TWO, 8, KC>
+                        : grouped_gemm_bf16_2sm_wide_kernel<EPI, TWO, 4, KC>;
+}
+template <int EPI, bool TWO>
+Bf16Kernel wide_kernel(int epi_warps, bool k128) {
+  return k128 ? wide_kernel_k<EPI, TWO, 2>(epi_warps) : wide_kernel_k<EPI, TWO, 1>(epi_warps);
+}
+
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const TokenMaps& tmB,
                                 const GemmArgs& a, int grid, cudaStream_t stream, const SecondProblem* two) {
-  if (!e4m3 && a.cta_stride > 0) {
+  if (!e4m3 && a.cta_stride > 0 && a.wide) {
+    const int epiw = a.epi_warps == 8 || a.epi_warps == 12 ? a.epi_warps : 4;
+    const bool pair2 = two != nullptr;
+    const bool k128 = a.kc == 2;
+    Bf16Kernel kern = epi == EPI_SWIGLU ? (pair2 ? wide_kernel<EPI_SWIGLU, true>(epiw, k128)
+                                                 : wide_kernel<EPI_SWIGLU, false>(epiw, k128))
+                                        : (pair2 ? wide_kernel<EPI_WEIGHTED, true>(epiw, k128)
+                                                 : wide_kernel<EPI_WEIGHTED, false>(epiw, k128));
+    const size_t smem = gemm_bf16_2sm_wide_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    if (pair2)
+      kern<<<grid & ~1, 64 + 32 * epiw, smem, stream>>>(tmA, tmB, a, two->tmA, two->tmB, two->a);
+    else
+      kern<<<grid & ~1, 64 + 32 * epiw, smem, stream>>>(tmA, tmB, a, tmA, tmB, a);
+  } else if (!e4m3 && a.cta_stride > 0) {
     const size_t smem = gemm_bf16_2sm_smem_bytes();
     auto kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_2sm_kernel<EPI_SWIGLU>
                                   : grouped_gemm_bf16_2sm_kernel<EPI_WEIGHTED>;

@@ -38,6 +38,8 @@ struct GemmArgs {
   // number of tokens (rows of the fp32 accumulator `out`)
   const int32_t* scatter_tok;
   int32_t scatter_T;
+  // CTA-pair kernel with two weight sub-tiles per CTA (512 weight rows a pair)
+  int32_t wide;
 };
 
 struct RouteArgs {

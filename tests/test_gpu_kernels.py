@@ -257,18 +257,26 @@ def _ref_grouped(a, w13, w2, off, row_w):
     return out, hs
 
 
-@pytest.fixture(params=["pair", "1sm-sb", "1sm-sb-epi4", "1sm-sb-epi8", "1sm-db", "1sm-db-k64"])
+@pytest.fixture(params=["pair", "wide", "wide-epi8", "wide-k128", "1sm-sb", "1sm-sb-epi4", "1sm-sb-epi8", "1sm-db",
+                        "1sm-db-k64"])
 def gemm_variant(request, monkeypatch):
-    """bf16 grouped GEMMs, each kernel forced: CTA pairs, or single CTAs with
-    one TMEM accumulator pair (epilogue warps per GEMM: 4 gate/up, 12 down; or
-    4 / 8 for both) or
-    with two (stages of 128 K, or of 64 K for k64)."""
-    for var in ("MOE_GEMM_1SM", "MOE_GEMM_PAIR", "MOE_GEMM_DB", "MOE_GEMM_SB", "MOE_DOWN_K64",
-                "MOE_DOWN_DB", "MOE_EPI4", "MOE_EPI8"):
+    """bf16 grouped GEMMs, each kernel forced: CTA pairs (one 128-row weight
+    sub-tile per CTA, or two: "wide", where the shape allows, with stages of
+    64 K or of 128 K), or single CTAs
+    with one TMEM accumulator pair (epilogue warps per GEMM: 4 gate/up, 12
+    down; or 4 / 8 for both) or with two (stages of 128 K, or of 64 K for k64)."""
+    for var in ("MOE_GEMM_1SM", "MOE_GEMM_PAIR", "MOE_GEMM_WIDE", "MOE_WIDE_K128", "MOE_GEMM_DB", "MOE_GEMM_SB",
+                "MOE_DOWN_K64", "MOE_DOWN_DB", "MOE_EPI4", "MOE_EPI8"):
         monkeypatch.delenv(var, raising=False)
     v = request.param
     if v == "pair":
         monkeypatch.setenv("MOE_GEMM_PAIR", "1")
+    elif v.startswith("wide"):
+        monkeypatch.setenv("MOE_GEMM_WIDE", "1")
+        if v.endswith("epi8"):
+            monkeypatch.setenv("MOE_EPI8", "1")
+        if v.endswith("k128"):
+            monkeypatch.setenv("MOE_WIDE_K128", "1")
     else:
         monkeypatch.setenv("MOE_GEMM_1SM", "1")
         monkeypatch.setenv("MOE_GEMM_DB" if v.startswith("1sm-db") else "MOE_GEMM_SB", "1")
