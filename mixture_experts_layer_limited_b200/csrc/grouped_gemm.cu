@@ -180,6 +180,7 @@ __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __e
 // async proxy; it keeps one stage of copies in flight ahead of that.
 constexpr int kGatherThreads = 64;
 
+
 // TWO: a second single-group problem a2 (the shared expert: its own weights
 // tmA2, token rows tmB2 and output) runs in the same launch. Its tiles come
 // first in the tile order, so the routed experts' ragged tiles fill the tail.
@@ -391,10 +392,33 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       const int feat_sub1 = sh ? a2.feat_sub1 : a.feat_sub1;
       const float* row_w = sh ? a2.row_w : a.row_w;
       const uint32_t bi = nbuf == 2 ? (it & 1u) : 0u, use = nbuf == 2 ? (it >> 1) : it;
+      const int nchunk = (ti.N + 31) / 32;
+      // GEMM2: the routing weights (and, for the scatter, the tokens) of this
+      // warp's 32-row chunks, fetched before the accumulator is ready so that
+      // their latency overlaps the wait instead of each chunk's epilogue
+      // 32-row chunks of a tile (at most 8) an epilogue warp handles at most
+      constexpr int kEpiChunks = (8 + EPIW / 4 - 1) / (EPIW / 4);
+      float wpre[kEpiChunks];
+      int tpre[kEpiChunks];
+      if (EPI != EPI_SWIGLU) {
+        const int32_t* src = sh ? a2.scatter_tok : a.scatter_tok;
+        const int ntok = sh ? a2.scatter_T : a.scatter_T;
+#pragma unroll
+        for (int u = 0; u < kEpiChunks; ++u) {
+          const int r = (c0 + u * cstep) * 32 + lane;            // row within the tile
+          const bool valid = c0 + u * cstep < nchunk && r < ti.n_valid;
+          wpre[u] = (row_w && valid) ? __ldg(row_w + ti.row0 + r) : 0.0f;
+          int tok = -1;
+          if (EPI == EPI_SCATTER && valid) {
+            tok = src ? __ldg(src + ti.row0 + r) : ti.row0 + r;   // routed rows through src_token
+            if (tok >= ntok) { flag_status(a.status, MOE_DEVSTAT_BAD_EXPERT_ID); tok = -1; }
+          }
+          tpre[u] = tok;
+        }
+      }
       if (!mbar_wait(&tmem_full[bi], use & 1u, &abort_flag, a.status)) break;
       tc_fence_after();
       const uint32_t acc_addr = lane_addr + bi * 2u * sub_cols;
-      const int nchunk = (ti.N + 31) / 32;
       __nv_bfloat16* stg = stage_out[warp - 2];
       if (EPI == EPI_SWIGLU) {
         const int feat0 = ti.mb * feat_stride + 32 * q;            // this warp's 32 features
@@ -411,26 +435,22 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll 1
         for (int s = 0; s < 2; ++s) {
           const int feat0 = ti.mb * feat_stride + s * feat_sub1 + 32 * q;
-          for (int c = c0; c < nchunk; c += cstep) {
+#pragma unroll
+          for (int u = 0; u < kEpiChunks; ++u) {
+            const int c = c0 + u * cstep;
+            if (c >= nchunk) break;                                  // warp-uniform
             float v[32];
             tmem_ld32(acc_addr + s * sub_cols + c * 32, v);
             tmem_ld_wait();
             if (row_w) {
-              const float wl = (c * 32 + lane < ti.n_valid) ? __ldg(row_w + ti.row0 + c * 32 + lane) : 0.0f;
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wl, j);
+              for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wpre[u], j);
             }
             if (EPI == EPI_SCATTER) {
-              // row -> token (routed rows through src_token, shared rows are tokens)
-              const int32_t* src = sh ? a2.scatter_tok : a.scatter_tok;
-              const int ntok = sh ? a2.scatter_T : a.scatter_T;
-              const int r = ti.row0 + c * 32 + lane;
-              int tok = c * 32 + lane < ti.n_valid ? (src ? __ldg(src + r) : r) : -1;
-              if (tok >= ntok) { flag_status(a.status, MOE_DEVSTAT_BAD_EXPERT_ID); tok = -1; }
               float* acc_out = reinterpret_cast<float*>(sh ? a2.out : a.out);
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
-                const int tj = __shfl_sync(0xffffffffu, tok, j);
+                const int tj = __shfl_sync(0xffffffffu, tpre[u], j);
                 if (tj >= 0) atomicAdd(acc_out + static_cast<size_t>(tj) * out_ld + feat0 + lane, v[j]);
               }
             } else {
