@@ -109,6 +109,10 @@ typedef int32_t moe_scoring;
  * Limits: 1 <= k <= 16, E % 16 == 0, 16 <= E <= 256, E % n_group == 0,
  *   n_group <= 32, topk_group <= n_group, k <= topk_group * E / n_group,
  *   H % 64 == 0 when x != NULL. Otherwise MOE_ERR_INVALID_ARG/UNSUPPORTED.
+ * A token none of whose candidate experts has a score that compares (all
+ *   NaN; with n_group > 1 the dropped groups' experts score -inf and still
+ *   compare) gets ids -1 and weights 0, is counted nowhere, and flags
+ *   MOE_DEVSTAT_BAD_EXPERT_ID in p->dev_status.
  * ------------------------------------------------------------------------ */
 typedef struct {
     int32_t T, H, E, k;

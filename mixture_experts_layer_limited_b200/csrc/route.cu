@@ -17,6 +17,8 @@
 //       groups are scored by the sum of their two best selection scores and
 //       ranked with shuffles, and the top-k is k rounds of a warp arg-max
 //       (larger score first, lower expert index on ties).
+#include <cstdlib>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -299,22 +301,173 @@ route_tokens_kernel(const RouteArgs r) {
         const int oe = __shfl_xor_sync(0xffffffffu, be, d);
         if (beats(v, be, ov, oe)) { v = ov; be = oe; }
       }
-      const int owner = be & 31, slot = be >> 5;
+      const bool found = be < r.E;                     // false only when no score compares (NaN)
+      const int owner = be & 31, slot = found ? be >> 5 : 0;
       float u = 0.0f;
 #pragma unroll
       for (int i = 0; i < kEpl; ++i)
         if (i == slot) u = unb[i];
       u = __shfl_sync(0xffffffffu, u, owner);
-      if (lane == owner) taken |= 1u << slot;
-      if (lane == j) { my_id = be; my_w = u; }
+      if (found && lane == owner) taken |= 1u << slot;
+      if (lane == j) { my_id = found ? be : -1; my_w = found ? u : 0.0f; }
     }
     float sum = 0.0f;
     for (int j = 0; j < r.k; ++j) sum += __shfl_sync(0xffffffffu, my_w, j);
     if (lane < r.k) {
       const float w = (r.norm ? my_w / sum : my_w) * r.scale;
       r.ids[static_cast<size_t>(tok) * r.k + lane] = my_id;
-      r.w[static_cast<size_t>(tok) * r.k + lane] = w;
-      atomicAdd(&hist[my_id], 1);
+      r.w[static_cast<size_t>(tok) * r.k + lane] = my_id >= 0 ? w : 0.0f;
+      if (my_id >= 0) atomicAdd(&hist[my_id], 1);
+      else flag_status(r.status, MOE_DEVSTAT_BAD_EXPERT_ID);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < r.E; e += blockDim.x)
+    if (hist[e]) atomicAdd(r.counts + e, hist[e]);
+}
+
+// ------------------------------------------------------------------------
+// Routing, eight threads per token (E = 8C experts, C <= 32; n_group | 8;
+// k <= 8): thread p of a token holds experts [pC, pC + C) in registers, so
+// a group of E / n_group experts is whole threads and its top-2 merges over
+// 8 / n_group threads by shuffles; the top-k is k rounds of an arg-max over
+// the 8 threads; thread j < k writes slot j. The same decisions and weights
+// as route_tokens_kernel (same scores, same order, same sums), in about half
+// the instructions per token.
+// ------------------------------------------------------------------------
+template <int C>
+__device__ __forceinline__ void load_scores(const float* src, float (&s)[C]) {
+  if constexpr (C % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < C / 4; ++i) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(src) + i);
+      s[4 * i] = v.x; s[4 * i + 1] = v.y; s[4 * i + 2] = v.z; s[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < C / 2; ++i) {
+      const float2 v = __ldg(reinterpret_cast<const float2*>(src) + i);
+      s[2 * i] = v.x; s[2 * i + 1] = v.y;
+    }
+  }
+}
+
+template <int C>
+__global__ void __launch_bounds__(256, 2)
+route_tokens_g8_kernel(const RouteArgs r) {
+  __shared__ int hist[256];
+  __shared__ float bias_s[256];
+  for (int e = threadIdx.x; e < r.E; e += blockDim.x) {
+    hist[e] = 0;
+    bias_s[e] = r.bias ? r.bias[e] : 0.0f;
+  }
+  __syncthreads();
+  constexpr uint32_t kAll = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const int p = lane & 7;                            // this thread's part of its token
+  const int gl0 = lane & 24;                         // the token's first lane
+  const bool sig = r.scoring == MOE_SIGMOID;
+  const bool has_bias = r.bias != nullptr;
+  const bool raw_logit = !sig && r.G == 1 && !has_bias;   // softmax, one group: select on logits
+  const int tpg = 8 / r.G;                           // threads per group
+  const int e0 = p * C;
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  // a warp routes four tokens per pass; every lane takes part in every shuffle
+  for (int wq = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wq * 4 < r.T; wq += nwarps) {
+    const int tok = wq * 4 + (lane >> 3);
+    const bool valid = tok < r.T;
+    const float* L = r.logits + static_cast<size_t>(valid ? tok : 0) * r.E;
+    float s[C];
+    load_scores<C>(L + e0, s);
+    // softmax: max and denominator over the token's E logits
+    float lmax = 0.0f;
+    double den = 1.0;
+    if (!sig) {
+      lmax = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < C; ++i) lmax = fmaxf(lmax, s[i]);
+#pragma unroll
+      for (int d = 1; d < 8; d <<= 1) lmax = fmaxf(lmax, __shfl_xor_sync(kAll, lmax, d));
+      double sum = 0.0;
+#pragma unroll
+      for (int i = 0; i < C; ++i) sum += exp(static_cast<double>(s[i]) - static_cast<double>(lmax));
+#pragma unroll
+      for (int d = 1; d < 8; d <<= 1) sum += __shfl_xor_sync(kAll, sum, d);
+      den = sum;
+    }
+    // selection scores, in place
+    if (!raw_logit) {
+#pragma unroll
+      for (int i = 0; i < C; ++i) {
+        const float u = sig ? sigmoid_rn(s[i])
+                            : static_cast<float>(exp(static_cast<double>(s[i]) - static_cast<double>(lmax)) / den);
+        s[i] = has_bias ? u + bias_s[e0 + i] : u;
+      }
+    }
+    if (r.G > 1) {
+      // group score = fp32 sum of the group's two largest selection scores
+      float m1 = -INFINITY, m2 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < C; ++i) {
+        const float v = s[i];
+        if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
+      }
+      for (int d = 1; d < tpg; d <<= 1) {             // the two largest of both halves
+        const float o1 = __shfl_xor_sync(kAll, m1, d), o2 = __shfl_xor_sync(kAll, m2, d);
+        const float hi = fmaxf(m1, o1), lo = fminf(m1, o1);
+        m2 = fmaxf(lo, fmaxf(m2, o2));
+        m1 = hi;
+      }
+      const float gs = m1 + m2;
+      // keep the topk_group best groups (lower group index first on ties)
+      const int my_g = p / tpg;
+      int rank_g = 0;
+      for (int j = 0; j < r.G; ++j) {
+        const float o = __shfl_sync(kAll, gs, gl0 + j * tpg);
+        rank_g += (o > gs || (o == gs && j < my_g)) ? 1 : 0;
+      }
+      if (rank_g >= r.g) {
+#pragma unroll
+        for (int i = 0; i < C; ++i) s[i] = -INFINITY;
+      }
+    }
+    // top-k: k rounds of an arg-max over the token's 8 threads
+    uint32_t taken = 0;
+    int my_id = 0;
+    for (int j = 0; j < r.k; ++j) {
+      float v = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < C; ++i)
+        if (!((taken >> i) & 1u) && beats(v, be, s[i], e0 + i)) { v = s[i]; be = e0 + i; }
+#pragma unroll
+      for (int d = 1; d < 8; d <<= 1) {
+        const float ov = __shfl_xor_sync(kAll, v, d);
+        const int oe = __shfl_xor_sync(kAll, be, d);
+        if (beats(v, be, ov, oe)) { v = ov; be = oe; }
+      }
+      const int rel = be - e0;
+      if (rel >= 0 && rel < C) taken |= 1u << rel;
+      if (p == j) my_id = be;
+    }
+    // weights: the unbiased score of slot p's expert, renormalised over the
+    // k slots in slot order, times the scaling factor
+    // (no expert wins a round only when no score compares, i.e. all are
+    // NaN: the slot gets id -1, flagged, and counts nowhere)
+    const bool has_id = my_id >= 0 && my_id < r.E;
+    float u = 0.0f;
+    if (p < r.k && valid && has_id) {
+      const float lv = L[my_id];
+      u = sig ? sigmoid_rn(lv) : static_cast<float>(exp(static_cast<double>(lv) - static_cast<double>(lmax)) / den);
+    }
+    float sum = 0.0f;
+    for (int j = 0; j < r.k; ++j) sum += __shfl_sync(kAll, u, gl0 + j);
+    if (p < r.k && valid) {
+      const float w = (r.norm ? u / sum : u) * r.scale;
+      r.ids[static_cast<size_t>(tok) * r.k + p] = has_id ? my_id : -1;
+      r.w[static_cast<size_t>(tok) * r.k + p] = has_id ? w : 0.0f;
+      if (has_id) atomicAdd(&hist[my_id], 1);
+      else flag_status(r.status, MOE_DEVSTAT_BAD_EXPERT_ID);
     }
   }
   __syncthreads();
@@ -339,6 +492,22 @@ cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, con
 }
 
 cudaError_t launch_route_tokens(const RouteArgs& r, int num_sms, cudaStream_t stream) {
+  // eight threads per token where the shape allows (MOE_ROUTE_WARP=1: always a warp)
+  const char* force_warp = std::getenv("MOE_ROUTE_WARP");
+  const int C = r.E / 8;
+  if (!(force_warp && force_warp[0] == '1') && r.E % 8 == 0 && r.k <= 8 && 8 % r.G == 0 &&
+      (C == 2 || C == 4 || C == 8 || C == 16 || C == 32)) {
+    const int need = (r.T + 31) / 32;                 // 32 tokens per CTA of 256 threads
+    const int grid = need < 4 * num_sms ? need : 4 * num_sms;
+    switch (C) {
+      case 2: route_tokens_g8_kernel<2><<<grid, 256, 0, stream>>>(r); break;
+      case 4: route_tokens_g8_kernel<4><<<grid, 256, 0, stream>>>(r); break;
+      case 8: route_tokens_g8_kernel<8><<<grid, 256, 0, stream>>>(r); break;
+      case 16: route_tokens_g8_kernel<16><<<grid, 256, 0, stream>>>(r); break;
+      default: route_tokens_g8_kernel<32><<<grid, 256, 0, stream>>>(r); break;
+    }
+    return cudaGetLastError();
+  }
   const int need = (r.T + kRouteWarps - 1) / kRouteWarps;
   const int grid = need < 8 * num_sms ? need : 8 * num_sms;
   route_tokens_kernel<<<grid, kRouteWarps * 32, 0, stream>>>(r);

@@ -138,6 +138,66 @@ def test_route_gate_gemm(name, T):
     print(f"{name} T={T}: near-tie tokens excluded {int(flagged.sum())}")
 
 
+@pytest.mark.parametrize("name,T,topk_group", [("tiny", None, None), ("tiny_grouped", None, None),
+                                               ("v2lite", None, None), ("v3", None, None), ("v3", 1001, 2),
+                                               ("v3", 77, 8), ("v3_ties", 777, None), ("v2lite", 1, None)])
+def test_route_eight_threads_per_token_matches_warp_per_token(name, T, topk_group, monkeypatch):
+    """The two routing kernels (eight threads per token, the default where the
+    shape allows; one warp per token) take the same decisions: ids and counts
+    bit for bit, weights bit for bit with sigmoid scores and to the last bit
+    of the softmax denominator's summation order otherwise."""
+    cfg = _cfg(name)
+    if topk_group:
+        cfg = dataclasses.replace(cfg, topk_group=topk_group)
+    T = T or cfg.T
+    L = make_logits(cfg, device=DEV, T=T)
+    bias = uniform_bias(cfg.E, cfg.seed + 5) if cfg.scoring == "sigmoid" else None
+    if name == "v3_ties":
+        L = torch.round(L * 4) / 4
+        bias = torch.round(bias * 50) / 50
+    monkeypatch.delenv("MOE_ROUTE_WARP", raising=False)
+    ids0, w0, c0, _ = gpu_route(cfg, T, bias=bias, logits=L)
+    monkeypatch.setenv("MOE_ROUTE_WARP", "1")
+    ids1, w1, c1, _ = gpu_route(cfg, T, bias=bias, logits=L)
+    torch.cuda.synchronize()
+    assert torch.equal(ids0, ids1) and torch.equal(c0, c1)
+    if cfg.scoring == "sigmoid":
+        assert torch.equal(w0, w1)
+    else:
+        torch.testing.assert_close(w0, w1, rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("warp", [False, True])
+def test_route_token_with_nan_scores_is_flagged_not_routed(warp, monkeypatch):
+    """Without a group limit, a token whose logits are all NaN has no winner
+    in any round: its slots get id -1 and weight 0, the status word is
+    flagged, nothing is counted for it, and the other tokens route as usual.
+    (With a group limit the experts of the dropped groups score -inf, which
+    still compares, so such a token is routed there with NaN weights.)"""
+    if warp:
+        monkeypatch.setenv("MOE_ROUTE_WARP", "1")
+    else:
+        monkeypatch.delenv("MOE_ROUTE_WARP", raising=False)
+    cfg = dataclasses.replace(get_config("v3"), n_group=1, topk_group=1)
+    T = 64
+    L = make_logits(cfg, device=DEV, T=T)
+    L[5] = float("nan")
+    bias = uniform_bias(cfg.E, cfg.seed + 5)
+    ids = torch.empty(T, cfg.k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, cfg.k, dtype=torch.float32, device=DEV)
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    N.moe_route(T, cfg.H, cfg.E, cfg.k, cfg.n_group, cfg.topk_group, N.MOE_SIGMOID, cfg.norm_topk_prob,
+                cfg.scale, None, None, bias, L, ids, w, counts, status)
+    torch.cuda.synchronize()
+    assert N.moe_read_device_status(status) & N.MOE_DEVSTAT_BAD_EXPERT_ID
+    assert torch.all(ids[5] == -1) and torch.all(w[5] == 0)
+    keep = np.array([t for t in range(T) if t != 5])
+    r = oracle_route(np32(L[torch.as_tensor(keep, device=DEV)]), cfg, np32(bias))
+    assert np.array_equal(ids.cpu().numpy()[keep], r.ids)
+    assert int(counts.sum()) == (T - 1) * cfg.k
+
+
 @pytest.mark.parametrize("name,T", [("tiny", None), ("v3", None), ("v3", 1000)])
 def test_gate_logits_then_route_equals_route(name, T):
     """moe_gate_logits followed by moe_route on those logits (x = NULL) is
