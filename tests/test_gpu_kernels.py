@@ -224,10 +224,22 @@ def _ids_from_oracle(T, k, E, seed, skew=0.0):
     return r.ids, r.weights.astype(np.float32)
 
 
+@pytest.fixture(params=["lsu", "bulk"])
+def perm_copy(request, monkeypatch):
+    """The permutation's row copies: by the threads' own 16-byte loads and
+    stores (the default) or on the bulk-copy engine."""
+    if request.param == "bulk":
+        monkeypatch.setenv("MOE_PERM_BULK", "1")
+    else:
+        monkeypatch.delenv("MOE_PERM_BULK", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("T,k,E,H,skew", [(64, 4, 16, 256, 0.0), (8192, 8, 256, 7168, 0.0),
                                           (1000, 6, 64, 2048, 0.0), (2000, 8, 256, 512, 3.0),
-                                          (1, 1, 16, 256, 0.0), (3, 16, 16, 128, 0.0)])
-def test_permute_bit_exact(T, k, E, H, skew):
+                                          (1, 1, 16, 256, 0.0), (3, 16, 16, 128, 0.0),
+                                          (50, 2, 16, 28672, 0.0)])
+def test_permute_bit_exact(T, k, E, H, skew, perm_copy):
     ids_np, w_np = _ids_from_oracle(T, k, E, seed=T + E, skew=skew)
     offsets_o, src_o, s2r_o = oracle.permute(ids_np, E)
     ids = torch.from_numpy(ids_np).to(DEV)
@@ -250,7 +262,7 @@ def test_permute_bit_exact(T, k, E, H, skew):
     assert torch.equal(xp, x[torch.from_numpy(src_o).to(DEV)])
 
 
-def test_permute_e4m3_rows_and_scales():
+def test_permute_e4m3_rows_and_scales(perm_copy):
     T, k, E, H = 300, 8, 64, 512
     ids_np, w_np = _ids_from_oracle(T, k, E, seed=9)
     _, src_o, _ = oracle.permute(ids_np, E)
@@ -270,7 +282,7 @@ def test_permute_e4m3_rows_and_scales():
     assert torch.equal(xps, xs[idx])
 
 
-def test_permute_flags_out_of_range_ids_without_writing_outside():
+def test_permute_flags_out_of_range_ids_without_writing_outside(perm_copy):
     T, k, E, H = 128, 4, 16, 256
     ids_np, w_np = _ids_from_oracle(T, k, E, seed=10)
     ids_np = ids_np.copy()
