@@ -7,16 +7,19 @@
 // top-2, topk_group = 4 kept, top-8 within, renormalise, x routed_scaling_factor);
 // the xxqk.cn digest §2.2 (bias only steers selection; device-limited routing).
 //
-// Two kernels:
+// Two launches:
 //   gate_gemm_pair_kernel  logits = x . gate^T on tcgen05. A cluster of two
 //       CTAs takes 128 tokens: CTA r accumulates over half r of the hidden
 //       size in its own TMEM (M = 128 tokens, N = E, fp32), then the two swap,
 //       through distributed shared memory, the partial sums of the 64 tokens
 //       the other one writes out. Every logit is (first half) + (second half).
-//   route_tokens_kernel  one warp per token: lane l scores experts l, l+32, ...,
-//       groups are scored by the sum of their two best selection scores and
-//       ranked with shuffles, and the top-k is k rounds of a warp arg-max
-//       (larger score first, lower expert index on ties).
+//   route_tokens_g8_kernel  eight threads per token, each holding E/8
+//       consecutive experts (where E, n_group and k allow; otherwise
+//       route_tokens_kernel, one warp per token, lane l holding experts l,
+//       l+32, ...): groups are scored by the sum of their two best selection
+//       scores and ranked with shuffles, and the top-k is k rounds of an
+//       arg-max over the token's threads (larger score first, lower expert
+//       index on ties).
 #include <cstdlib>
 
 #include "kernels.cuh"
