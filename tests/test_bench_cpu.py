@@ -29,3 +29,30 @@ def test_reference_arm_other_ranks_exit_quietly():
                          capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
     assert out.returncode == 0
     assert not [l for l in out.stdout.splitlines() if l.startswith("{")]
+
+
+def test_every_layer_stage_has_a_launch_count_and_a_cost_model():
+    """Each stage name a layer can produce (default, shared expert apart,
+    gather, fused combine; E4M3 adds quantize_x) is known to the benchmark's
+    launch count and per-stage cost model, for every configuration."""
+    sys.path.insert(0, ROOT)
+    import torch
+    import bench
+    from moe_inputs import CONFIGS
+    from mixture_experts_layer_limited_b200 import MoELayer, LayerSpec
+    for name, cfg in CONFIGS.items():
+        if cfg.dtype != "bf16":
+            continue
+        spec = LayerSpec.from_config(cfg)
+        H, E, I, Is, T = cfg.H, cfg.E, cfg.I, cfg.I_s, 4
+        z = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+        model = bench.stage_model(cfg)
+        for kw in ({}, {"fuse_shared": False}, {"gather": True}, {"fuse_combine": True}):
+            # shapes only: stages() builds the launch closures without running them
+            lay = MoELayer(spec, z(E, 8), z(1, 1), z(1, 1), z(1, 1) if Is else None,
+                           z(1, 1) if Is else None, None, T, **kw)
+            names = [n for n, _ in lay.stages(z(T, H))] + ["bias_update"]
+            for n in names:
+                assert n in bench.LAUNCHES and n in model, (name, kw, n)
+                assert bench.launches_of(n, cfg) >= 1
+    assert "quantize_x" in bench.LAUNCHES
