@@ -217,10 +217,10 @@ def gemm_source_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(stage):
+def profiled_traffic(stage, workload):
     """DRAM bytes per launch of the gate/up GEMM from the committed ncu
-    summary, only if it was taken of this stage's launch and the GEMM source
-    has not changed since."""
+    summary, only if it was taken of this stage's launch, scaled to this
+    workload, and the GEMM source has not changed since."""
     if not os.path.exists(PROFILE_TRAFFIC):
         return None
     kv = {}
@@ -228,7 +228,8 @@ def profiled_traffic(stage):
         if ":" in line:
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
-    if kv.get("gemm_source_sha256_16") != gemm_source_hash() or kv.get("stage") != stage:
+    if (kv.get("gemm_source_sha256_16") != gemm_source_hash() or kv.get("stage") != stage
+            or kv.get("workload") != workload):
         return None
     try:
         return float(kv["traffic_bytes_per_launch_full_size"])
@@ -368,7 +369,7 @@ def run_ours(args):
     what = "routed experts + shared expert, one launch" if dom == "gate_up" else "routed experts"
     roofline = {"kernel": f"grouped_gemm_bf16 (gate/up + SwiGLU, {what})", "bound": "tensor",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(dom),
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(dom, cfg.name),
                 "peak_note": f"bf16 sustained, {peaks['source']} (MEASURED_PEAKS.json)",
                 "algorithmic_flops_per_launch": model[dom]["flops"],
                 "algorithmic_bytes_per_launch": model[dom]["bytes"]}
