@@ -126,3 +126,41 @@ def test_host_validation_rejects_before_launch():
     assert lib.moe_quantize_rows(4, 128, odd, fake, fake, None) == N.MOE_ERR_ALIGNMENT
     assert lib.moe_read_device_status(None, None, None) == N.MOE_ERR_INVALID_ARG
     assert lib.moe_last_cuda_error() == 0
+
+
+def test_header_is_plain_c_and_a_c_program_links_and_calls_it(tmp_path):
+    """include/moe.h compiles as C99 (no C++ or torch types in the
+    boundary), and a C program linked against libmoe.so calls it: the ABI
+    version, a workspace size, and an argument check that fails before any
+    launch (no GPU needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    from mixture_experts_layer_limited_b200.build import lib_path
+    lib = lib_path()
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "use_moe.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "moe.h"
+int main(void) {
+  size_t ws = 0;
+  moe_status s = moe_permute_workspace_size(8192, 8, 256, &ws);
+  moe_status bad = moe_combine(0, 8, 7168, NULL, NULL, NULL, NULL, NULL, NULL);
+  printf("%d %d %zu %d %s\n", (int)moe_abi_version(), (int)s, ws, (int)bad, moe_status_string(bad));
+  return 0;
+}
+''')
+    exe = tmp_path / "use_moe"
+    cmd = [gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"), str(src), "-o", str(exe),
+           lib, "-Wl,-rpath," + os.path.dirname(lib)]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    ver, s, ws, bad, *msg = out.stdout.split()
+    assert int(ver) == N.load_library().moe_abi_version()
+    assert int(s) == N.MOE_OK and int(ws) == N.moe_permute_workspace_size(8192, 8, 256)
+    assert int(bad) == N.MOE_ERR_INVALID_ARG
