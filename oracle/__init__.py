@@ -16,7 +16,10 @@ Parity status per function (what pins each one is listed in the tests):
   gate_logits                                   pinned (identity gate)
   route_from_logits                             pinned (brute force, invariants)
   permute                                       pinned (worked example)
-  swiglu_ffn                                    pinned (closed form SiLU(1))
+  swiglu_hidden / swiglu_ffn                    pinned (closed forms SiLU(+-1),
+                                                SiLU(ln 3) = 3/4 ln 3; gate/up order)
+  combine                                       pinned (hand example, equals the
+                                                layer's own sum over slots)
   moe_forward                                   pinned (dense brute force,
                                                 combine identities)
   bias_update / load_cv                         pinned (closed forms)
@@ -26,12 +29,13 @@ Parity status per function (what pins each one is listed in the tests):
 from .moe_oracle import (
     e4m3_values, quantize_e4m3, dequantize_e4m3, round_to_e4m3, fp8_quantize_blocks,
     fp8_quantize_rows, fp8_qdq_blocks, fp8_qdq_rows, gate_logits, selection_scores, route_from_logits,
-    RouteResult, permute, swiglu_ffn, moe_forward, bias_update, load_cv, seq_aux_loss,
+    RouteResult, permute, swiglu_hidden, swiglu_ffn, moe_forward, combine, bias_update, load_cv,
+    seq_aux_loss,
 )
 
 __all__ = [
     "e4m3_values", "quantize_e4m3", "dequantize_e4m3", "round_to_e4m3",
     "fp8_quantize_blocks", "fp8_quantize_rows", "fp8_qdq_blocks", "fp8_qdq_rows", "gate_logits", "selection_scores",
-    "route_from_logits", "RouteResult", "permute", "swiglu_ffn",
-    "moe_forward", "bias_update", "load_cv", "seq_aux_loss",
+    "route_from_logits", "RouteResult", "permute", "swiglu_hidden", "swiglu_ffn",
+    "moe_forward", "combine", "bias_update", "load_cv", "seq_aux_loss",
 ]

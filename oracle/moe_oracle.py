@@ -305,16 +305,21 @@ def permute(ids: np.ndarray, E: int):
 # --------------------------------------------------------------------------
 # Experts ([MoE-walk] §3.3.1 SwiGLU, §3.3.2 shared experts).
 # --------------------------------------------------------------------------
-def swiglu_ffn(x: np.ndarray, w13: np.ndarray, w2: np.ndarray) -> np.ndarray:
-    """gate_up = x @ w13^T; gate, up = first / last I columns;
-    h = SiLU(gate) * up with SiLU(v) = v * sigmoid(v); out = h @ w2^T."""
+def swiglu_hidden(x: np.ndarray, w13: np.ndarray) -> np.ndarray:
+    """The expert's intermediate activation: gate_up = x @ w13^T; gate, up =
+    its first / last I columns (w13 stacks w1 over w3); h = SiLU(gate) * up
+    with SiLU(v) = v * sigmoid(v)."""
     x = np.asarray(x, np.float64)
     w13 = np.asarray(w13, np.float64)
     I = w13.shape[0] // 2
     gu = x @ w13.T
     g, u = gu[:, :I], gu[:, I:]
-    h = g * (1.0 / (1.0 + np.exp(-g))) * u
-    return h @ np.asarray(w2, np.float64).T
+    return g * (1.0 / (1.0 + np.exp(-g))) * u
+
+
+def swiglu_ffn(x: np.ndarray, w13: np.ndarray, w2: np.ndarray) -> np.ndarray:
+    """One SwiGLU expert: out = h @ w2^T with h = swiglu_hidden(x, w13)."""
+    return swiglu_hidden(x, w13) @ np.asarray(w2, np.float64).T
 
 
 def _swiglu_fp8(xd, w13, w2, w2_rows=None):
@@ -322,10 +327,7 @@ def _swiglu_fp8(xd, w13, w2, w2_rows=None):
     1x128 tile (xd = the dequantised activations), h re-quantised per 1x128.
     `w2_rows` optionally restricts the output to those features (the blocks
     holding them are quantised exactly as in the whole matrix)."""
-    I = w13.shape[0] // 2
-    gu = xd @ fp8_qdq_blocks(w13).T
-    g, u = gu[:, :I], gu[:, I:]
-    h = g * (1.0 / (1.0 + np.exp(-g))) * u
+    h = swiglu_hidden(xd, fp8_qdq_blocks(w13))
     hd = fp8_qdq_rows(h.astype(np.float32))
     if w2_rows is None:
         return hd @ fp8_qdq_blocks(w2).T
@@ -340,13 +342,15 @@ def _swiglu_fp8(xd, w13, w2, w2_rows=None):
 def moe_forward(x: np.ndarray, route: RouteResult,
                 expert_weights: Callable[[int], Tuple[np.ndarray, np.ndarray]],
                 shared: Optional[Tuple[np.ndarray, np.ndarray]], fp8: bool = False,
-                return_parts: bool = False, out_features=None):
+                return_parts: bool = False, out_features=None, map_fn=map):
     """y_t = shared(x_t) + sum_j w_tj * E_{id_tj}(x_t)  ([MoE-walk] §3.4).
 
     `x` holds the tokens to evaluate (any subset; the layer is per token), and
     `route` their routing. `expert_weights(e)` returns (w13_e, w2_e) for one
     expert, so the caller can widen one expert at a time. `out_features`
-    (optional) limits the output to those hidden features.
+    (optional) limits the output to those hidden features. `map_fn` evaluates
+    the experts (default: one after another; a thread pool's map runs them
+    side by side); their outputs are summed in expert order either way.
     """
     x = np.asarray(x, np.float64)
     T, H = x.shape
@@ -356,7 +360,8 @@ def moe_forward(x: np.ndarray, route: RouteResult,
     Hout = H if out_features is None else len(out_features)
     routed = np.zeros((T, Hout), dtype=np.float64)
     per_slot = np.zeros((T, k, Hout), dtype=np.float64) if return_parts else None
-    for e in np.unique(ids):
+
+    def expert_rows(e):
         tt, jj = np.nonzero(ids == e)
         w13, w2 = expert_weights(int(e))
         if fp8:
@@ -365,6 +370,9 @@ def moe_forward(x: np.ndarray, route: RouteResult,
         else:
             w2s = w2 if out_features is None else np.asarray(w2)[out_features]
             out = swiglu_ffn(x[tt], w13, w2s)
+        return tt, jj, out
+
+    for tt, jj, out in map_fn(expert_rows, np.unique(ids)):
         contrib = route.weights[tt, jj][:, None] * out
         np.add.at(routed, tt, contrib)
         if return_parts:
@@ -380,6 +388,25 @@ def moe_forward(x: np.ndarray, route: RouteResult,
     y = routed + sh
     if return_parts:
         return y, routed, sh, per_slot
+    return y
+
+
+def combine(expert_out: np.ndarray, slot_to_row: np.ndarray, k: int,
+            weights: Optional[np.ndarray] = None, shared: Optional[np.ndarray] = None) -> np.ndarray:
+    """Unpermute and combine ([MoE-walk] §3.4): token t's output is its shared
+    expert row plus the sum over its k slots j of w_tj times the expert output
+    row that slot's copy was computed in, row slot_to_row[t*k + j] of
+    expert_out. weights = None: the rows already carry their routing weight
+    (w = 1). Slots whose row is negative (dropped) contribute nothing."""
+    eo = np.asarray(expert_out, np.float64)
+    s2r = np.asarray(slot_to_row).reshape(-1, k)
+    T = s2r.shape[0]
+    w = np.ones((T, k)) if weights is None else np.asarray(weights, np.float64).reshape(T, k)
+    y = np.zeros((T, eo.shape[1])) if shared is None else np.array(shared, np.float64)
+    for t in range(T):
+        for j in range(k):
+            if s2r[t, j] >= 0:
+                y[t] += w[t, j] * eo[s2r[t, j]]
     return y
 
 

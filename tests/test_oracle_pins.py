@@ -281,6 +281,55 @@ def test_swiglu_closed_form():
     np.testing.assert_allclose(out2, 3.0 * (-2.0) * (-0.2689414213699951), rtol=1e-15)
 
 
+def test_swiglu_hidden_closed_form_and_gate_up_order():
+    # x = (ln 3, 2): w1 picks x0 (gate), w3 picks x1 (up):
+    # sigmoid(ln 3) = 3/4, so h = SiLU(ln 3) * 2 = (3/4) ln 3 * 2 = 1.5 ln 3
+    x = np.array([[np.log(3.0), 2.0]])
+    w13 = np.array([[1.0, 0.0], [0.0, 1.0]])          # [w1; w3], I = 1
+    np.testing.assert_allclose(oracle.swiglu_hidden(x, w13), [[1.5 * np.log(3.0)]], rtol=1e-15)
+    # gate and up swapped: SiLU(2) * ln 3 = 2 / (1 + e^-2) * ln 3, not the same
+    swapped = oracle.swiglu_hidden(x, w13[::-1])
+    np.testing.assert_allclose(swapped, [[2.0 / (1.0 + np.exp(-2.0)) * np.log(3.0)]], rtol=1e-15)
+    assert abs(swapped[0, 0] - 1.5 * np.log(3.0)) > 0.1
+    # the expert is h followed by the down projection
+    rng = np.random.default_rng(11)
+    xr, w13r, w2r = rng.standard_normal((5, 16)), rng.standard_normal((12, 16)), rng.standard_normal((16, 6))
+    np.testing.assert_allclose(oracle.swiglu_ffn(xr, w13r, w2r), oracle.swiglu_hidden(xr, w13r) @ w2r.T,
+                               rtol=1e-14)
+
+
+def test_combine_hand_example():
+    # 2 tokens, k = 2; expert rows (already permuted): r0=(1,2) r1=(10,20) r2=(100,200) r3=(-1,-1)
+    # token 0 -> rows 2, 0 with weights 0.5, 2; token 1 -> rows 3, 1 with weights 1, 0.1
+    eo = np.array([[1.0, 2.0], [10.0, 20.0], [100.0, 200.0], [-1.0, -1.0]])
+    s2r = np.array([2, 0, 3, 1])
+    w = np.array([[0.5, 2.0], [1.0, 0.1]])
+    sh = np.array([[7.0, 8.0], [0.0, 1.0]])
+    y = oracle.combine(eo, s2r, 2, w, sh)
+    np.testing.assert_array_equal(y, [[7 + 50 + 2, 8 + 100 + 4], [0 - 1 + 1, 1 - 1 + 2]])
+    # weights already in the rows, no shared expert; a dropped slot (-1) adds nothing
+    np.testing.assert_array_equal(oracle.combine(eo, np.array([2, 0, -1, 1]), 2),
+                                  [[101.0, 202.0], [10.0, 20.0]])
+
+
+def test_combine_of_permuted_expert_rows_equals_layer_sum():
+    """combine over the permutation's rows gives moe_forward's output: the
+    per-slot expert outputs laid out in the permuted row order, unpermuted by
+    slot_to_row and summed with the routing weights and the shared expert."""
+    cfg = tiny_grouped_config()
+    inp = make_inputs(cfg)
+    x = inp.x.float().numpy()
+    w13, w2 = inp.w13.float().numpy(), inp.w2.float().numpy()
+    sh = (inp.sw13.float().numpy(), inp.sw2.float().numpy())
+    L32 = oracle.gate_logits(x, inp.gate.float().numpy()).astype(np.float32)
+    r = oracle.route_from_logits(L32, cfg.k, cfg.n_group, cfg.topk_group, cfg.scoring,
+                                 cfg.norm_topk_prob, cfg.scale, inp.bias.numpy())
+    y, _, shared, per_slot = oracle.moe_forward(x, r, lambda e: (w13[e], w2[e]), sh, return_parts=True)
+    _, src, s2r = oracle.permute(r.ids, cfg.E)
+    rows = per_slot.reshape(cfg.T * cfg.k, -1)[np.argsort(s2r)]       # row p holds slot s with s2r[s] = p
+    np.testing.assert_allclose(oracle.combine(rows, s2r, cfg.k, r.weights, shared), y, rtol=1e-12, atol=1e-12)
+
+
 def _dense_bruteforce(x, route, w13, w2, sw13, sw2, E):
     """Every expert on every token, masked by the routing weights."""
     x = x.astype(np.float64)
@@ -476,3 +525,21 @@ def test_seq_aux_loss_two_token_hand_example(scoring, row0):
     assert oracle.seq_aux_loss(L, both_on_0, 2, 1, scoring, 2, 1.0) == pytest.approx(1.25, rel=1e-6)
     assert oracle.seq_aux_loss(L, split, 2, 1, scoring, 2, 1.0) == pytest.approx(1.0, rel=1e-6)
     assert oracle.seq_aux_loss(L, np.array([[1], [1]]), 2, 1, scoring, 2, 1.0) == pytest.approx(0.75, rel=1e-6)
+
+
+def test_moe_forward_thread_pool_map_gives_identical_result():
+    """Evaluating the experts side by side changes nothing: their outputs are
+    summed in expert order either way."""
+    from concurrent.futures import ThreadPoolExecutor
+    cfg = tiny_grouped_config()
+    inp = make_inputs(cfg)
+    x = inp.x.float().numpy()
+    w13, w2 = inp.w13.float().numpy(), inp.w2.float().numpy()
+    sh = (inp.sw13.float().numpy(), inp.sw2.float().numpy())
+    L32 = oracle.gate_logits(x, inp.gate.float().numpy()).astype(np.float32)
+    r = oracle.route_from_logits(L32, cfg.k, cfg.n_group, cfg.topk_group, cfg.scoring,
+                                 cfg.norm_topk_prob, cfg.scale, inp.bias.numpy())
+    y0 = oracle.moe_forward(x, r, lambda e: (w13[e], w2[e]), sh)
+    with ThreadPoolExecutor(4) as ex:
+        y1 = oracle.moe_forward(x, r, lambda e: (w13[e], w2[e]), sh, map_fn=ex.map)
+    np.testing.assert_array_equal(y0, y1)
