@@ -18,8 +18,10 @@
  *
  * Conventions for every call:
  *   - Tensor pointers are DEVICE pointers to dense row-major arrays, allocated
- *     and owned by the caller. The library allocates no memory and keeps no
- *     mutable global state between calls (moe_last_cuda_error aside).
+ *     and owned by the caller. The library allocates no memory. Its only
+ *     mutable global state is the per-thread moe_last_cuda_error and the
+ *     process-wide wait limit of moe_set_wait_limit_ns (a debugging knob,
+ *     2 s unless changed); moe_permute_static_ws keeps its own array.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL means the
  *     legacy default stream). Outputs are valid once the stream reaches it.
  *   - Arguments are checked on the host before any launch. On a non-OK
@@ -29,7 +31,8 @@
  *   - `dev_status`, where taken, is an optional device int32 (NULL = off).
  *     Kernels never trap: a bounds check that fails or a bounded wait that
  *     runs out ORs a code into it (MOE_DEVSTAT_*) and the kernel returns.
- *     Read it with moe_read_device_status.
+ *     Read it with moe_read_device_status. After a wait runs out, the
+ *     kernel's outputs are incomplete, but the CUDA context stays usable.
  *   - No C++ exception crosses this interface.
  */
 #ifndef MOE_B200_MOE_H
@@ -194,6 +197,11 @@ MOE_API moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H,
  * on the GPU (other streams, other host threads) race and give wrong
  * results; serialise them. Nothing needs clearing between calls (every call
  * rewrites the part of the array it reads).
+ * The looked-up address is cached per device index for the life of the
+ * process: after cudaDeviceReset (or anything else that destroys and
+ * recreates the device's primary context) it is stale, and the next call
+ * would write through it. Do not call this entry point again in a process
+ * that has reset the device.
  * ------------------------------------------------------------------------ */
 MOE_API moe_status moe_permute_static_ws(int32_t T, int32_t k, int32_t E, int32_t H,
                        const int32_t* topk_ids, const float* topk_w,
@@ -271,8 +279,8 @@ MOE_API moe_status moe_down_proj(int32_t rows, int32_t H, const moe_ffn_weights*
  * dtype; its I may differ from w's). rows / sh_rows: T*k / T. Other
  * arguments, limits and errors as moe_gate_up_swiglu / moe_down_proj; E4M3
  * scales as there (sh_a_scale / sh_h_scale for the shared rows). bf16 layers
- * run as one launch; E4M3 layers (and MOE_GEMM_PAIR=1) as two launches of the
- * same calls in this order. */
+ * run as one launch; E4M3 layers as two launches of the same calls in this
+ * order. */
 MOE_API moe_status moe_gate_up_swiglu_with_shared(int32_t rows, int32_t H, const moe_ffn_weights* w,
                               const void* a, const float* a_scale, const int32_t* offsets,
                               void* h_ws, float* h_scale_ws,
@@ -396,6 +404,21 @@ MOE_API moe_status moe_quantize_rows(int32_t M, int32_t K, const void* a, void* 
  * ------------------------------------------------------------------------ */
 MOE_API moe_status moe_read_device_status(const int32_t* dev_status, int32_t* out, void* stream);
 MOE_API int32_t moe_last_cuda_error(void);
+
+/* ------------------------------------------------------------------------ *
+ * Bounded device waits (debugging). The pages have no counterpart.
+ * Every kernel that waits on an mbarrier (the grouped GEMMs, the gate GEMM)
+ * gives up a wait after a limit of wall time, sets MOE_DEVSTAT_TIMEOUT in
+ * its dev_status, lets its in-flight copies and MMAs finish, frees its
+ * tensor memory and returns; its outputs are then incomplete.
+ * moe_set_wait_limit_ns: the limit for launches issued after the call, in
+ *   nanoseconds, process-wide; 0 restores the default (2 s). A limit far
+ *   below a kernel's normal waits (a few ns) makes it time out on purpose,
+ *   which is how the timeout path is tested. Always MOE_OK.
+ * moe_wait_limit_ns: the current limit.
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_set_wait_limit_ns(uint64_t ns);
+MOE_API uint64_t moe_wait_limit_ns(void);
 MOE_API const char* moe_status_string(moe_status s);
 MOE_API int32_t moe_abi_version(void);
 

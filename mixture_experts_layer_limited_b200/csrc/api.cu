@@ -1,7 +1,7 @@
 // C-ABI entry points of libmoe (declared in include/moe.h): argument checks on
 // the host, TMA tensor-map encoding, kernel launches. No allocation happens
 // here; every buffer belongs to the caller.
-#include <cstdlib>
+#include <atomic>
 #include <mutex>
 
 #include "kernels.cuh"
@@ -92,46 +92,10 @@ moe_status sm_count(int* n) {
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-// Kernel choice for the bf16 grouped GEMMs, by measurement at the V3 shape:
-// the gate/up GEMM (SwiGLU epilogue) runs on single CTAs, the down GEMM on
-// CTA pairs (tcgen05 cta_group::2, epilogue overlapped with the next tile).
-// MOE_GEMM_1SM=1 puts both on single CTAs, MOE_GEMM_PAIR=1 both on pairs
-// (same results; for comparison). Read at each call.
-bool env_on(const char* name) {
-  const char* v = std::getenv(name);
-  return v && v[0] == '1';
-}
-// Kernel choice per bf16 GEMM (measured at the V3 shape on B200): both run on
-// single CTAs with 256-token tiles and one TMEM accumulator pair (two pairs
-// of 128-token tiles would overlap the epilogue with the next tile's MMAs but
-// halve the reuse of each weight tile). The down projection's epilogue stores
-// twice the features of gate/up's, so it runs on 12 epilogue warps (three per
-// TMEM lane quarter), gate/up on 4.
-// Switches, for comparisons: MOE_GEMM_PAIR=1 / MOE_GEMM_1SM=1 force CTA pairs
-// / single CTAs for both GEMMs, MOE_GEMM_PAIR_DOWN=1 pairs for down only;
-// MOE_GEMM_DB=1 / MOE_GEMM_SB=1 force two / one accumulator pairs for both,
-// MOE_DOWN_DB=1 two for down only; MOE_EPI8=1 / MOE_EPI4=1 force 8 / 4
-// epilogue warps for both; MOE_GEMM_WIDE=1 runs both on CTA pairs with two
-// weight sub-tiles per CTA where the shape allows (gate/up: I % 256 == 0,
-// down: H % 512 == 0).
-bool wide_pairs(bool gate_up, int I, int H) {
-  if (env_on("MOE_GEMM_1SM") || !env_on("MOE_GEMM_WIDE")) return false;
-  return gate_up ? I % 256 == 0 : H % 512 == 0;
-}
-bool bf16_on_pairs(bool gate_up) {
-  if (env_on("MOE_GEMM_1SM")) return false;
-  return env_on("MOE_GEMM_PAIR") || (!gate_up && env_on("MOE_GEMM_PAIR_DOWN"));
-}
-int one_cta_buffers(bool gate_up) {
-  if (env_on("MOE_GEMM_DB")) return 2;
-  if (env_on("MOE_GEMM_SB")) return 1;
-  return (!gate_up && env_on("MOE_DOWN_DB")) ? 2 : 1;
-}
-int epilogue_warps(bool gate_up) {
-  if (env_on("MOE_EPI8")) return 8;
-  if (env_on("MOE_EPI4")) return 4;
-  return gate_up ? 4 : 12;
-}
+// Limit of every bounded device-side wait, passed to the kernels at launch
+// (moe_set_wait_limit_ns; 2 s unless changed).
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
+uint64_t wait_limit() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 }  // namespace
 
@@ -140,6 +104,13 @@ extern "C" {
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 
 int32_t moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+moe_status moe_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : ns, std::memory_order_relaxed);
+  return MOE_OK;
+}
+
+uint64_t moe_wait_limit_ns(void) { return wait_limit(); }
 
 const char* moe_status_string(moe_status s) {
   switch (s) {
@@ -175,6 +146,7 @@ moe_status moe_gate_logits(int32_t T, int32_t H, int32_t E, const void* x, const
   r.E = E;
   r.logits = logits;
   r.status = dev_status;
+  r.wait_ns = wait_limit();
   return gate_gemm(r, x, gate_w, as_stream(stream));
 }
 
@@ -196,7 +168,8 @@ moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_
   if (s != MOE_OK) return s;
   cudaStream_t st = as_stream(stream);
   RouteArgs r{p->T, p->H, p->E, p->k, p->n_group, p->topk_group, p->scoring, p->norm_topk_prob ? 1 : 0,
-              p->routed_scaling_factor, sel_bias, logits, topk_ids, topk_w, expert_counts, p->dev_status};
+              p->routed_scaling_factor, sel_bias, logits, topk_ids, topk_w, expert_counts, p->dev_status,
+              wait_limit()};
   cudaError_t e = cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * p->E, st);
   if (e != cudaSuccess) return cuda_fail(e);
   if (x && (s = gate_gemm(r, x, gate_w, st)) != MOE_OK) return s;
@@ -272,85 +245,80 @@ struct GemmPlan {
   bool fp8;
 };
 
+// Kernel choice for the bf16 grouped GEMMs, by measurement at the V3 shape on
+// B200: single CTAs, 256-token tiles with one TMEM accumulator pair, three
+// 64-K stages; 4 epilogue warps for gate/up and 12 for down, whose output
+// rows are twice as wide (three warps per TMEM lane quarter take turns on
+// its 32-token chunks). E4M3: at most 32 tokens a tile.
 moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a, const float* a_scale,
                         const int32_t* offsets, void* h_ws, float* h_scale_ws, int32_t* dev_status, GemmPlan* p) {
   const bool fp8 = w->dtype == MOE_E4M3;
-  const bool pair = !fp8 && bf16_on_pairs(true);
   const int I = w->I;
-  if (!fp8 && wide_pairs(true, I, H)) {
-    moe_status s = make_tmap(&p->tmA, w->w13, false, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
-    if (s != MOE_OK) return s;
-    if ((s = make_token_tmaps(&p->tmB, a, false, H, rows)) != MOE_OK) return s;
-    // pair tile: 256 features; CTA r: gate rows [mb*256 + 128r, +128) and their up rows
-    p->g = GemmArgs{rows, H, w->groups, offsets, 2 * I, I / 256, 256, I, 256, 0, 256, 128, 1, 0,
-                    h_ws, I, nullptr, nullptr, nullptr, nullptr, dev_status};
-    p->g.kc = env_on("MOE_WIDE_K128") ? 2 : 1;   // 2 stages of 128 K instead of 4 of 64 K
-    p->g.epi_warps = epilogue_warps(true);
-    p->g.wide = 1;
-    p->fp8 = false;
-    return MOE_OK;
-  }
-  moe_status s = make_tmap(&p->tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, pair ? 64 : 128);
+  moe_status s = make_tmap(&p->tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
   if (s != MOE_OK) return s;
-  s = make_token_tmaps(&p->tmB, a, fp8, H, rows);
-  if (s != MOE_OK) return s;
-  const int nb = (fp8 || pair) ? 1 : one_cta_buffers(true);
-  p->g = GemmArgs{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, fp8 ? 32 : (nb == 2 ? 128 : 256),
-                  pair ? 64 : 0, nb, 0, h_ws, I, nullptr, w->w13_scale, a_scale, h_scale_ws, dev_status};
-  // with two accumulators (128-token tiles) the stages carry 128 K, as for down
-  p->g.kc = (!fp8 && !pair && nb == 2 && !env_on("MOE_DOWN_K64")) ? 2 : 1;
-  p->g.epi_warps = epilogue_warps(true);
+  if ((s = make_token_tmaps(&p->tmB, a, fp8, H, rows)) != MOE_OK) return s;
+  GemmArgs& g = p->g;
+  g = GemmArgs{};
+  g.rows = rows;
+  g.K = H;
+  g.groups = w->groups;
+  g.offsets = offsets;
+  g.a_rows_per_group = 2 * I;            // w13[e]: gate rows [0, I), up rows [I, 2I)
+  g.n_mblk = I / 128;
+  g.mblk_stride = 128;
+  g.sub1_off = I;                        // sub-tile 1: the up rows of the same 128 features
+  g.feat_stride = 128;
+  g.bn_max = fp8 ? 32 : 256;
+  g.out = h_ws;
+  g.out_ld = I;
+  g.a_scale = w->w13_scale;
+  g.b_scale = a_scale;
+  g.out_scale = h_scale_ws;
+  g.status = dev_status;
+  g.epi_warps = 4;
+  g.wait_ns = wait_limit();
   p->fp8 = fp8;
   return MOE_OK;
 }
 
 moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* h, const float* h_scale,
-                     const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status, GemmPlan* p,
-                     bool scatter = false) {
+                     const int32_t* offsets, const float* row_w, void* out, int32_t* dev_status, GemmPlan* p) {
   const bool fp8 = w->dtype == MOE_E4M3;
-  // the scatter form (combine fused in) runs on single CTAs, one accumulator pair
-  const bool pair = !fp8 && !scatter && bf16_on_pairs(false);
   const int I = w->I;
-  if (!fp8 && !scatter && wide_pairs(false, I, H)) {
-    moe_status s = make_tmap(&p->tmA, w->w2, false, I, static_cast<uint64_t>(w->groups) * H, 128);
-    if (s != MOE_OK) return s;
-    if ((s = make_token_tmaps(&p->tmB, h, false, I, rows)) != MOE_OK) return s;
-    // pair tile: 512 output features; CTA r sub-tile s: w2 rows [mb*512 + 256s + 128r, +128)
-    p->g = GemmArgs{rows, I, w->groups, offsets, H, H / 512, 512, 256, 512, 256, 256, 128, 1, 0,
-                    out, H, row_w, nullptr, nullptr, nullptr, dev_status};
-    p->g.kc = env_on("MOE_WIDE_K128") ? 2 : 1;   // 2 stages of 128 K instead of 4 of 64 K
-    p->g.epi_warps = epilogue_warps(false);
-    p->g.wide = 1;
-    p->fp8 = false;
-    return MOE_OK;
-  }
-  // the single-CTA bf16 kernel reads its 256 contiguous w2 rows as one box
-  const bool one_box = !fp8;
-  moe_status s = make_tmap(&p->tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H,
-                           (fp8 || pair) ? 128 : 256);
+  // bf16: a tile's 256 contiguous w2 rows are one TMA box
+  moe_status s = make_tmap(&p->tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H, fp8 ? 128 : 256);
   if (s != MOE_OK) return s;
-  s = make_token_tmaps(&p->tmB, h, fp8, I, rows);
-  if (s != MOE_OK) return s;
-  const int nb = (fp8 || pair || scatter) ? 1 : one_cta_buffers(false);
-  p->g = GemmArgs{rows, I, w->groups, offsets, H, H / 256, 256, pair ? 64 : 128, 256, 128,
-                  fp8 ? 32 : (nb == 2 ? 128 : 256), pair ? 128 : 0, nb, one_box ? 1 : 0,
-                  out, H, row_w, w->w2_scale, h_scale, nullptr, dev_status};
-  // two accumulators on single CTAs: stages of 128 K (2 x 96 KB), measured a
-  // little faster than 4 x 48 KB stages of 64 K; MOE_DOWN_K64=1 keeps 64 K
-  p->g.kc = (!fp8 && !pair && nb == 2 && !env_on("MOE_DOWN_K64")) ? 2 : 1;
-  p->g.epi_warps = epilogue_warps(false);
+  if ((s = make_token_tmaps(&p->tmB, h, fp8, I, rows)) != MOE_OK) return s;
+  GemmArgs& g = p->g;
+  g = GemmArgs{};
+  g.rows = rows;
+  g.K = I;
+  g.groups = w->groups;
+  g.offsets = offsets;
+  g.a_rows_per_group = H;
+  g.n_mblk = H / 256;
+  g.mblk_stride = 256;
+  g.sub1_off = 128;                      // sub-tiles: w2 rows [mb*256, +128) and [mb*256 + 128, +128)
+  g.feat_stride = 256;
+  g.feat_sub1 = 128;
+  g.bn_max = fp8 ? 32 : 256;
+  g.a_one_box = fp8 ? 0 : 1;
+  g.out = out;
+  g.out_ld = H;
+  g.row_w = row_w;
+  g.a_scale = w->w2_scale;
+  g.b_scale = h_scale;
+  g.status = dev_status;
+  g.epi_warps = 12;
+  g.wait_ns = wait_limit();
   p->fp8 = fp8;
   return MOE_OK;
 }
 
 moe_status launch_plan(const GemmPlan& p, int epi, cudaStream_t st, int nsm, const GemmPlan* second = nullptr) {
 
-  // one launch needs the same kernel form for both: single-CTA bf16, same tile shape
-  // (or both on wide CTA pairs)
-  const bool same_form = (p.g.cta_stride == 0 && second && second->g.cta_stride == 0) ||
-                         (p.g.wide && second && second->g.wide);
-  const bool one = second && !p.fp8 && !second->fp8 && same_form &&
-                   p.g.bn_max == second->g.bn_max && p.g.nbuf == second->g.nbuf && p.g.kc == second->g.kc &&
+  // one launch needs the same kernel form for both: bf16, same tile shape
+  const bool one = second && !p.fp8 && !second->fp8 && p.g.bn_max == second->g.bn_max &&
                    p.g.epi_warps == second->g.epi_warps;
   if (second && !one) {
     moe_status s = check_launch(launch_grouped_gemm(p.fp8, epi, p.tmA, p.tmB, p.g, nsm, st));
@@ -413,8 +381,23 @@ moe_status moe_gate_up_swiglu_gather(int32_t rows, int32_t H, const moe_ffn_weig
   if (s != MOE_OK) return s;
   s = make_token_tmaps(&tmB, x, false, H, T);      // not read: token rows are gathered
   if (s != MOE_OK) return s;
-  GemmArgs g1{rows, H, w->groups, offsets, 2 * I, I / 128, 128, I, 128, 0, 256, 0, 1, 0,
-              h_ws, I, nullptr, nullptr, nullptr, nullptr, dev_status, x, src_token, T};
+  GemmArgs g1{};
+  g1.rows = rows;
+  g1.K = H;
+  g1.groups = w->groups;
+  g1.offsets = offsets;
+  g1.a_rows_per_group = 2 * I;
+  g1.n_mblk = I / 128;
+  g1.mblk_stride = 128;
+  g1.sub1_off = I;
+  g1.feat_stride = 128;
+  g1.out = h_ws;
+  g1.out_ld = I;
+  g1.status = dev_status;
+  g1.gather_src = x;
+  g1.gather_rows = src_token;
+  g1.gather_src_rows = T;
+  g1.wait_ns = wait_limit();
   return check_launch(launch_grouped_gemm(false, EPI_SWIGLU, tmA, tmB, g1, nsm, as_stream(stream)));
 }
 
@@ -465,9 +448,7 @@ moe_status moe_gate_up_swiglu_with_shared(int32_t rows, int32_t H, const moe_ffn
   if ((s = plan_gate_up(sh_rows, H, sw, sh_a, sh_a_scale, nullptr, sh_h_ws, sh_h_scale_ws, dev_status, &q)) !=
       MOE_OK)
     return s;
-  if (!env_on("MOE_SHARED_APART")) return launch_plan(p, EPI_SWIGLU, st, nsm, &q);
-  if ((s = launch_plan(p, EPI_SWIGLU, st, nsm)) != MOE_OK) return s;
-  return launch_plan(q, EPI_SWIGLU, st, nsm);
+  return launch_plan(p, EPI_SWIGLU, st, nsm, &q);
 }
 
 moe_status moe_down_proj_with_shared(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* h,
@@ -486,9 +467,7 @@ moe_status moe_down_proj_with_shared(int32_t rows, int32_t H, const moe_ffn_weig
   if ((s = plan_down(rows, H, w, h, h_scale, offsets, row_w, out, dev_status, &p)) != MOE_OK) return s;
   if ((s = plan_down(sh_rows, H, sw, sh_h, sh_h_scale, nullptr, nullptr, sh_out, dev_status, &q)) != MOE_OK)
     return s;
-  if (!env_on("MOE_SHARED_APART")) return launch_plan(p, EPI_WEIGHTED, st, nsm, &q);
-  if ((s = launch_plan(p, EPI_WEIGHTED, st, nsm)) != MOE_OK) return s;
-  return launch_plan(q, EPI_WEIGHTED, st, nsm);
+  return launch_plan(p, EPI_WEIGHTED, st, nsm, &q);
 }
 
 moe_status moe_down_proj_combine(int32_t rows, int32_t T, int32_t H, const moe_ffn_weights* w, const void* h,
@@ -509,13 +488,12 @@ moe_status moe_down_proj_combine(int32_t rows, int32_t T, int32_t H, const moe_f
   cudaStream_t st = as_stream(stream);
   cudaError_t e = cudaMemsetAsync(acc_ws, 0, static_cast<size_t>(T) * H * sizeof(float), st);
   if (e != cudaSuccess) return cuda_fail(e);
-  // the scatter runs on the single-CTA kernel: one accumulator pair, 256 tokens
   GemmPlan p, q;
-  if ((s = plan_down(rows, H, w, h, nullptr, offsets, row_w, acc_ws, dev_status, &p, true)) != MOE_OK) return s;
+  if ((s = plan_down(rows, H, w, h, nullptr, offsets, row_w, acc_ws, dev_status, &p)) != MOE_OK) return s;
   p.g.scatter_tok = src_token;
   p.g.scatter_T = T;
   if (sw) {
-    if ((s = plan_down(T, H, sw, sh_h, nullptr, nullptr, nullptr, acc_ws, dev_status, &q, true)) != MOE_OK) return s;
+    if ((s = plan_down(T, H, sw, sh_h, nullptr, nullptr, nullptr, acc_ws, dev_status, &q)) != MOE_OK) return s;
     q.g.scatter_tok = nullptr;
     q.g.scatter_T = T;
   }

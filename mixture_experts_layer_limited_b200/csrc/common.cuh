@@ -1,9 +1,12 @@
 // Device-side building blocks for sm_100a: mbarriers with bounded waits,
 // TMA tile loads, tcgen05 tensor-core MMA / TMEM access, and small helpers.
 //
-// Every spin on an mbarrier is bounded: after kWaitLimitNs of wall time the
-// waiting thread raises the CTA's abort flag and ORs MOE_DEVSTAT_TIMEOUT into
-// the caller's status word, so kernels return instead of hanging.
+// Every spin on an mbarrier is bounded: after the launch's wait limit (a
+// kernel argument, 2 s unless the caller set another with
+// moe_set_wait_limit_ns) the waiting thread raises the CTA's abort flag and
+// ORs MOE_DEVSTAT_TIMEOUT into the caller's status word, so kernels return
+// instead of hanging. Waits that drain in-flight work after an abort always
+// allow kDrainLimitNs, whatever the launch's limit.
 #pragma once
 
 #include <cstdint>
@@ -16,7 +19,8 @@
 
 namespace moe {
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // 2 s per wait
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -68,14 +72,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Waits for the phase with the given parity to complete. Returns false when
 // the CTA aborted (another thread timed out) or this wait itself timed out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status) {
+                                          int32_t* status, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         flag_status(status, MOE_DEVSTAT_TIMEOUT);
         return false;
@@ -88,7 +92,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+    if (globaltimer_ns() - t0 > kDrainLimitNs) return;
   }
 }
 

@@ -20,24 +20,25 @@
 //          feature in the same thread and fuses SiLU(gate) * up.
 //   GEMM2: sub-tiles = w2 rows [mb*256, +128) and [mb*256 + 128, +128); the
 //          epilogue multiplies by the routing weight of the row.
-// TMEM (512 fp32 columns): one accumulator pair of up to 256 tokens (GEMM1),
-// or two pairs of up to 128 tokens (GEMM2), so that the epilogue of one tile
-// runs while the MMAs of the next fill the other pair.
+// TMEM (512 fp32 columns) holds one accumulator pair of up to 256 tokens.
+// 256-token tiles read each 3.7 MB weight tile (V3 gate/up) half as often as
+// 128-token tiles would, which at the V3 shape on B200 was measured to be
+// worth more than double-buffering the accumulator (which would halve the
+// tile) to overlap the epilogue with the next tile's MMAs.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over tiles):
+// Warp roles (one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer (A: the weight rows, B: the tile's token rows in
 //               boxes of 256/128/64/32/16 rows, 128-byte swizzle) into a ring
-//               of stages of one or two 64-K chunks;
+//               of three 64-K stages;
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer;
-//   warps 2..5  epilogue: tcgen05.ld (warp w owns TMEM lanes 32*(w%4)..+31),
-//               fused activation / weighting, bf16 stores.
+//   warps 2..   epilogue (4 warps for GEMM1, 12 for GEMM2, whose output is
+//               twice as wide): tcgen05.ld (warp w reads TMEM lanes
+//               32*(w%4)..+31), fused activation / weighting, bf16 stores.
 // A launch may carry a second, single-group problem (the shared expert) whose
 // tiles come first in the tile order.
 // The E4M3 variant accumulates each 128-wide K block separately in a TMEM
 // ring and promotes it with the fp32 block scales on the CUDA cores, since
 // the weight scale is per 128x128 block and the activation scale per 1x128.
-// Two CTA-pair variants (tcgen05 cta_group::2: one or two weight sub-tiles
-// per CTA) are kept as options; at the V3 shape both are slower.
 #include "kernels.cuh"
 
 namespace moe {
@@ -184,7 +185,7 @@ constexpr int kGatherThreads = 64;
 // TWO: a second single-group problem a2 (the shared expert: its own weights
 // tmA2, token rows tmB2 and output) runs in the same launch. Its tiles come
 // first in the tile order, so the routed experts' ragged tiles fill the tail.
-template <int EPI, int STAGES, bool GATHER, bool TWO, int KC = 1, int EPIW = 4>
+template <int EPI, int STAGES, bool GATHER, bool TWO, int EPIW = 4>
 __global__ void __launch_bounds__(64 + 32 * EPIW + (GATHER ? kGatherThreads : 0), 1)
 grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ TokenMaps tmB, const GemmArgs a,
@@ -196,7 +197,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   __shared__ Sched sched;
   __shared__ __align__(16) __nv_bfloat16 stage_out[EPIW][32 * 32];
   __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
-  __shared__ uint64_t tmem_full[2], tmem_empty[2], drain_bar;
+  __shared__ uint64_t tmem_full, tmem_empty, drain_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ int issued_parity[STAGES];
   __shared__ volatile int abort_flag;
@@ -204,15 +205,13 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   const uint32_t b_stage_bytes = static_cast<uint32_t>(a.bn_max) * 128u;
-  // TMEM: nbuf accumulators of two sub-tiles; sub-tile s of buffer b starts at
-  // column b * 2 * sub_cols + s * sub_cols
-  const int nbuf = a.nbuf == 2 ? 2 : 1;
-  const uint32_t sub_cols = nbuf == 2 ? 128u : 256u;
-  // a stage holds KC chunks of 64 K, each [A sub-tile 0][A sub-tile 1][B rows]
-  const uint32_t chunk_bytes = 2 * A_SUB_BYTES + b_stage_bytes;
-  const uint32_t stage_bytes = KC * chunk_bytes;
-  auto sA = [&](int st, int sub, int c = 0) { return smem + st * stage_bytes + c * chunk_bytes + sub * A_SUB_BYTES; };
-  auto sB = [&](int st, int c = 0) { return smem + st * stage_bytes + c * chunk_bytes + 2 * A_SUB_BYTES; };
+  // TMEM: one accumulator pair, sub-tile s in columns [s * 256, +256)
+  constexpr uint32_t sub_cols = 256u;
+  const uint64_t wait_ns = a.wait_ns;
+  // a stage holds 64 K: [A sub-tile 0][A sub-tile 1][B rows]
+  const uint32_t stage_bytes = 2 * A_SUB_BYTES + b_stage_bytes;
+  auto sA = [&](int st, int sub) { return smem + st * stage_bytes + sub * A_SUB_BYTES; };
+  auto sB = [&](int st) { return smem + st * stage_bytes + 2 * A_SUB_BYTES; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -220,10 +219,8 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       mbar_init(&empty_bar[i], 1);
       issued_parity[i] = -1;
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tmem_full[b], 1);
-      mbar_init(&tmem_empty[b], 32 * EPIW);
-    }
+    mbar_init(&tmem_full, 1);
+    mbar_init(&tmem_empty, 32 * EPIW);
     mbar_init(&drain_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
@@ -265,23 +262,19 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         const int a_row1 = a_row0 + (sh ? a2.sub1_off : a.sub1_off);
         const bool one_box = sh ? a2.a_one_box != 0 : a.a_one_box != 0;
         const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;   // re-read by sibling token blocks
-        const uint32_t bytes = KC * (2 * A_SUB_BYTES + (GATHER ? 0u : static_cast<uint32_t>(ti.N) * 128u));
+        const uint32_t bytes = 2 * A_SUB_BYTES + (GATHER ? 0u : static_cast<uint32_t>(ti.N) * 128u);
         bool ok = true;
-        for (int ks = 0; ks < nk / KC; ++ks) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status, wait_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
-#pragma unroll
-          for (int c = 0; c < KC; ++c) {
-            const int kb = ks * KC + c;
-            tma_load_2d(sA(stage, 0, c), mA, &full_bar[stage], kb * KB, a_row0, pol_w);
-            if (!one_box) tma_load_2d(sA(stage, 1, c), mA, &full_bar[stage], kb * KB, a_row1, pol_w);
-            if (!GATHER) {
-              uint8_t* bdst = sB(stage, c);
-              uint64_t* fb = &full_bar[stage];
-              load_token_rows(ti.N, [&](int which, int off) {
-                tma_load_2d(bdst + off * 128, &mB->box[which], fb, kb * KB, ti.row0 + off, pol_x);
-              });
-            }
+          tma_load_2d(sA(stage, 0), mA, &full_bar[stage], kb * KB, a_row0, pol_w);
+          if (!one_box) tma_load_2d(sA(stage, 1), mA, &full_bar[stage], kb * KB, a_row1, pol_w);
+          if (!GATHER) {
+            uint8_t* bdst = sB(stage);
+            uint64_t* fb = &full_bar[stage];
+            load_token_rows(ti.N, [&](int which, int off) {
+              tma_load_2d(bdst + off * 128, &mB->box[which], fb, kb * KB, ti.row0 + off, pol_x);
+            });
           }
           issued_parity[stage] = static_cast<int>(phase);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -312,7 +305,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         srow[i] = sr;
       }
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status, wait_ns)) { ok = false; break; }
         const uint32_t bbase = smem_u32(sB(stage));
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -345,31 +338,27 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         const TileInfo ti = sh ? decode_in_segment(a2, 0, 0, a2.rows, t) : decode_tile(sched, a, t - total2);
         const int nk = (sh ? a2.K : a.K) / KB;
         const uint32_t idesc = make_idesc(1u, 128u, static_cast<uint32_t>(ti.N));
-        const uint32_t bi = nbuf == 2 ? (it & 1u) : 0u, use = nbuf == 2 ? (it >> 1) : it;
-        const uint32_t d0 = tmem_base + bi * 2u * sub_cols;
-        if (!mbar_wait(&tmem_empty[bi], (use & 1u) ^ 1u, &abort_flag, a.status)) break;
+        const uint32_t d0 = tmem_base;
+        if (!mbar_wait(&tmem_empty, (it & 1u) ^ 1u, &abort_flag, a.status, wait_ns)) break;
         tc_fence_after();
         bool ok = true;
-        for (int ks = 0; ks < nk / KC; ++ks) {
-          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status)) { ok = false; break; }
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status, wait_ns)) { ok = false; break; }
           tc_fence_after();
+          const uint32_t a0 = smem_u32(sA(stage, 0)), a1 = smem_u32(sA(stage, 1));
+          const uint32_t b0 = smem_u32(sB(stage));
 #pragma unroll
-          for (int c = 0; c < KC; ++c) {
-            const uint32_t a0 = smem_u32(sA(stage, 0, c)), a1 = smem_u32(sA(stage, 1, c));
-            const uint32_t b0 = smem_u32(sB(stage, c));
-#pragma unroll
-            for (int kk = 0; kk < KB / 16; ++kk) {
-              const uint32_t acc = (ks | c | kk) != 0;
-              const uint64_t bd = sw128_desc(b0 + kk * 32);
-              umma_bf16(d0, sw128_desc(a0 + kk * 32), bd, idesc, acc);
-              umma_bf16(d0 + sub_cols, sw128_desc(a1 + kk * 32), bd, idesc, acc);
-            }
+          for (int kk = 0; kk < KB / 16; ++kk) {
+            const uint32_t acc = (kb | kk) != 0;
+            const uint64_t bd = sw128_desc(b0 + kk * 32);
+            umma_bf16(d0, sw128_desc(a0 + kk * 32), bd, idesc, acc);
+            umma_bf16(d0 + sub_cols, sw128_desc(a1 + kk * 32), bd, idesc, acc);
           }
           umma_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tmem_full[bi]);
+        umma_commit(&tmem_full);
       }
       // all issued MMAs must finish before TMEM is released
       umma_commit(&drain_bar);
@@ -391,7 +380,6 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       const int feat_stride = sh ? a2.feat_stride : a.feat_stride;
       const int feat_sub1 = sh ? a2.feat_sub1 : a.feat_sub1;
       const float* row_w = sh ? a2.row_w : a.row_w;
-      const uint32_t bi = nbuf == 2 ? (it & 1u) : 0u, use = nbuf == 2 ? (it >> 1) : it;
       const int nchunk = (ti.N + 31) / 32;
       // GEMM2: the routing weights (and, for the scatter, the tokens) of this
       // warp's 32-row chunks, fetched before the accumulator is ready so that
@@ -416,9 +404,9 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
           tpre[u] = tok;
         }
       }
-      if (!mbar_wait(&tmem_full[bi], use & 1u, &abort_flag, a.status)) break;
+      if (!mbar_wait(&tmem_full, it & 1u, &abort_flag, a.status, wait_ns)) break;
       tc_fence_after();
-      const uint32_t acc_addr = lane_addr + bi * 2u * sub_cols;
+      const uint32_t acc_addr = lane_addr;
       __nv_bfloat16* stg = stage_out[warp - 2];
       if (EPI == EPI_SWIGLU) {
         const int feat0 = ti.mb * feat_stride + 32 * q;            // this warp's 32 features
@@ -460,7 +448,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         }
       }
       tc_fence_before();
-      mbar_arrive(&tmem_empty[bi]);
+      mbar_arrive(&tmem_empty);
     }
   }
 
@@ -468,456 +456,6 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, 512);
-}
-
-// ========================================================================
-// BF16 kernel on CTA pairs (tcgen05 cta_group::2), double-buffered TMEM
-// ========================================================================
-// A CTA pair computes a 256 x N tile with one MMA stream issued by the leader
-// (cluster rank 0): each CTA stages its own 128 weight rows and N/2 of the
-// tokens, and holds the 128 x N fp32 accumulator of its rows in its TMEM.
-// Per SM that halves the token traffic of a 1-CTA 256-row tile and leaves
-// TMEM room for two accumulators (2 x 256 columns), so the epilogue of one
-// tile runs while the next tile's MMAs fill the other buffer.
-//   GEMM1: CTA r holds gate rows [f + 64r, +64) in TMEM lanes 0..63 and the
-//          matching up rows in lanes 64..127 (f = mb*128); the epilogue
-//          warps of lanes 64..127 pass the up values through shared memory
-//          to the warps of lanes 0..63, which compute SiLU(gate) * up.
-//   GEMM2: CTA r holds w2 rows [mb*256 + 128r, +128).
-constexpr int k2smStages = 3;
-constexpr int k2smChunks = 2;              // 64-K chunks per stage: 128 K, 64 KB a stage per CTA
-constexpr int kXStride = 33;               // padded row of the lane exchange buffer
-
-template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-grouped_gemm_bf16_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
-                             const __grid_constant__ TokenMaps tmB, const GemmArgs a) {
-  constexpr int KB = 64;
-  constexpr int KC = k2smChunks;
-  constexpr int STAGES = k2smStages;
-  constexpr uint32_t A_BYTES = 128 * 128;       // this CTA's 128 weight rows x 64 K
-  constexpr uint32_t B_BYTES = 128 * 128;       // up to 128 token rows x 64 K
-  constexpr uint32_t CHUNK_BYTES = A_BYTES + B_BYTES;
-  constexpr uint32_t STAGE_BYTES = KC * CHUNK_BYTES;
-  extern __shared__ __align__(1024) uint8_t dsmem[];
-  __shared__ Sched sched;
-  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
-  __shared__ uint64_t tmem_full[2], tmem_empty[2];
-  __shared__ uint64_t drain_bar, epi_bar;
-  __shared__ uint32_t tmem_base_s;
-  __shared__ volatile int abort_flag;
-  __shared__ float xbuf[2][64 * kXStride];
-  __shared__ __align__(16) __nv_bfloat16 stage_out[4][32 * 32];
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-  const int pair = static_cast<int>(cluster_id_x());
-  const int npairs = static_cast<int>(nclusters_x());
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
-  auto sA = [&](int st, int c) { return smem + st * STAGE_BYTES + c * CHUNK_BYTES; };
-  auto sB = [&](int st, int c) { return smem + st * STAGE_BYTES + c * CHUNK_BYTES + A_BYTES; };
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tmem_full[b], 1);
-      mbar_init(&tmem_empty[b], 8);               // 4 epilogue warps x 2 CTAs
-    }
-    mbar_init(&drain_bar, 1);
-    mbar_init(&epi_bar, 128);
-    abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&tmB.box[i]);
-  }
-  if (warp == 1) {
-    tmem_alloc_2sm(&tmem_base_s, 512);
-    tmem_relinquish_2sm();
-  }
-  if (warp == 2) build_schedule(sched, a, lane);
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();                                 // the peer's barriers exist before any remote signal
-  tc_fence_after();
-  const uint32_t tmem_base = tmem_base_s;
-  const int total = sched.tile_start[a.groups];
-  const int nk = a.K / KB;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      const uint64_t pol_once = policy_evict_first();
-      const uint64_t pol_reuse = policy_evict_normal();
-      const uint64_t pol_x = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int t = pair; t < total && !abort_flag; t += npairs) {
-        const TileInfo ti = decode_tile(sched, a, t);
-        const int half = ti.N >> 1;                       // tokens staged by each CTA
-        const int rows = (half + 15) & ~15;               // rows fetched (multiple of 16)
-        const uint32_t tx = 2u * KC * (A_BYTES + static_cast<uint32_t>(rows) * 128u);
-        const int a_lo = ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride + static_cast<int>(rank) * a.cta_stride;
-        const int a_hi = a_lo + a.sub1_off;
-        const int b0 = ti.row0 + static_cast<int>(rank) * half;
-        const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;
-        bool ok = true;
-        for (int ks = 0; ks < nk / KC; ++ks) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
-          const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
-#pragma unroll
-          for (int c = 0; c < KC; ++c) {
-            const int kb = ks * KC + c;
-            tma_load_2d_2sm(sA(stage, c), &tmA, fb, kb * KB, a_lo, pol_w);
-            if (!a.a_one_box) tma_load_2d_2sm(sA(stage, c) + A_BYTES / 2, &tmA, fb, kb * KB, a_hi, pol_w);
-            uint8_t* bdst = sB(stage, c);
-            load_token_rows(rows, [&](int which, int off) {
-              tma_load_2d_2sm(bdst + off * 128, &tmB.box[which], fb, kb * KB, b0 + off, pol_x);
-            });
-          }
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-      }
-      if (abort_flag) {   // copies complete on the leader's barrier: give them time to land
-        const uint64_t t0 = globaltimer_ns();
-        while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
-      }
-    }
-  } else if (warp == 1) {
-    if (leader && lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, it = 0;
-      for (int t = pair; t < total && !abort_flag; t += npairs, ++it) {
-        const TileInfo ti = decode_tile(sched, a, t);
-        const uint32_t b = it & 1u, use = it >> 1;
-        if (!mbar_wait(&tmem_empty[b], (use & 1u) ^ 1u, &abort_flag, a.status)) break;
-        tc_fence_after();
-        const uint32_t idesc = make_idesc(1u, 256u, static_cast<uint32_t>(ti.N));
-        const uint32_t d = tmem_base + b * 256u;
-        bool ok = true;
-        for (int ks = 0; ks < nk / KC; ++ks) {
-          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < KC; ++c) {
-            const uint32_t a0 = smem_u32(sA(stage, c)), b0 = smem_u32(sB(stage, c));
-#pragma unroll
-            for (int kk = 0; kk < KB / 16; ++kk)
-              umma_bf16_2sm(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (ks | c | kk) != 0);
-          }
-          umma_commit_2sm(&empty_bar[stage], 0x3);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-        umma_commit_2sm(&tmem_full[b], 0x3);
-      }
-      umma_commit_2sm(&drain_bar, 0x1);             // every MMA done before TMEM is freed
-      mbar_wait_drain(&drain_bar, 0);
-    }
-  } else {
-    const int q = warp & 3;
-    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-    const uint32_t empty_addr0 = mapa_shared(smem_u32(&tmem_empty[0]), 0);
-    const uint32_t empty_addr1 = mapa_shared(smem_u32(&tmem_empty[1]), 0);
-    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
-    uint32_t it = 0, epi_phase = 0, xslot = 0;
-    auto epi_sync = [&]() -> bool {
-      mbar_arrive(&epi_bar);
-      const bool r = mbar_wait(&epi_bar, epi_phase, &abort_flag, a.status);
-      epi_phase ^= 1u;
-      return r;
-    };
-    bool ok = true;
-    for (int t = pair; t < total && ok; t += npairs, ++it) {
-      const TileInfo ti = decode_tile(sched, a, t);
-      const uint32_t b = it & 1u, use = it >> 1;
-      if (!mbar_wait(&tmem_full[b], use & 1u, &abort_flag, a.status)) break;
-      tc_fence_after();
-      const uint32_t acc = lane_addr + b * 256u;
-      const int nchunk = (ti.N + 31) / 32;
-      __nv_bfloat16* stg = stage_out[q];
-      if (EPI == EPI_SWIGLU) {
-        // Lanes 0..63 hold gate, 64..127 up, of the same 64 features. Gate
-        // warps finish tokens 0..15 of each chunk, up warps tokens 16..31:
-        // each hands the other half of its values over through xbuf.
-        const bool gate_warp = q < 2;
-        const int fl = 32 * (q & 1) + lane;                                   // feature within the 64
-        const int feat0 = ti.mb * 128 + 64 * static_cast<int>(rank) + 32 * (q & 1);
-        for (int c = 0; c < nchunk; ++c) {
-          float v[32];
-          tmem_ld32(acc + c * 32, v);
-          tmem_ld_wait();
-          float* row = xbuf[xslot & 1u] + fl * kXStride;
-          if (gate_warp) {
-#pragma unroll
-            for (int j = 16; j < 32; ++j) row[j] = v[j];
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) row[j] = v[j];
-          }
-          if (!epi_sync()) { ok = false; break; }
-          float hh[16];
-          if (gate_warp) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) hh[j] = silu(v[j]) * row[j];
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) hh[j] = silu(row[16 + j]) * v[16 + j];
-          }
-          const int t0 = c * 32 + (gate_warp ? 0 : 16);
-          store_tile<16>(stg, hh, lane, out, a.out_ld, ti.row0 + t0, ti.n_valid - t0, feat0);
-          ++xslot;
-        }
-        if (!ok) break;
-      } else {
-        const int feat0 = ti.mb * 256 + 128 * static_cast<int>(rank) + 32 * q;
-        for (int c = 0; c < nchunk; ++c) {
-          float v[32];
-          tmem_ld32(acc + c * 32, v);
-          tmem_ld_wait();
-          if (a.row_w) {
-            const float wl = (c * 32 + lane < ti.n_valid) ? __ldg(a.row_w + ti.row0 + c * 32 + lane) : 0.0f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wl, j);
-          }
-          store_tile<32>(stg, v, lane, out, a.out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(b ? empty_addr1 : empty_addr0);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();                                 // the pair is done with each other's memory
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc_2sm(tmem_base, 512);
-}
-
-// ========================================================================
-// BF16 kernel on CTA pairs, two weight sub-tiles per CTA ("wide" pairs)
-// ========================================================================
-// A CTA pair computes a 512 x N tile: two tcgen05 cta_group::2 MMA streams
-// (M = 256 each) share the pair's token rows. Each CTA stages two 128-row
-// weight sub-tiles and N/2 of the tokens and holds 2 x 128 x N fp32 in its
-// TMEM (512 columns, one accumulator pair, as the single-CTA kernel). Per SM
-// and per 64 K that is 48 KB staged for the same 1024 MMA cycles the
-// single-CTA kernel stages 64 KB for (its 256 tokens are read by both CTAs
-// there), so four stages fit where that kernel holds three.
-//   GEMM1: CTA r sub-tile 0 = gate rows [mb*256 + 128r, +128), sub-tile 1 =
-//          the up rows of the same features: SiLU(gate) * up in-thread.
-//   GEMM2: CTA r sub-tile s = w2 rows [mb*512 + 256s + 128r, +128).
-// TWO: a second single-group problem (the shared expert) whose tiles come
-// first, as in the single-CTA kernel.
-constexpr int kWideStages = 4;           // of 64 K (KC = 1), or 2 of 128 K (KC = 2)
-
-template <int EPI, bool TWO, int EPIW, int KC>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * EPIW, 1)
-grouped_gemm_bf16_2sm_wide_kernel(const __grid_constant__ CUtensorMap tmA,
-                                  const __grid_constant__ TokenMaps tmB, const GemmArgs a,
-                                  const __grid_constant__ CUtensorMap tmA2,
-                                  const __grid_constant__ TokenMaps tmB2, const GemmArgs a2) {
-  constexpr int KB = 64;
-  constexpr int STAGES = kWideStages / KC;
-  constexpr uint32_t A_SUB = 128 * 128;         // one 128-row weight sub-tile x 64 K
-  constexpr uint32_t B_BYTES = 128 * 128;       // up to 128 token rows x 64 K
-  constexpr uint32_t CHUNK_BYTES = 2 * A_SUB + B_BYTES;
-  constexpr uint32_t STAGE_BYTES = KC * CHUNK_BYTES;
-  extern __shared__ __align__(1024) uint8_t dsmem[];
-  __shared__ Sched sched;
-  __shared__ __align__(16) __nv_bfloat16 stage_out[EPIW][32 * 32];
-  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
-  __shared__ uint64_t tmem_full, tmem_empty, drain_bar;
-  __shared__ uint32_t tmem_base_s;
-  __shared__ volatile int abort_flag;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-  const int pair = static_cast<int>(cluster_id_x());
-  const int npairs = static_cast<int>(nclusters_x());
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
-  auto sA = [&](int st, int sub, int c) { return smem + st * STAGE_BYTES + c * CHUNK_BYTES + sub * A_SUB; };
-  auto sB = [&](int st, int c) { return smem + st * STAGE_BYTES + c * CHUNK_BYTES + 2 * A_SUB; };
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
-    }
-    mbar_init(&tmem_full, 1);
-    mbar_init(&tmem_empty, 2 * EPIW);             // every epilogue warp of both CTAs
-    mbar_init(&drain_bar, 1);
-    abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&tmB.box[i]);
-    if (TWO) {
-      tma_prefetch_desc(&tmA2);
-      for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&tmB2.box[i]);
-    }
-  }
-  if (warp == 1) {
-    tmem_alloc_2sm(&tmem_base_s, 512);
-    tmem_relinquish_2sm();
-  }
-  if (warp == 2) build_schedule(sched, a, lane);
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();                                 // the peer's barriers exist before any remote signal
-  tc_fence_after();
-  const uint32_t tmem_base = tmem_base_s;
-  const int total2 = TWO ? tiles_of(a2.rows, a.bn_max, a2.n_mblk) : 0;
-  const int total = total2 + sched.tile_start[a.groups];
-
-  if (warp == 0) {
-    if (lane == 0) {
-      const uint64_t pol_once = policy_evict_first();
-      const uint64_t pol_reuse = policy_evict_normal();
-      const uint64_t pol_x = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int t = pair; t < total && !abort_flag; t += npairs) {
-        const bool sh = TWO && t < total2;
-        const GemmArgs& g = sh ? a2 : a;
-        const TileInfo ti = sh ? decode_in_segment(a2, 0, 0, a2.rows, t) : decode_tile(sched, a, t - total2);
-        const CUtensorMap* mA = sh ? &tmA2 : &tmA;
-        const TokenMaps* mB = sh ? &tmB2 : &tmB;
-        const int nk = g.K / KB;
-        const int half = ti.N >> 1;                       // tokens staged by each CTA
-        const int rows = (half + 15) & ~15;               // rows fetched (multiple of 16)
-        const uint32_t tx = 2u * KC * (2u * A_SUB + static_cast<uint32_t>(rows) * 128u);
-        const int a_lo = ti.g * g.a_rows_per_group + ti.mb * g.mblk_stride + static_cast<int>(rank) * g.cta_stride;
-        const int a_hi = a_lo + g.sub1_off;
-        const int b0 = ti.row0 + static_cast<int>(rank) * half;
-        const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;   // re-read by sibling token blocks
-        bool ok = true;
-        for (int ks = 0; ks < nk / KC; ++ks) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
-          const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
-#pragma unroll
-          for (int c = 0; c < KC; ++c) {
-            const int kb = ks * KC + c;
-            tma_load_2d_2sm(sA(stage, 0, c), mA, fb, kb * KB, a_lo, pol_w);
-            tma_load_2d_2sm(sA(stage, 1, c), mA, fb, kb * KB, a_hi, pol_w);
-            uint8_t* bdst = sB(stage, c);
-            load_token_rows(rows, [&](int which, int off) {
-              tma_load_2d_2sm(bdst + off * 128, &mB->box[which], fb, kb * KB, b0 + off, pol_x);
-            });
-          }
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-      }
-      if (abort_flag) {   // copies complete on the leader's barrier: give them time to land
-        const uint64_t t0 = globaltimer_ns();
-        while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
-      }
-    }
-  } else if (warp == 1) {
-    if (leader && lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, it = 0;
-      for (int t = pair; t < total && !abort_flag; t += npairs, ++it) {
-        const bool sh = TWO && t < total2;
-        const TileInfo ti = sh ? decode_in_segment(a2, 0, 0, a2.rows, t) : decode_tile(sched, a, t - total2);
-        const int nk = (sh ? a2.K : a.K) / KB;
-        if (!mbar_wait(&tmem_empty, (it & 1u) ^ 1u, &abort_flag, a.status)) break;
-        tc_fence_after();
-        const uint32_t idesc = make_idesc(1u, 256u, static_cast<uint32_t>(ti.N));
-        bool ok = true;
-        for (int ks = 0; ks < nk / KC; ++ks) {
-          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < KC; ++c) {
-            const uint32_t a0 = smem_u32(sA(stage, 0, c)), a1 = smem_u32(sA(stage, 1, c));
-            const uint32_t b0 = smem_u32(sB(stage, c));
-#pragma unroll
-            for (int kk = 0; kk < KB / 16; ++kk) {
-              const uint32_t acc = (ks | c | kk) != 0;
-              const uint64_t bd = sw128_desc(b0 + kk * 32);
-              umma_bf16_2sm(tmem_base, sw128_desc(a0 + kk * 32), bd, idesc, acc);
-              umma_bf16_2sm(tmem_base + 256u, sw128_desc(a1 + kk * 32), bd, idesc, acc);
-            }
-          }
-          umma_commit_2sm(&empty_bar[stage], 0x3);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-        umma_commit_2sm(&tmem_full, 0x3);
-      }
-      umma_commit_2sm(&drain_bar, 0x1);             // every MMA done before TMEM is freed
-      mbar_wait_drain(&drain_bar, 0);
-    }
-  } else {
-    // epilogue warps 2 .. 1+EPIW: warp w reads TMEM lanes 32*(w%4)..+31 of
-    // both sub-tiles; with 8 or 12 warps, two or three share each lane
-    // quarter and take turns on its 32-token chunks
-    const int q = warp & 3;
-    const int c0 = (warp - 2) / 4, cstep = EPIW / 4;
-    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-    const uint32_t empty_addr = mapa_shared(smem_u32(&tmem_empty), 0);
-    __nv_bfloat16* stg = stage_out[warp - 2];
-    uint32_t it = 0;
-    for (int t = pair; t < total; t += npairs, ++it) {
-      const bool sh = TWO && t < total2;
-      const GemmArgs& g = sh ? a2 : a;
-      const TileInfo ti = sh ? decode_in_segment(a2, 0, 0, a2.rows, t) : decode_tile(sched, a, t - total2);
-      if (!mbar_wait(&tmem_full, it & 1u, &abort_flag, a.status)) break;
-      tc_fence_after();
-      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out);
-      const int nchunk = (ti.N + 31) / 32;
-      const int fbase = ti.mb * g.feat_stride + 128 * static_cast<int>(rank) + 32 * q;
-      if (EPI == EPI_SWIGLU) {
-        for (int c = c0; c < nchunk; c += cstep) {
-          float gt[32], up[32];
-          tmem_ld32(lane_addr + c * 32, gt);
-          tmem_ld32(lane_addr + 256u + c * 32, up);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) gt[j] = silu(gt[j]) * up[j];
-          store_tile<32>(stg, gt, lane, out, g.out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, fbase);
-        }
-      } else {
-#pragma unroll 1
-        for (int s = 0; s < 2; ++s) {
-          for (int c = c0; c < nchunk; c += cstep) {
-            float v[32];
-            tmem_ld32(lane_addr + s * 256u + c * 32, v);
-            tmem_ld_wait();
-            if (g.row_w) {
-              const float wl = (c * 32 + lane < ti.n_valid) ? __ldg(g.row_w + ti.row0 + c * 32 + lane) : 0.0f;
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wl, j);
-            }
-            store_tile<32>(stg, v, lane, out, g.out_ld, ti.row0 + c * 32, ti.n_valid - c * 32,
-                           fbase + s * g.feat_sub1);
-          }
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(empty_addr);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();                                 // the pair is done with each other's memory
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc_2sm(tmem_base, 512);
 }
 
 // ========================================================================
@@ -998,7 +536,7 @@ grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status, a.wait_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
           tma_load_2d(sA(stage, 0), &tmA, &full_bar[stage], kb * KB, a_row0, pol_w);
           tma_load_2d(sA(stage, 1), &tmA, &full_bar[stage], kb * KB, a_row1, pol_w);
@@ -1025,8 +563,8 @@ grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int kb = 0; kb < nk; ++kb, ++kbg) {
           const uint32_t slot = kbg % kF8Slots;
           const uint32_t slot_phase = (kbg / kF8Slots) & 1u;
-          if (!mbar_wait(&part_empty[slot], slot_phase ^ 1u, &abort_flag, a.status)) { ok = false; break; }
-          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait(&part_empty[slot], slot_phase ^ 1u, &abort_flag, a.status, a.wait_ns)) { ok = false; break; }
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, a.status, a.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem_base + slot * kF8SlotCols;
           const uint32_t a0 = smem_u32(sA(stage, 0)), a1 = smem_u32(sA(stage, 1));
@@ -1057,7 +595,7 @@ grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
     // Bounded sync of the 128 epilogue threads (an abort ends it, never hangs).
     auto epi_sync = [&]() -> bool {
       mbar_arrive(&epi_bar);
-      const bool r = mbar_wait(&epi_bar, epi_phase, &abort_flag, a.status);
+      const bool r = mbar_wait(&epi_bar, epi_phase, &abort_flag, a.status, a.wait_ns);
       epi_phase ^= 1u;
       return r;
     };
@@ -1081,7 +619,7 @@ grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int kb = 0; kb < nk; ++kb, ++kbg) {
         const uint32_t slot = kbg % kF8Slots;
         const uint32_t slot_phase = (kbg / kF8Slots) & 1u;
-        if (!mbar_wait(&part_full[slot], slot_phase, &abort_flag, a.status)) { ok = false; break; }
+        if (!mbar_wait(&part_full[slot], slot_phase, &abort_flag, a.status, a.wait_ns)) { ok = false; break; }
         tc_fence_after();
         float v0[32], v1[32];
         tmem_ld32(lane_addr + slot * kF8SlotCols, v0);
@@ -1149,101 +687,44 @@ grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
 // ------------------------------------------------------------------------
 // host-side launch helpers (called from api.cu)
 // ------------------------------------------------------------------------
-size_t gemm_bf16_smem_bytes(int stages, int bn_max) {
-  return static_cast<size_t>(stages) * (2 * 128 * 128 + static_cast<size_t>(bn_max) * 128) + 1024;
-}
-size_t gemm_bf16_2sm_smem_bytes() {
-  return static_cast<size_t>(k2smStages) * k2smChunks * (2 * 128 * 128) + 1024;
-}
-size_t gemm_bf16_2sm_wide_smem_bytes() {
-  return static_cast<size_t>(kWideStages) * (3 * 128 * 128) + 1024;
-}
-size_t gemm_e4m3_smem_bytes(int stages) {
-  return static_cast<size_t>(stages) * (2 * 128 * 128 + kF8Bn * 128) + 1024;
-}
-
 constexpr int kBf16Stages = 3;
-constexpr int kBf16StagesDb = 4;
-constexpr int kBf16StagesK128 = 1;        // 128 K per stage (two 64-K chunks)
-constexpr int kBf16StagesDbK128 = 2;
 constexpr int kE4m3Stages = 4;
+
+size_t gemm_bf16_smem_bytes(int bn_max) {
+  return static_cast<size_t>(kBf16Stages) * (2 * 128 * 128 + static_cast<size_t>(bn_max) * 128) + 1024;
+}
+size_t gemm_e4m3_smem_bytes() {
+  return static_cast<size_t>(kE4m3Stages) * (2 * 128 * 128 + kF8Bn * 128) + 1024;
+}
 
 using Bf16Kernel = void (*)(CUtensorMap, TokenMaps, GemmArgs, CUtensorMap, TokenMaps, GemmArgs);
 
-// The single-CTA bf16 kernel: (one problem | two) x (64 | 128 K per stage)
-// x (4 | 8 | 12 epilogue warps).
-template <int EPI, int STAGES, int STAGES_K128, int EPIW>
-Bf16Kernel bf16_kernel_w(bool two, bool k128) {
-  if (k128)
-    return two ? grouped_gemm_bf16_kernel<EPI, STAGES_K128, false, true, 2, EPIW>
-               : grouped_gemm_bf16_kernel<EPI, STAGES_K128, false, false, 2, EPIW>;
-  return two ? grouped_gemm_bf16_kernel<EPI, STAGES, false, true, 1, EPIW>
-             : grouped_gemm_bf16_kernel<EPI, STAGES, false, false, 1, EPIW>;
-}
-template <int EPI, int STAGES, int STAGES_K128>
-Bf16Kernel bf16_kernel(bool two, bool k128, int epi_warps) {
-  if (epi_warps == 12) return bf16_kernel_w<EPI, STAGES, STAGES_K128, 12>(two, k128);
-  return epi_warps == 8 ? bf16_kernel_w<EPI, STAGES, STAGES_K128, 8>(two, k128)
-                        : bf16_kernel_w<EPI, STAGES, STAGES_K128, 4>(two, k128);
-}
-
-template <int EPI, bool TWO, int KC>
-Bf16Kernel wide_kernel_k(int epi_warps) {
-  if (epi_warps == 12) return grouped_gemm_bf16_2sm_wide_kernel<EPI, TWO, 12, KC>;
-  return epi_warps == 8 ? grouped_gemm_bf16_2sm_wide_kernel<EPI, TWO, 8, KC>
-                        : grouped_gemm_bf16_2sm_wide_kernel<EPI, TWO, 4, KC>;
-}
-template <int EPI, bool TWO>
-Bf16Kernel wide_kernel(int epi_warps, bool k128) {
-  return k128 ? wide_kernel_k<EPI, TWO, 2>(epi_warps) : wide_kernel_k<EPI, TWO, 1>(epi_warps);
+// The bf16 kernel forms: (one problem | two) x (4 | 12 epilogue warps).
+template <int EPI>
+Bf16Kernel bf16_kernel(bool two, int epi_warps) {
+  if (epi_warps == 12)
+    return two ? grouped_gemm_bf16_kernel<EPI, kBf16Stages, false, true, 12>
+               : grouped_gemm_bf16_kernel<EPI, kBf16Stages, false, false, 12>;
+  return two ? grouped_gemm_bf16_kernel<EPI, kBf16Stages, false, true, 4>
+             : grouped_gemm_bf16_kernel<EPI, kBf16Stages, false, false, 4>;
 }
 
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const TokenMaps& tmB,
                                 const GemmArgs& a, int grid, cudaStream_t stream, const SecondProblem* two) {
-  if (!e4m3 && a.cta_stride > 0 && a.wide) {
-    const int epiw = a.epi_warps == 8 || a.epi_warps == 12 ? a.epi_warps : 4;
-    const bool pair2 = two != nullptr;
-    const bool k128 = a.kc == 2;
-    Bf16Kernel kern = epi == EPI_SWIGLU ? (pair2 ? wide_kernel<EPI_SWIGLU, true>(epiw, k128)
-                                                 : wide_kernel<EPI_SWIGLU, false>(epiw, k128))
-                                        : (pair2 ? wide_kernel<EPI_WEIGHTED, true>(epiw, k128)
-                                                 : wide_kernel<EPI_WEIGHTED, false>(epiw, k128));
-    const size_t smem = gemm_bf16_2sm_wide_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    if (pair2)
-      kern<<<grid & ~1, 64 + 32 * epiw, smem, stream>>>(tmA, tmB, a, two->tmA, two->tmB, two->a);
-    else
-      kern<<<grid & ~1, 64 + 32 * epiw, smem, stream>>>(tmA, tmB, a, tmA, tmB, a);
-  } else if (!e4m3 && a.cta_stride > 0) {
-    const size_t smem = gemm_bf16_2sm_smem_bytes();
-    auto kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_2sm_kernel<EPI_SWIGLU>
-                                  : grouped_gemm_bf16_2sm_kernel<EPI_WEIGHTED>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    kern<<<grid & ~1, kThreads, smem, stream>>>(tmA, tmB, a);
-  } else if (!e4m3) {
+  if (!e4m3) {
     const bool gather = a.gather_rows != nullptr;
-    // two accumulators hold <= 128-token tiles: 48 KB stages, four of them
-    const bool db = a.nbuf == 2 && !gather;
-    const bool k128 = a.kc == 2 && !gather;
-    const int epiw = gather ? 4 : (a.epi_warps == 8 || a.epi_warps == 12 ? a.epi_warps : 4);
+    const int epiw = gather ? 4 : (a.epi_warps == 12 ? 12 : 4);
     const int threads = 64 + 32 * epiw + (gather ? kGatherThreads : 0);
-    const int stages = k128 ? (db ? kBf16StagesDbK128 : kBf16StagesK128) : (db ? kBf16StagesDb : kBf16Stages);
-    const size_t smem = gemm_bf16_smem_bytes(stages, a.bn_max) * (k128 ? 2 : 1) - (k128 ? 1024 : 0);
+    const size_t smem = gemm_bf16_smem_bytes(a.bn_max);
     const bool pair2 = two != nullptr && !gather;
     Bf16Kernel kern;
     if (gather)
       kern = epi == EPI_SWIGLU ? grouped_gemm_bf16_kernel<EPI_SWIGLU, kBf16Stages, true, false>
                                : grouped_gemm_bf16_kernel<EPI_WEIGHTED, kBf16Stages, true, false>;
     else if (epi == EPI_SCATTER)
-      kern = bf16_kernel<EPI_SCATTER, kBf16Stages, kBf16StagesK128>(pair2, false, epiw);
-    else if (db)
-      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128, epiw)
-                               : bf16_kernel<EPI_WEIGHTED, kBf16StagesDb, kBf16StagesDbK128>(pair2, k128, epiw);
+      kern = bf16_kernel<EPI_SCATTER>(pair2, epiw);
     else
-      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU, kBf16Stages, kBf16StagesK128>(pair2, k128, epiw)
-                               : bf16_kernel<EPI_WEIGHTED, kBf16Stages, kBf16StagesK128>(pair2, k128, epiw);
+      kern = epi == EPI_SWIGLU ? bf16_kernel<EPI_SWIGLU>(pair2, epiw) : bf16_kernel<EPI_WEIGHTED>(pair2, epiw);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     if (pair2)
@@ -1251,7 +732,7 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
     else
       kern<<<grid, threads, smem, stream>>>(tmA, tmB, a, tmA, tmB, a);
   } else {
-    const size_t smem = gemm_e4m3_smem_bytes(kE4m3Stages);
+    const size_t smem = gemm_e4m3_smem_bytes();
     auto kern = epi == EPI_SWIGLU ? grouped_gemm_e4m3_kernel<EPI_SWIGLU, kE4m3Stages>
                                   : grouped_gemm_e4m3_kernel<EPI_WEIGHTED, kE4m3Stages>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -6,40 +6,36 @@
 namespace moe {
 
 struct GemmArgs {
-  int32_t rows;              // activation rows (B operand)
-  int32_t K;                 // reduction length
-  int32_t groups;            // number of segments
-  const int32_t* offsets;    // [groups + 1] or nullptr (one segment)
-  int32_t a_rows_per_group;  // weight rows per group (2I or H)
-  int32_t n_mblk;            // weight blocks per group
-  int32_t mblk_stride;       // weight-row stride between blocks (128 / 256)
-  int32_t sub1_off;          // weight-row offset of sub-tile 1 (I / 128)
-  int32_t feat_stride;       // output-feature stride between blocks (128 / 256)
-  int32_t feat_sub1;         // output-feature offset of sub-tile 1 (0 / 128)
-  int32_t bn_max;            // max tokens per tile (multiple of 32, <= 256)
-  int32_t cta_stride;        // CTA-pair kernel: weight-row offset of the second CTA (0 = 1-CTA kernel)
-  int32_t nbuf;              // 1-CTA kernel: TMEM accumulators (2 needs bn_max <= 128)
-  int32_t a_one_box;         // a CTA's weight rows are contiguous: one TMA box (256 rows, pair: 128)
-  void* out;                 // [rows, out_ld] bf16, or e4m3 codes (GEMM1 FP8)
-  int32_t out_ld;
-  const float* row_w;        // [rows] or nullptr
-  const float* a_scale;      // E4M3: [groups, a_rows_per_group/128, K/128]
-  const float* b_scale;      // E4M3: [rows, K/128]
-  float* out_scale;          // E4M3 GEMM1: [rows, out_ld/128]
-  int32_t* status;
+  int32_t rows = 0;                // activation rows (B operand)
+  int32_t K = 0;                   // reduction length
+  int32_t groups = 1;              // number of segments
+  const int32_t* offsets = nullptr;  // [groups + 1] or nullptr (one segment)
+  int32_t a_rows_per_group = 0;    // weight rows per group (2I or H)
+  int32_t n_mblk = 0;              // weight blocks per group
+  int32_t mblk_stride = 0;         // weight-row stride between blocks (128 / 256)
+  int32_t sub1_off = 0;            // weight-row offset of sub-tile 1 (I / 128)
+  int32_t feat_stride = 0;         // output-feature stride between blocks (128 / 256)
+  int32_t feat_sub1 = 0;           // output-feature offset of sub-tile 1 (0 / 128)
+  int32_t bn_max = 256;            // max tokens per tile (multiple of 32, <= 256)
+  int32_t a_one_box = 0;           // a tile's 256 weight rows are contiguous: one TMA box
+  void* out = nullptr;             // [rows, out_ld] bf16, or e4m3 codes (GEMM1 FP8)
+  int32_t out_ld = 0;
+  const float* row_w = nullptr;    // [rows] or nullptr
+  const float* a_scale = nullptr;  // E4M3: [groups, a_rows_per_group/128, K/128]
+  const float* b_scale = nullptr;  // E4M3: [rows, K/128]
+  float* out_scale = nullptr;      // E4M3 GEMM1: [rows, out_ld/128]
+  int32_t* status = nullptr;
   // Gathered token rows (gate/up GEMM of the routed experts): B row p is
   // row gather_rows[p] of gather_src [*, K] instead of row p of the B map.
-  const void* gather_src;
-  const int32_t* gather_rows;
-  int32_t gather_src_rows;   // rows of gather_src (indices outside [0, this) are flagged, not read)
-  int32_t kc;                // 1-CTA bf16 kernel: 64-K chunks per pipeline stage (1 or 2)
-  int32_t epi_warps;         // 1-CTA bf16 kernel: epilogue warps (4, 8 or 12)
+  const void* gather_src = nullptr;
+  const int32_t* gather_rows = nullptr;
+  int32_t gather_src_rows = 0;     // rows of gather_src (indices outside [0, this) are flagged, not read)
+  int32_t epi_warps = 4;           // bf16 kernel: epilogue warps (4 or 12)
   // EPI_SCATTER: token of each row ([rows], NULL: the row is the token) and the
   // number of tokens (rows of the fp32 accumulator `out`)
-  const int32_t* scatter_tok;
-  int32_t scatter_T;
-  // CTA-pair kernel with two weight sub-tiles per CTA (512 weight rows a pair)
-  int32_t wide;
+  const int32_t* scatter_tok = nullptr;
+  int32_t scatter_T = 0;
+  uint64_t wait_ns = kDefaultWaitLimitNs;  // limit of each bounded mbarrier wait
 };
 
 struct RouteArgs {
@@ -52,14 +48,13 @@ struct RouteArgs {
   float* w;                 // [T, k]
   int32_t* counts;          // [E], zeroed beforehand
   int32_t* status;
+  uint64_t wait_ns;         // limit of each bounded mbarrier wait
 };
 
 // EPI_SCATTER: GEMM2 with the combine fused in: the weighted fp32 rows are
 // added atomically into a [tokens, H] fp32 accumulator at their token.
 enum { EPI_SWIGLU = 0, EPI_WEIGHTED = 1, EPI_SCATTER = 2 };
 
-// tmB: token-row tensor maps with 64-, 32- and 16-row boxes (bf16), or one
-// 32-row map (e4m3).
 // Token-row tensor maps: bf16 boxes of 256, 128, 64, 32 and 16 rows (a tile's
 // rows are fetched with the fewest boxes); e4m3 uses box[0] of 32 rows.
 constexpr int kTokBoxes = 5;
@@ -67,7 +62,7 @@ struct TokenMaps {
   CUtensorMap box[kTokBoxes];
 };
 
-// A second single-group problem for the same launch (bf16, single-CTA kernel).
+// A second single-group problem for the same launch (bf16).
 struct SecondProblem {
   CUtensorMap tmA;
   TokenMaps tmB;

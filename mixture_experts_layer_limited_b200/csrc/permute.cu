@@ -12,7 +12,6 @@
 //   3. perm_place : one warp per token ranks its slots among the earlier
 //                   slots of its block (ballots), writes the metadata, reads
 //                   the token's row once and writes it to its k rows.
-#include <cstdlib>
 
 #include "kernels.cuh"
 
@@ -221,84 +220,6 @@ perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ top
   }
 }
 
-// ------------------------------------------------------------------------
-// perm_place with the row copies on the bulk-copy (TMA) engine (an option,
-// MOE_PERM_BULK=1; the threads' own copies measured faster): lane 0 of a
-// token's warp loads the row into shared memory with one cp.async.bulk
-// (issued before the slot ranks are computed, so the load overlaps them) and
-// writes it to the token's k rows with k bulk stores; the warp's threads only
-// compute ranks and metadata. E4M3 scales (a few hundred bytes a row) are
-// copied by the warp as in perm_place_kernel.
-// ------------------------------------------------------------------------
-constexpr int kBulkSmemBytes = 100 * 1024;   // row buffers per CTA (two CTAs per SM)
-
-__device__ __forceinline__ void bulk_load_row(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(smem_dst)),
-               "l"(static_cast<uint64_t>(__cvta_generic_to_global(gsrc))), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void bulk_store_row(void* gdst, const void* smem_src, uint32_t bytes, uint64_t policy) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(
-                   static_cast<uint64_t>(__cvta_generic_to_global(gdst))),
-               "r"(smem_u32(smem_src)), "r"(bytes), "l"(policy)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-  return true;
-}
-
-__global__ void __launch_bounds__(256)
-perm_place_bulk_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T, int k, int E,
-                       const int32_t* __restrict__ blockbase, int32_t* __restrict__ slot_to_row,
-                       int32_t* __restrict__ src_token, float* __restrict__ row_w,
-                       const uint8_t* __restrict__ x, int row_bytes, uint8_t* __restrict__ x_perm,
-                       const float* __restrict__ x_scale, float* __restrict__ x_perm_scale, int nscale,
-                       int32_t* status) {
-  extern __shared__ __align__(128) uint8_t rowbuf[];
-  __shared__ uint64_t bar[8];
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int t = blockIdx.x * (blockDim.x >> 5) + w;
-  if (t >= T) return;                                  // warp-uniform
-  uint8_t* buf = rowbuf + static_cast<size_t>(w) * row_bytes;
-  if (lane == 0) {
-    mbar_init(&bar[w], 1);
-    fence_barrier_init();
-    mbar_arrive_expect_tx(&bar[w], static_cast<uint32_t>(row_bytes));
-    bulk_load_row(buf, x + static_cast<size_t>(t) * row_bytes, static_cast<uint32_t>(row_bytes), &bar[w]);
-  }
-  const int my_row = perm_rows_of_token(t, lane, ids, topk_w, T, k, E, blockbase, slot_to_row, src_token, row_w);
-  int landed = 1;
-  if (lane == 0) landed = mbar_wait_bounded(&bar[w], 0) ? 1 : 0;
-  landed = __shfl_sync(0xffffffffu, landed, 0);
-  if (!landed) {                                       // the row never arrived: flag, write nothing
-    if (lane == 0) flag_status(status, MOE_DEVSTAT_TIMEOUT);
-    return;
-  }
-  const uint64_t pol = policy_evict_first();           // x_perm is far larger than L2
-  for (int j = 0; j < k; ++j) {                        // warp-uniform trip count
-    const int row = __shfl_sync(0xffffffffu, my_row, j);
-    if (lane == 0 && row >= 0)
-      bulk_store_row(x_perm + static_cast<size_t>(row) * row_bytes, buf, static_cast<uint32_t>(row_bytes), pol);
-  }
-  if (lane == 0) {
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // the buffer has been read
-  }
-  if (x_scale) {
-    for (int j = 0; j < k; ++j) {
-      const int row = __shfl_sync(0xffffffffu, my_row, j);
-      if (row < 0) continue;                              // warp-uniform
-      for (int i = lane; i < nscale; i += 32)
-        x_perm_scale[static_cast<size_t>(row) * nscale + i] = x_scale[static_cast<size_t>(t) * nscale + i];
-    }
-  }
-}
-
 size_t permute_workspace_bytes(int T, int E) {
   const int nb = (T + kTokBlock - 1) / kTokBlock;
   return static_cast<size_t>(nb) * E * sizeof(int32_t);
@@ -314,22 +235,6 @@ cudaError_t launch_permute(int T, int k, int E, int row_bytes, const int32_t* id
   const int parts = 1024 / E;
   const size_t scan_smem = (static_cast<size_t>(parts) * E + E + 32) * sizeof(int);
   perm_scan_kernel<<<1, 1024, scan_smem, stream>>>(blockhist, nb, E, T * k, offsets);
-  // rows to copy: by the threads' own 16-byte loads and stores, or with
-  // MOE_PERM_BULK=1 on the bulk-copy engine (when a row buffer per warp
-  // fits; measured about 5 % slower for the V3 layer's 14 KB rows)
-  const char* bulk = std::getenv("MOE_PERM_BULK");
-  const int bulk_warps = row_bytes > 0 ? kBulkSmemBytes / row_bytes : 0;
-  if (x_perm && bulk_warps >= 1 && row_bytes % 16 == 0 && bulk && bulk[0] == '1') {
-    const int warps = bulk_warps < 8 ? bulk_warps : 8;
-    const size_t smem = static_cast<size_t>(warps) * row_bytes;
-    cudaError_t e = cudaFuncSetAttribute(perm_place_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    perm_place_bulk_kernel<<<(T + warps - 1) / warps, warps * 32, smem, stream>>>(
-        ids, topk_w, T, k, E, blockhist, slot_to_row, src_token, row_w, static_cast<const uint8_t*>(x),
-        row_bytes, static_cast<uint8_t*>(x_perm), x_scale, x_perm_scale, nscale, status);
-    return cudaGetLastError();
-  }
   const int warps = 8;
   perm_place_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
       ids, topk_w, T, k, E, blockhist, slot_to_row, src_token, row_w, reinterpret_cast<const uint4*>(x),

@@ -20,7 +20,6 @@
 //       scores and ranked with shuffles, and the top-k is k rounds of an
 //       arg-max over the token's threads (larger score first, lower expert
 //       index on ties).
-#include <cstdlib>
 
 #include "kernels.cuh"
 
@@ -95,7 +94,7 @@ gate_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
       uint32_t phase = 0;
       for (int i = 0; i < kb_count; ++i) {
         const int kb = kb_begin + i;
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, r.status)) break;
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, r.status, r.wait_ns)) break;
         mbar_arrive_expect_tx(&full_bar[stage], stage_bytes);
         uint8_t* st = smem + stage * stage_bytes;
         tma_load_2d(st, &tmX, &full_bar[stage], kb * KB, m0, pol_x);
@@ -115,7 +114,7 @@ gate_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
       uint32_t phase = 0;
       bool ok = true;
       for (int i = 0; i < kb_count; ++i) {
-        if (!mbar_wait(&full_bar[stage], phase, &abort_flag, r.status)) { ok = false; break; }
+        if (!mbar_wait(&full_bar[stage], phase, &abort_flag, r.status, r.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a0 = smem_u32(smem + stage * stage_bytes);
         const uint32_t b0 = a0 + a_bytes;
@@ -130,7 +129,7 @@ gate_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
       mbar_wait_drain(&drain_bar, 0);
     }
   } else if (kb_count > 0) {
-    mbar_wait(&tmem_full, 0, &abort_flag, r.status);   // an abort still reaches the cluster barriers
+    mbar_wait(&tmem_full, 0, &abort_flag, r.status, r.wait_ns);   // an abort still reaches the cluster barriers
     tc_fence_after();
   }
   // both CTAs: every MMA has completed (epilogue threads arrive only after
@@ -495,11 +494,9 @@ cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, con
 }
 
 cudaError_t launch_route_tokens(const RouteArgs& r, int num_sms, cudaStream_t stream) {
-  // eight threads per token where the shape allows (MOE_ROUTE_WARP=1: always a warp)
-  const char* force_warp = std::getenv("MOE_ROUTE_WARP");
+  // eight threads per token where the shape allows, else one warp per token
   const int C = r.E / 8;
-  if (!(force_warp && force_warp[0] == '1') && r.E % 8 == 0 && r.k <= 8 && 8 % r.G == 0 &&
-      (C == 2 || C == 4 || C == 8 || C == 16 || C == 32)) {
+  if (r.E % 8 == 0 && r.k <= 8 && 8 % r.G == 0 && (C == 2 || C == 4 || C == 8 || C == 16 || C == 32)) {
     const int need = (r.T + 31) / 32;                 // 32 tokens per CTA of 256 threads
     const int grid = need < 4 * num_sms ? need : 4 * num_sms;
     switch (C) {

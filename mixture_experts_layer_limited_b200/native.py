@@ -33,6 +33,7 @@ EXPORTED = [
     "moe_combine", "moe_bias_update", "moe_aux_loss_workspace_size", "moe_aux_loss",
     "moe_quantize_blocks", "moe_quantize_rows",
     "moe_read_device_status", "moe_last_cuda_error", "moe_status_string", "moe_abi_version",
+    "moe_set_wait_limit_ns", "moe_wait_limit_ns",
 ]
 
 
@@ -97,11 +98,14 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_last_cuda_error": [],
         "moe_status_string": [_I],
         "moe_abi_version": [],
+        "moe_set_wait_limit_ns": [ctypes.c_uint64],
+        "moe_wait_limit_ns": [],
     }
+    restype = {"moe_status_string": ctypes.c_char_p, "moe_wait_limit_ns": ctypes.c_uint64}
     for name, args in sig.items():
         f = getattr(lib, name)
         f.argtypes = args
-        f.restype = ctypes.c_char_p if name == "moe_status_string" else ctypes.c_int32
+        f.restype = restype.get(name, ctypes.c_int32)
     _LIB = lib
     return lib
 
@@ -271,3 +275,13 @@ def moe_read_device_status(dev_status, stream=None) -> int:
     if st not in (MOE_OK, MOE_ERR_DEVICE_CHECK, MOE_ERR_DEVICE_TIMEOUT):
         _check("moe_read_device_status", st)
     return out.value
+
+
+def moe_set_wait_limit_ns(ns: int):
+    """Limit of every bounded device-side wait for later launches (0: the
+    default, 2 s). A debugging knob; process-wide."""
+    _check("moe_set_wait_limit_ns", load_library().moe_set_wait_limit_ns(int(ns)))
+
+
+def moe_wait_limit_ns() -> int:
+    return int(load_library().moe_wait_limit_ns())

@@ -164,3 +164,14 @@ int main(void) {
     assert int(ver) == N.load_library().moe_abi_version()
     assert int(s) == N.MOE_OK and int(ws) == N.moe_permute_workspace_size(8192, 8, 256)
     assert int(bad) == N.MOE_ERR_INVALID_ARG
+
+
+def test_wait_limit_knob_round_trip_is_host_only():
+    """moe_set_wait_limit_ns only records the limit for later launches."""
+    assert N.moe_wait_limit_ns() == 2_000_000_000
+    try:
+        N.moe_set_wait_limit_ns(12345)
+        assert N.moe_wait_limit_ns() == 12345
+    finally:
+        N.moe_set_wait_limit_ns(0)
+    assert N.moe_wait_limit_ns() == 2_000_000_000

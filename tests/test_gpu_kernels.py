@@ -3,6 +3,7 @@
 Bit-exact: E4M3 codes and scales, routing ids / counts given identical fp32
 logits, the permutation, the bias trajectory. Floating point: within the
 tolerance each test states."""
+import ctypes
 import dataclasses
 
 import numpy as np
@@ -138,47 +139,45 @@ def test_route_gate_gemm(name, T):
     print(f"{name} T={T}: near-tie tokens excluded {int(flagged.sum())}")
 
 
-@pytest.mark.parametrize("name,T,topk_group", [("tiny", None, None), ("tiny_grouped", None, None),
-                                               ("v2lite", None, None), ("v3", None, None), ("v3", 1001, 2),
-                                               ("v3", 77, 8), ("v3_ties", 777, None), ("v2lite", 1, None)])
-def test_route_eight_threads_per_token_matches_warp_per_token(name, T, topk_group, monkeypatch):
-    """The two routing kernels (eight threads per token, the default where the
-    shape allows; one warp per token) take the same decisions: ids and counts
-    bit for bit, weights bit for bit with sigmoid scores and to the last bit
-    of the softmax denominator's summation order otherwise."""
-    cfg = _cfg(name)
-    if topk_group:
-        cfg = dataclasses.replace(cfg, topk_group=topk_group)
+# Shapes outside the eight-threads-per-token kernel's range (k > 8, n_group
+# not dividing 8, E / 8 not a power of two from 2 to 32) are routed by the
+# general one-warp-per-token kernel: ids, counts and weights against the
+# oracle as for the default kernel.
+WARP_ROUTE_CASES = [
+    ("v3 k=9", "v3", dict(k=9), 2048),
+    ("v3 16 groups keep 8", "v3", dict(n_group=16, topk_group=8), 2048),
+    ("E=48 softmax top-6", "v2lite", dict(E=48), 1500),
+    ("tiny k=12", "tiny", dict(k=12), None),
+    ("tiny_grouped k=9 ties", "tiny_grouped", dict(k=9, topk_group=3), 500),
+]
+
+
+@pytest.mark.parametrize("label,name,over,T", WARP_ROUTE_CASES, ids=[c[0] for c in WARP_ROUTE_CASES])
+def test_route_warp_per_token_shapes_bit_exact(label, name, over, T):
+    cfg = dataclasses.replace(_cfg(name), **over)
     T = T or cfg.T
     L = make_logits(cfg, device=DEV, T=T)
     bias = uniform_bias(cfg.E, cfg.seed + 5) if cfg.scoring == "sigmoid" else None
-    if name == "v3_ties":
+    if "ties" in label:
         L = torch.round(L * 4) / 4
         bias = torch.round(bias * 50) / 50
-    monkeypatch.delenv("MOE_ROUTE_WARP", raising=False)
-    ids0, w0, c0, _ = gpu_route(cfg, T, bias=bias, logits=L)
-    monkeypatch.setenv("MOE_ROUTE_WARP", "1")
-    ids1, w1, c1, _ = gpu_route(cfg, T, bias=bias, logits=L)
+    ids, w, counts, _ = gpu_route(cfg, T, bias=bias, logits=L)
     torch.cuda.synchronize()
-    assert torch.equal(ids0, ids1) and torch.equal(c0, c1)
-    if cfg.scoring == "sigmoid":
-        assert torch.equal(w0, w1)
-    else:
-        torch.testing.assert_close(w0, w1, rtol=1e-6, atol=0)
+    r = oracle_route(np32(L), cfg, np32(bias) if bias is not None else None)
+    assert np.array_equal(ids.cpu().numpy(), r.ids)
+    assert np.array_equal(counts.cpu().numpy(), r.counts)
+    np.testing.assert_allclose(w.cpu().numpy(), r.weights, rtol=5e-6, atol=1e-7)
 
 
-@pytest.mark.parametrize("warp", [False, True])
-def test_route_token_with_nan_scores_is_flagged_not_routed(warp, monkeypatch):
+@pytest.mark.parametrize("k", [8, 9], ids=["eight-threads-kernel", "warp-kernel"])
+def test_route_token_with_nan_scores_is_flagged_not_routed(k):
     """Without a group limit, a token whose logits are all NaN has no winner
     in any round: its slots get id -1 and weight 0, the status word is
     flagged, nothing is counted for it, and the other tokens route as usual.
     (With a group limit the experts of the dropped groups score -inf, which
-    still compares, so such a token is routed there with NaN weights.)"""
-    if warp:
-        monkeypatch.setenv("MOE_ROUTE_WARP", "1")
-    else:
-        monkeypatch.delenv("MOE_ROUTE_WARP", raising=False)
-    cfg = dataclasses.replace(get_config("v3"), n_group=1, topk_group=1)
+    still compares, so such a token is routed there with NaN weights.)
+    k = 8 runs the eight-threads-per-token kernel, k = 9 the warp kernel."""
+    cfg = dataclasses.replace(get_config("v3"), n_group=1, topk_group=1, k=k)
     T = 64
     L = make_logits(cfg, device=DEV, T=T)
     L[5] = float("nan")
@@ -224,22 +223,11 @@ def _ids_from_oracle(T, k, E, seed, skew=0.0):
     return r.ids, r.weights.astype(np.float32)
 
 
-@pytest.fixture(params=["lsu", "bulk"])
-def perm_copy(request, monkeypatch):
-    """The permutation's row copies: by the threads' own 16-byte loads and
-    stores (the default) or on the bulk-copy engine."""
-    if request.param == "bulk":
-        monkeypatch.setenv("MOE_PERM_BULK", "1")
-    else:
-        monkeypatch.delenv("MOE_PERM_BULK", raising=False)
-    return request.param
-
-
 @pytest.mark.parametrize("T,k,E,H,skew", [(64, 4, 16, 256, 0.0), (8192, 8, 256, 7168, 0.0),
                                           (1000, 6, 64, 2048, 0.0), (2000, 8, 256, 512, 3.0),
                                           (1, 1, 16, 256, 0.0), (3, 16, 16, 128, 0.0),
                                           (50, 2, 16, 28672, 0.0)])
-def test_permute_bit_exact(T, k, E, H, skew, perm_copy):
+def test_permute_bit_exact(T, k, E, H, skew):
     ids_np, w_np = _ids_from_oracle(T, k, E, seed=T + E, skew=skew)
     offsets_o, src_o, s2r_o = oracle.permute(ids_np, E)
     ids = torch.from_numpy(ids_np).to(DEV)
@@ -262,7 +250,7 @@ def test_permute_bit_exact(T, k, E, H, skew, perm_copy):
     assert torch.equal(xp, x[torch.from_numpy(src_o).to(DEV)])
 
 
-def test_permute_e4m3_rows_and_scales(perm_copy):
+def test_permute_e4m3_rows_and_scales():
     T, k, E, H = 300, 8, 64, 512
     ids_np, w_np = _ids_from_oracle(T, k, E, seed=9)
     _, src_o, _ = oracle.permute(ids_np, E)
@@ -282,7 +270,7 @@ def test_permute_e4m3_rows_and_scales(perm_copy):
     assert torch.equal(xps, xs[idx])
 
 
-def test_permute_flags_out_of_range_ids_without_writing_outside(perm_copy):
+def test_permute_flags_out_of_range_ids_without_writing_outside():
     T, k, E, H = 128, 4, 16, 256
     ids_np, w_np = _ids_from_oracle(T, k, E, seed=10)
     ids_np = ids_np.copy()
@@ -316,49 +304,14 @@ def _ref_grouped(a, w13, w2, off, row_w):
     rw = np32(row_w).astype(np.float64) if row_w is not None else None
     out = np.zeros((a.shape[0], w2.shape[1]))
     hs = np.zeros((a.shape[0], w2.shape[2]))
-    I = w2.shape[2]
     for g in range(len(off) - 1):
         s, e = off[g], off[g + 1]
         if e == s:
             continue
-        gu = a64[s:e] @ w13_64[g].T
-        h = gu[:, :I] / (1 + np.exp(-gu[:, :I])) * gu[:, I:]
-        hs[s:e] = h
+        hs[s:e] = oracle.swiglu_hidden(a64[s:e], w13_64[g])
         o = oracle.swiglu_ffn(a64[s:e], w13_64[g], w2_64[g])
         out[s:e] = o * (rw[s:e, None] if rw is not None else 1.0)
     return out, hs
-
-
-@pytest.fixture(params=["pair", "wide", "wide-epi8", "wide-k128", "1sm-sb", "1sm-sb-epi4", "1sm-sb-epi8", "1sm-db",
-                        "1sm-db-k64"])
-def gemm_variant(request, monkeypatch):
-    """bf16 grouped GEMMs, each kernel forced: CTA pairs (one 128-row weight
-    sub-tile per CTA, or two: "wide", where the shape allows, with stages of
-    64 K or of 128 K), or single CTAs
-    with one TMEM accumulator pair (epilogue warps per GEMM: 4 gate/up, 12
-    down; or 4 / 8 for both) or with two (stages of 128 K, or of 64 K for k64)."""
-    for var in ("MOE_GEMM_1SM", "MOE_GEMM_PAIR", "MOE_GEMM_WIDE", "MOE_WIDE_K128", "MOE_GEMM_DB", "MOE_GEMM_SB",
-                "MOE_DOWN_K64", "MOE_DOWN_DB", "MOE_EPI4", "MOE_EPI8"):
-        monkeypatch.delenv(var, raising=False)
-    v = request.param
-    if v == "pair":
-        monkeypatch.setenv("MOE_GEMM_PAIR", "1")
-    elif v.startswith("wide"):
-        monkeypatch.setenv("MOE_GEMM_WIDE", "1")
-        if v.endswith("epi8"):
-            monkeypatch.setenv("MOE_EPI8", "1")
-        if v.endswith("k128"):
-            monkeypatch.setenv("MOE_WIDE_K128", "1")
-    else:
-        monkeypatch.setenv("MOE_GEMM_1SM", "1")
-        monkeypatch.setenv("MOE_GEMM_DB" if v.startswith("1sm-db") else "MOE_GEMM_SB", "1")
-        if v.endswith("k64"):
-            monkeypatch.setenv("MOE_DOWN_K64", "1")
-        if v.endswith("epi4"):
-            monkeypatch.setenv("MOE_EPI4", "1")
-        if v.endswith("epi8"):
-            monkeypatch.setenv("MOE_EPI8", "1")
-    return v
 
 
 @pytest.mark.parametrize("H,I,sizes", [
@@ -367,8 +320,12 @@ def gemm_variant(request, monkeypatch):
     (7168, 2048, [300, 77]),
     (2048, 1408, [384, 0, 5, 513]),
     (512, 256, [1200, 2, 8]),
+    # segments of more than 8 token blocks of 256: the tile order's last,
+    # partial chunk of token blocks (5000 rows = 20 blocks = 8 + 8 + 4)
+    (512, 256, [2300, 5000, 3]),
+    (7168, 2048, [2100, 0, 17]),
 ])
-def test_grouped_swiglu_bf16(H, I, sizes, gemm_variant):
+def test_grouped_swiglu_bf16(H, I, sizes):
     G = len(sizes)
     off = _segments(sizes)
     rows = int(off[-1])
@@ -385,7 +342,7 @@ def test_grouped_swiglu_bf16(H, I, sizes, gemm_variant):
     assert N.moe_read_device_status(status) == 0
     ref, href = _ref_grouped(a, w13, w2, off, row_w)
     eh, eo = rel_err(np64(h), href), rel_err(np64(out), ref)
-    print(f"{gemm_variant} H={H} I={I}: h err {eh:.2e}, out err {eo:.2e}")
+    print(f"H={H} I={I} sizes={sizes}: h err {eh:.2e}, out err {eo:.2e}")
     assert eh < 1e-2 and eo < BF16_TOL
 
 
@@ -394,7 +351,7 @@ def test_grouped_swiglu_bf16(H, I, sizes, gemm_variant):
     (7168, 2048, 2048, [300, 77, 512, 1], 1000),
     (2048, 1408, 2816, [384, 0, 5, 513], 129),
 ])
-def test_routed_and_shared_in_one_launch(H, I, I_s, sizes, T, gemm_variant):
+def test_routed_and_shared_in_one_launch(H, I, I_s, sizes, T):
     """moe_*_with_shared: the routed segments and a shared FFN of T rows (its
     own I_s, weight 1) in one launch per GEMM. Every output tile is computed as
     in the separate launches, so the results must be bit-identical to them,
@@ -425,15 +382,15 @@ def test_routed_and_shared_in_one_launch(H, I, I_s, sizes, T, gemm_variant):
     N.moe_down_proj(T, H, sw2, N.MOE_BF16, 1, I_s, sh_h2, None, None, sh_o2)
     assert N.moe_read_device_status(status) == 0
     for got, sep, name in ((h, h2, "h"), (sh_h, sh_h2, "shared h"), (o, o2, "out"), (sh_o, sh_o2, "shared out")):
-        assert torch.equal(got, sep), f"{gemm_variant}: {name} differs from the separate launches"
+        assert torch.equal(got, sep), f"{name} differs from the separate launches"
     ref, href = _ref_grouped(xp, w13, w2, off, row_w)
     sref, shref = _ref_grouped(x, sw13, sw2, np.array([0, T], np.int32), None)
     errs = [rel_err(np64(h), href), rel_err(np64(o), ref), rel_err(np64(sh_h), shref), rel_err(np64(sh_o), sref)]
-    print(f"{gemm_variant} H={H} I={I} I_s={I_s}: errors {[f'{v:.2e}' for v in errs]}")
+    print(f"H={H} I={I} I_s={I_s}: errors {[f'{v:.2e}' for v in errs]}")
     assert errs[0] < 1e-2 and errs[2] < 1e-2 and errs[1] < BF16_TOL and errs[3] < BF16_TOL
 
 
-def test_grouped_swiglu_bf16_single_group_no_offsets(gemm_variant):
+def test_grouped_swiglu_bf16_single_group_no_offsets():
     rows, H, I = 300, 512, 384
     g = _gen(77)
     a = torch.randn(rows, H, generator=g, device=DEV).to(torch.bfloat16)
@@ -497,12 +454,9 @@ def test_combine(weighted, shared):
     sh = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16) if shared else None
     y = torch.empty(T, H, dtype=torch.bfloat16, device=DEV)
     N.moe_combine(T, k, H, eo, perm, tw, sh, y)
-    rows = perm.cpu().numpy().reshape(T, k)
-    e64 = np64(eo)
-    w64 = np32(tw).astype(np.float64) if weighted else np.ones((T, k))
-    ref = np.einsum("tj,tjh->th", w64, e64[rows])
-    if shared:
-        ref = ref + np64(sh)
+    ref = oracle.combine(np64(eo), perm.cpu().numpy(), k, np32(tw) if weighted else None,
+                         np64(sh) if shared else None)
+    # fp32 sum, one bf16 rounding: within half an ulp of bf16 (2^-8 relative)
     assert np.all(np.abs(np64(y) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)
 
 
@@ -547,8 +501,7 @@ def test_gate_up_gather_matches_permuted_copy_and_oracle():
     href = np.zeros((R, I))
     for e in range(E):
         s, t = off_np[e], off_np[e + 1]
-        gu = x64[src_np[s:t]] @ w64[e].T
-        href[s:t] = gu[:, :I] / (1 + np.exp(-gu[:, :I])) * gu[:, I:]
+        href[s:t] = oracle.swiglu_hidden(x64[src_np[s:t]], w64[e])
     assert rel_err(np64(h_gat), href) < 1e-2
 
 
@@ -566,3 +519,45 @@ def test_gate_up_gather_flags_bad_rows():
     N.moe_gate_up_swiglu_gather(T * k, H, w13, E, I, x, T, torch.from_numpy(src_np).to(DEV),
                                 torch.from_numpy(off_np.astype(np.int32)).to(DEV), h, dev_status=status)
     assert N.moe_read_device_status(status) & N.MOE_DEVSTAT_BAD_EXPERT_ID
+
+
+# -------------------------------------------------- bounded waits time out
+def test_wait_limit_runs_out_then_the_same_call_is_correct():
+    """With a wait limit of a few nanoseconds every wait of the grouped GEMM
+    that does not succeed at once gives up: the kernel sets MOE_DEVSTAT_TIMEOUT
+    in its status word (moe_read_device_status maps it to
+    MOE_ERR_DEVICE_TIMEOUT), drains its in-flight copies and MMAs, frees its
+    tensor memory and returns, without a trap. The context stays usable: the
+    same call with the default limit on the same stream matches the oracle."""
+    H, I, sizes = 512, 256, [300, 17, 0, 129]
+    G = len(sizes)
+    off = _segments(sizes)
+    rows = int(off[-1])
+    g = _gen(4242)
+    a = torch.randn(rows, H, generator=g, device=DEV).to(torch.bfloat16)
+    w13 = (torch.randn(G, 2 * I, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w2 = (torch.randn(G, H, I, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    row_w = torch.rand(rows, generator=g, device=DEV) + 0.5
+    offd = torch.from_numpy(off).to(DEV)
+    h = torch.empty(rows, I, dtype=torch.bfloat16, device=DEV)
+    out = torch.empty(rows, H, dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    assert N.moe_wait_limit_ns() == 2_000_000_000
+    N.moe_set_wait_limit_ns(5)
+    try:
+        assert N.moe_wait_limit_ns() == 5
+        N.moe_grouped_swiglu(rows, H, w13, w2, N.MOE_BF16, G, I, a, offd, row_w, h, out, dev_status=status)
+        raw = N.moe_read_device_status(status)
+    finally:
+        N.moe_set_wait_limit_ns(0)
+    assert N.moe_wait_limit_ns() == 2_000_000_000
+    assert raw == N.MOE_DEVSTAT_TIMEOUT, raw
+    code = ctypes.c_int32(0)
+    assert N.load_library().moe_read_device_status(
+        ctypes.c_void_p(status.data_ptr()), ctypes.byref(code),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == N.MOE_ERR_DEVICE_TIMEOUT
+    status.zero_()
+    N.moe_grouped_swiglu(rows, H, w13, w2, N.MOE_BF16, G, I, a, offd, row_w, h, out, dev_status=status)
+    assert N.moe_read_device_status(status) == 0
+    ref, href = _ref_grouped(a, w13, w2, off, row_w)
+    assert rel_err(np64(h), href) < 1e-2 and rel_err(np64(out), ref) < BF16_TOL

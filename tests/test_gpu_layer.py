@@ -4,6 +4,9 @@ Routing is compared id for id on every token whose k-th / (k+1)-th selection
 scores (or g-th / (g+1)-th group scores) are at least 1e-5 apart in the
 oracle; closer tokens are excluded and counted. Outputs are compared as
 max|y - y_oracle| / max|y_oracle| over the compared tokens."""
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import pytest
 import torch
@@ -43,8 +46,9 @@ def _check_permutation_properties(layer, T, k, E):
         assert np.all(np.diff(src[off[e]:off[e + 1]]) > 0)
 
 
-def _oracle_tokens(cfg, inp, toks, feats=None, fp8=False):
-    """Oracle routing + output for the given tokens (and features)."""
+def _oracle_tokens(cfg, inp, toks, feats=None, fp8=False, threads=1):
+    """Oracle routing + output for the given tokens (and features); the
+    experts are evaluated on `threads` host threads."""
     x64 = np64(inp.x[toks])
     L = oracle.gate_logits(x64, np64(inp.gate)).astype(np.float32)
     bias = np32(inp.bias) if inp.bias is not None else None
@@ -53,8 +57,70 @@ def _oracle_tokens(cfg, inp, toks, feats=None, fp8=False):
         return np32(inp.w13[e]), np32(inp.w2[e])
 
     shared = (np32(inp.sw13), np32(inp.sw2)) if inp.sw13 is not None else None
-    y = oracle.moe_forward(x64, r, ew, shared, fp8=fp8, out_features=feats)
+    if threads > 1:
+        with ThreadPoolExecutor(threads) as ex:
+            y = oracle.moe_forward(x64, r, ew, shared, fp8=fp8, out_features=feats, map_fn=ex.map)
+    else:
+        y = oracle.moe_forward(x64, r, ew, shared, fp8=fp8, out_features=feats)
     return r, y
+
+
+def _host_threads():
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 1
+    return max(1, min(16, n))
+
+
+TOKEN_BLOCK = 256      # token rows per grouped-GEMM tile (bf16)
+CHUNK_BLOCKS = 8       # token blocks per rasterisation chunk
+
+
+def coverage_tokens(layer, T, k, E, n_min=256, seed=0):
+    """Tokens whose full output rows are compared with the oracle: tokens 0
+    and T-1; one token of every expert segment that received rows (so every
+    expert's weights are exercised); the tokens of the first and last rows of
+    the longest segment; for every segment longer than 8 token blocks, the
+    tokens of the first and last rows of its last token block (the grouped
+    GEMM's last, partial chunk of token blocks); then random tokens up to
+    n_min. Chosen from the GPU's permutation, which the caller has already
+    checked for its invariants."""
+    off = layer.offsets.cpu().numpy().astype(np.int64)
+    src = layer.src_token[:T * k].cpu().numpy().astype(np.int64)
+    counts = np.diff(off)
+    rng = np.random.default_rng(seed)
+    toks = {0, T - 1}
+    for e in range(E):
+        if counts[e] > 0:
+            toks.add(int(src[off[e] + rng.integers(counts[e])]))
+    e_long = int(np.argmax(counts))
+    toks |= {int(src[off[e_long]]), int(src[off[e_long + 1] - 1])}
+    tail = 0
+    for e in np.nonzero(counts > CHUNK_BLOCKS * TOKEN_BLOCK)[0]:
+        n = int(counts[e])
+        ntb = -(-n // TOKEN_BLOCK)
+        bn = -(-(-(-n // ntb)) // 16) * 16
+        toks |= {int(src[off[e] + (ntb - 1) * bn]), int(src[off[e + 1] - 1])}
+        tail += 1
+    extra = [t for t in rng.permutation(T) if t not in toks]
+    toks |= set(int(t) for t in extra[:max(0, n_min - len(toks))])
+    return np.array(sorted(toks)), tail
+
+
+def _compare_full_rows(cfg, inp, layer, y, toks, tol, fp8=False):
+    """Every feature of the given tokens' outputs against the oracle; routing
+    ids on the same tokens; near ties excluded and counted."""
+    r, yref = _oracle_tokens(cfg, inp, toks, fp8=fp8, threads=_host_threads())
+    flagged = near_tie_mask(r)
+    ids_g = layer.ids[torch.as_tensor(toks, device=DEV)].cpu().numpy()
+    mism = routing_mismatch(ids_g, r)
+    assert not np.any(mism & ~flagged), describe_mismatch(ids_g, r, np.nonzero(mism & ~flagged)[0])
+    ok = ~flagged & ~mism
+    yg = np64(y[torch.as_tensor(toks, device=DEV)])
+    err = rel_err(yg[ok], yref[ok])
+    assert np.all(np.isfinite(yg))
+    return err, int(flagged.sum()), int(ok.sum())
 
 
 @pytest.mark.parametrize("name", ["tiny", "tiny_grouped", "v2lite"])
@@ -77,7 +143,10 @@ def test_layer_full_oracle(name):
     assert err < BF16_TOL
 
 
-def test_layer_v3_full_size_sampled():
+def test_layer_v3_full_size_every_expert_all_features():
+    """The V3 layer at its full size (T = 8192): >= 256 tokens covering every
+    expert segment, tokens 0 and T-1 and the ends of the longest segment,
+    compared with the oracle on all 7168 features."""
     cfg = get_config("v3")
     inp = make_inputs(cfg, device=DEV)
     layer = _layer(cfg, inp)
@@ -85,22 +154,13 @@ def test_layer_v3_full_size_sampled():
     torch.cuda.synchronize()
     assert layer.device_status() == 0
     _check_permutation_properties(layer, cfg.T, cfg.k, cfg.E)
-    rng = np.random.default_rng(31)
-    toks = np.sort(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 10, replace=False)]))
-    feats = np.sort(rng.choice(cfg.H, 384, replace=False))
-    r, yref = _oracle_tokens(cfg, inp, toks, feats)
-    flagged = near_tie_mask(r)
-    ids_g = layer.ids[toks].cpu().numpy()
-    mism = routing_mismatch(ids_g, r)
-    assert not np.any(mism & ~flagged), describe_mismatch(ids_g, r, np.nonzero(mism & ~flagged)[0])
-    ok = ~flagged & ~mism
-    yg = np64(y[toks][:, torch.as_tensor(feats, device=DEV)])
-    err = rel_err(yg[ok], yref[ok])
-    print(f"v3 T=8192: sampled err {err:.2e}, excluded {int(flagged.sum())}")
-    assert err < BF16_TOL
+    toks, _ = coverage_tokens(layer, cfg.T, cfg.k, cfg.E, seed=31)
+    err, excl, n = _compare_full_rows(cfg, inp, layer, y, toks, BF16_TOL)
+    print(f"v3 T=8192: {n} tokens x {cfg.H} features compared, err {err:.2e}, near ties excluded {excl}")
+    assert len(toks) >= 256 and err < BF16_TOL
 
 
-def test_layer_v3_fp8_decode():
+def test_layer_v3_fp8_decode_all_tokens_all_features():
     cfg = get_config("v3_fp8_decode")
     inp = make_inputs(cfg, device=DEV)
     layer = _layer(cfg, inp)
@@ -112,18 +172,9 @@ def test_layer_v3_fp8_decode():
     qo, so = oracle.fp8_quantize_rows(np32(inp.x))
     assert np.array_equal(layer.xq[:cfg.T].cpu().numpy(), qo)
     assert np.array_equal(layer.xs[:cfg.T].cpu().numpy(), so)
-    rng = np.random.default_rng(32)
-    toks = np.sort(rng.choice(cfg.T, 3, replace=False))
-    feats = np.sort(rng.choice(cfg.H, 256, replace=False))
-    r, yref = _oracle_tokens(cfg, inp, toks, feats, fp8=True)
-    flagged = near_tie_mask(r)
-    ids_g = layer.ids[toks].cpu().numpy()
-    mism = routing_mismatch(ids_g, r)
-    assert not np.any(mism & ~flagged), describe_mismatch(ids_g, r, np.nonzero(mism & ~flagged)[0])
-    ok = ~flagged & ~mism
-    yg = np64(y[toks][:, torch.as_tensor(feats, device=DEV)])
-    err = rel_err(yg[ok], yref[ok])
-    print(f"v3 fp8 decode: sampled err {err:.2e}")
+    toks = np.arange(cfg.T)
+    err, excl, n = _compare_full_rows(cfg, inp, layer, y, toks, FP8_TOL, fp8=True)
+    print(f"v3 fp8 decode: {n} tokens x {cfg.H} features compared, err {err:.2e}, near ties excluded {excl}")
     assert err < FP8_TOL
 
 
@@ -157,25 +208,22 @@ def test_layer_v3_skewed_bias_loop():
         assert abs(float(layer.load_cv.item()) - cvs[-1]) < 1e-6
     print("load CV per step:", " ".join(f"{c:.4f}" for c in cvs))
     print("share of experts 0-15 per step:", " ".join(f"{h:.3f}" for h in hot))
-    assert cvs[-1] < cvs[0]
-    # (b) a full forward from x at this size, sampled against the oracle
+    # the load CV drops step over step (never rises) and ends below its start
+    assert all(b <= a for a, b in zip(cvs, cvs[1:])), cvs
+    assert cvs[cfg.bias_steps] < cvs[0]
+    # (b) a full forward from x at this size with the final bias: >= 256 tokens
+    #     covering every expert segment (and the last token blocks of the hot
+    #     experts' long segments) against the oracle on all features
     y = layer.forward(inp.x)
     torch.cuda.synchronize()
     assert layer.device_status() == 0
     _check_permutation_properties(layer, T, k, E)
     inp.bias = layer.bias.clone()             # the bias the forward used
-    rng = np.random.default_rng(33)
-    toks = np.sort(rng.choice(T, 6, replace=False))
-    feats = np.sort(rng.choice(cfg.H, 256, replace=False))
-    r, yref = _oracle_tokens(cfg, inp, toks, feats)
-    flagged = near_tie_mask(r)
-    ids_g = layer.ids[toks].cpu().numpy()
-    mism = routing_mismatch(ids_g, r)
-    assert not np.any(mism & ~flagged), describe_mismatch(ids_g, r, np.nonzero(mism & ~flagged)[0])
-    ok = ~flagged & ~mism
-    err = rel_err(np64(y[toks][:, torch.as_tensor(feats, device=DEV)])[ok], yref[ok])
-    print(f"v3 skewed: sampled err {err:.2e}")
-    assert err < BF16_TOL
+    toks, tail = coverage_tokens(layer, T, k, E, seed=33)
+    err, excl, n = _compare_full_rows(cfg, inp, layer, y, toks, BF16_TOL)
+    print(f"v3 skewed: {n} tokens x {cfg.H} features compared ({tail} segments longer than 8 token "
+          f"blocks), err {err:.2e}, near ties excluded {excl}")
+    assert tail > 0 and err < BF16_TOL
 
 
 def test_layer_gather_variant_matches_default():
@@ -332,10 +380,11 @@ def test_layer_cuda_graph_replay_matches_eager(name):
         assert torch.equal(layer.bias, eager.bias)
 
 
-def test_layer_v3_largest_batch_sampled():
+def test_layer_v3_largest_batch():
     """T = 65536 tokens (524288 routed rows, 7.5 GB of permuted activations):
-    the permutation's invariants on every row and sampled outputs against
-    the oracle."""
+    the permutation's invariants on every row, and >= 256 tokens covering
+    every expert segment and the last token blocks of every segment longer
+    than 8 token blocks against the oracle on all features."""
     cfg = get_config("v3", T=65536)
     inp = make_inputs(cfg, device=DEV)
     layer = _layer(cfg, inp)
@@ -343,19 +392,11 @@ def test_layer_v3_largest_batch_sampled():
     torch.cuda.synchronize()
     assert layer.device_status() == 0
     _check_permutation_properties(layer, cfg.T, cfg.k, cfg.E)
-    rng = np.random.default_rng(65536)
-    toks = np.sort(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 4, replace=False)]))
-    feats = np.sort(rng.choice(cfg.H, 256, replace=False))
-    r, yref = _oracle_tokens(cfg, inp, toks, feats)
-    flagged = near_tie_mask(r)
-    ids_g = layer.ids[toks].cpu().numpy()
-    mism = routing_mismatch(ids_g, r)
-    assert not np.any(mism & ~flagged), describe_mismatch(ids_g, r, np.nonzero(mism & ~flagged)[0])
-    ok = ~flagged & ~mism
-    yg = np64(y[toks][:, torch.as_tensor(feats, device=DEV)])
-    err = rel_err(yg[ok], yref[ok])
-    print(f"v3 T=65536: sampled err {err:.2e}, excluded {int(flagged.sum())}")
-    assert err < BF16_TOL
+    toks, tail = coverage_tokens(layer, cfg.T, cfg.k, cfg.E, seed=65536)
+    err, excl, n = _compare_full_rows(cfg, inp, layer, y, toks, BF16_TOL)
+    print(f"v3 T=65536: {n} tokens x {cfg.H} features compared ({tail} segments longer than 8 token "
+          f"blocks), err {err:.2e}, near ties excluded {excl}")
+    assert tail > 0 and err < BF16_TOL
 
 
 @pytest.mark.parametrize("name", ["tiny", "v2lite", "v3"])
