@@ -282,7 +282,7 @@ def profiled_traffic(stage, workload):
         return None
 
 
-LAUNCHES = {"route": 2, "quantize_x": 1, "permute": 3, "gate_up_routed": 1, "down_routed": 1,
+LAUNCHES = {"route": 2, "permute": 3, "gate_up_routed": 1, "down_routed": 1,
             "gate_up_shared": 1, "down_shared": 1, "gate_up": 1, "down": 1, "combine": 1, "bias_update": 1,
             "down_combine": 2}
 
@@ -302,8 +302,10 @@ def stage_model(cfg):
     ab = 1 if cfg.dtype == "e4m3" else 2
     m = {
         "route": {"flops": 2.0 * T * H * E, "bytes": T * H * 2 + E * H * 2 + T * E * 4 + R * 8},
-        "quantize_x": {"flops": 0.0, "bytes": T * H * 2 + T * H + T * (H // 128) * 4},
-        "permute": {"flops": 0.0, "bytes": T * H * ab + R * H * ab + R * 8 + R * 12},
+        # E4M3 layers read x in bf16 and write codes + 1x128 scales (also the
+        # shared expert's unpermuted codes)
+        "permute": {"flops": 0.0, "bytes": (T * H * 2 + R * (H + H // 32) + T * (H + H // 32) + R * 20)
+                    if ab == 1 else (T * H * 2 + R * H * 2 + R * 20)},
         "gate_up_routed": {"flops": 2.0 * R * H * 2 * I, "bytes": E * 2 * I * H * ab + R * H * ab + R * I * ab},
         "down_routed": {"flops": 2.0 * R * I * H, "bytes": E * H * I * ab + R * I * ab + R * H * 2},
         "gate_up_shared": {"flops": 2.0 * T * H * 2 * Is, "bytes": 2 * Is * H * ab + T * H * ab + T * Is * ab},

@@ -51,7 +51,7 @@ extern "C" {
 #define MOE_API
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 typedef int32_t moe_status;
 #define MOE_OK                 0
@@ -156,11 +156,20 @@ MOE_API moe_status moe_gate_logits(int32_t T, int32_t H, int32_t E, const void* 
  *   slot_to_row    [T*k] int32 out, t*k + j -> row (inv_permuted_idx)
  *   row_w          [T*k] fp32 out,  topk_w[t][j] at row slot_to_row[t*k+j]
  *                  (may be NULL, then topk_w may be NULL too)
- *   x / x_perm     x_dtype MOE_BF16: x [T, H] bf16 -> x_perm [T*k, H] bf16.
- *                  x_dtype MOE_E4M3: x [T, H] e4m3 codes (moe_quantize_rows)
- *                  with x_scale [T, H/128] -> x_perm [T*k, H] codes and
- *                  x_perm_scale [T*k, H/128]. x_perm may be NULL (metadata
- *                  only).
+ *   x / x_perm     x_dtype -> perm_dtype:
+ *                  BF16 -> BF16: x [T, H] bf16 -> x_perm [T*k, H] bf16.
+ *                  BF16 -> E4M3: x [T, H] bf16 is quantised here, per 1x128
+ *                    tile along H ([FP8-infer] 1x128 activation tiles,
+ *                    dynamic; the bytes of moe_quantize_rows): x_perm
+ *                    [T*k, H] codes and x_perm_scale [T*k, H/128]; x_q /
+ *                    x_q_scale [T, H] / [T, H/128] (optional, both or
+ *                    neither) also receive the token's own codes and scales
+ *                    (the shared expert's operand). H % 128 == 0.
+ *                  E4M3 -> E4M3: x [T, H] codes with x_scale [T, H/128] ->
+ *                    x_perm [T*k, H] codes and x_perm_scale [T*k, H/128].
+ *                  E4M3 -> BF16 is MOE_ERR_UNSUPPORTED. x_q / x_q_scale are
+ *                  NULL unless quantising. x_perm may be NULL (metadata,
+ *                  and x_q if given, only).
  *   workspace      device scratch of moe_permute_workspace_size() bytes.
  * topk_ids outside [0, E) are counted nowhere and flag
  * MOE_DEVSTAT_BAD_EXPERT_ID in dev_status (outputs are then undefined).
@@ -170,7 +179,8 @@ MOE_API moe_status moe_permute_workspace_size(int32_t T, int32_t k, int32_t E, s
 MOE_API moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H,
                        const int32_t* topk_ids, const float* topk_w,
                        const void* x, moe_dtype x_dtype, const float* x_scale,
-                       void* x_perm, float* x_perm_scale,
+                       void* x_perm, moe_dtype perm_dtype, float* x_perm_scale,
+                       void* x_q, float* x_q_scale,
                        int32_t* expert_offsets, int32_t* src_token,
                        int32_t* slot_to_row, float* row_w,
                        void* workspace, size_t workspace_bytes,
@@ -185,7 +195,8 @@ MOE_API moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H,
  * and must not be taken around it, code that must not risk the implicit
  * device synchronisation a cudaMalloc can cause, and plugin interfaces that
  * hand in only input and output buffers. Arguments, outputs and errors are
- * those of moe_permute, minus `workspace` / `workspace_bytes`.
+ * those of moe_permute with perm_dtype = x_dtype and no x_q / x_q_scale,
+ * minus `workspace` / `workspace_bytes`.
  *
  * The scratch is a 1 MiB array in the library's own device memory (every GPU
  * that loads the library holds it until the process exits). It fits

@@ -184,33 +184,35 @@ moe_status moe_permute_workspace_size(int32_t T, int32_t k, int32_t E, size_t* b
 
 moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t* topk_ids,
                        const float* topk_w, const void* x, moe_dtype x_dtype, const float* x_scale,
-                       void* x_perm, float* x_perm_scale, int32_t* expert_offsets, int32_t* src_token,
-                       int32_t* slot_to_row, float* row_w, void* workspace, size_t workspace_bytes,
-                       int32_t* dev_status, void* stream) {
+                       void* x_perm, moe_dtype perm_dtype, float* x_perm_scale, void* x_q, float* x_q_scale,
+                       int32_t* expert_offsets, int32_t* src_token, int32_t* slot_to_row, float* row_w,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
   if (T < 1 || k < 1 || E < 1 || H < 1 || k > E) return MOE_ERR_INVALID_ARG;
   if (!topk_ids || !expert_offsets || !src_token || !slot_to_row || !workspace) return MOE_ERR_INVALID_ARG;
   if (row_w && !topk_w) return MOE_ERR_INVALID_ARG;
-  if (x_perm && !x) return MOE_ERR_INVALID_ARG;
+  if ((x_perm || x_q) && !x) return MOE_ERR_INVALID_ARG;
   if (x_dtype != MOE_BF16 && x_dtype != MOE_E4M3) return MOE_ERR_INVALID_ARG;
+  if (perm_dtype != MOE_BF16 && perm_dtype != MOE_E4M3) return MOE_ERR_INVALID_ARG;
+  if (x_dtype == MOE_E4M3 && perm_dtype != MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  const bool quant = x_dtype == MOE_BF16 && perm_dtype == MOE_E4M3;
+  if ((x_q || x_q_scale) && (!quant || !x_q || !x_q_scale)) return MOE_ERR_INVALID_ARG;
   if (k > 16 || E > 1024) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(T) * k > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
-  int row_bytes = 0, nscale = 0;
-  if (x_dtype == MOE_BF16) {
+  if (perm_dtype == MOE_BF16) {
     if (H % 8 != 0) return MOE_ERR_UNSUPPORTED;
-    row_bytes = 2 * H;
   } else {
     if (H % 128 != 0) return MOE_ERR_UNSUPPORTED;
-    if (x_perm && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
-    row_bytes = H;
-    nscale = H / 128;
+    if (x_perm && !x_perm_scale) return MOE_ERR_INVALID_ARG;
+    if (x_dtype == MOE_E4M3 && x_perm && !x_scale) return MOE_ERR_INVALID_ARG;
   }
   if (workspace_bytes < permute_workspace_bytes(T, E)) return MOE_ERR_INVALID_ARG;
-  if (any_misaligned(topk_ids, topk_w, x, x_scale, x_perm, x_perm_scale, expert_offsets, src_token,
-                     slot_to_row, row_w, workspace))
+  if (any_misaligned(topk_ids, topk_w, x, x_scale, x_perm, x_perm_scale, x_q, x_q_scale, expert_offsets,
+                     src_token, slot_to_row, row_w, workspace))
     return MOE_ERR_ALIGNMENT;
-  return check_launch(launch_permute(T, k, E, row_bytes, topk_ids, topk_w, x, x_dtype == MOE_E4M3 ? x_scale : nullptr,
-                                     nscale, x_perm, x_perm_scale, expert_offsets, src_token, slot_to_row,
-                                     row_w, static_cast<int32_t*>(workspace), dev_status, as_stream(stream)));
+  return check_launch(launch_permute(T, k, E, H, x_dtype == MOE_E4M3, perm_dtype == MOE_E4M3, topk_ids, topk_w, x,
+                                     x_scale, x_perm, x_perm_scale, x_q, x_q_scale, expert_offsets, src_token,
+                                     slot_to_row, row_w, static_cast<int32_t*>(workspace), dev_status,
+                                     as_stream(stream)));
 }
 
 }  // extern "C"

@@ -75,11 +75,14 @@ cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, con
                              cudaStream_t stream);
 cudaError_t launch_route_tokens(const RouteArgs& r, int num_sms, cudaStream_t stream);
 size_t permute_workspace_bytes(int T, int E);
-cudaError_t launch_permute(int T, int k, int E, int row_bytes, const int32_t* ids, const float* topk_w,
-                           const void* x, const float* x_scale, int nscale, void* x_perm,
-                           float* x_perm_scale, int32_t* offsets, int32_t* src_token,
-                           int32_t* slot_to_row, float* row_w, int32_t* blockhist, int32_t* status,
-                           cudaStream_t stream);
+// x_e4m3: x holds E4M3 codes (+ x_scale); perm_e4m3: x_perm receives codes
+// (+ x_perm_scale), quantised here when x is bf16 (x_q / x_q_scale, optional,
+// then also receive the token's own codes).
+cudaError_t launch_permute(int T, int k, int E, int H, bool x_e4m3, bool perm_e4m3, const int32_t* ids,
+                           const float* topk_w, const void* x, const float* x_scale, void* x_perm,
+                           float* x_perm_scale, void* x_q, float* x_q_scale, int32_t* offsets,
+                           int32_t* src_token, int32_t* slot_to_row, float* row_w, int32_t* blockhist,
+                           int32_t* status, cudaStream_t stream);
 cudaError_t launch_combine(int T, int k, int H, const void* eo, const int32_t* slot_to_row,
                            const float* topk_w, const void* shared, void* y, cudaStream_t stream);
 constexpr int kAuxChunk = 128;   // tokens per aux-loss partial

@@ -220,25 +220,106 @@ perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ top
   }
 }
 
+// bf16 rows quantised to E4M3 on their way to the k rows (x_perm E4M3):
+// per 1x128 tile along H, scale = amax / 448 (1 for an all-zero tile) and
+// code = RNE-saturated E4M3 of v / scale, both IEEE fp32 (the FP8 inference
+// post's 1x128 dynamic activation tiles; the same bytes as
+// moe_quantize_rows). Lane l holds 16 consecutive values of the row, 8 lanes
+// one tile, so a warp step covers 4 tiles and every store is 16 bytes. x_q /
+// x_q_scale (optional) receive the token's own codes and scales, unpermuted.
+__global__ void __launch_bounds__(256, 3)
+perm_place_quant_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T, int k, int E,
+                        const int32_t* __restrict__ blockbase, int32_t* __restrict__ slot_to_row,
+                        int32_t* __restrict__ src_token, float* __restrict__ row_w,
+                        const __nv_bfloat16* __restrict__ x, int H, uint8_t* __restrict__ x_perm,
+                        float* __restrict__ x_perm_scale, uint8_t* __restrict__ x_q,
+                        float* __restrict__ x_q_scale) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;                                  // warp-uniform
+  const int my_row = perm_rows_of_token(t, lane, ids, topk_w, T, k, E, blockbase, slot_to_row, src_token, row_w);
+  if (!x_perm && !x_q) return;                         // metadata only
+  const int ntiles = H / 128;
+  const __nv_bfloat16* src = x + static_cast<size_t>(t) * H;
+  for (int tb = 0; tb < ntiles; tb += 4) {             // same trip count on every lane
+    const int tile = tb + (lane >> 3);
+    const bool valid = tile < ntiles;                  // uniform within each 8-lane group
+    const int e0 = tile * 128 + (lane & 7) * 16;
+    float v[16];
+    if (valid) {
+      const uint4 r0 = __ldg(reinterpret_cast<const uint4*>(src + e0));
+      const uint4 r1 = __ldg(reinterpret_cast<const uint4*>(src + e0 + 8));
+      const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&r0);
+      const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&r1);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 a = __bfloat1622float2(h0[i]), b = __bfloat1622float2(h1[i]);
+        v[2 * i] = a.x;
+        v[2 * i + 1] = a.y;
+        v[8 + 2 * i] = b.x;
+        v[8 + 2 * i + 1] = b.y;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+    for (int d = 4; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+    const float sc = amax == 0.0f ? 1.0f : amax / 448.0f;
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      w[i] = static_cast<uint32_t>(to_e4m3(v[4 * i] / sc)) | (static_cast<uint32_t>(to_e4m3(v[4 * i + 1] / sc)) << 8) |
+             (static_cast<uint32_t>(to_e4m3(v[4 * i + 2] / sc)) << 16) |
+             (static_cast<uint32_t>(to_e4m3(v[4 * i + 3] / sc)) << 24);
+    const uint4 codes = make_uint4(w[0], w[1], w[2], w[3]);
+    if (x_perm) {
+#pragma unroll
+      for (int j = 0; j < kPermKMax; ++j) {
+        if (j >= k) break;                               // warp-uniform
+        const int row = __shfl_sync(0xffffffffu, my_row, j);
+        if (row >= 0 && valid) {
+          *reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(row) * H + e0) = codes;
+          if ((lane & 7) == 0) x_perm_scale[static_cast<size_t>(row) * ntiles + tile] = sc;
+        }
+      }
+    }
+    if (x_q && valid) {
+      *reinterpret_cast<uint4*>(x_q + static_cast<size_t>(t) * H + e0) = codes;
+      if ((lane & 7) == 0) x_q_scale[static_cast<size_t>(t) * ntiles + tile] = sc;
+    }
+  }
+}
+
 size_t permute_workspace_bytes(int T, int E) {
   const int nb = (T + kTokBlock - 1) / kTokBlock;
   return static_cast<size_t>(nb) * E * sizeof(int32_t);
 }
 
-cudaError_t launch_permute(int T, int k, int E, int row_bytes, const int32_t* ids, const float* topk_w,
-                           const void* x, const float* x_scale, int nscale, void* x_perm,
-                           float* x_perm_scale, int32_t* offsets, int32_t* src_token,
-                           int32_t* slot_to_row, float* row_w, int32_t* blockhist, int32_t* status,
-                           cudaStream_t stream) {
+cudaError_t launch_permute(int T, int k, int E, int H, bool x_e4m3, bool perm_e4m3, const int32_t* ids,
+                           const float* topk_w, const void* x, const float* x_scale, void* x_perm,
+                           float* x_perm_scale, void* x_q, float* x_q_scale, int32_t* offsets,
+                           int32_t* src_token, int32_t* slot_to_row, float* row_w, int32_t* blockhist,
+                           int32_t* status, cudaStream_t stream) {
   const int nb = (T + kTokBlock - 1) / kTokBlock;
   perm_hist_kernel<<<nb, 256, E * sizeof(int), stream>>>(ids, T, k, E, blockhist, status);
   const int parts = 1024 / E;
   const size_t scan_smem = (static_cast<size_t>(parts) * E + E + 32) * sizeof(int);
   perm_scan_kernel<<<1, 1024, scan_smem, stream>>>(blockhist, nb, E, T * k, offsets);
   const int warps = 8;
+  if (!x_e4m3 && perm_e4m3) {
+    perm_place_quant_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
+        ids, topk_w, T, k, E, blockhist, slot_to_row, src_token, row_w, static_cast<const __nv_bfloat16*>(x), H,
+        static_cast<uint8_t*>(x_perm), x_perm_scale, static_cast<uint8_t*>(x_q), x_q_scale);
+    return cudaGetLastError();
+  }
+  const int row_bytes = x_e4m3 ? H : 2 * H;
   perm_place_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
       ids, topk_w, T, k, E, blockhist, slot_to_row, src_token, row_w, reinterpret_cast<const uint4*>(x),
-      row_bytes / 16, reinterpret_cast<uint4*>(x_perm), x_scale, x_perm_scale, nscale);
+      row_bytes / 16, reinterpret_cast<uint4*>(x_perm), x_e4m3 ? x_scale : nullptr, x_perm_scale, H / 128);
   return cudaGetLastError();
 }
 
@@ -286,6 +367,7 @@ extern "C" moe_status moe_permute_static_ws(int32_t T, int32_t k, int32_t E, int
     }
     ws = g_static_ws_ptr[dev];
   }
-  return moe_permute(T, k, E, H, topk_ids, topk_w, x, x_dtype, x_scale, x_perm, x_perm_scale, expert_offsets,
-                     src_token, slot_to_row, row_w, ws, kStaticWsBytes, dev_status, stream);
+  return moe_permute(T, k, E, H, topk_ids, topk_w, x, x_dtype, x_scale, x_perm, x_dtype, x_perm_scale, nullptr,
+                     nullptr, expert_offsets, src_token, slot_to_row, row_w, ws, kStaticWsBytes, dev_status,
+                     stream);
 }

@@ -127,19 +127,21 @@ class MoELayer:
                     logits_in if logits_in is not None else self.logits[:T],
                     self.ids[:T], self.topk_w[:T], self.counts, self.status)
 
-    def quantize_x(self, x: torch.Tensor, T: int):
-        """E4M3 layers: x -> 1x128-tile codes + scales (once per token)."""
-        N.moe_quantize_rows(T, self.spec.H, x, self.xq[:T], self.xs[:T])
-
     def permute(self, x: torch.Tensor, T: int):
+        """The permutation; E4M3 layers quantise x per 1x128 tile inside it
+        (x_perm codes + scales, and the unpermuted codes xq / xs the shared
+        expert reads)."""
         s = self.spec
-        if self.fp8:
-            src, dt, src_s = self.xq[:T], N.MOE_E4M3, self.xs[:T]
-        else:
-            src, dt, src_s = x, N.MOE_BF16, None
         R = T * s.k
-        N.moe_permute(T, s.k, s.E, s.H, self.ids[:T], self.topk_w[:T], src, dt, src_s,
-                      None if self.gather else self.x_perm[:R], self.x_perm_s[:R] if self.fp8 else None,
+        if self.fp8:
+            N.moe_permute(T, s.k, s.E, s.H, self.ids[:T], self.topk_w[:T], x, N.MOE_BF16, None,
+                          self.x_perm[:R], self.x_perm_s[:R], self.offsets, self.src_token[:R],
+                          self.slot_to_row[:R], self.row_w[:R], self.ws, self.status,
+                          perm_dtype=N.MOE_E4M3, x_q=self.xq[:T] if self.sh_h is not None else None,
+                          x_q_scale=self.xs[:T] if self.sh_h is not None else None)
+            return
+        N.moe_permute(T, s.k, s.E, s.H, self.ids[:T], self.topk_w[:T], x, N.MOE_BF16, None,
+                      None if self.gather else self.x_perm[:R], None,
                       self.offsets, self.src_token[:R], self.slot_to_row[:R], self.row_w[:R],
                       self.ws, self.status)
 
@@ -219,10 +221,8 @@ class MoELayer:
         """The forward as named steps, each one or more libmoe launches."""
         T = x.shape[0]
         assert T <= self.T_max and x.dtype == torch.bfloat16 and x.is_contiguous()
-        st = [("route", lambda: self.route(x, write_logits))]
-        if self.fp8:
-            st.append(("quantize_x", lambda: self.quantize_x(x, T)))
-        st.append(("permute", lambda: self.permute(x, T)))
+        st = [("route", lambda: self.route(x, write_logits)),
+              ("permute", lambda: self.permute(x, T))]
         if self.fuse_combine:
             if self.sh_h is not None and not self.gather:
                 st.append(("gate_up", lambda: self.gate_up_with_shared(x, T)))

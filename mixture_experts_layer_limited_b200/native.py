@@ -75,7 +75,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_route": [ctypes.POINTER(RouteParams), _P, _P, _P, _P, _P, _P, _P, _P],
         "moe_gate_logits": [_I, _I, _I, _P, _P, _P, _P, _P],
         "moe_permute_workspace_size": [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
-        "moe_permute": [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
+        "moe_permute": [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
                         ctypes.c_size_t, _P, _P],
         "moe_permute_static_ws": [_I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P],
         "moe_grouped_swiglu": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P, _P, _P, _P],
@@ -158,12 +158,16 @@ def moe_permute_workspace_size(T, k, E) -> int:
 
 
 def moe_permute(T, k, E, H, topk_ids, topk_w, x, x_dtype, x_scale, x_perm, x_perm_scale,
-                expert_offsets, src_token, slot_to_row, row_w, workspace, dev_status=None, stream=None):
+                expert_offsets, src_token, slot_to_row, row_w, workspace, dev_status=None, stream=None,
+                perm_dtype=None, x_q=None, x_q_scale=None):
+    """perm_dtype defaults to x_dtype (a copy); MOE_E4M3 with bf16 x quantises
+    the rows per 1x128 tile on the way (x_q / x_q_scale: the token's own codes)."""
     ws_bytes = workspace.numel() * workspace.element_size()
+    pdt = x_dtype if perm_dtype is None else perm_dtype
     _check("moe_permute", load_library().moe_permute(
-        T, k, E, H, _ptr(topk_ids), _ptr(topk_w), _ptr(x), x_dtype, _ptr(x_scale), _ptr(x_perm),
-        _ptr(x_perm_scale), _ptr(expert_offsets), _ptr(src_token), _ptr(slot_to_row), _ptr(row_w),
-        _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+        T, k, E, H, _ptr(topk_ids), _ptr(topk_w), _ptr(x), x_dtype, _ptr(x_scale), _ptr(x_perm), pdt,
+        _ptr(x_perm_scale), _ptr(x_q), _ptr(x_q_scale), _ptr(expert_offsets), _ptr(src_token),
+        _ptr(slot_to_row), _ptr(row_w), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
 
 
 def moe_grouped_swiglu(rows, H, w13, w2, dtype, groups, I, a, offsets, row_w, h_ws, out,

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = N.load_library()
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
     assert lib.moe_status_string(0) == b"ok"
     assert b"invalid" in lib.moe_status_string(N.MOE_ERR_INVALID_ARG)
     assert lib.moe_status_string(99) == b"unknown status"
@@ -78,10 +78,21 @@ def test_host_validation_rejects_before_launch():
     assert lib.moe_gate_logits(8, 256, 16, fake, None, fake, None, None) == N.MOE_ERR_INVALID_ARG
     assert lib.moe_gate_logits(8, 256, 16, fake, fake, odd, None, None) == N.MOE_ERR_ALIGNMENT
     # moe_permute: missing workspace, too small workspace, unsupported E
-    args = [fake, fake, fake, N.MOE_BF16, None, fake, None, fake, fake, fake, fake]
+    args = [fake, fake, fake, N.MOE_BF16, None, fake, N.MOE_BF16, None, None, None, fake, fake, fake, fake]
     assert lib.moe_permute(64, 4, 16, 256, *args, None, 0, None, None) == N.MOE_ERR_INVALID_ARG
     assert lib.moe_permute(64, 4, 16, 256, *args, fake, 4, None, None) == N.MOE_ERR_INVALID_ARG
     assert lib.moe_permute(64, 4, 2048, 256, *args, fake, 1 << 20, None, None) == N.MOE_ERR_UNSUPPORTED
+    # perm_dtype: E4M3 codes cannot become bf16 rows; quantising needs x_perm_scale and H % 128;
+    # x_q only when quantising, and with its scales
+    def perm(x_dt, p_dt, xps, xq, xqs, H=256):
+        return lib.moe_permute(64, 4, 16, H, fake, fake, fake, x_dt, fake, fake, p_dt, xps, xq, xqs,
+                               fake, fake, fake, fake, fake, 1 << 20, None, None)
+    assert perm(N.MOE_E4M3, N.MOE_BF16, None, None, None) == N.MOE_ERR_UNSUPPORTED
+    assert perm(N.MOE_BF16, N.MOE_E4M3, None, None, None) == N.MOE_ERR_INVALID_ARG
+    assert perm(N.MOE_BF16, N.MOE_E4M3, fake, None, None, H=200) == N.MOE_ERR_UNSUPPORTED
+    assert perm(N.MOE_BF16, N.MOE_BF16, None, fake, fake) == N.MOE_ERR_INVALID_ARG
+    assert perm(N.MOE_BF16, N.MOE_E4M3, fake, fake, None) == N.MOE_ERR_INVALID_ARG
+    assert perm(N.MOE_BF16, 7, fake, None, None) == N.MOE_ERR_INVALID_ARG
     # moe_grouped_swiglu: H not a multiple of 256, offsets NULL with groups > 1
     w = N.FFNWeights(fake, fake, None, None, N.MOE_BF16, 4, 128)
     assert lib.moe_grouped_swiglu(64, 200, ctypes.byref(w), fake, None, fake, None, fake, None, fake,

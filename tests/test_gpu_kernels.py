@@ -270,6 +270,44 @@ def test_permute_e4m3_rows_and_scales():
     assert torch.equal(xps, xs[idx])
 
 
+@pytest.mark.parametrize("T,k,E,H", [(256, 8, 256, 7168), (300, 6, 64, 640), (1, 1, 16, 128)])
+def test_permute_quantises_bf16_rows_to_e4m3(T, k, E, H):
+    """perm_dtype E4M3 with bf16 x: every row of x_perm holds its token's
+    1x128-tile E4M3 codes and scales, byte for byte the oracle's
+    fp8_quantize_rows of x, and x_q / x_q_scale the token's own (H = 640:
+    five tiles, so a warp step covers a partial group of four)."""
+    ids_np, w_np = _ids_from_oracle(T, k, E, seed=T + H)
+    off_o, src_o, s2r_o = oracle.permute(ids_np, E)
+    g = _gen(T + 7)
+    x = (torch.randn(T, H, generator=g, device=DEV) * 3).to(torch.bfloat16)
+    x[0, 128:256] = 0                                  # an all-zero tile: scale 1, zero codes
+    if T > 1:
+        x[1, :128] = -x[1, :128].abs()                 # a tile of negative values only
+    R = T * k
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    src = torch.empty(R, dtype=torch.int32, device=DEV)
+    s2r = torch.empty(R, dtype=torch.int32, device=DEV)
+    roww = torch.empty(R, dtype=torch.float32, device=DEV)
+    xp = torch.empty(R, H, dtype=torch.uint8, device=DEV)
+    xps = torch.empty(R, H // 128, dtype=torch.float32, device=DEV)
+    xq = torch.empty(T, H, dtype=torch.uint8, device=DEV)
+    xqs = torch.empty(T, H // 128, dtype=torch.float32, device=DEV)
+    ws = torch.empty(N.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    N.moe_permute(T, k, E, H, torch.from_numpy(ids_np).to(DEV), torch.from_numpy(w_np).to(DEV), x, N.MOE_BF16,
+                  None, xp, xps, offsets, src, s2r, roww, ws, status, perm_dtype=N.MOE_E4M3, x_q=xq,
+                  x_q_scale=xqs)
+    assert N.moe_read_device_status(status) == 0
+    qo, so = oracle.fp8_quantize_rows(np32(x))
+    assert np.array_equal(xq.cpu().numpy(), qo)
+    assert np.array_equal(xqs.cpu().numpy(), so)
+    assert np.array_equal(xp.cpu().numpy(), qo[src_o])
+    assert np.array_equal(xps.cpu().numpy(), so[src_o])
+    assert np.array_equal(offsets.cpu().numpy(), off_o)
+    assert np.array_equal(s2r.cpu().numpy(), s2r_o)
+    assert np.array_equal(roww.cpu().numpy(), w_np.reshape(-1)[np.argsort(s2r_o)])
+
+
 def test_permute_flags_out_of_range_ids_without_writing_outside():
     T, k, E, H = 128, 4, 16, 256
     ids_np, w_np = _ids_from_oracle(T, k, E, seed=10)
