@@ -125,14 +125,15 @@ const char* moe_status_string(moe_status s) {
   }
 }
 
-// logits = x @ gate^T on the CTA-pair gate GEMM (r carries T, H, E, logits, status)
-moe_status gate_gemm(const RouteArgs& r, const void* x, const void* gate_w, cudaStream_t st) {
+// logits = x @ gate^T on the CTA-pair gate GEMM (r carries T, H, E, logits,
+// status), and with `route` the routing of every token in the same launch
+moe_status gate_gemm(const RouteArgs& r, const void* x, const void* gate_w, bool route, cudaStream_t st) {
   CUtensorMap tmX, tmG;
   moe_status s = make_tmap(&tmX, x, false, r.H, r.T, 128);
   if (s != MOE_OK) return s;
   s = make_tmap(&tmG, gate_w, false, r.H, r.E, static_cast<uint32_t>(r.E));
   if (s != MOE_OK) return s;
-  return check_launch(launch_gate_gemm(tmX, tmG, r, st));
+  return check_launch(launch_gate_gemm(tmX, tmG, r, route, st));
 }
 
 moe_status moe_gate_logits(int32_t T, int32_t H, int32_t E, const void* x, const void* gate_w, float* logits,
@@ -147,7 +148,7 @@ moe_status moe_gate_logits(int32_t T, int32_t H, int32_t E, const void* x, const
   r.logits = logits;
   r.status = dev_status;
   r.wait_ns = wait_limit();
-  return gate_gemm(r, x, gate_w, as_stream(stream));
+  return gate_gemm(r, x, gate_w, false, as_stream(stream));
 }
 
 moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_w, const float* sel_bias,
@@ -172,7 +173,12 @@ moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_
               wait_limit()};
   cudaError_t e = cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * p->E, st);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (x && (s = gate_gemm(r, x, gate_w, st)) != MOE_OK) return s;
+  // from x: one launch (projection + routing) where the shape allows
+  if (x) {
+    const bool fused = route8_experts_per_thread(r) > 0;
+    if ((s = gate_gemm(r, x, gate_w, fused, st)) != MOE_OK) return s;
+    if (fused) return MOE_OK;
+  }
   return check_launch(launch_route_tokens(r, nsm, st));
 }
 

@@ -69,21 +69,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with an explicit bound on how long the thread may be suspended
+// inside the instruction (it resumes as soon as the phase completes).
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete. Returns false when
-// the CTA aborted (another thread timed out) or this wait itself timed out.
+// the CTA aborted (another thread timed out) or this wait itself ran past
+// limit_ns. Each suspension inside try_wait is bounded by the limit (at most
+// 1 ms), so a short limit is seen even by a wait whose phase would complete
+// within the hardware's own suspension window.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int32_t* status, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t suspend = limit_ns < 1000000ull ? static_cast<uint32_t>(limit_ns) : 1000000u;
+  if (mbar_try_wait_for(bar, parity, suspend)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort_flag = 1;
-        flag_status(status, MOE_DEVSTAT_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_for(bar, parity, suspend)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      flag_status(status, MOE_DEVSTAT_TIMEOUT);
+      return false;
     }
   }
 }

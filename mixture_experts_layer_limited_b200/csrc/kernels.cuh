@@ -71,8 +71,11 @@ struct SecondProblem {
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const TokenMaps& tmB,
                                 const GemmArgs& a, int grid, cudaStream_t stream,
                                 const SecondProblem* two = nullptr);
-cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
+// route: also route the tokens in the same launch where the shape allows
+// (route8_experts_per_thread(r) > 0); counts must be zeroed beforehand.
+cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r, bool route,
                              cudaStream_t stream);
+int route8_experts_per_thread(const RouteArgs& r);
 cudaError_t launch_route_tokens(const RouteArgs& r, int num_sms, cudaStream_t stream);
 size_t permute_workspace_bytes(int T, int E);
 // x_e4m3: x holds E4M3 codes (+ x_scale); perm_e4m3: x_perm receives codes

@@ -7,19 +7,21 @@
 // top-2, topk_group = 4 kept, top-8 within, renormalise, x routed_scaling_factor);
 // the xxqk.cn digest §2.2 (bias only steers selection; device-limited routing).
 //
-// Two launches:
-//   gate_gemm_pair_kernel  logits = x . gate^T on tcgen05. A cluster of two
-//       CTAs takes 128 tokens: CTA r accumulates over half r of the hidden
-//       size in its own TMEM (M = 128 tokens, N = E, fp32), then the two swap,
-//       through distributed shared memory, the partial sums of the 64 tokens
-//       the other one writes out. Every logit is (first half) + (second half).
-//   route_tokens_g8_kernel  eight threads per token, each holding E/8
-//       consecutive experts (where E, n_group and k allow; otherwise
-//       route_tokens_kernel, one warp per token, lane l holding experts l,
-//       l+32, ...): groups are scored by the sum of their two best selection
-//       scores and ranked with shuffles, and the top-k is k rounds of an
-//       arg-max over the token's threads (larger score first, lower expert
-//       index on ties).
+// gate_route_pair_kernel computes logits = x . gate^T on tcgen05: a cluster
+// of two CTAs takes 128 tokens; CTA r accumulates over half r of the hidden
+// size in its own TMEM (M = 128 tokens, N = E, fp32), then the two swap,
+// through distributed shared memory, the partial sums of the 64 tokens the
+// other one owns. Every logit is (first half) + (second half). Where the
+// shape allows (E = 8C with C in {2, 4, 8, 16, 32}, n_group | 8, k <= 8:
+// every layer here) the same launch then routes the CTA's 64 tokens from
+// their logits in shared memory, eight threads per token, each holding E/8
+// consecutive experts: groups are scored by the sum of their two best
+// selection scores and ranked with shuffles, and the top-k is k rounds of
+// an arg-max over the token's threads (larger score first, lower expert
+// index on ties). route_tokens_g8_kernel does the same from logits in
+// global memory (routing given logits); other shapes are routed by
+// route_tokens_kernel, one warp per token, lane l holding experts l, l+32,
+// ..., in the same decision order.
 
 #include "kernels.cuh"
 
@@ -33,167 +35,6 @@ constexpr int kRouteWarps = 8;       // tokens in flight per routing CTA
 // Score -> fp32 as the library states it: sigmoid in double, rounded once.
 __device__ __forceinline__ float sigmoid_rn(float v) {
   return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(v))));
-}
-
-// ------------------------------------------------------------------------
-// Gate GEMM on CTA pairs, split along K.
-// ------------------------------------------------------------------------
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-gate_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
-                      const RouteArgs r, uint32_t tmem_cols) {
-  constexpr int KB = 64;
-  extern __shared__ __align__(1024) uint8_t dsmem[];
-  __shared__ uint64_t full_bar[kRouteStages], empty_bar[kRouteStages];
-  __shared__ uint64_t tmem_full, drain_bar;
-  __shared__ uint32_t tmem_base_s;
-  __shared__ int issued_parity[kRouteStages];
-  __shared__ volatile int abort_flag;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
-  const uint32_t a_bytes = 128u * 128u;
-  const uint32_t b_bytes = static_cast<uint32_t>(r.E) * 128u;
-  const uint32_t stage_bytes = a_bytes + b_bytes;
-  const int m0 = static_cast<int>(cluster_id_x()) * kRouteRows;
-  const int nk = r.H / KB;
-  const int nk0 = (nk + 1) / 2;
-  const int kb_begin = rank ? nk0 : 0;
-  const int kb_count = rank ? nk - nk0 : nk0;
-  float* recv = reinterpret_cast<float*>(smem);        // peer partials, after the main loop
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kRouteStages; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
-      issued_parity[i] = -1;
-    }
-    mbar_init(&tmem_full, 1);
-    mbar_init(&drain_bar, 1);
-    abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmX);
-    tma_prefetch_desc(&tmG);
-  }
-  if (warp == 1) {
-    tmem_alloc(&tmem_base_s, tmem_cols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = tmem_base_s;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      const uint64_t pol_x = policy_evict_first();
-      const uint64_t pol_g = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int i = 0; i < kb_count; ++i) {
-        const int kb = kb_begin + i;
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, r.status, r.wait_ns)) break;
-        mbar_arrive_expect_tx(&full_bar[stage], stage_bytes);
-        uint8_t* st = smem + stage * stage_bytes;
-        tma_load_2d(st, &tmX, &full_bar[stage], kb * KB, m0, pol_x);
-        tma_load_2d(st + a_bytes, &tmG, &full_bar[stage], kb * KB, 0, pol_g);
-        issued_parity[stage] = static_cast<int>(phase);
-        if (++stage == kRouteStages) { stage = 0; phase ^= 1u; }
-      }
-      if (abort_flag) {
-        for (int i = 0; i < kRouteStages; ++i)
-          if (issued_parity[i] >= 0) mbar_wait_drain(&full_bar[i], static_cast<uint32_t>(issued_parity[i]));
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = make_idesc(1u, 128u, static_cast<uint32_t>(r.E));
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int i = 0; i < kb_count; ++i) {
-        if (!mbar_wait(&full_bar[stage], phase, &abort_flag, r.status, r.wait_ns)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t a0 = smem_u32(smem + stage * stage_bytes);
-        const uint32_t b0 = a0 + a_bytes;
-#pragma unroll
-        for (int kk = 0; kk < KB / 16; ++kk)
-          umma_bf16(tmem_base, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (i | kk) != 0);
-        umma_commit(&empty_bar[stage]);
-        if (++stage == kRouteStages) { stage = 0; phase ^= 1u; }
-      }
-      if (ok && kb_count > 0) umma_commit(&tmem_full);
-      umma_commit(&drain_bar);
-      mbar_wait_drain(&drain_bar, 0);
-    }
-  } else if (kb_count > 0) {
-    mbar_wait(&tmem_full, 0, &abort_flag, r.status, r.wait_ns);   // an abort still reaches the cluster barriers
-    tc_fence_after();
-  }
-  // both CTAs: every MMA has completed (epilogue threads arrive only after
-  // tmem_full), so the operand rings are free for the exchange
-  cluster_sync();
-
-  const int q = warp & 3;
-  const int row = 32 * q + lane;                       // TMEM lane == token row of the tile
-  const bool epi = warp >= 2;
-  const bool mine = (row >> 6) == static_cast<int>(rank);   // CTA r writes rows [64r, 64r + 64)
-  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-  auto partial = [&](int c, float (&v)[32]) {
-    if (kb_count > 0) {
-      tmem_ld32(lane_addr + c * 32, v);
-      tmem_ld_wait();
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-    }
-  };
-  if (epi && !mine) {                                  // send to the CTA that writes this token
-    const uint32_t dst = mapa_shared(smem_u32(recv), rank ^ 1u) + static_cast<uint32_t>((row & 63) * r.E) * 4u;
-    for (int c = 0; c * 32 < r.E; ++c) {
-      float v[32];
-      partial(c, v);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (c * 32 + 4 * j < r.E)
-          asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (c * 32 + 4 * j) * 4u),
-                       "f"(v[4 * j]), "f"(v[4 * j + 1]), "f"(v[4 * j + 2]), "f"(v[4 * j + 3])
-                       : "memory");
-      }
-    }
-  }
-  cluster_sync();                                      // the peer's partials have landed
-
-  if (epi && mine) {
-    const int tok = m0 + row;
-    const float* peer = recv + static_cast<size_t>(row & 63) * r.E;
-    for (int c = 0; c * 32 < r.E; ++c) {
-      float v[32];
-      partial(c, v);
-      if (tok < r.T) {
-        float4* dst = reinterpret_cast<float4*>(r.logits + static_cast<size_t>(tok) * r.E + c * 32);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (c * 32 + 4 * j < r.E) {
-            float o[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float p = peer[c * 32 + 4 * j + u];
-              o[u] = rank ? p + v[4 * j + u] : v[4 * j + u] + p;      // first half + second half
-            }
-            dst[j] = make_float4(o[0], o[1], o[2], o[3]);
-          }
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
 }
 
 // ------------------------------------------------------------------------
@@ -337,20 +178,132 @@ route_tokens_kernel(const RouteArgs r) {
 // as route_tokens_kernel (same scores, same order, same sums), in about half
 // the instructions per token.
 // ------------------------------------------------------------------------
+// C consecutive scores from global or shared memory (generic loads).
 template <int C>
 __device__ __forceinline__ void load_scores(const float* src, float (&s)[C]) {
   if constexpr (C % 4 == 0) {
 #pragma unroll
     for (int i = 0; i < C / 4; ++i) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(src) + i);
+      const float4 v = reinterpret_cast<const float4*>(src)[i];
       s[4 * i] = v.x; s[4 * i + 1] = v.y; s[4 * i + 2] = v.z; s[4 * i + 3] = v.w;
     }
   } else {
 #pragma unroll
     for (int i = 0; i < C / 2; ++i) {
-      const float2 v = __ldg(reinterpret_cast<const float2*>(src) + i);
+      const float2 v = reinterpret_cast<const float2*>(src)[i];
       s[2 * i] = v.x; s[2 * i + 1] = v.y;
     }
+  }
+}
+
+// Routes token `tok` (valid: tok < T) from its E logits at L, eight
+// threads per token: lane bits 0..2 pick the thread's part (experts
+// [pC, pC + C)), lane bits 3..4 the token of the warp's four. Every lane of
+// the warp must call it (all lanes take part in every shuffle). Counts go to
+// the shared histogram `hist`.
+template <int C>
+__device__ __forceinline__ void route_token8(const RouteArgs& r, const float* __restrict__ L, int tok, bool valid,
+                                             const float* bias_s, int* hist) {
+  constexpr uint32_t kAll = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const int p = lane & 7;                            // this thread's part of its token
+  const int gl0 = lane & 24;                         // the token's first lane
+  const bool sig = r.scoring == MOE_SIGMOID;
+  const bool has_bias = r.bias != nullptr;
+  const bool raw_logit = !sig && r.G == 1 && !has_bias;   // softmax, one group: select on logits
+  const int tpg = 8 / r.G;                           // threads per group
+  const int e0 = p * C;
+  float s[C];
+  load_scores<C>(L + e0, s);
+  // softmax: max and denominator over the token's E logits
+  float lmax = 0.0f;
+  double den = 1.0;
+  if (!sig) {
+    lmax = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < C; ++i) lmax = fmaxf(lmax, s[i]);
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) lmax = fmaxf(lmax, __shfl_xor_sync(kAll, lmax, d));
+    double sum = 0.0;
+#pragma unroll
+    for (int i = 0; i < C; ++i) sum += exp(static_cast<double>(s[i]) - static_cast<double>(lmax));
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) sum += __shfl_xor_sync(kAll, sum, d);
+    den = sum;
+  }
+  // selection scores, in place
+  if (!raw_logit) {
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      const float u = sig ? sigmoid_rn(s[i])
+                          : static_cast<float>(exp(static_cast<double>(s[i]) - static_cast<double>(lmax)) / den);
+      s[i] = has_bias ? u + bias_s[e0 + i] : u;
+    }
+  }
+  if (r.G > 1) {
+    // group score = fp32 sum of the group's two largest selection scores
+    float m1 = -INFINITY, m2 = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      const float v = s[i];
+      if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
+    }
+    for (int d = 1; d < tpg; d <<= 1) {             // the two largest of both halves
+      const float o1 = __shfl_xor_sync(kAll, m1, d), o2 = __shfl_xor_sync(kAll, m2, d);
+      const float hi = fmaxf(m1, o1), lo = fminf(m1, o1);
+      m2 = fmaxf(lo, fmaxf(m2, o2));
+      m1 = hi;
+    }
+    const float gs = m1 + m2;
+    // keep the topk_group best groups (lower group index first on ties)
+    const int my_g = p / tpg;
+    int rank_g = 0;
+    for (int j = 0; j < r.G; ++j) {
+      const float o = __shfl_sync(kAll, gs, gl0 + j * tpg);
+      rank_g += (o > gs || (o == gs && j < my_g)) ? 1 : 0;
+    }
+    if (rank_g >= r.g) {
+#pragma unroll
+      for (int i = 0; i < C; ++i) s[i] = -INFINITY;
+    }
+  }
+  // top-k: k rounds of an arg-max over the token's 8 threads
+  uint32_t taken = 0;
+  int my_id = 0;
+  for (int j = 0; j < r.k; ++j) {
+    float v = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < C; ++i)
+      if (!((taken >> i) & 1u) && beats(v, be, s[i], e0 + i)) { v = s[i]; be = e0 + i; }
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) {
+      const float ov = __shfl_xor_sync(kAll, v, d);
+      const int oe = __shfl_xor_sync(kAll, be, d);
+      if (beats(v, be, ov, oe)) { v = ov; be = oe; }
+    }
+    const int rel = be - e0;
+    if (rel >= 0 && rel < C) taken |= 1u << rel;
+    if (p == j) my_id = be;
+  }
+  // weights: the unbiased score of slot p's expert, renormalised over the
+  // k slots in slot order, times the scaling factor
+  // (no expert wins a round only when no score compares, i.e. all are
+  // NaN: the slot gets id -1, flagged, and counts nowhere)
+  const bool has_id = my_id >= 0 && my_id < r.E;
+  float u = 0.0f;
+  if (p < r.k && valid && has_id) {
+    const float lv = L[my_id];
+    u = sig ? sigmoid_rn(lv) : static_cast<float>(exp(static_cast<double>(lv) - static_cast<double>(lmax)) / den);
+  }
+  float sum = 0.0f;
+  for (int j = 0; j < r.k; ++j) sum += __shfl_sync(kAll, u, gl0 + j);
+  if (p < r.k && valid) {
+    const float w = (r.norm ? u / sum : u) * r.scale;
+    r.ids[static_cast<size_t>(tok) * r.k + p] = has_id ? my_id : -1;
+    r.w[static_cast<size_t>(tok) * r.k + p] = has_id ? w : 0.0f;
+    if (has_id) atomicAdd(&hist[my_id], 1);
+    else flag_status(r.status, MOE_DEVSTAT_BAD_EXPERT_ID);
   }
 }
 
@@ -364,113 +317,13 @@ route_tokens_g8_kernel(const RouteArgs r) {
     bias_s[e] = r.bias ? r.bias[e] : 0.0f;
   }
   __syncthreads();
-  constexpr uint32_t kAll = 0xffffffffu;
   const int lane = threadIdx.x & 31;
-  const int p = lane & 7;                            // this thread's part of its token
-  const int gl0 = lane & 24;                         // the token's first lane
-  const bool sig = r.scoring == MOE_SIGMOID;
-  const bool has_bias = r.bias != nullptr;
-  const bool raw_logit = !sig && r.G == 1 && !has_bias;   // softmax, one group: select on logits
-  const int tpg = 8 / r.G;                           // threads per group
-  const int e0 = p * C;
   const int nwarps = gridDim.x * (blockDim.x >> 5);
   // a warp routes four tokens per pass; every lane takes part in every shuffle
   for (int wq = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wq * 4 < r.T; wq += nwarps) {
     const int tok = wq * 4 + (lane >> 3);
     const bool valid = tok < r.T;
-    const float* L = r.logits + static_cast<size_t>(valid ? tok : 0) * r.E;
-    float s[C];
-    load_scores<C>(L + e0, s);
-    // softmax: max and denominator over the token's E logits
-    float lmax = 0.0f;
-    double den = 1.0;
-    if (!sig) {
-      lmax = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < C; ++i) lmax = fmaxf(lmax, s[i]);
-#pragma unroll
-      for (int d = 1; d < 8; d <<= 1) lmax = fmaxf(lmax, __shfl_xor_sync(kAll, lmax, d));
-      double sum = 0.0;
-#pragma unroll
-      for (int i = 0; i < C; ++i) sum += exp(static_cast<double>(s[i]) - static_cast<double>(lmax));
-#pragma unroll
-      for (int d = 1; d < 8; d <<= 1) sum += __shfl_xor_sync(kAll, sum, d);
-      den = sum;
-    }
-    // selection scores, in place
-    if (!raw_logit) {
-#pragma unroll
-      for (int i = 0; i < C; ++i) {
-        const float u = sig ? sigmoid_rn(s[i])
-                            : static_cast<float>(exp(static_cast<double>(s[i]) - static_cast<double>(lmax)) / den);
-        s[i] = has_bias ? u + bias_s[e0 + i] : u;
-      }
-    }
-    if (r.G > 1) {
-      // group score = fp32 sum of the group's two largest selection scores
-      float m1 = -INFINITY, m2 = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < C; ++i) {
-        const float v = s[i];
-        if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
-      }
-      for (int d = 1; d < tpg; d <<= 1) {             // the two largest of both halves
-        const float o1 = __shfl_xor_sync(kAll, m1, d), o2 = __shfl_xor_sync(kAll, m2, d);
-        const float hi = fmaxf(m1, o1), lo = fminf(m1, o1);
-        m2 = fmaxf(lo, fmaxf(m2, o2));
-        m1 = hi;
-      }
-      const float gs = m1 + m2;
-      // keep the topk_group best groups (lower group index first on ties)
-      const int my_g = p / tpg;
-      int rank_g = 0;
-      for (int j = 0; j < r.G; ++j) {
-        const float o = __shfl_sync(kAll, gs, gl0 + j * tpg);
-        rank_g += (o > gs || (o == gs && j < my_g)) ? 1 : 0;
-      }
-      if (rank_g >= r.g) {
-#pragma unroll
-        for (int i = 0; i < C; ++i) s[i] = -INFINITY;
-      }
-    }
-    // top-k: k rounds of an arg-max over the token's 8 threads
-    uint32_t taken = 0;
-    int my_id = 0;
-    for (int j = 0; j < r.k; ++j) {
-      float v = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < C; ++i)
-        if (!((taken >> i) & 1u) && beats(v, be, s[i], e0 + i)) { v = s[i]; be = e0 + i; }
-#pragma unroll
-      for (int d = 1; d < 8; d <<= 1) {
-        const float ov = __shfl_xor_sync(kAll, v, d);
-        const int oe = __shfl_xor_sync(kAll, be, d);
-        if (beats(v, be, ov, oe)) { v = ov; be = oe; }
-      }
-      const int rel = be - e0;
-      if (rel >= 0 && rel < C) taken |= 1u << rel;
-      if (p == j) my_id = be;
-    }
-    // weights: the unbiased score of slot p's expert, renormalised over the
-    // k slots in slot order, times the scaling factor
-    // (no expert wins a round only when no score compares, i.e. all are
-    // NaN: the slot gets id -1, flagged, and counts nowhere)
-    const bool has_id = my_id >= 0 && my_id < r.E;
-    float u = 0.0f;
-    if (p < r.k && valid && has_id) {
-      const float lv = L[my_id];
-      u = sig ? sigmoid_rn(lv) : static_cast<float>(exp(static_cast<double>(lv) - static_cast<double>(lmax)) / den);
-    }
-    float sum = 0.0f;
-    for (int j = 0; j < r.k; ++j) sum += __shfl_sync(kAll, u, gl0 + j);
-    if (p < r.k && valid) {
-      const float w = (r.norm ? u / sum : u) * r.scale;
-      r.ids[static_cast<size_t>(tok) * r.k + p] = has_id ? my_id : -1;
-      r.w[static_cast<size_t>(tok) * r.k + p] = has_id ? w : 0.0f;
-      if (has_id) atomicAdd(&hist[my_id], 1);
-      else flag_status(r.status, MOE_DEVSTAT_BAD_EXPERT_ID);
-    }
+    route_token8<C>(r, r.logits + static_cast<size_t>(valid ? tok : 0) * r.E, tok, valid, bias_s, hist);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < r.E; e += blockDim.x)
@@ -478,25 +331,241 @@ route_tokens_g8_kernel(const RouteArgs r) {
 }
 
 // ------------------------------------------------------------------------
-cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
+// Gate GEMM on CTA pairs, split along K, and (C > 0) the routing of the
+// tile's tokens in the same launch.
+// ------------------------------------------------------------------------
+// 256 threads: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer,
+// warps 2..5 read the accumulator (warp w: TMEM lanes 32*(w%4)..+31); after
+// the exchange every warp routes. The CTAs of a pair start their K loop at
+// a rotation that differs from pair to pair, so the pairs running side by
+// side do not all read the same gate rows at the same moment (each pair
+// still sums its K blocks in one fixed order).
+constexpr int kGateThreads = 256;
+
+template <int C>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGateThreads, 1)
+gate_route_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
+                       const RouteArgs r, uint32_t tmem_cols) {
+  constexpr int KB = 64;
+  extern __shared__ __align__(1024) uint8_t dsmem[];
+  __shared__ uint64_t full_bar[kRouteStages], empty_bar[kRouteStages];
+  __shared__ uint64_t tmem_full, drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int issued_parity[kRouteStages];
+  __shared__ volatile int abort_flag;
+  __shared__ int hist[C > 0 ? 256 : 1];
+  __shared__ float bias_s[C > 0 ? 256 : 1];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  const uint32_t a_bytes = 128u * 128u;
+  const uint32_t b_bytes = static_cast<uint32_t>(r.E) * 128u;
+  const uint32_t stage_bytes = a_bytes + b_bytes;
+  const int m0 = static_cast<int>(cluster_id_x()) * kRouteRows;
+  const int nk = r.H / KB;
+  const int nk0 = (nk + 1) / 2;
+  const int kb_begin = rank ? nk0 : 0;
+  const int kb_count = rank ? nk - nk0 : nk0;
+  float* recv = reinterpret_cast<float*>(smem);        // peer partials, after the main loop
+  const int rot = kb_count > 0 ? static_cast<int>((cluster_id_x() * 7u) % static_cast<uint32_t>(kb_count)) : 0;
+
+  if constexpr (C > 0) {
+    for (int e = threadIdx.x; e < r.E; e += blockDim.x) {
+      hist[e] = 0;
+      bias_s[e] = r.bias ? r.bias[e] : 0.0f;
+    }
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRouteStages; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+      issued_parity[i] = -1;
+    }
+    mbar_init(&tmem_full, 1);
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmG);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_x = policy_evict_first();
+      const uint64_t pol_g = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int i = 0; i < kb_count; ++i) {
+        const int kb = kb_begin + (i + rot < kb_count ? i + rot : i + rot - kb_count);
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, r.status, r.wait_ns)) break;
+        mbar_arrive_expect_tx(&full_bar[stage], stage_bytes);
+        uint8_t* st = smem + stage * stage_bytes;
+        tma_load_2d(st, &tmX, &full_bar[stage], kb * KB, m0, pol_x);
+        tma_load_2d(st + a_bytes, &tmG, &full_bar[stage], kb * KB, 0, pol_g);
+        issued_parity[stage] = static_cast<int>(phase);
+        if (++stage == kRouteStages) { stage = 0; phase ^= 1u; }
+      }
+      if (abort_flag) {
+        for (int i = 0; i < kRouteStages; ++i)
+          if (issued_parity[i] >= 0) mbar_wait_drain(&full_bar[i], static_cast<uint32_t>(issued_parity[i]));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(1u, 128u, static_cast<uint32_t>(r.E));
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; i < kb_count; ++i) {
+        if (!mbar_wait(&full_bar[stage], phase, &abort_flag, r.status, r.wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(smem + stage * stage_bytes);
+        const uint32_t b0 = a0 + a_bytes;
+#pragma unroll
+        for (int kk = 0; kk < KB / 16; ++kk)
+          umma_bf16(tmem_base, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (i | kk) != 0);
+        umma_commit(&empty_bar[stage]);
+        if (++stage == kRouteStages) { stage = 0; phase ^= 1u; }
+      }
+      if (ok && kb_count > 0) umma_commit(&tmem_full);
+      umma_commit(&drain_bar);
+      mbar_wait_drain(&drain_bar, 0);
+    }
+  } else if (kb_count > 0) {
+    mbar_wait(&tmem_full, 0, &abort_flag, r.status, r.wait_ns);   // an abort still reaches the cluster barriers
+    tc_fence_after();
+  }
+  // both CTAs: every MMA has completed (epilogue threads arrive only after
+  // tmem_full), so the operand rings are free for the exchange
+  cluster_sync();
+
+  const int q = warp & 3;
+  const int row = 32 * q + lane;                       // TMEM lane == token row of the tile
+  const bool epi = warp >= 2 && warp < 6;
+  const bool mine = (row >> 6) == static_cast<int>(rank);   // CTA r writes rows [64r, 64r + 64)
+  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+  auto partial = [&](int c, float (&v)[32]) {
+    if (kb_count > 0) {
+      tmem_ld32(lane_addr + c * 32, v);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+    }
+  };
+  if (epi && !mine) {                                  // send to the CTA that writes this token
+    const uint32_t dst = mapa_shared(smem_u32(recv), rank ^ 1u) + static_cast<uint32_t>((row & 63) * r.E) * 4u;
+    for (int c = 0; c * 32 < r.E; ++c) {
+      float v[32];
+      partial(c, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (c * 32 + 4 * j < r.E)
+          asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (c * 32 + 4 * j) * 4u),
+                       "f"(v[4 * j]), "f"(v[4 * j + 1]), "f"(v[4 * j + 2]), "f"(v[4 * j + 3])
+                       : "memory");
+      }
+    }
+  }
+  cluster_sync();                                      // the peer's partials have landed
+
+  if (epi && mine) {
+    const int tok = m0 + row;
+    float* peer = recv + static_cast<size_t>(row & 63) * r.E;   // becomes this token's full logits
+    for (int c = 0; c * 32 < r.E; ++c) {
+      float v[32];
+      partial(c, v);
+      if (tok < r.T) {
+        float4* dst = reinterpret_cast<float4*>(r.logits + static_cast<size_t>(tok) * r.E + c * 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (c * 32 + 4 * j < r.E) {
+            float o[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float p = peer[c * 32 + 4 * j + u];
+              o[u] = rank ? p + v[4 * j + u] : v[4 * j + u] + p;      // first half + second half
+            }
+            dst[j] = make_float4(o[0], o[1], o[2], o[3]);
+            if constexpr (C > 0) reinterpret_cast<float4*>(peer + c * 32)[j] = make_float4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+    }
+  }
+  if constexpr (C > 0) {
+    // route this CTA's 64 tokens from their logits in shared memory: each
+    // warp four tokens a pass (eight threads per token), 32 tokens a pass
+    __syncthreads();
+    const int tok_base = m0 + 64 * static_cast<int>(rank);
+    for (int pass = 0; pass < 64; pass += 4 * (kGateThreads / 32)) {
+      const int i = pass + 4 * warp + (lane >> 3);
+      const int tok = tok_base + i;
+      const bool valid = i < 64 && tok < r.T;
+      route_token8<C>(r, recv + static_cast<size_t>(valid ? i : 0) * r.E, tok, valid, bias_s, hist);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < r.E; e += blockDim.x)
+      if (hist[e]) atomicAdd(r.counts + e, hist[e]);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
+}
+
+// ------------------------------------------------------------------------
+int route8_experts_per_thread(const RouteArgs& r) {
+  const int C = r.E / 8;
+  const bool ok = r.E % 8 == 0 && r.k <= 8 && r.G >= 1 && 8 % r.G == 0 &&
+                  (C == 2 || C == 4 || C == 8 || C == 16 || C == 32);
+  return ok ? C : 0;
+}
+
+template <int C>
+cudaError_t launch_gate_route(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r, size_t smem,
+                              uint32_t cols, int grid, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(gate_route_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  gate_route_pair_kernel<C><<<grid, kGateThreads, smem, stream>>>(tmX, tmG, r, cols);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r, bool route,
                              cudaStream_t stream) {
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(r.E)) cols <<= 1;
   const size_t ring = static_cast<size_t>(kRouteStages) * (128 * 128 + static_cast<size_t>(r.E) * 128);
   const size_t recv = static_cast<size_t>(64) * r.E * sizeof(float);
   const size_t smem = (ring > recv ? ring : recv) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(gate_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  const int tiles = (r.T + kRouteRows - 1) / kRouteRows;
-  gate_gemm_pair_kernel<<<2 * tiles, 192, smem, stream>>>(tmX, tmG, r, cols);
-  return cudaGetLastError();
+  const int grid = 2 * ((r.T + kRouteRows - 1) / kRouteRows);
+  switch (route ? route8_experts_per_thread(r) : 0) {
+    case 2: return launch_gate_route<2>(tmX, tmG, r, smem, cols, grid, stream);
+    case 4: return launch_gate_route<4>(tmX, tmG, r, smem, cols, grid, stream);
+    case 8: return launch_gate_route<8>(tmX, tmG, r, smem, cols, grid, stream);
+    case 16: return launch_gate_route<16>(tmX, tmG, r, smem, cols, grid, stream);
+    case 32: return launch_gate_route<32>(tmX, tmG, r, smem, cols, grid, stream);
+    default: return launch_gate_route<0>(tmX, tmG, r, smem, cols, grid, stream);
+  }
 }
 
 cudaError_t launch_route_tokens(const RouteArgs& r, int num_sms, cudaStream_t stream) {
   // eight threads per token where the shape allows, else one warp per token
-  const int C = r.E / 8;
-  if (r.E % 8 == 0 && r.k <= 8 && 8 % r.G == 0 && (C == 2 || C == 4 || C == 8 || C == 16 || C == 32)) {
+  const int C = route8_experts_per_thread(r);
+  if (C > 0) {
     const int need = (r.T + 31) / 32;                 // 32 tokens per CTA of 256 threads
     const int grid = need < 4 * num_sms ? need : 4 * num_sms;
     switch (C) {
