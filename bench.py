@@ -282,7 +282,7 @@ def profiled_traffic(stage, workload):
         return None
 
 
-LAUNCHES = {"route": 2, "permute": 3, "gate_up_routed": 1, "down_routed": 1,
+LAUNCHES = {"route": 1, "permute": 3, "gate_up_routed": 1, "down_routed": 1,
             "gate_up_shared": 1, "down_shared": 1, "gate_up": 1, "down": 1, "combine": 1, "bias_update": 1,
             "down_combine": 2}
 

@@ -88,6 +88,65 @@ def test_route_from_logits_bit_exact(name, T):
     np.testing.assert_allclose(w.cpu().numpy(), r.weights, rtol=5e-6, atol=1e-7)
 
 
+def _near_tie_logits(T, E, G, gaps, rng):
+    """Sigmoid-scored logits (no bias) where token t's 8th and 9th best
+    experts, or its 4th and 5th best groups, are a chosen distance apart.
+    Groups of E/G experts; every token has two strong experts in each of
+    four groups (0, 2, 4, 6), then the tie is placed either between two
+    experts of group 0 (the k-th / (k+1)-th boundary) or between groups 1
+    and 3 (the kept / dropped group boundary)."""
+    gsz = E // G
+    L = np.full((T, E), -6.0, dtype=np.float32) + rng.uniform(0, 0.01, (T, E)).astype(np.float32)
+    sig = lambda v: 1.0 / (1.0 + np.exp(-np.float64(v)))
+    for t in range(T):
+        gap = gaps[t % len(gaps)]
+        for gi, g in enumerate((0, 2, 4, 6)):
+            L[t, g * gsz + 3] = 4.0 - gi * 0.25
+            L[t, g * gsz + 5] = 3.9 - gi * 0.25
+        if (t // len(gaps)) % 2 == 0:
+            # experts: seven clear winners in groups 0, 2, 4, 6 (two each but
+            # group 6's second is weak), then the 8th / 9th pair in group 0
+            L[t, 6 * gsz + 5] = -1.0
+            a = np.float32(1.0)
+            L[t, 0 * gsz + 7] = a
+            # find b with sigmoid(a) - sigmoid(b) ~ gap in fp32 (the scores the oracle compares)
+            target = np.float32(sig(a)) - np.float32(gap)
+            b = np.float32(np.log(target / (1 - target)))
+            L[t, 0 * gsz + 9] = b
+        else:
+            # groups: groups 1 and 3 compete for the 4th place, their top-2
+            # sums a chosen distance apart; groups 2, 4, 6 strong, 0 weak
+            L[t, 0 * gsz + 3] = -2.0
+            L[t, 0 * gsz + 5] = -2.0
+            L[t, 1 * gsz + 1] = 0.5
+            L[t, 1 * gsz + 2] = 0.5
+            s1 = np.float32(np.float32(sig(0.5)) + np.float32(sig(0.5)))
+            target = np.float32(s1 - np.float32(gap)) - np.float32(sig(0.5))
+            L[t, 3 * gsz + 1] = 0.5
+            L[t, 3 * gsz + 2] = np.float32(np.log(target / (1 - target)))
+    return L
+
+
+def test_route_sigmoid_decisions_at_tiny_score_gaps_bit_exact():
+    """Tokens whose k-th / (k+1)-th selection scores, or whose last kept and
+    first dropped group scores, differ by 0 to 1e-4 (fp32 distances of a few
+    ulp and up): routed on identical fp32 logits, ids, counts and weights
+    must be the oracle's, bit for bit where the decision is taken."""
+    cfg = dataclasses.replace(get_config("v3"), n_group=8, topk_group=4, k=8)
+    rng = np.random.default_rng(77)
+    gaps = [0.0, 1e-7, 5e-7, 1e-6, 2e-6, 3e-6, 4e-6, 5e-6, 7e-6, 8e-6, 9e-6, 1.2e-5, 3e-5, 1e-4]
+    T = 28 * 20
+    L = _near_tie_logits(T, cfg.E, cfg.n_group, gaps, rng)
+    Ld = torch.from_numpy(L).to(DEV)
+    for bias in (None, uniform_bias(cfg.E, 91) * 0.0):
+        ids, w, counts, _ = gpu_route(cfg, T, bias=bias, logits=Ld)
+        torch.cuda.synchronize()
+        r = oracle_route(L, cfg, np32(bias) if bias is not None else None)
+        assert np.array_equal(ids.cpu().numpy(), r.ids)
+        assert np.array_equal(counts.cpu().numpy(), r.counts)
+        np.testing.assert_allclose(w.cpu().numpy(), r.weights, rtol=5e-6, atol=1e-7)
+
+
 @pytest.mark.parametrize("topk_group", [1, 2, 4, 8])
 def test_route_topk_group_sweep_bit_exact_with_load_cv(topk_group):
     """The group-limit sweep at the V3 shape (8 groups): ids and counts
