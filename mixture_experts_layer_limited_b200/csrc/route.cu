@@ -334,13 +334,13 @@ route_tokens_g8_kernel(const RouteArgs r) {
 // Gate GEMM on CTA pairs, split along K, and (C > 0) the routing of the
 // tile's tokens in the same launch.
 // ------------------------------------------------------------------------
-// 256 threads: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer,
+// 512 threads: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer,
 // warps 2..5 read the accumulator (warp w: TMEM lanes 32*(w%4)..+31); after
-// the exchange every warp routes. The CTAs of a pair start their K loop at
+// the exchange all sixteen warps route, the CTA's 64 tokens in one pass. The CTAs of a pair start their K loop at
 // a rotation that differs from pair to pair, so the pairs running side by
 // side do not all read the same gate rows at the same moment (each pair
 // still sums its K blocks in one fixed order).
-constexpr int kGateThreads = 256;
+constexpr int kGateThreads = 512;
 
 template <int C>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGateThreads, 1)
@@ -506,7 +506,7 @@ gate_route_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
   }
   if constexpr (C > 0) {
     // route this CTA's 64 tokens from their logits in shared memory: each
-    // warp four tokens a pass (eight threads per token), 32 tokens a pass
+    // warp four tokens (eight threads per token)
     __syncthreads();
     const int tok_base = m0 + 64 * static_cast<int>(rank);
     for (int pass = 0; pass < 64; pass += 4 * (kGateThreads / 32)) {
