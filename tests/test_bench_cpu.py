@@ -55,3 +55,33 @@ def test_every_layer_stage_has_a_launch_count_and_a_cost_model():
             for n in names:
                 assert n in bench.LAUNCHES and n in model, (name, kw, n)
                 assert bench.launches_of(n, cfg) >= 1
+
+
+def test_cpu_sample_holds_every_token_of_the_hottest_and_coldest_expert():
+    """The CPU baseline's sample: at least n_min tokens, every token of the
+    expert with the most rows and of the one with the fewest (non-empty)
+    rows, no token twice."""
+    sys.path.insert(0, ROOT)
+    import types
+    import numpy as np
+    import torch
+    import bench
+    import oracle
+    from moe_inputs import get_config
+    rng = np.random.default_rng(5)
+    T, k, E = 4096, 8, 64
+    L = rng.standard_normal((T, E)).astype(np.float32)
+    L[:, 3] += 2.0                                   # a hot expert
+    L[:, 17] -= 3.0                                  # a cold one
+    ids = oracle.route_from_logits(L, k, 1, 1, "softmax", False, 1.0).ids
+    off, src, _ = oracle.permute(ids, E)
+    layer = types.SimpleNamespace(offsets=torch.from_numpy(off.astype(np.int32)),
+                                  src_token=torch.from_numpy(src.astype(np.int32)))
+    cfg = types.SimpleNamespace(T=T, k=k)
+    toks, hot, n_hot, cold, n_cold = bench.cpu_sample_tokens(layer, cfg, 1024)
+    counts = np.diff(off)
+    assert hot == int(np.argmax(counts)) and n_hot == counts.max()
+    assert cold == int(np.argmin(np.where(counts > 0, counts, 10 ** 9))) and n_cold > 0
+    assert len(toks) >= 1024 and len(set(toks.tolist())) == len(toks)
+    for e in (hot, cold):
+        assert set(src[off[e]:off[e + 1]].tolist()) <= set(toks.tolist())
