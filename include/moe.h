@@ -106,9 +106,15 @@ typedef int32_t moe_scoring;
  *                 x == NULL.
  *   topk_ids      [T, k] int32 out;  topk_w [T, k] fp32 out.
  *   expert_counts [E] int32 out.
- * Work: with x, a tcgen05 gate GEMM on CTA pairs (each CTA of a pair sums
- * half the hidden size; every logit is first half + second half); then one
- * warp routes each token.
+ * Work: with x, a tcgen05 gate GEMM on clusters of 2, 4 or 8 CTAs per 128
+ * tokens (each CTA sums one slice of the hidden size; every logit is the
+ * slices' partial sums added in order; the split depends on T and the SM
+ * count only, so moe_gate_logits gives the same logits) and, in the same
+ * launch where the shape allows (E = 8C, C in {2,4,8,16,32}, n_group | 8,
+ * k <= 8), the routing of every token, eight threads per token. With
+ * x == NULL, or from x for other shapes, the routing is its own launch
+ * (eight threads per token where the shape allows, else one warp per token;
+ * the same decisions either way).
  * Limits: 1 <= k <= 16, E % 16 == 0, 16 <= E <= 256, E % n_group == 0,
  *   n_group <= 32, topk_group <= n_group, k <= topk_group * E / n_group,
  *   H % 64 == 0 when x != NULL. Otherwise MOE_ERR_INVALID_ARG/UNSUPPORTED.

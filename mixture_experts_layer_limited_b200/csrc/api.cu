@@ -125,15 +125,15 @@ const char* moe_status_string(moe_status s) {
   }
 }
 
-// logits = x @ gate^T on the CTA-pair gate GEMM (r carries T, H, E, logits,
+// logits = x @ gate^T on the clustered gate GEMM (r carries T, H, E, logits,
 // status), and with `route` the routing of every token in the same launch
-moe_status gate_gemm(const RouteArgs& r, const void* x, const void* gate_w, bool route, cudaStream_t st) {
+moe_status gate_gemm(const RouteArgs& r, const void* x, const void* gate_w, bool route, int nsm, cudaStream_t st) {
   CUtensorMap tmX, tmG;
   moe_status s = make_tmap(&tmX, x, false, r.H, r.T, 128);
   if (s != MOE_OK) return s;
   s = make_tmap(&tmG, gate_w, false, r.H, r.E, static_cast<uint32_t>(r.E));
   if (s != MOE_OK) return s;
-  return check_launch(launch_gate_gemm(tmX, tmG, r, route, st));
+  return check_launch(launch_gate_gemm(tmX, tmG, r, route, nsm, st));
 }
 
 moe_status moe_gate_logits(int32_t T, int32_t H, int32_t E, const void* x, const void* gate_w, float* logits,
@@ -141,6 +141,9 @@ moe_status moe_gate_logits(int32_t T, int32_t H, int32_t E, const void* x, const
   if (T < 1 || H < 64 || !x || !gate_w || !logits) return MOE_ERR_INVALID_ARG;
   if (H % 64 != 0 || E > 256 || E < 16 || E % 16 != 0) return MOE_ERR_UNSUPPORTED;
   if (any_misaligned(x, gate_w, logits)) return MOE_ERR_ALIGNMENT;
+  int nsm = 0;
+  moe_status s = sm_count(&nsm);
+  if (s != MOE_OK) return s;
   RouteArgs r{};
   r.T = T;
   r.H = H;
@@ -148,7 +151,7 @@ moe_status moe_gate_logits(int32_t T, int32_t H, int32_t E, const void* x, const
   r.logits = logits;
   r.status = dev_status;
   r.wait_ns = wait_limit();
-  return gate_gemm(r, x, gate_w, false, as_stream(stream));
+  return gate_gemm(r, x, gate_w, false, nsm, as_stream(stream));
 }
 
 moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_w, const float* sel_bias,
@@ -176,7 +179,7 @@ moe_status moe_route(const moe_route_params* p, const void* x, const void* gate_
   // from x: one launch (projection + routing) where the shape allows
   if (x) {
     const bool fused = route8_experts_per_thread(r) > 0;
-    if ((s = gate_gemm(r, x, gate_w, fused, st)) != MOE_OK) return s;
+    if ((s = gate_gemm(r, x, gate_w, fused, nsm, st)) != MOE_OK) return s;
     if (fused) return MOE_OK;
   }
   return check_launch(launch_route_tokens(r, nsm, st));

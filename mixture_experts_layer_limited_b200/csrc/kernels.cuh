@@ -72,9 +72,11 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
                                 const GemmArgs& a, int grid, cudaStream_t stream,
                                 const SecondProblem* two = nullptr);
 // route: also route the tokens in the same launch where the shape allows
-// (route8_experts_per_thread(r) > 0); counts must be zeroed beforehand.
+// (route8_experts_per_thread(r) > 0); counts must be zeroed beforehand. The
+// split of the hidden size over a cluster's CTAs depends on T and num_sms only,
+// so the logits of a given T are the same with and without routing.
 cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r, bool route,
-                             cudaStream_t stream);
+                             int num_sms, cudaStream_t stream);
 int route8_experts_per_thread(const RouteArgs& r);
 cudaError_t launch_route_tokens(const RouteArgs& r, int num_sms, cudaStream_t stream);
 size_t permute_workspace_bytes(int T, int E);

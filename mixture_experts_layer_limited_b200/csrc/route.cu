@@ -7,13 +7,15 @@
 // top-2, topk_group = 4 kept, top-8 within, renormalise, x routed_scaling_factor);
 // the xxqk.cn digest §2.2 (bias only steers selection; device-limited routing).
 //
-// gate_route_pair_kernel computes logits = x . gate^T on tcgen05: a cluster
-// of two CTAs takes 128 tokens; CTA r accumulates over half r of the hidden
-// size in its own TMEM (M = 128 tokens, N = E, fp32), then the two swap,
-// through distributed shared memory, the partial sums of the 64 tokens the
-// other one owns. Every logit is (first half) + (second half). Where the
-// shape allows (E = 8C with C in {2, 4, 8, 16, 32}, n_group | 8, k <= 8:
-// every layer here) the same launch then routes the CTA's 64 tokens from
+// gate_route_kernel computes logits = x . gate^T on tcgen05: a cluster of
+// SPLIT CTAs (2, 4 or 8; the most that still keeps every CTA of the grid
+// resident at once) takes 128 tokens; CTA r accumulates over the r-th of SPLIT
+// slices of the hidden size in its own TMEM (M = 128 tokens, N = E, fp32),
+// then each CTA sends, through distributed shared memory, its partial sums of
+// the 128/SPLIT tokens every other CTA owns. Every logit is the sum of the
+// SPLIT partials in slice order. Where the shape allows (E = 8C with C in
+// {2, 4, 8, 16, 32}, n_group | 8, k <= 8: every layer here) the same launch
+// then routes the CTA's 128/SPLIT tokens from
 // their logits in shared memory, eight threads per token, each holding E/8
 // consecutive experts: groups are scored by the sum of their two best
 // selection scores and ranked with shuffles, and the top-k is k rounds of
@@ -342,11 +344,13 @@ route_tokens_g8_kernel(const RouteArgs r) {
 // still sums its K blocks in one fixed order).
 constexpr int kGateThreads = 512;
 
-template <int C>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGateThreads, 1)
-gate_route_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
-                       const RouteArgs r, uint32_t tmem_cols) {
+template <int C, int SPLIT>
+__global__ void __launch_bounds__(kGateThreads, 1)
+gate_route_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
+                  const RouteArgs r, uint32_t tmem_cols) {
+  static_assert(SPLIT == 2 || SPLIT == 4 || SPLIT == 8, "clusters of 2, 4 or 8 CTAs");
   constexpr int KB = 64;
+  constexpr int OWN = kRouteRows / SPLIT;              // tokens each CTA owns (and routes)
   extern __shared__ __align__(1024) uint8_t dsmem[];
   __shared__ uint64_t full_bar[kRouteStages], empty_bar[kRouteStages];
   __shared__ uint64_t tmem_full, drain_bar;
@@ -364,10 +368,14 @@ gate_route_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
   const uint32_t stage_bytes = a_bytes + b_bytes;
   const int m0 = static_cast<int>(cluster_id_x()) * kRouteRows;
   const int nk = r.H / KB;
-  const int nk0 = (nk + 1) / 2;
-  const int kb_begin = rank ? nk0 : 0;
-  const int kb_count = rank ? nk - nk0 : nk0;
-  float* recv = reinterpret_cast<float*>(smem);        // peer partials, after the main loop
+  // CTA r: the K blocks [r * nk / SPLIT, (r + 1) * nk / SPLIT)
+  const int kb_begin = (static_cast<int>(rank) * nk) / SPLIT;
+  const int kb_count = ((static_cast<int>(rank) + 1) * nk) / SPLIT - kb_begin;
+  // after the main loop: recv[slot][OWN][LD], the other CTAs' partial sums of
+  // this CTA's tokens (slot = the sender's rank with this CTA's left out);
+  // rows padded by 16 bytes so that 32 rows' same column spread over the banks
+  float* recv = reinterpret_cast<float*>(smem);
+  const int LD = r.E + 4;
   const int rot = kb_count > 0 ? static_cast<int>((cluster_id_x() * 7u) % static_cast<uint32_t>(kb_count)) : 0;
 
   if constexpr (C > 0) {
@@ -453,8 +461,9 @@ gate_route_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
   const int q = warp & 3;
   const int row = 32 * q + lane;                       // TMEM lane == token row of the tile
   const bool epi = warp >= 2 && warp < 6;
-  const bool mine = (row >> 6) == static_cast<int>(rank);   // CTA r writes rows [64r, 64r + 64)
+  const int owner = row / OWN;                         // CTA owner writes rows [OWN * owner, +OWN)
   const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+  // every lane of a warp reads the accumulator (tcgen05.ld is warp-collective)
   auto partial = [&](int c, float (&v)[32]) {
     if (kb_count > 0) {
       tmem_ld32(lane_addr + c * 32, v);
@@ -464,57 +473,74 @@ gate_route_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_con
       for (int j = 0; j < 32; ++j) v[j] = 0.0f;
     }
   };
-  if (epi && !mine) {                                  // send to the CTA that writes this token
-    const uint32_t dst = mapa_shared(smem_u32(recv), rank ^ 1u) + static_cast<uint32_t>((row & 63) * r.E) * 4u;
+  // a warp whose 32 rows are all this CTA's sends nothing; otherwise every
+  // lane whose row another CTA owns sends it there
+  const bool warp_all_mine = (32 * q) / OWN == static_cast<int>(rank) && (32 * q + 31) / OWN == static_cast<int>(rank);
+  if (epi && !warp_all_mine) {
+    const int slot = static_cast<int>(rank) < owner ? static_cast<int>(rank) : static_cast<int>(rank) - 1;
+    const uint32_t dst = mapa_shared(smem_u32(recv), static_cast<uint32_t>(owner)) +
+                         static_cast<uint32_t>((slot * OWN + row % OWN) * LD) * 4u;
     for (int c = 0; c * 32 < r.E; ++c) {
       float v[32];
       partial(c, v);
+      if (owner != static_cast<int>(rank)) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (c * 32 + 4 * j < r.E)
-          asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (c * 32 + 4 * j) * 4u),
-                       "f"(v[4 * j]), "f"(v[4 * j + 1]), "f"(v[4 * j + 2]), "f"(v[4 * j + 3])
-                       : "memory");
+        for (int j = 0; j < 8; ++j) {
+          if (c * 32 + 4 * j < r.E)
+            asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (c * 32 + 4 * j) * 4u),
+                         "f"(v[4 * j]), "f"(v[4 * j + 1]), "f"(v[4 * j + 2]), "f"(v[4 * j + 3])
+                         : "memory");
+        }
       }
     }
   }
-  cluster_sync();                                      // the peer's partials have landed
+  cluster_sync();                                      // every partial has landed
 
-  if (epi && mine) {
+  // this CTA's own rows [OWN * rank, +OWN): the warps holding them add the
+  // SPLIT partial sums in rank order and write the logits (and, to route
+  // them, keep them in slot 0 of recv)
+  const bool warp_has_mine = (32 * q) / OWN <= static_cast<int>(rank) && static_cast<int>(rank) <= (32 * q + 31) / OWN;
+  if (epi && warp_has_mine) {
+    const bool mine = owner == static_cast<int>(rank);
     const int tok = m0 + row;
-    float* peer = recv + static_cast<size_t>(row & 63) * r.E;   // becomes this token's full logits
+    const int i = row % OWN;
     for (int c = 0; c * 32 < r.E; ++c) {
       float v[32];
       partial(c, v);
-      if (tok < r.T) {
+      if (mine && tok < r.T) {
         float4* dst = reinterpret_cast<float4*>(r.logits + static_cast<size_t>(tok) * r.E + c * 32);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (c * 32 + 4 * j < r.E) {
-            float o[4];
+            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float p = peer[c * 32 + 4 * j + u];
-              o[u] = rank ? p + v[4 * j + u] : v[4 * j + u] + p;      // first half + second half
+            for (int src = 0; src < SPLIT; ++src) {           // partials added in rank order
+              const int sl = src < static_cast<int>(rank) ? src : src - 1;
+              const float4 pv = src == static_cast<int>(rank)
+                                    ? make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3])
+                                    : *reinterpret_cast<const float4*>(recv + (sl * OWN + i) * LD + c * 32 + 4 * j);
+              if (src == 0) {
+                acc = pv;
+              } else {
+                acc.x += pv.x; acc.y += pv.y; acc.z += pv.z; acc.w += pv.w;
+              }
             }
-            dst[j] = make_float4(o[0], o[1], o[2], o[3]);
-            if constexpr (C > 0) reinterpret_cast<float4*>(peer + c * 32)[j] = make_float4(o[0], o[1], o[2], o[3]);
+            dst[j] = acc;
+            if constexpr (C > 0) *reinterpret_cast<float4*>(recv + i * LD + c * 32 + 4 * j) = acc;
           }
         }
       }
     }
   }
   if constexpr (C > 0) {
-    // route this CTA's 64 tokens from their logits in shared memory: each
-    // warp four tokens (eight threads per token)
+    // route this CTA's OWN tokens from their logits in shared memory: each
+    // warp four tokens (eight threads per token), all in one pass
     __syncthreads();
-    const int tok_base = m0 + 64 * static_cast<int>(rank);
-    for (int pass = 0; pass < 64; pass += 4 * (kGateThreads / 32)) {
-      const int i = pass + 4 * warp + (lane >> 3);
-      const int tok = tok_base + i;
-      const bool valid = i < 64 && tok < r.T;
-      route_token8<C>(r, recv + static_cast<size_t>(valid ? i : 0) * r.E, tok, valid, bias_s, hist);
-    }
+    const int tok_base = m0 + OWN * static_cast<int>(rank);
+    const int i = 4 * warp + (lane >> 3);
+    const int tok = tok_base + i;
+    const bool valid = i < OWN && tok < r.T;
+    route_token8<C>(r, recv + static_cast<size_t>(valid ? i : 0) * LD, tok, valid, bias_s, hist);
     __syncthreads();
     for (int e = threadIdx.x; e < r.E; e += blockDim.x)
       if (hist[e]) atomicAdd(r.counts + e, hist[e]);
@@ -534,31 +560,62 @@ int route8_experts_per_thread(const RouteArgs& r) {
   return ok ? C : 0;
 }
 
-template <int C>
-cudaError_t launch_gate_route(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r, size_t smem,
-                              uint32_t cols, int grid, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(gate_route_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+// Clusters of SPLIT CTAs per 128-token tile: the largest of 8, 4, 2 that still
+// leaves every CTA resident at once (tiles * SPLIT <= the SM count), so few
+// tokens still spread over many SMs while V3's 64 tiles keep pairs.
+int gate_split(int T, int num_sms) {
+  const int tiles = (T + kRouteRows - 1) / kRouteRows;
+  for (int split = 8; split > 2; split >>= 1)
+    if (tiles * split <= num_sms) return split;
+  return 2;
+}
+
+template <int C, int SPLIT>
+cudaError_t launch_gate_route_split(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r,
+                                    uint32_t cols, cudaStream_t stream) {
+  const size_t ring = static_cast<size_t>(kRouteStages) * (128 * 128 + static_cast<size_t>(r.E) * 128);
+  const size_t recv = static_cast<size_t>(SPLIT - 1) * (kRouteRows / SPLIT) * (r.E + 4) * sizeof(float);
+  const size_t smem = (ring > recv ? ring : recv) + 1024;
+  auto kern = gate_route_kernel<C, SPLIT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  gate_route_pair_kernel<C><<<grid, kGateThreads, smem, stream>>>(tmX, tmG, r, cols);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(SPLIT * ((r.T + kRouteRows - 1) / kRouteRows));
+  cfg.blockDim = dim3(kGateThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = SPLIT;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tmX, tmG, r, cols);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
+template <int C>
+cudaError_t launch_gate_route(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r, uint32_t cols,
+                              int split, cudaStream_t stream) {
+  if (split == 8) return launch_gate_route_split<C, 8>(tmX, tmG, r, cols, stream);
+  if (split == 4) return launch_gate_route_split<C, 4>(tmX, tmG, r, cols, stream);
+  return launch_gate_route_split<C, 2>(tmX, tmG, r, cols, stream);
+}
+
 cudaError_t launch_gate_gemm(const CUtensorMap& tmX, const CUtensorMap& tmG, const RouteArgs& r, bool route,
-                             cudaStream_t stream) {
+                             int num_sms, cudaStream_t stream) {
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(r.E)) cols <<= 1;
-  const size_t ring = static_cast<size_t>(kRouteStages) * (128 * 128 + static_cast<size_t>(r.E) * 128);
-  const size_t recv = static_cast<size_t>(64) * r.E * sizeof(float);
-  const size_t smem = (ring > recv ? ring : recv) + 1024;
-  const int grid = 2 * ((r.T + kRouteRows - 1) / kRouteRows);
+  const int split = gate_split(r.T, num_sms);
   switch (route ? route8_experts_per_thread(r) : 0) {
-    case 2: return launch_gate_route<2>(tmX, tmG, r, smem, cols, grid, stream);
-    case 4: return launch_gate_route<4>(tmX, tmG, r, smem, cols, grid, stream);
-    case 8: return launch_gate_route<8>(tmX, tmG, r, smem, cols, grid, stream);
-    case 16: return launch_gate_route<16>(tmX, tmG, r, smem, cols, grid, stream);
-    case 32: return launch_gate_route<32>(tmX, tmG, r, smem, cols, grid, stream);
-    default: return launch_gate_route<0>(tmX, tmG, r, smem, cols, grid, stream);
+    case 2: return launch_gate_route<2>(tmX, tmG, r, cols, split, stream);
+    case 4: return launch_gate_route<4>(tmX, tmG, r, cols, split, stream);
+    case 8: return launch_gate_route<8>(tmX, tmG, r, cols, split, stream);
+    case 16: return launch_gate_route<16>(tmX, tmG, r, cols, split, stream);
+    case 32: return launch_gate_route<32>(tmX, tmG, r, cols, split, stream);
+    default: return launch_gate_route<0>(tmX, tmG, r, cols, split, stream);
   }
 }
 

@@ -171,8 +171,12 @@ def test_route_topk_group_sweep_bit_exact_with_load_cv(topk_group):
     assert max(len(set(row)) for row in groups_used.tolist()) <= topk_group
 
 
+# T picks the gate GEMM's cluster size (CTAs sharing one 128-token tile's
+# hidden size): 8 up to 18 tiles (tiny, where some CTAs get no K block; 1000;
+# 1; 129), 4 up to 37 (v2lite 4096; 3000 with a 56-token tail), 2 beyond (v3).
 @pytest.mark.parametrize("name,T", [("tiny", None), ("tiny_grouped", None), ("v2lite", None),
-                                    ("v3", None), ("v3", 1000), ("v3", 1), ("v2lite", 129)])
+                                    ("v3", None), ("v3", 1000), ("v3", 1), ("v2lite", 129),
+                                    ("v3", 3000)])
 def test_route_gate_gemm(name, T):
     cfg = _cfg(name)
     T = T or cfg.T
@@ -256,7 +260,7 @@ def test_route_token_with_nan_scores_is_flagged_not_routed(k):
     assert int(counts.sum()) == (T - 1) * cfg.k
 
 
-@pytest.mark.parametrize("name,T", [("tiny", None), ("v3", None), ("v3", 1000)])
+@pytest.mark.parametrize("name,T", [("tiny", None), ("v3", None), ("v3", 1000), ("v3", 3000)])
 def test_gate_logits_then_route_equals_route(name, T):
     """moe_gate_logits followed by moe_route on those logits (x = NULL) is
     moe_route in two calls: logits, ids, weights and counts bit for bit."""
