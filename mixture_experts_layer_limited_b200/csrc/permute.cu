@@ -6,12 +6,14 @@
 // gives expert_first_token_offset as the segment boundaries. That is a stable
 // counting sort of the T*k (token, slot) pairs keyed by expert, done here in
 // three launches:
-//   1. perm_hist  : per block of kTokBlock tokens, an expert histogram;
+//   1. perm_hist  : per block of kTokBlock tokens, an expert histogram and
+//                   each slot's rank among the block's slots of its expert
+//                   (kept in slot_to_row until step 3 replaces it);
 //   2. perm_scan  : expert offsets (exclusive scan of the totals) and, per
 //                   block, the first row of each expert's part of the segment;
-//   3. perm_place : one warp per token ranks its slots among the earlier
-//                   slots of its block (ballots), writes the metadata, reads
-//                   the token's row once and writes it to its k rows.
+//   3. perm_place : one warp per token adds the two for each of its slots,
+//                   writes the metadata, reads the token's row once and
+//                   writes it to its k rows.
 
 #include "kernels.cuh"
 
@@ -19,21 +21,57 @@ namespace moe {
 
 constexpr int kTokBlock = 64;        // tokens per rank block
 
-__global__ void perm_hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E,
-                                 int32_t* __restrict__ blockhist, int32_t* status) {
+// 256 threads; the block's slots (token-major, then slot) are taken 256 at a
+// time in order. A slot's rank = its expert's count over the earlier rounds
+// + the counts of the earlier warps of this round + the earlier lanes of its
+// own warp with the same expert (match_any), so equal experts keep slot
+// order: the stable sort's order inside the block.
+constexpr int kHistThreads = 256;
+
+__global__ void __launch_bounds__(kHistThreads)
+perm_hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int32_t* __restrict__ blockhist,
+                 int32_t* __restrict__ local_rank, int32_t* status) {
+  constexpr int kWarps = kHistThreads / 32;
   extern __shared__ int hist_dyn[];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist_dyn[e] = 0;
-  __syncthreads();
+  int* cnt = hist_dyn;                                  // [E]: the earlier rounds' slots per expert
+  int* wcnt = hist_dyn + E;                             // [kWarps][E]: this round's slots per warp and expert
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < E; e += kHistThreads) cnt[e] = 0;
   const int s0 = blockIdx.x * kTokBlock * k;
   const int s1 = min(T, (blockIdx.x + 1) * kTokBlock) * k;
-  for (int s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
-    const int e = ids[s];
-    if (e >= 0 && e < E) atomicAdd(&hist_dyn[e], 1);
-    else flag_status(status, MOE_DEVSTAT_BAD_EXPERT_ID);
+  for (int base = s0; base < s1; base += kHistThreads) {   // same trip count in the whole CTA
+    for (int i = threadIdx.x; i < kWarps * E; i += kHistThreads) wcnt[i] = 0;
+    __syncthreads();
+    const int s = base + threadIdx.x;
+    int e = -1;
+    if (s < s1) {
+      e = ids[s];
+      if (e < 0 || e >= E) {
+        flag_status(status, MOE_DEVSTAT_BAD_EXPERT_ID);
+        e = -1;
+      }
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int intra = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && intra == 0) wcnt[warp * E + e] = __popc(peers);
+    __syncthreads();
+    if (e >= 0) {
+      int rank = cnt[e] + intra;
+      for (int w = 0; w < warp; ++w) rank += wcnt[w * E + e];
+      local_rank[s] = rank;
+    } else if (s < s1) {
+      local_rank[s] = -1;
+    }
+    __syncthreads();                                    // cnt read before it advances
+    for (int x = threadIdx.x; x < E; x += kHistThreads) {
+      int add = 0;
+      for (int w = 0; w < kWarps; ++w) add += wcnt[w * E + x];
+      cnt[x] += add;
+    }
+    __syncthreads();                                    // wcnt read before the next round clears it
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    blockhist[static_cast<size_t>(blockIdx.x) * E + e] = hist_dyn[e];
+  for (int e = threadIdx.x; e < E; e += kHistThreads)
+    blockhist[static_cast<size_t>(blockIdx.x) * E + e] = cnt[e];
 }
 
 // One CTA of 1024 threads. Thread (e, part) owns expert e for blocks
@@ -115,17 +153,17 @@ perm_scan_kernel(int32_t* __restrict__ blockhist, int nb, int E, int total,
 
 // One warp per token t: its rows, then the copies.
 //   row of slot (t, j) = first row of (block of t, expert e) from perm_scan
-//                        + the number of earlier slots of the block with expert e
-// (token order, then slot order: the stable counting sort). The warp counts
-// the earlier slots 32 at a time with one ballot per slot of t, writes
-// slot_to_row / src_token / row_w, reads the token's row once and writes it
-// to its k rows with 16-byte vector loads and stores (fp8 rows also carry
-// their 1x128 scales). Slots with ids outside [0, E) get row -1 (flagged by
-// perm_hist) and are not written.
+//                        + the slot's rank inside the block from perm_hist
+// (token order, then slot order: the stable counting sort). Lane j < k
+// writes slot j's slot_to_row / src_token / row_w; the warp reads the token's
+// row once and writes it to its k rows with 16-byte vector loads and stores
+// (fp8 rows also carry their 1x128 scales). Slots with ids outside [0, E)
+// get row -1 (flagged by perm_hist) and are not written.
 constexpr int kPermKMax = 16;
 
 // The rows of token t's k slots (lane j < k returns slot j's row, -1 for an
-// invalid id) and their metadata; called by the whole warp.
+// invalid id) and their metadata; slot_to_row holds perm_hist's ranks on
+// entry and the rows on return.
 __device__ __forceinline__ int perm_rows_of_token(int t, int lane, const int32_t* __restrict__ ids,
                                                   const float* __restrict__ topk_w, int T, int k, int E,
                                                   const int32_t* __restrict__ blockbase,
@@ -133,45 +171,19 @@ __device__ __forceinline__ int perm_rows_of_token(int t, int lane, const int32_t
                                                   int32_t* __restrict__ src_token, float* __restrict__ row_w) {
   const int nrows = T * k;
   const int b = t / kTokBlock;
-  const size_t s_me = static_cast<size_t>(t) * k;
-  int my_e = -1;
-  if (lane < k) {
-    my_e = ids[s_me + lane];
-    if (my_e < 0 || my_e >= E) my_e = -1;
-  }
-  // earlier slots of the block with my expert
-  int cnt = 0;
-  const size_t s_blk = static_cast<size_t>(b) * kTokBlock * k;
-  for (size_t base = s_blk; base < s_me; base += 32) {  // same trip count on every lane
-    const size_t s = base + lane;
-    const int e = s < s_me ? ids[s] : -1;
-#pragma unroll
-    for (int j = 0; j < kPermKMax; ++j) {
-      if (j < k) {
-        const int ej = __shfl_sync(0xffffffffu, my_e, j);
-        const int c = __popc(__ballot_sync(0xffffffffu, ej >= 0 && e == ej));
-        if (lane == j) cnt += c;
-      }
-    }
-  }
-  // earlier slots of this token with the same expert (repeated ids)
-#pragma unroll
-  for (int j = 0; j < kPermKMax; ++j) {
-    if (j < k) {
-      const int ej = __shfl_sync(0xffffffffu, my_e, j);
-      if (j < lane && ej == my_e) ++cnt;
-    }
-  }
+  const size_t s = static_cast<size_t>(t) * k + lane;
   int my_row = -1;
-  if (lane < k && my_e >= 0) {
-    my_row = blockbase[static_cast<size_t>(b) * E + my_e] + cnt;
-    if (my_row >= nrows) my_row = -1;                 // never write outside the rows
-  }
   if (lane < k) {
-    slot_to_row[s_me + lane] = my_row;
+    const int e = ids[s];
+    const int rank = slot_to_row[s];
+    if (e >= 0 && e < E && rank >= 0) {
+      my_row = blockbase[static_cast<size_t>(b) * E + e] + rank;
+      if (my_row >= nrows) my_row = -1;                 // never write outside the rows
+    }
+    slot_to_row[s] = my_row;
     if (my_row >= 0) {
       src_token[my_row] = t;
-      if (row_w) row_w[my_row] = topk_w[s_me + lane];
+      if (row_w) row_w[my_row] = topk_w[s];
     }
   }
   return my_row;
@@ -186,15 +198,24 @@ perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ top
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;                                  // warp-uniform
-  const int my_row = perm_rows_of_token(t, lane, ids, topk_w, T, k, E, blockbase, slot_to_row, src_token, row_w);
-  if (!x_perm) return;                                 // metadata only
   const uint4* src = x + static_cast<size_t>(t) * vec_per_row;
-  for (int base = 0; base < vec_per_row; base += 128) {   // same trip count on every lane
-    uint4 val[4];
+  uint4 val[4];
+  if (x_perm) {                                        // the row's first chunk in flight during the metadata
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int v = base + u * 32 + lane;
+      const int v = u * 32 + lane;
       if (v < vec_per_row) val[u] = __ldg(src + v);
+    }
+  }
+  const int my_row = perm_rows_of_token(t, lane, ids, topk_w, T, k, E, blockbase, slot_to_row, src_token, row_w);
+  if (!x_perm) return;                                 // metadata only
+  for (int base = 0; base < vec_per_row; base += 128) {   // same trip count on every lane
+    if (base > 0) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = base + u * 32 + lane;
+        if (v < vec_per_row) val[u] = __ldg(src + v);
+      }
     }
 #pragma unroll
     for (int j = 0; j < kPermKMax; ++j) {
@@ -294,7 +315,7 @@ perm_place_quant_kernel(const int32_t* __restrict__ ids, const float* __restrict
   }
 }
 
-size_t permute_workspace_bytes(int T, int E) {
+size_t permute_workspace_bytes(int T, int E) {   // blockhist[nb][E]
   const int nb = (T + kTokBlock - 1) / kTokBlock;
   return static_cast<size_t>(nb) * E * sizeof(int32_t);
 }
@@ -305,7 +326,8 @@ cudaError_t launch_permute(int T, int k, int E, int H, bool x_e4m3, bool perm_e4
                            int32_t* src_token, int32_t* slot_to_row, float* row_w, int32_t* blockhist,
                            int32_t* status, cudaStream_t stream) {
   const int nb = (T + kTokBlock - 1) / kTokBlock;
-  perm_hist_kernel<<<nb, 256, E * sizeof(int), stream>>>(ids, T, k, E, blockhist, status);
+  perm_hist_kernel<<<nb, kHistThreads, (kHistThreads / 32 + 1) * E * sizeof(int), stream>>>(
+      ids, T, k, E, blockhist, slot_to_row, status);
   const int parts = 1024 / E;
   const size_t scan_smem = (static_cast<size_t>(parts) * E + E + 32) * sizeof(int);
   perm_scan_kernel<<<1, 1024, scan_smem, stream>>>(blockhist, nb, E, T * k, offsets);

@@ -292,6 +292,23 @@ def _ids_from_oracle(T, k, E, seed, skew=0.0):
                                           (50, 2, 16, 28672, 0.0)])
 def test_permute_bit_exact(T, k, E, H, skew):
     ids_np, w_np = _ids_from_oracle(T, k, E, seed=T + E, skew=skew)
+    _check_permute(ids_np, w_np, E, H)
+
+
+@pytest.mark.parametrize("T,k,E", [(200, 16, 16), (1000, 4, 4), (129, 8, 256), (64, 16, 1024)])
+def test_permute_repeated_ids_keep_slot_order(T, k, E):
+    """ids drawn with replacement, so a token may name one expert in several
+    of its slots, and k = 16 puts a block's slots over several rounds of the
+    histogram kernel: rows still follow the stable order, token then slot."""
+    rng = np.random.default_rng(T * k + E)
+    ids_np = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    ids_np[0, :] = ids_np[0, 0]                        # one token with a single expert in every slot
+    w_np = rng.random((T, k)).astype(np.float32)
+    _check_permute(ids_np, w_np, E, 128)
+
+
+def _check_permute(ids_np, w_np, E, H):
+    T, k = ids_np.shape
     offsets_o, src_o, s2r_o = oracle.permute(ids_np, E)
     ids = torch.from_numpy(ids_np).to(DEV)
     tw = torch.from_numpy(w_np).to(DEV)
