@@ -199,20 +199,20 @@ perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ top
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;                                  // warp-uniform
   const uint4* src = x + static_cast<size_t>(t) * vec_per_row;
-  uint4 val[4];
+  uint4 val[8];
   if (x_perm) {                                        // the row's first chunk in flight during the metadata
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u) {
       const int v = u * 32 + lane;
       if (v < vec_per_row) val[u] = __ldg(src + v);
     }
   }
   const int my_row = perm_rows_of_token(t, lane, ids, topk_w, T, k, E, blockbase, slot_to_row, src_token, row_w);
   if (!x_perm) return;                                 // metadata only
-  for (int base = 0; base < vec_per_row; base += 128) {   // same trip count on every lane
+  for (int base = 0; base < vec_per_row; base += 256) {   // same trip count on every lane
     if (base > 0) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int v = base + u * 32 + lane;
         if (v < vec_per_row) val[u] = __ldg(src + v);
       }
@@ -224,7 +224,7 @@ perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ top
       if (row >= 0) {
         uint4* dst = x_perm + static_cast<size_t>(row) * vec_per_row;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           const int v = base + u * 32 + lane;
           if (v < vec_per_row) __stcs(dst + v, val[u]);        // streamed: x_perm is far larger than L2
         }
