@@ -578,6 +578,28 @@ def test_combine(weighted, shared):
     assert np.all(np.abs(np64(y) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)
 
 
+def test_combine_full_size_sampled_tokens():
+    """The V3 shape (T = 8192, k = 8, H = 7168: 1.2 GB moved in one launch):
+    every token combined on the GPU; the first, the last and 62 random tokens
+    compared on every feature with the oracle's combine of those tokens."""
+    T, k, H = 8192, 8, 7168
+    g = _gen(9)
+    eo = torch.randn(T * k, H, generator=g, device=DEV).to(torch.bfloat16)
+    perm = torch.randperm(T * k, generator=g, device=DEV).to(torch.int32)
+    tw = torch.rand(T, k, generator=g, device=DEV)
+    sh = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
+    y = torch.empty(T, H, dtype=torch.bfloat16, device=DEV)
+    N.moe_combine(T, k, H, eo, perm, tw, sh, y)
+    rng = np.random.default_rng(3)
+    S = np.unique(np.concatenate([[0, T - 1], rng.choice(np.arange(1, T - 1), 62, replace=False)]))
+    rows = perm.cpu().numpy().reshape(T, k)[S].reshape(-1)          # the sampled tokens' rows, slot order
+    St = torch.from_numpy(S).to(DEV)
+    ref = oracle.combine(np64(eo[torch.from_numpy(rows).to(DEV)]), np.arange(len(rows)), k,
+                         np32(tw[St]), np64(sh[St]))
+    got = np64(y[St])
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)
+
+
 # ----------------------------------------------------------- bias update
 def test_bias_update_bit_exact_ten_steps():
     E, T, k, gamma = 256, 8192, 8, 0.001
