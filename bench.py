@@ -49,6 +49,8 @@ def parse_args():
                          "of the hottest and the coldest expert)")
     ap.add_argument("--fuse-combine", action="store_true",
                     help="run the combine inside the down GEMM (atomic fp32 scatter-add) instead of after it")
+    ap.add_argument("--split-ffn", action="store_true",
+                    help="run the experts' two GEMMs as two launches (gate/up, then down) instead of one")
     ap.add_argument("--routing-sweep", action="store_true",
                     help="instead of the throughput line: load CV, aux loss and router time for "
                          "topk_group 8/4/2/1 of 8 groups on the V3 and skewed inputs (one line each)")
@@ -284,7 +286,7 @@ def profiled_traffic(stage, workload):
 
 LAUNCHES = {"route": 1, "permute": 3, "gate_up_routed": 1, "down_routed": 1,
             "gate_up_shared": 1, "down_shared": 1, "gate_up": 1, "down": 1, "combine": 1, "bias_update": 1,
-            "down_combine": 2}
+            "down_combine": 2, "ffn": 1}
 
 
 def launches_of(name, cfg):
@@ -316,6 +318,8 @@ def stage_model(cfg):
     # routed + shared expert in one launch per GEMM
     for fused, parts in (("gate_up", ("gate_up_routed", "gate_up_shared")), ("down", ("down_routed", "down_shared"))):
         m[fused] = {key: sum(m[p][key] for p in parts) for key in ("flops", "bytes")}
+    # both GEMMs, routed + shared expert, in one launch (h still makes its round trip)
+    m["ffn"] = {key: m["gate_up"][key] + m["down"][key] for key in ("flops", "bytes")}
     # down GEMMs with the combine in the epilogue: weights and h in, y out
     m["down_combine"] = {"flops": m["down"]["flops"],
                          "bytes": E * H * I * ab + R * I * ab + H * Is * ab + T * Is * ab + T * H * 2}
@@ -346,7 +350,7 @@ def run_ours(args):
         g.manual_seed(cfg.seed + 100003 * rank)
         inp.x = torch.randn(cfg.T, cfg.H, generator=g, device="cuda").to(torch.bfloat16)
     layer = MoELayer(LayerSpec.from_config(cfg), inp.gate, inp.w13, inp.w2, inp.sw13, inp.sw2,
-                     inp.bias, cfg.T, fuse_combine=args.fuse_combine)
+                     inp.bias, cfg.T, fuse_combine=args.fuse_combine, fuse_ffn=not args.split_ffn)
     T_global = cfg.T * world
     stream = torch.cuda.current_stream()
     stages = layer.stages(inp.x)
@@ -410,14 +414,16 @@ def run_ours(args):
     tokens = cfg.T * world * K
     value = tokens / (ms * 1e-3)
     flops_step = cfg.flops()
-    dom = "gate_up" if "gate_up" in avg else "gate_up_routed"
+    dom = "ffn" if "ffn" in avg else "gate_up" if "gate_up" in avg else "gate_up_routed"
     achieved = model[dom]["flops"] / (avg[dom] * 1e-3) / 1e12
     # the timed region is well under a second, at the clock the sampler saw:
     # the peak is the burst figure (a GEMM timed alone); the sustained one
     # (seconds under the power cap, at a lower clock) only as a second number
     peak = peaks["bf16_tflops"]
-    what = "routed experts + shared expert, one launch" if dom == "gate_up" else "routed experts"
-    roofline = {"kernel": f"grouped_gemm_bf16 (gate/up + SwiGLU, {what})", "bound": "tensor",
+    what = "routed experts + shared expert, one launch" if dom in ("gate_up", "ffn") else "routed experts"
+    kname = ("grouped_ffn_bf16 (gate/up + SwiGLU and down + routing weight, " if dom == "ffn"
+             else "grouped_gemm_bf16 (gate/up + SwiGLU, ") + what + ")"
+    roofline = {"kernel": kname, "bound": "tensor",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": profiled_traffic(dom, cfg.name),
                 "sm_mhz": clk.get("sm_mhz"),

@@ -312,6 +312,32 @@ MOE_API moe_status moe_down_proj_with_shared(int32_t rows, int32_t H, const moe_
                               const void* sh_h, const float* sh_h_scale, void* sh_out,
                               int32_t* dev_status, void* stream);
 
+/* moe_swiglu_ffn_with_shared -- both GEMMs of the routed experts and of the
+ * shared expert in ONE persistent launch ([MoE-walk] §3.3: SwiGLU experts as
+ * one grouped GEMM, the merged shared expert as one more group):
+ *   h_ws    = SiLU(a w1^T) * (a w3^T) per segment of offsets,
+ *   out     = row_w * (h_ws w2^T),
+ *   sh_h_ws = SwiGLU of (sh_a, sw13),  sh_out = sh_h_ws sw2^T,
+ * the same values, bit for bit, as moe_gate_up_swiglu_with_shared followed by
+ * moe_down_proj_with_shared. The CTAs take the tiles of both GEMMs from one
+ * counter, in order, and a token block's down tiles start as soon as its h
+ * rows are stored (a counter per token block in sync_ws, bounded waits), so
+ * no SM idles while the last gate/up tiles end.
+ *   sync_ws        device scratch of at least moe_swiglu_ffn_sync_size()
+ *                  bytes, 16-byte aligned; zeroed by the call (stream order),
+ *                  so it may not be shared by calls in flight at once.
+ * bf16 only (MOE_ERR_UNSUPPORTED otherwise); other arguments, limits and
+ * errors as the two calls it replaces. A wait that runs out flags
+ * MOE_DEVSTAT_TIMEOUT in dev_status. */
+MOE_API moe_status moe_swiglu_ffn_sync_size(int32_t rows, int32_t groups, int32_t sh_rows, size_t* bytes);
+MOE_API moe_status moe_swiglu_ffn_with_shared(int32_t rows, int32_t H, const moe_ffn_weights* w,
+                              const void* a, const int32_t* offsets, const float* row_w,
+                              void* h_ws, void* out,
+                              int32_t sh_rows, const moe_ffn_weights* sw, const void* sh_a,
+                              void* sh_h_ws, void* sh_out,
+                              void* sync_ws, size_t sync_ws_bytes,
+                              int32_t* dev_status, void* stream);
+
 /* moe_down_proj_combine -- the second GEMM with the combine fused into its
  * epilogue ([MoE-walk] §3.3.1 + §3.4): every routed row's weighted output
  * row_w[r] * (h[r] w2[e]^T) is added in fp32 straight into the row of its token

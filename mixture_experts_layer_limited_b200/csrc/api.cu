@@ -248,6 +248,12 @@ moe_status check_ffn(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
   return MOE_OK;
 }
 
+// Token blocks (of at most 256 rows) of `rows` rows in one segment, and an
+// upper bound over `groups` segments of `rows` rows in all (each non-empty
+// segment adds at most one partial block).
+int32_t ffn_blocks(int32_t rows) { return (rows + 255) / 256; }
+int32_t ffn_routed_blocks(int32_t rows, int32_t groups) { return ffn_blocks(rows) + groups; }
+
 // Tensor maps and kernel arguments of one grouped GEMM.
 struct GemmPlan {
   CUtensorMap tmA;
@@ -479,6 +485,51 @@ moe_status moe_down_proj_with_shared(int32_t rows, int32_t H, const moe_ffn_weig
   if ((s = plan_down(sh_rows, H, sw, sh_h, sh_h_scale, nullptr, nullptr, sh_out, dev_status, &q)) != MOE_OK)
     return s;
   return launch_plan(p, EPI_WEIGHTED, st, nsm, &q);
+}
+
+moe_status moe_swiglu_ffn_sync_size(int32_t rows, int32_t groups, int32_t sh_rows, size_t* bytes) {
+  if (!bytes || rows < 1 || groups < 1 || sh_rows < 1) return MOE_ERR_INVALID_ARG;
+  *bytes = sizeof(int32_t) * (ffn_routed_blocks(rows, groups) + ffn_blocks(sh_rows) + 1);
+  return MOE_OK;
+}
+
+moe_status moe_swiglu_ffn_with_shared(int32_t rows, int32_t H, const moe_ffn_weights* w, const void* a,
+                                      const int32_t* offsets, const float* row_w, void* h_ws, void* out,
+                                      int32_t sh_rows, const moe_ffn_weights* sw, const void* sh_a, void* sh_h_ws,
+                                      void* sh_out, void* sync_ws, size_t sync_ws_bytes, int32_t* dev_status,
+                                      void* stream) {
+  moe_status s = check_ffn(rows, H, w, a, nullptr, true, true);
+  if (s != MOE_OK) return s;
+  if ((s = check_ffn(sh_rows, H, sw, sh_a, nullptr, true, true)) != MOE_OK) return s;
+  if (!offsets || !h_ws || !out || !sh_h_ws || !sh_out || !sync_ws || sw->groups != 1) return MOE_ERR_INVALID_ARG;
+  if (w->dtype != MOE_BF16 || sw->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  const size_t nctr = ffn_routed_blocks(rows, w->groups) + ffn_blocks(sh_rows);
+  const size_t need = sizeof(int32_t) * (nctr + 1);   // token-block counters, then the tile counter
+  if (sync_ws_bytes < need) return MOE_ERR_INVALID_ARG;
+  if (any_misaligned(offsets, row_w, h_ws, out, sh_h_ws, sh_out, sync_ws)) return MOE_ERR_ALIGNMENT;
+  int nsm = 0;
+  if ((s = sm_count(&nsm)) != MOE_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  GemmPlan gu, sgu, dn, sdn;
+  if ((s = plan_gate_up(sh_rows, H, sw, sh_a, nullptr, nullptr, sh_h_ws, nullptr, dev_status, &sgu)) != MOE_OK)
+    return s;
+  if ((s = plan_gate_up(rows, H, w, a, nullptr, offsets, h_ws, nullptr, dev_status, &gu)) != MOE_OK) return s;
+  if ((s = plan_down(sh_rows, H, sw, sh_h_ws, nullptr, nullptr, nullptr, sh_out, dev_status, &sdn)) != MOE_OK)
+    return s;
+  if ((s = plan_down(rows, H, w, h_ws, nullptr, offsets, row_w, out, dev_status, &dn)) != MOE_OK) return s;
+  FfnArgs f{};
+  const GemmPlan* plans[4] = {&sgu, &gu, &sdn, &dn};
+  for (int i = 0; i < 4; ++i) {
+    f.tmA[i] = plans[i]->tmA;
+    f.tmB[i] = plans[i]->tmB;
+    f.g[i] = plans[i]->g;
+  }
+  f.ready = static_cast<int32_t*>(sync_ws);
+  f.tile_counter = f.ready + nctr;
+  f.shared_base = ffn_routed_blocks(rows, w->groups);
+  cudaError_t e = cudaMemsetAsync(sync_ws, 0, need, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return check_launch(launch_ffn_bf16(f, nsm, st));
 }
 
 moe_status moe_down_proj_combine(int32_t rows, int32_t T, int32_t H, const moe_ffn_weights* w, const void* h,

@@ -282,6 +282,38 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Orders global-memory data this thread has acquired (written by other SMs
+// with ordinary stores) before its later async-proxy (TMA) reads of it.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait until *count >= target (a counter other CTAs raise with
+// release semantics). On the limit: sets the CTA's abort flag, flags
+// MOE_DEVSTAT_TIMEOUT and returns false; returns false at once if another
+// thread of the CTA has aborted.
+__device__ __forceinline__ bool wait_count(const int32_t* count, int32_t target, volatile int* abort_flag,
+                                           int32_t* status, uint64_t limit_ns) {
+  if (ld_acquire_gpu(count) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    __nanosleep(200);
+    if (ld_acquire_gpu(count) >= target) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      flag_status(status, MOE_DEVSTAT_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // E4M3 code of v (round to nearest even, saturate to +-448).
 __device__ __forceinline__ uint8_t to_e4m3(float v) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));

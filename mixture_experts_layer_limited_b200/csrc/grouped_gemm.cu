@@ -49,6 +49,7 @@ constexpr int kThreads = 192;
 struct TileInfo {
   int g, mb, row0, n_valid, N;
   int ntb;              // token blocks of this segment
+  int tb;               // this tile's token block in the segment
 };
 
 // Token blocks per rasterisation chunk: inside a segment, tiles run in chunks
@@ -57,10 +58,17 @@ struct TileInfo {
 // and the chunk's token blocks (L2).
 constexpr int kTbChunk = 8;
 
-// Per-CTA copy of the tile schedule: tile_start[g] = first tile of group g.
+// Pipeline stages of 64 K: bf16 (64 KB each), E4M3.
+constexpr int kBf16Stages = 3;
+constexpr int kE4m3Stages = 4;
+
+// Per-CTA copy of the tile schedule: tb_start[g] = first token block of
+// group g (over all groups), tile_start[g] = its first tile (tb_start[g] x
+// the problem's weight blocks).
 struct Sched {
   int tile_start[kMaxGroups + 1];
   int seg_start[kMaxGroups + 1];
+  int tb_start[kMaxGroups + 1];
 };
 
 __device__ __forceinline__ int tiles_of(int n, int bn_max, int n_mblk) {
@@ -82,7 +90,7 @@ __device__ void build_schedule(Sched& s, const GemmArgs& a, int lane) {
         n = a.rows;
       }
     }
-    int t = (g < a.groups) ? tiles_of(n, a.bn_max, a.n_mblk) : 0;
+    int t = (g < a.groups) ? tiles_of(n, a.bn_max, 1) : 0;   // token blocks
     int incl = t;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -90,13 +98,15 @@ __device__ void build_schedule(Sched& s, const GemmArgs& a, int lane) {
       if (lane >= d) incl += v;
     }
     if (g < a.groups) {
-      s.tile_start[g] = carry + incl - t;
+      s.tb_start[g] = carry + incl - t;
+      s.tile_start[g] = (carry + incl - t) * a.n_mblk;
       s.seg_start[g] = st;
     }
     carry += __shfl_sync(0xffffffffu, incl, 31);
   }
   if (lane == 0) {
-    s.tile_start[a.groups] = carry;
+    s.tb_start[a.groups] = carry;
+    s.tile_start[a.groups] = carry * a.n_mblk;
     s.seg_start[a.groups] = a.offsets ? a.offsets[a.groups] : a.rows;
   }
 }
@@ -114,6 +124,7 @@ __device__ __forceinline__ TileInfo decode_in_segment(const GemmArgs& a, int g, 
   ti.mb = r / c_tb;
   const int tb = chunk * kTbChunk + (r - ti.mb * c_tb);
   ti.ntb = ntb;
+  ti.tb = tb;
   ti.row0 = seg0 + tb * bn;
   ti.n_valid = min(bn, n - tb * bn);
   ti.N = ((ti.n_valid + 15) / 16) * 16;
@@ -128,6 +139,19 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, const GemmArgs& 
   }
   return decode_in_segment(a, lo, s.seg_start[lo], s.seg_start[lo + 1] - s.seg_start[lo],
                            t - s.tile_start[lo]);
+}
+
+// Tile t of problem a over the schedule's segments when a's weight blocks per
+// group differ from those the schedule was built with (its token blocks are
+// the same: same offsets and bn_max).
+__device__ __forceinline__ TileInfo decode_tile_nb(const Sched& s, const GemmArgs& a, int t) {
+  int lo = 0, hi = a.groups - 1;   // last g with tb_start[g] * n_mblk <= t
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (s.tb_start[mid] * a.n_mblk <= t) lo = mid; else hi = mid - 1;
+  }
+  return decode_in_segment(a, lo, s.seg_start[lo], s.seg_start[lo + 1] - s.seg_start[lo],
+                           t - s.tb_start[lo] * a.n_mblk);
 }
 
 // Token rows of one stage (a multiple of 16, at most 256) are fetched with at
@@ -459,6 +483,273 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
 }
 
 // ========================================================================
+// Both GEMMs of the SwiGLU experts in one persistent launch (bf16)
+// ========================================================================
+// Tiles in order: shared gate/up, routed gate/up, shared down, routed down,
+// each problem rasterised as in the kernel above, all on 256-token tiles with
+// one accumulator pair and 12 epilogue warps. The CTAs take tiles from a
+// global counter, in order, so the work is shared out to the end (a CTA
+// whose tiles ran fast takes more) and the down tiles start on the SMs that
+// finish their gate/up share first. A down tile reads the h rows of one
+// token block: the gate/up epilogue warps, after storing their part of a
+// tile, fence and add 1 to that token block's counter, and the down tile's
+// producer waits (bounded) for n_mblk(gate/up) x 4 x kGuQ arrivals, then
+// fences the async proxy before its TMA loads of those rows. Tiles are
+// handed out in increasing order and a producer only waits after issuing
+// every load of its earlier tiles, so each awaited gate/up tile completes.
+// The tile a stage holds travels with the stage (stage_tile), the tile in
+// the accumulator from the MMA warp to the epilogue warps (acc_tile,
+// tile_bar); -1 marks the end.
+__global__ void __launch_bounds__(64 + 32 * kFfnEpiWarps, 1)
+grouped_ffn_bf16_kernel(const __grid_constant__ FfnArgs f) {
+  constexpr int EPIW = kFfnEpiWarps;
+  constexpr int STAGES = kBf16Stages;
+  constexpr int KB = 64;
+  constexpr uint32_t A_SUB_BYTES = 128 * 128;
+  constexpr uint32_t sub_cols = 256u;
+  extern __shared__ __align__(1024) uint8_t dsmem[];
+  __shared__ Sched sched;
+  __shared__ __align__(16) __nv_bfloat16 stage_out[EPIW][32 * 32];
+  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
+  __shared__ uint64_t tmem_full, tmem_empty, drain_bar, tile_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int issued_parity[STAGES];
+  __shared__ int stage_tile[STAGES];
+  __shared__ int acc_tile;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const GemmArgs& gr = f.g[1];                       // routed gate/up: the schedule's segments
+  int32_t* status = gr.status;
+  const uint64_t wait_ns = gr.wait_ns;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  const uint32_t stage_bytes = 2 * A_SUB_BYTES + static_cast<uint32_t>(gr.bn_max) * 128u;
+  auto sA = [&](int st, int sub) { return smem + st * stage_bytes + sub * A_SUB_BYTES; };
+  auto sB = [&](int st) { return smem + st * stage_bytes + 2 * A_SUB_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+      issued_parity[i] = -1;
+    }
+    mbar_init(&tmem_full, 1);
+    mbar_init(&tmem_empty, 32 * EPIW);
+    mbar_init(&drain_bar, 1);
+    mbar_init(&tile_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int p = 0; p < 4; ++p) {
+      tma_prefetch_desc(&f.tmA[p]);
+      for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&f.tmB[p].box[i]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, 512);
+    tmem_relinquish();
+  }
+  if (warp == 2) build_schedule(sched, gr, lane);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int tb_routed = sched.tb_start[gr.groups];
+  // first tile of problems 1, 2, 3, and the total
+  const int first1 = tiles_of(f.g[0].rows, f.g[0].bn_max, f.g[0].n_mblk);
+  const int first2 = first1 + tb_routed * f.g[1].n_mblk;
+  const int first3 = first2 + tiles_of(f.g[2].rows, f.g[2].bn_max, f.g[2].n_mblk);
+  const int total = first3 + tb_routed * f.g[3].n_mblk;
+  // problem of tile t, its tile info and its token block's counter
+  auto locate = [&](int t, int& p, TileInfo& ti) -> int {
+    p = t < first1 ? 0 : t < first2 ? 1 : t < first3 ? 2 : 3;
+    const int base = p == 0 ? 0 : p == 1 ? first1 : p == 2 ? first2 : first3;
+    const GemmArgs& g = f.g[p];
+    if (p == 0 || p == 2) {
+      ti = decode_in_segment(g, 0, 0, g.rows, t - base);
+      return f.shared_base + ti.tb;
+    }
+    ti = decode_tile_nb(sched, g, t - base);
+    return sched.tb_start[ti.g] + ti.tb;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_once = policy_evict_first();
+      const uint64_t pol_reuse = policy_evict_normal();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int next = atomicAdd(f.tile_counter, 1);
+      while (next < total && !abort_flag) {
+        const int t = next;
+        int p;
+        TileInfo ti;
+        const int idx = locate(t, p, ti);
+        const GemmArgs& g = f.g[p];
+        if (p >= 2) {                                  // h rows of this token block stored and visible
+          const int32_t target = f.g[p - 2].n_mblk * 4 * kGuQ;
+          if (!wait_count(f.ready + idx, target, &abort_flag, status, wait_ns)) break;
+          fence_proxy_async_global();
+        }
+        const int nk = g.K / KB;
+        const CUtensorMap* mA = &f.tmA[p];
+        const TokenMaps* mB = &f.tmB[p];
+        const int a_row0 = ti.g * g.a_rows_per_group + ti.mb * g.mblk_stride;
+        const int a_row1 = a_row0 + g.sub1_off;
+        const bool one_box = g.a_one_box != 0;
+        const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;
+        const uint32_t bytes = 2 * A_SUB_BYTES + static_cast<uint32_t>(ti.N) * 128u;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, status, wait_ns)) { ok = false; break; }
+          stage_tile[stage] = t;
+          mbar_arrive_expect_tx(&full_bar[stage], bytes);
+          tma_load_2d(sA(stage, 0), mA, &full_bar[stage], kb * KB, a_row0, pol_w);
+          if (!one_box) tma_load_2d(sA(stage, 1), mA, &full_bar[stage], kb * KB, a_row1, pol_w);
+          uint8_t* bdst = sB(stage);
+          uint64_t* fb = &full_bar[stage];
+          load_token_rows(ti.N, [&](int which, int off) {
+            tma_load_2d(bdst + off * 128, &mB->box[which], fb, kb * KB, ti.row0 + off, pol_x);
+          });
+          issued_parity[stage] = static_cast<int>(phase);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (kb == nk - 1) next = atomicAdd(f.tile_counter, 1);   // the next tile, claimed as this one's
+        }                                                           // last stage is queued
+        if (!ok) break;
+      }
+      // the end marker: one more stage, no data
+      if (!abort_flag && mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, status, wait_ns)) {
+        stage_tile[stage] = -1;
+        mbar_arrive(&full_bar[stage]);
+      }
+      if (abort_flag) {   // let every issued copy land before the CTA exits
+        for (int i = 0; i < STAGES; ++i)
+          if (issued_parity[i] >= 0) mbar_wait_drain(&full_bar[i], static_cast<uint32_t>(issued_parity[i]));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (uint32_t it = 0;; ++it) {
+        // the tile whose k-blocks come next: its first stage names it
+        if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, wait_ns)) break;
+        const int t = stage_tile[stage];
+        if (!mbar_wait(&tmem_empty, (it & 1u) ^ 1u, &abort_flag, status, wait_ns)) break;
+        acc_tile = t;
+        mbar_arrive(&tile_bar);
+        if (t < 0) break;
+        int p;
+        TileInfo ti;
+        locate(t, p, ti);
+        const int nk = f.g[p].K / KB;
+        const uint32_t idesc = make_idesc(1u, 128u, static_cast<uint32_t>(ti.N));
+        const uint32_t d0 = tmem_base;
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (kb > 0 && !mbar_wait(&full_bar[stage], phase, &abort_flag, status, wait_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA(stage, 0)), a1 = smem_u32(sA(stage, 1));
+          const uint32_t b0 = smem_u32(sB(stage));
+#pragma unroll
+          for (int kk = 0; kk < KB / 16; ++kk) {
+            const uint32_t acc = (kb | kk) != 0;
+            const uint64_t bd = sw128_desc(b0 + kk * 32);
+            umma_bf16(d0, sw128_desc(a0 + kk * 32), bd, idesc, acc);
+            umma_bf16(d0 + sub_cols, sw128_desc(a1 + kk * 32), bd, idesc, acc);
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tmem_full);
+      }
+      // all issued MMAs must finish before TMEM is released
+      umma_commit(&drain_bar);
+      mbar_wait_drain(&drain_bar, 0);
+    }
+  } else {
+    // epilogue warps 2 .. 13: warp w reads TMEM lanes 32*(w%4)..+31; down
+    // tiles: every third 32-token chunk from (w-2)/4; gate/up tiles: the
+    // warps with (w-2)/4 < kGuQ, every kGuQ-th chunk
+    const int q = warp & 3;
+    const int c0 = (warp - 2) / 4;
+    constexpr int cstep = EPIW / 4;
+    constexpr int kEpiChunks = (8 + cstep - 1) / cstep;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    __nv_bfloat16* stg = stage_out[warp - 2];
+    for (uint32_t it = 0;; ++it) {
+      if (!mbar_wait(&tile_bar, it & 1u, &abort_flag, status, wait_ns)) break;
+      const int t = acc_tile;
+      if (t < 0) break;
+      int p;
+      TileInfo ti;
+      const int idx = locate(t, p, ti);
+      const GemmArgs& g = f.g[p];
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out);
+      const size_t out_ld = g.out_ld;
+      const int nchunk = (ti.N + 31) / 32;
+      float wpre[kEpiChunks];
+      if (p >= 2) {                                    // down: routing weights fetched ahead
+#pragma unroll
+        for (int u = 0; u < kEpiChunks; ++u) {
+          const int r = (c0 + u * cstep) * 32 + lane;
+          const bool valid = c0 + u * cstep < nchunk && r < ti.n_valid;
+          wpre[u] = (g.row_w && valid) ? __ldg(g.row_w + ti.row0 + r) : 0.0f;
+        }
+      }
+      if (!mbar_wait(&tmem_full, it & 1u, &abort_flag, status, wait_ns)) break;
+      tc_fence_after();
+      if (p < 2) {
+        const int feat0 = ti.mb * g.feat_stride + 32 * q;
+        for (int c = c0 < kGuQ ? c0 : nchunk; c < nchunk; c += kGuQ) {
+          float gv[32], uv[32];
+          tmem_ld32(lane_addr + c * 32, gv);
+          tmem_ld32(lane_addr + sub_cols + c * 32, uv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) gv[j] = silu(gv[j]) * uv[j];
+          store_tile<32>(stg, gv, lane, out, out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
+        }
+      } else {
+#pragma unroll 1
+        for (int s = 0; s < 2; ++s) {
+          const int feat0 = ti.mb * g.feat_stride + s * g.feat_sub1 + 32 * q;
+#pragma unroll
+          for (int u = 0; u < kEpiChunks; ++u) {
+            const int c = c0 + u * cstep;
+            if (c >= nchunk) break;                                  // warp-uniform
+            float v[32];
+            tmem_ld32(lane_addr + s * sub_cols + c * 32, v);
+            tmem_ld_wait();
+            if (g.row_w) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] *= __shfl_sync(0xffffffffu, wpre[u], j);
+            }
+            store_tile<32>(stg, v, lane, out, out_ld, ti.row0 + c * 32, ti.n_valid - c * 32, feat0);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tmem_empty);
+      if (p < 2 && c0 < kGuQ) {                        // this warp's part of the h tile is stored
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(f.ready + idx, 1);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+// ========================================================================
 // E4M3 kernel (block-scaled, promotion on CUDA cores), tokens per tile <= 32
 // ========================================================================
 constexpr int kF8Bn = 32;          // max tokens per tile
@@ -687,9 +978,6 @@ grouped_gemm_e4m3_kernel(const __grid_constant__ CUtensorMap tmA,
 // ------------------------------------------------------------------------
 // host-side launch helpers (called from api.cu)
 // ------------------------------------------------------------------------
-constexpr int kBf16Stages = 3;
-constexpr int kE4m3Stages = 4;
-
 size_t gemm_bf16_smem_bytes(int bn_max) {
   return static_cast<size_t>(kBf16Stages) * (2 * 128 * 128 + static_cast<size_t>(bn_max) * 128) + 1024;
 }
@@ -739,6 +1027,15 @@ cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, cons
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, smem, stream>>>(tmA, tmB.box[0], a);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ffn_bf16(const FfnArgs& f, int grid, cudaStream_t stream) {
+  const size_t smem = gemm_bf16_smem_bytes(f.g[1].bn_max);
+  cudaError_t e = cudaFuncSetAttribute(grouped_ffn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  grouped_ffn_bf16_kernel<<<grid, 64 + 32 * kFfnEpiWarps, smem, stream>>>(f);
   return cudaGetLastError();
 }
 

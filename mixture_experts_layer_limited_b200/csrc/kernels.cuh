@@ -71,6 +71,25 @@ struct SecondProblem {
 cudaError_t launch_grouped_gemm(bool e4m3, int epi, const CUtensorMap& tmA, const TokenMaps& tmB,
                                 const GemmArgs& a, int grid, cudaStream_t stream,
                                 const SecondProblem* two = nullptr);
+
+// Both bf16 GEMMs of the SwiGLU experts, routed and shared, in one persistent
+// launch: g[0] shared gate/up, g[1] routed gate/up, g[2] shared down, g[3]
+// routed down (g[1] and g[3] share offsets; all four bn_max = 256). ready:
+// one int32 counter per token block, zeroed before the launch: routed token
+// blocks from 0, the shared problem's from shared_base; tile_counter: the
+// next tile to hand out, zeroed before the launch.
+struct FfnArgs {
+  CUtensorMap tmA[4];
+  TokenMaps tmB[4];
+  GemmArgs g[4];
+  int32_t* ready;
+  int32_t* tile_counter;
+  int32_t shared_base;
+};
+static_assert(sizeof(FfnArgs) <= 4096, "FfnArgs must fit the kernel parameter space");
+constexpr int kFfnEpiWarps = 12;
+constexpr int kGuQ = 1;       // epilogue warps per TMEM lane quarter on the gate/up tiles
+cudaError_t launch_ffn_bf16(const FfnArgs& f, int grid, cudaStream_t stream);
 // route: also route the tokens in the same launch where the shape allows
 // (route8_experts_per_thread(r) > 0); counts must be zeroed beforehand. The
 // split of the hidden size over a cluster's CTAs depends on T and num_sms only,

@@ -40,7 +40,7 @@ class MoELayer:
     def __init__(self, spec: LayerSpec, gate: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
                  sw13: Optional[torch.Tensor], sw2: Optional[torch.Tensor],
                  bias: Optional[torch.Tensor], T_max: int, gather: bool = False,
-                 fuse_shared: bool = True, fuse_combine: bool = False):
+                 fuse_shared: bool = True, fuse_combine: bool = False, fuse_ffn: bool = True):
         self.spec = spec
         # gather=True: bf16 layers read the routed experts' token rows straight
         # from x (the permutation fused into the first GEMM; no x_perm). At the
@@ -51,6 +51,11 @@ class MoELayer:
         # fuse_combine: the combine runs inside the down GEMM (atomic fp32 adds
         # into a [T, H] accumulator); measured slower at the V3 shape, so off
         self.fuse_combine = fuse_combine and spec.dtype != "e4m3"
+        # fuse_ffn: bf16 layers with a shared expert run both GEMMs (routed and
+        # shared) as one persistent launch, down tiles starting as soon as
+        # their token block's h rows are stored
+        self.fuse_ffn = (fuse_ffn and spec.dtype != "e4m3" and fuse_shared and not self.gather
+                         and not self.fuse_combine and spec.I_s > 0 and sw13 is not None)
         dev = gate.device
         self.dev = dev
         self.gate = gate.contiguous()
@@ -107,6 +112,11 @@ class MoELayer:
             self.sh_o = z(T_max, H, dt=bf)
         else:
             self.sh_h = self.sh_o = None
+        if self.fuse_ffn:
+            n = N.moe_swiglu_ffn_sync_size(R, E, T_max)
+            self.ffn_ws = z((n + 15) // 16 * 16, dt=torch.uint8)
+        else:
+            self.ffn_ws = None
 
     def _quant_blocks(self, w):
         B, Nr, K = w.shape
@@ -203,6 +213,15 @@ class MoELayer:
             h_scale=self.h_s[:R] if self.fp8 else None, sw2_scale=self.sw2_s,
             sh_h_scale=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status)
 
+    def ffn_with_shared(self, x: torch.Tensor, T: int):
+        """Both GEMMs of the routed experts and of the shared expert in one launch."""
+        s = self.spec
+        R = T * s.k
+        N.moe_swiglu_ffn_with_shared(
+            R, s.H, self.w13, self.w2, s.E, s.I, self.x_perm[:R], self.offsets, self.row_w[:R], self.h[:R],
+            self.o[:R], T, self.sw13, self.sw2, s.I_s, x, self.sh_h[:T], self.sh_o[:T], self.ffn_ws,
+            dev_status=self.status)
+
     def down_with_combine(self, T: int):
         """The routed and shared down GEMMs with the combine in their epilogue."""
         s = self.spec
@@ -232,7 +251,10 @@ class MoELayer:
                     st.append(("gate_up_shared", lambda: self.shared_gate_up(x, T)))
             st.append(("down_combine", lambda: self.down_with_combine(T)))
             return st
-        if self.sh_h is not None and self.fuse_shared and not self.gather:
+        if self.fuse_ffn:
+            # routed + shared expert, both GEMMs, one launch
+            st.append(("ffn", lambda: self.ffn_with_shared(x, T)))
+        elif self.sh_h is not None and self.fuse_shared and not self.gather:
             # routed + shared expert in one launch per GEMM
             st += [("gate_up", lambda: self.gate_up_with_shared(x, T)),
                    ("down", lambda: self.down_with_shared(T))]

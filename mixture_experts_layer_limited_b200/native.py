@@ -30,6 +30,7 @@ EXPORTED = [
     "moe_grouped_swiglu",
     "moe_gate_up_swiglu", "moe_gate_up_swiglu_gather", "moe_down_proj",
     "moe_gate_up_swiglu_with_shared", "moe_down_proj_with_shared", "moe_down_proj_combine",
+    "moe_swiglu_ffn_sync_size", "moe_swiglu_ffn_with_shared",
     "moe_combine", "moe_bias_update", "moe_aux_loss_workspace_size", "moe_aux_loss",
     "moe_quantize_blocks", "moe_quantize_rows",
     "moe_read_device_status", "moe_last_cuda_error", "moe_status_string", "moe_abi_version",
@@ -86,6 +87,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
                                            _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P, _P],
         "moe_down_proj_with_shared": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P,
                                       _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P],
+        "moe_swiglu_ffn_sync_size": [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
+        "moe_swiglu_ffn_with_shared": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P,
+                                       _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, ctypes.c_size_t,
+                                       _P, _P],
         "moe_down_proj_combine": [_I, _I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P,
                                   ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P],
         "moe_combine": [_I, _I, _I, _P, _P, _P, _P, _P, _P],
@@ -224,6 +229,24 @@ def moe_down_proj_with_shared(rows, H, w2, dtype, groups, I, h, offsets, row_w, 
         rows, H, ctypes.byref(w), _ptr(h), _ptr(h_scale), _ptr(offsets), _ptr(row_w), _ptr(out),
         sh_rows, ctypes.byref(sw), _ptr(sh_h), _ptr(sh_h_scale), _ptr(sh_out),
         _ptr(dev_status), _stream(stream)))
+
+
+def moe_swiglu_ffn_sync_size(rows, groups, sh_rows):
+    n = ctypes.c_size_t(0)
+    _check("moe_swiglu_ffn_sync_size", load_library().moe_swiglu_ffn_sync_size(rows, groups, sh_rows,
+                                                                               ctypes.byref(n)))
+    return n.value
+
+
+def moe_swiglu_ffn_with_shared(rows, H, w13, w2, groups, I, a, offsets, row_w, h_ws, out,
+                               sh_rows, sw13, sw2, I_s, sh_a, sh_h_ws, sh_out, sync_ws,
+                               dev_status=None, stream=None):
+    w = FFNWeights(_ptr(w13), _ptr(w2), None, None, MOE_BF16, groups, I)
+    sw = FFNWeights(_ptr(sw13), _ptr(sw2), None, None, MOE_BF16, 1, I_s)
+    _check("moe_swiglu_ffn_with_shared", load_library().moe_swiglu_ffn_with_shared(
+        rows, H, ctypes.byref(w), _ptr(a), _ptr(offsets), _ptr(row_w), _ptr(h_ws), _ptr(out),
+        sh_rows, ctypes.byref(sw), _ptr(sh_a), _ptr(sh_h_ws), _ptr(sh_out),
+        _ptr(sync_ws), sync_ws.numel() * sync_ws.element_size(), _ptr(dev_status), _stream(stream)))
 
 
 def moe_down_proj_combine(rows, T, H, w2, groups, I, h, offsets, row_w, src_token, sw2, I_s, sh_h,

@@ -18,7 +18,7 @@ import torch
 from .layer import MoELayer
 
 # stages that read the forward's input x, and the stage that writes its output y
-_READS_X = ("route", "permute", "gate_up", "gate_up_routed", "gate_up_shared")
+_READS_X = ("route", "permute", "gate_up", "gate_up_routed", "gate_up_shared", "ffn")
 _WRITES_Y = ("combine", "down_combine")
 
 

@@ -508,6 +508,72 @@ def test_routed_and_shared_in_one_launch(H, I, I_s, sizes, T):
     assert errs[0] < 1e-2 and errs[2] < 1e-2 and errs[1] < BF16_TOL and errs[3] < BF16_TOL
 
 
+@pytest.mark.parametrize("H,I,I_s,sizes,T", [
+    (512, 256, 384, [0, 17, 300, 5, 256, 0, 129], 300),
+    (7168, 2048, 2048, [2100, 0, 17, 260, 513], 1000),
+    (2048, 1408, 2816, [384, 0, 5, 513], 129),
+])
+def test_swiglu_ffn_one_launch_equals_two_launches(H, I, I_s, sizes, T):
+    """moe_swiglu_ffn_with_shared runs both GEMMs, routed and shared, in one
+    launch whose down tiles wait on per-token-block counters of the gate/up
+    tiles: h, out, shared h and shared out must be bit-identical to
+    moe_gate_up_swiglu_with_shared followed by moe_down_proj_with_shared
+    (segments over 8 token blocks, empty segments, I_s != I), and out within
+    the bf16 tolerance of the oracle. Run twice on the same scratch: the
+    counters are zeroed by each call."""
+    G = len(sizes)
+    off = _segments(sizes)
+    R = int(off[-1])
+    g = _gen(H + I + I_s + T + 1)
+    xp = torch.randn(R, H, generator=g, device=DEV).to(torch.bfloat16)
+    x = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
+    w13 = (torch.randn(G, 2 * I, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w2 = (torch.randn(G, H, I, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    sw13 = (torch.randn(1, 2 * I_s, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    sw2 = (torch.randn(1, H, I_s, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    row_w = torch.rand(R, generator=g, device=DEV) + 0.5
+    offd = torch.from_numpy(off).to(DEV)
+    e = lambda *shape: torch.empty(*shape, dtype=torch.bfloat16, device=DEV)
+    h, sh_h, o, sh_o = e(R, I), e(T, I_s), e(R, H), e(T, H)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    N.moe_gate_up_swiglu_with_shared(R, H, w13, N.MOE_BF16, G, I, xp, offd, h, T, sw13, I_s, x, sh_h,
+                                     dev_status=status)
+    N.moe_down_proj_with_shared(R, H, w2, N.MOE_BF16, G, I, h, offd, row_w, o, T, sw2, I_s, sh_h, sh_o,
+                                dev_status=status)
+    sync = torch.empty(N.moe_swiglu_ffn_sync_size(R, G, T), dtype=torch.uint8, device=DEV)
+    for _ in range(2):
+        h2, sh_h2, o2, sh_o2 = e(R, I), e(T, I_s), e(R, H), e(T, H)
+        N.moe_swiglu_ffn_with_shared(R, H, w13, w2, G, I, xp, offd, row_w, h2, o2, T, sw13, sw2, I_s, x,
+                                     sh_h2, sh_o2, sync, dev_status=status)
+        assert N.moe_read_device_status(status) == 0
+        for got, ref, name in ((h2, h, "h"), (sh_h2, sh_h, "shared h"), (o2, o, "out"), (sh_o2, sh_o, "shared out")):
+            assert torch.equal(got, ref), f"{name} differs from the two launches"
+    ref, _ = _ref_grouped(xp, w13, w2, off, row_w)
+    assert rel_err(np64(o2), ref) < BF16_TOL
+
+
+def test_swiglu_ffn_rejects_e4m3_and_short_scratch():
+    """The one-launch FFN is bf16 only, and its scratch must hold a counter
+    per token block (checked on the host, nothing launched)."""
+    R, H, I, T, G = 64, 256, 128, 16, 4
+    z = lambda *shape, dt=torch.bfloat16: torch.zeros(*shape, dtype=dt, device=DEV)
+    offd = torch.tensor([0, 16, 32, 48, 64], dtype=torch.int32, device=DEV)
+    args = [R, H, z(G, 2 * I, H), z(G, H, I), G, I, z(R, H), offd, None, z(R, I), z(R, H), T,
+            z(1, 2 * I, H), z(1, H, I), I, z(T, H), z(T, I), z(T, H)]
+    n = N.moe_swiglu_ffn_sync_size(R, G, T)
+    with pytest.raises(N.MoEError):
+        N.moe_swiglu_ffn_with_shared(*args, torch.empty(n - 4, dtype=torch.uint8, device=DEV))
+    lib = N.load_library()
+    w = N.FFNWeights(args[2].data_ptr(), args[3].data_ptr(), None, None, N.MOE_E4M3, G, I)
+    sw = N.FFNWeights(args[12].data_ptr(), args[13].data_ptr(), None, None, N.MOE_E4M3, 1, I)
+    sync = torch.empty(n, dtype=torch.uint8, device=DEV)
+    st = lib.moe_swiglu_ffn_with_shared(R, H, ctypes.byref(w), args[6].data_ptr(), offd.data_ptr(), None,
+                                        args[9].data_ptr(), args[10].data_ptr(), T, ctypes.byref(sw),
+                                        args[15].data_ptr(), args[16].data_ptr(), args[17].data_ptr(),
+                                        sync.data_ptr(), n, None, None)
+    assert st != 0
+
+
 def test_grouped_swiglu_bf16_single_group_no_offsets():
     rows, H, I = 300, 512, 384
     g = _gen(77)
