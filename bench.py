@@ -49,8 +49,11 @@ def parse_args():
                          "of the hottest and the coldest expert)")
     ap.add_argument("--fuse-combine", action="store_true",
                     help="run the combine inside the down GEMM (atomic fp32 scatter-add) instead of after it")
-    ap.add_argument("--split-ffn", action="store_true",
-                    help="run the experts' two GEMMs as two launches (gate/up, then down) instead of one")
+    ffn = ap.add_mutually_exclusive_group()
+    ffn.add_argument("--split-ffn", action="store_true",
+                     help="always run the experts' two GEMMs as two launches (gate/up, then down)")
+    ffn.add_argument("--fuse-ffn", action="store_true",
+                     help="always run them as one launch (default: one launch from 512 routed rows per expert)")
     ap.add_argument("--routing-sweep", action="store_true",
                     help="instead of the throughput line: load CV, aux loss and router time for "
                          "topk_group 8/4/2/1 of 8 groups on the V3 and skewed inputs (one line each)")
@@ -350,7 +353,7 @@ def run_ours(args):
         g.manual_seed(cfg.seed + 100003 * rank)
         inp.x = torch.randn(cfg.T, cfg.H, generator=g, device="cuda").to(torch.bfloat16)
     layer = MoELayer(LayerSpec.from_config(cfg), inp.gate, inp.w13, inp.w2, inp.sw13, inp.sw2,
-                     inp.bias, cfg.T, fuse_combine=args.fuse_combine, fuse_ffn=not args.split_ffn)
+                     inp.bias, cfg.T, fuse_combine=args.fuse_combine, fuse_ffn=False if args.split_ffn else (True if args.fuse_ffn else None))
     T_global = cfg.T * world
     stream = torch.cuda.current_stream()
     stages = layer.stages(inp.x)

@@ -40,7 +40,7 @@ class MoELayer:
     def __init__(self, spec: LayerSpec, gate: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
                  sw13: Optional[torch.Tensor], sw2: Optional[torch.Tensor],
                  bias: Optional[torch.Tensor], T_max: int, gather: bool = False,
-                 fuse_shared: bool = True, fuse_combine: bool = False, fuse_ffn: bool = True):
+                 fuse_shared: bool = True, fuse_combine: bool = False, fuse_ffn: Optional[bool] = None):
         self.spec = spec
         # gather=True: bf16 layers read the routed experts' token rows straight
         # from x (the permutation fused into the first GEMM; no x_perm). At the
@@ -52,10 +52,14 @@ class MoELayer:
         # into a [T, H] accumulator); measured slower at the V3 shape, so off
         self.fuse_combine = fuse_combine and spec.dtype != "e4m3"
         # fuse_ffn: bf16 layers with a shared expert run both GEMMs (routed and
-        # shared) as one persistent launch, down tiles starting as soon as
-        # their token block's h rows are stored
-        self.fuse_ffn = (fuse_ffn and spec.dtype != "e4m3" and fuse_shared and not self.gather
-                         and not self.fuse_combine and spec.I_s > 0 and sw13 is not None)
+        # shared) as one persistent launch on a dynamic tile counter, down
+        # tiles starting as soon as their token block's h rows are stored.
+        # None: by shape, per forward: when the routed rows average at least
+        # two full 256-row token blocks per expert (measured on B200: 11 %
+        # faster at 1024 rows per expert, level at 256 and 384)
+        self.fuse_ffn = fuse_ffn
+        self.ffn_ok = (fuse_ffn is not False and spec.dtype != "e4m3" and fuse_shared and not self.gather
+                       and not self.fuse_combine and spec.I_s > 0 and sw13 is not None)
         dev = gate.device
         self.dev = dev
         self.gate = gate.contiguous()
@@ -112,7 +116,7 @@ class MoELayer:
             self.sh_o = z(T_max, H, dt=bf)
         else:
             self.sh_h = self.sh_o = None
-        if self.fuse_ffn:
+        if self.ffn_ok:
             n = N.moe_swiglu_ffn_sync_size(R, E, T_max)
             self.ffn_ws = z((n + 15) // 16 * 16, dt=torch.uint8)
         else:
@@ -251,7 +255,7 @@ class MoELayer:
                     st.append(("gate_up_shared", lambda: self.shared_gate_up(x, T)))
             st.append(("down_combine", lambda: self.down_with_combine(T)))
             return st
-        if self.fuse_ffn:
+        if self.ffn_ok and (self.fuse_ffn or T * self.spec.k >= 512 * self.spec.E):
             # routed + shared expert, both GEMMs, one launch
             st.append(("ffn", lambda: self.ffn_with_shared(x, T)))
         elif self.sh_h is not None and self.fuse_shared and not self.gather:
