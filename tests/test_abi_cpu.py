@@ -48,6 +48,32 @@ def test_workspace_size_is_host_only():
         N.moe_permute_workspace_size(0, 8, 256)
 
 
+def test_ffn_sync_size_and_host_validation():
+    """The one-launch FFN's scratch: an int32 counter per possible token block
+    of the routed rows (one partial block per group at most) and of the
+    shared rows, plus the tile counter; short, misaligned or missing scratch
+    and a non-bf16 layer are rejected on the host, before any launch."""
+    R, E, T = 65536, 256, 8192
+    assert N.moe_swiglu_ffn_sync_size(R, E, T) == 4 * ((R + 255) // 256 + E + (T + 255) // 256 + 1)
+    with pytest.raises(N.MoEError):
+        N.moe_swiglu_ffn_sync_size(0, E, T)
+    lib = N.load_library()
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    w = N.FFNWeights(fake, fake, None, None, N.MOE_BF16, 4, 256)
+    sw = N.FFNWeights(fake, fake, None, None, N.MOE_BF16, 1, 256)
+    need = N.moe_swiglu_ffn_sync_size(64, 4, 16)
+
+    def call(sync, nbytes, weights=w):
+        return lib.moe_swiglu_ffn_with_shared(64, 512, ctypes.byref(weights), fake, fake, None, fake, fake,
+                                              16, ctypes.byref(sw), fake, fake, fake, sync, nbytes, None, None)
+    assert call(fake, need - 4) == N.MOE_ERR_INVALID_ARG
+    assert call(None, need) == N.MOE_ERR_INVALID_ARG
+    assert call(P(0x1004), need) == N.MOE_ERR_ALIGNMENT
+    e4 = N.FFNWeights(fake, fake, fake, fake, N.MOE_E4M3, 4, 256)
+    assert call(fake, need, e4) != N.MOE_OK
+
+
 def _raw(lib, fn, *args):
     return getattr(lib, fn)(*args)
 
