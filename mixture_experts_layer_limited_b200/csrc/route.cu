@@ -333,15 +333,16 @@ route_tokens_g8_kernel(const RouteArgs r) {
 }
 
 // ------------------------------------------------------------------------
-// Gate GEMM on CTA pairs, split along K, and (C > 0) the routing of the
-// tile's tokens in the same launch.
+// Gate GEMM on clusters of SPLIT CTAs, split along K, and (C > 0) the
+// routing of the tile's tokens in the same launch.
 // ------------------------------------------------------------------------
 // 512 threads: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer,
 // warps 2..5 read the accumulator (warp w: TMEM lanes 32*(w%4)..+31); after
-// the exchange all sixteen warps route, the CTA's 64 tokens in one pass. The CTAs of a pair start their K loop at
-// a rotation that differs from pair to pair, so the pairs running side by
-// side do not all read the same gate rows at the same moment (each pair
-// still sums its K blocks in one fixed order).
+// the exchange all sixteen warps route the CTA's 128/SPLIT tokens in one
+// pass. The CTAs of a cluster start their K loop at a rotation that differs
+// from cluster to cluster, so the clusters running side by side do not all
+// read the same gate rows at the same moment (each CTA still sums its K
+// blocks in one fixed order).
 constexpr int kGateThreads = 512;
 
 template <int C, int SPLIT>
