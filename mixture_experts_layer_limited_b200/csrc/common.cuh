@@ -282,6 +282,16 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the kernel before it in the stream still
+// runs; griddep_wait() blocks until that kernel has completed and its memory
+// is visible, griddep_launch_dependents() lets the next such kernel start.
+// Both are no-ops for kernels launched the ordinary way.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Orders global-memory data this thread has acquired (written by other SMs
 // with ordinary stores) before its later async-proxy (TMA) reads of it.
 __device__ __forceinline__ void fence_proxy_async_global() {

@@ -31,6 +31,7 @@ constexpr int kHistThreads = 256;
 __global__ void __launch_bounds__(kHistThreads)
 perm_hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int32_t* __restrict__ blockhist,
                  int32_t* __restrict__ local_rank, int32_t* status) {
+  griddep_launch_dependents();                         // the scan may be scheduled now
   constexpr int kWarps = kHistThreads / 32;
   extern __shared__ int hist_dyn[];
   int* cnt = hist_dyn;                                  // [E]: the earlier rounds' slots per expert
@@ -79,6 +80,8 @@ perm_hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int32_t* 
 __global__ void __launch_bounds__(1024)
 perm_scan_kernel(int32_t* __restrict__ blockhist, int nb, int E, int total,
                  int32_t* __restrict__ offsets) {
+  griddep_wait();                                      // the histograms are complete
+  griddep_launch_dependents();                         // the copy kernel's CTAs may start their row loads
   extern __shared__ int sdyn[];
   const int parts = blockDim.x / E;                 // >= 1 (E <= 1024)
   int* part_sum = sdyn;                             // [parts][E]
@@ -207,6 +210,7 @@ perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ top
       if (v < vec_per_row) val[u] = __ldg(src + v);
     }
   }
+  griddep_wait();                                      // ranks and first rows complete
   const int my_row = perm_rows_of_token(t, lane, ids, topk_w, T, k, E, blockbase, slot_to_row, src_token, row_w);
   if (!x_perm) return;                                 // metadata only
   for (int base = 0; base < vec_per_row; base += 256) {   // same trip count on every lane
@@ -258,6 +262,7 @@ perm_place_quant_kernel(const int32_t* __restrict__ ids, const float* __restrict
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;                                  // warp-uniform
+  griddep_wait();                                      // ranks and first rows complete
   const int my_row = perm_rows_of_token(t, lane, ids, topk_w, T, k, E, blockbase, slot_to_row, src_token, row_w);
   if (!x_perm && !x_q) return;                         // metadata only
   const int ntiles = H / 128;
@@ -315,6 +320,25 @@ perm_place_quant_kernel(const int32_t* __restrict__ ids, const float* __restrict
   }
 }
 
+// Launches kern as a programmatic dependent of the kernel before it in the
+// stream (see griddep_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 size_t permute_workspace_bytes(int T, int E) {   // blockhist[nb][E]
   const int nb = (T + kTokBlock - 1) / kTokBlock;
   return static_cast<size_t>(nb) * E * sizeof(int32_t);
@@ -330,19 +354,25 @@ cudaError_t launch_permute(int T, int k, int E, int H, bool x_e4m3, bool perm_e4
       ids, T, k, E, blockhist, slot_to_row, status);
   const int parts = 1024 / E;
   const size_t scan_smem = (static_cast<size_t>(parts) * E + E + 32) * sizeof(int);
-  perm_scan_kernel<<<1, 1024, scan_smem, stream>>>(blockhist, nb, E, T * k, offsets);
+  // the scan and the copy kernel are launched as programmatic dependents: each
+  // may be scheduled before the kernel ahead of it ends, and waits for it
+  // (griddep_wait) before reading its output; the copy kernel's row loads,
+  // which need none, start during the scan
+  cudaError_t e = launch_dependent(perm_scan_kernel, dim3(1), dim3(1024), scan_smem, stream, blockhist, nb, E,
+                                   T * k, offsets);
+  if (e != cudaSuccess) return e;
   const int warps = 8;
-  if (!x_e4m3 && perm_e4m3) {
-    perm_place_quant_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
-        ids, topk_w, T, k, E, blockhist, slot_to_row, src_token, row_w, static_cast<const __nv_bfloat16*>(x), H,
-        static_cast<uint8_t*>(x_perm), x_perm_scale, static_cast<uint8_t*>(x_q), x_q_scale);
-    return cudaGetLastError();
-  }
+  const dim3 grid((T + warps - 1) / warps), block(warps * 32);
+  if (!x_e4m3 && perm_e4m3)
+    return launch_dependent(perm_place_quant_kernel, grid, block, 0, stream, ids, topk_w, T, k, E,
+                            static_cast<const int32_t*>(blockhist), slot_to_row, src_token, row_w,
+                            static_cast<const __nv_bfloat16*>(x), H, static_cast<uint8_t*>(x_perm), x_perm_scale,
+                            static_cast<uint8_t*>(x_q), x_q_scale);
   const int row_bytes = x_e4m3 ? H : 2 * H;
-  perm_place_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
-      ids, topk_w, T, k, E, blockhist, slot_to_row, src_token, row_w, reinterpret_cast<const uint4*>(x),
-      row_bytes / 16, reinterpret_cast<uint4*>(x_perm), x_e4m3 ? x_scale : nullptr, x_perm_scale, H / 128);
-  return cudaGetLastError();
+  return launch_dependent(perm_place_kernel, grid, block, 0, stream, ids, topk_w, T, k, E,
+                          static_cast<const int32_t*>(blockhist), slot_to_row, src_token, row_w,
+                          reinterpret_cast<const uint4*>(x), row_bytes / 16, reinterpret_cast<uint4*>(x_perm),
+                          x_e4m3 ? x_scale : static_cast<const float*>(nullptr), x_perm_scale, H / 128);
 }
 
 }  // namespace moe
