@@ -22,8 +22,8 @@ namespace moe {
 constexpr int kTokBlock = 64;        // tokens per rank block
 
 // 256 threads; the block's slots (token-major, then slot) are taken 256 at a
-// time in order. A slot's rank = its expert's count over the earlier rounds
-// + the counts of the earlier warps of this round + the earlier lanes of its
+// time in order. A slot's rank = its expert's count over the earlier passes
+// + the counts of the earlier warps of this pass + the earlier lanes of its
 // own warp with the same expert (match_any), so equal experts keep slot
 // order: the stable sort's order inside the block.
 constexpr int kHistThreads = 256;
@@ -34,8 +34,8 @@ perm_hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int32_t* 
   griddep_launch_dependents();                         // the scan may be scheduled now
   constexpr int kWarps = kHistThreads / 32;
   extern __shared__ int hist_dyn[];
-  int* cnt = hist_dyn;                                  // [E]: the earlier rounds' slots per expert
-  int* wcnt = hist_dyn + E;                             // [kWarps][E]: this round's slots per warp and expert
+  int* cnt = hist_dyn;                                  // [E]: the earlier passes' slots per expert
+  int* wcnt = hist_dyn + E;                             // [kWarps][E]: this pass's slots per warp and expert
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += kHistThreads) cnt[e] = 0;
   const int s0 = blockIdx.x * kTokBlock * k;
@@ -69,7 +69,7 @@ perm_hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int32_t* 
       for (int w = 0; w < kWarps; ++w) add += wcnt[w * E + x];
       cnt[x] += add;
     }
-    __syncthreads();                                    // wcnt read before the next round clears it
+    __syncthreads();                                    // wcnt read before the next pass clears it
   }
   for (int e = threadIdx.x; e < E; e += kHistThreads)
     blockhist[static_cast<size_t>(blockIdx.x) * E + e] = cnt[e];

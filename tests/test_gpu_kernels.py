@@ -298,7 +298,7 @@ def test_permute_bit_exact(T, k, E, H, skew):
 @pytest.mark.parametrize("T,k,E", [(200, 16, 16), (1000, 4, 4), (129, 8, 256), (64, 16, 1024)])
 def test_permute_repeated_ids_keep_slot_order(T, k, E):
     """ids drawn with replacement, so a token may name one expert in several
-    of its slots, and k = 16 puts a block's slots over several rounds of the
+    of its slots, and k = 16 puts a block's slots over several passes of the
     histogram kernel: rows still follow the stable order, token then slot."""
     rng = np.random.default_rng(T * k + E)
     ids_np = rng.integers(0, E, size=(T, k)).astype(np.int32)
