@@ -47,7 +47,8 @@ def test_every_layer_stage_has_a_launch_count_and_a_cost_model():
         H, E, I, Is, T = cfg.H, cfg.E, cfg.I, cfg.I_s, 4
         z = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
         model = bench.stage_model(cfg)
-        for kw in ({}, {"fuse_shared": False}, {"gather": True}, {"fuse_combine": True}):
+        for kw in ({}, {"fuse_shared": False}, {"gather": True}, {"fuse_combine": True}, {"fuse_ffn": True},
+                   {"fuse_ffn": False}):
             # shapes only: stages() builds the launch closures without running them
             lay = MoELayer(spec, z(E, 8), z(1, 1), z(1, 1), z(1, 1) if Is else None,
                            z(1, 1) if Is else None, None, T, **kw)
@@ -55,6 +56,26 @@ def test_every_layer_stage_has_a_launch_count_and_a_cost_model():
             for n in names:
                 assert n in bench.LAUNCHES and n in model, (name, kw, n)
                 assert bench.launches_of(n, cfg) >= 1
+
+
+def test_one_launch_ffn_is_chosen_from_512_routed_rows_per_expert():
+    """bf16 layers with a shared expert run both GEMMs in one launch when the
+    routed rows average at least two full token blocks per expert (T*k >=
+    512*E), as two launches below; fuse_ffn True / False force either."""
+    sys.path.insert(0, ROOT)
+    import torch
+    from moe_inputs import get_config
+    from mixture_experts_layer_limited_b200 import MoELayer, LayerSpec
+    cfg = get_config("v3")
+    spec = LayerSpec.from_config(cfg)
+    z = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    E, k, H = cfg.E, cfg.k, cfg.H
+    T_max = 512 * E // k                                  # exactly two token blocks per expert
+    for fuse, T, want in ((None, T_max, "ffn"), (None, T_max - 1, "gate_up"), (True, 8, "ffn"),
+                          (False, T_max, "gate_up")):
+        lay = MoELayer(spec, z(E, 8), z(1, 1), z(1, 1), z(1, 1), z(1, 1), None, T_max, fuse_ffn=fuse)
+        names = [n for n, _ in lay.stages(z(T, H))]
+        assert want in names, (fuse, T, names)
 
 
 def test_cpu_sample_holds_every_token_of_the_hottest_and_coldest_expert():
