@@ -256,6 +256,28 @@ def test_layer_shared_expert_in_routed_launches_matches_separate(name):
     assert torch.equal(y0, y1)
 
 
+@pytest.mark.parametrize("name", ["v2lite", "v3", "v3_skewed"])
+def test_layer_one_launch_ffn_matches_two_launches(name):
+    """Both expert GEMMs in one launch (tiles from a counter, down tiles waiting
+    on their token block's gate/up tiles) give the layer output of the two
+    launches bit for bit, at the full sizes of three layers."""
+    cfg = get_config(name)
+    inp = make_inputs(cfg, device=DEV)
+    mk = lambda fuse: MoELayer(LayerSpec.from_config(cfg), inp.gate, inp.w13, inp.w2, inp.sw13, inp.sw2,
+                               inp.bias, cfg.T, fuse_ffn=fuse)
+    one = mk(True)
+    assert any(n == "ffn" for n, _ in one.stages(inp.x))
+    y1 = one.forward(inp.x).clone()
+    torch.cuda.synchronize()
+    assert one.device_status() == 0
+    del one
+    two = mk(False)
+    y2 = two.forward(inp.x)
+    torch.cuda.synchronize()
+    assert two.device_status() == 0
+    assert torch.equal(y1, y2)
+
+
 @pytest.mark.parametrize("name", ["v2lite", "v3"])
 def test_host_pipeline_matches_one_forward_at_a_time(name):
     """HostPipeline overlaps each batch's copies with its neighbours' compute;
