@@ -51,7 +51,7 @@ extern "C" {
 #define MOE_API
 #endif
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 
 typedef int32_t moe_status;
 #define MOE_OK                 0
@@ -238,7 +238,9 @@ MOE_API moe_status moe_permute_static_ws(int32_t T, int32_t k, int32_t E, int32_
  *   rows      number of activation rows (T*k routed, T shared).
  *   H         hidden size (K of the first GEMM, N of the second).
  *   w         weights: w13 [groups, 2I, H], w2 [groups, H, I] (out-major,
- *             i.e. K contiguous). MOE_E4M3 weights carry fp32 block scales
+ *             i.e. K contiguous), or, bf16 with w->tiled = 1, the same
+ *             values in the tiled layout moe_tile_ffn_weights writes.
+ *             MOE_E4M3 weights carry fp32 block scales
  *             w13_scale [groups, 2I/128, H/128], w2_scale [groups, H/128,
  *             I/128] (moe_quantize_blocks).
  *   a         [rows, H] activations: bf16, or e4m3 codes with a_scale
@@ -262,6 +264,7 @@ typedef struct {
     moe_dtype dtype;          /* MOE_BF16 or MOE_E4M3 */
     int32_t groups;
     int32_t I;
+    int32_t tiled;            /* bf16 only: 1 = w13 / w2 in the tiled layout, 0 = row-major */
 } moe_ffn_weights;
 
 MOE_API moe_status moe_grouped_swiglu(int32_t rows, int32_t H, const moe_ffn_weights* w,
@@ -421,6 +424,25 @@ MOE_API moe_status moe_aux_loss_workspace_size(int32_t T, int32_t E, int32_t seq
 MOE_API moe_status moe_aux_loss(int32_t T, int32_t E, int32_t k, int32_t seq_len, int32_t scoring,
                         const float* logits, const int32_t* topk_ids, float alpha, float* aux_out,
                         void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * moe_tile_ffn_weights -- the bf16 expert weights in the layout the grouped
+ * GEMMs stream fastest: each tile the GEMM loads in one step (128 rows of
+ * w13 or 256 rows of w2, by 64 K) is one contiguous 16 / 32 KB block, the
+ * tiles of a row block in K order:
+ *   w13_t[((g*(2I/128) + rb)*(H/64) + kb)*128 + r][c] = w13[g][rb*128 + r][kb*64 + c]
+ *   w2_t [((g*(H/256)  + rb)*(I/64) + kb)*256 + r][c] = w2 [g][rb*256 + r][kb*64 + c]
+ * (c < 64). The values are unchanged, so results are bit-identical to the
+ * row-major weights; pass the tiled copies with w->tiled = 1. The pages
+ * state the weights only as [E, 2I, H] / [E, H, I] matrices; the tiling is
+ * a layout of this library.
+ *   src   row-major weights (src->tiled must be 0, dtype MOE_BF16).
+ *   w13_t / w2_t  device outputs of the same sizes as src->w13 / src->w2 (either
+ *         may be NULL to skip it); they may not overlap the inputs.
+ * Limits: those of moe_grouped_swiglu (I % 128 == 0, H % 256 == 0).
+ * ------------------------------------------------------------------------ */
+MOE_API moe_status moe_tile_ffn_weights(int32_t H, const moe_ffn_weights* src, void* w13_t, void* w2_t,
+                                        void* stream);
 
 /* ------------------------------------------------------------------------ *
  * FP8 E4M3 quantisers ([V3-teardown] §3 infer.toml: weight_block_size

@@ -236,6 +236,8 @@ moe_status check_ffn(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
   if ((need_w13 && !w->w13) || (need_w2 && !w->w2)) return MOE_ERR_INVALID_ARG;
   if (rows < 1 || H < 1 || w->I < 1 || w->groups < 1) return MOE_ERR_INVALID_ARG;
   if (w->dtype != MOE_BF16 && w->dtype != MOE_E4M3) return MOE_ERR_INVALID_ARG;
+  if (w->tiled != 0 && w->tiled != 1) return MOE_ERR_INVALID_ARG;
+  if (w->tiled && w->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (H % 256 != 0 || w->I % 128 != 0 || w->groups > 512) return MOE_ERR_UNSUPPORTED;
   if (w->dtype == MOE_E4M3) {
     if ((need_w13 && !w->w13_scale) || (need_w2 && !w->w2_scale) || !a_scale) return MOE_ERR_INVALID_ARG;
@@ -271,7 +273,9 @@ moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const
                         const int32_t* offsets, void* h_ws, float* h_scale_ws, int32_t* dev_status, GemmPlan* p) {
   const bool fp8 = w->dtype == MOE_E4M3;
   const int I = w->I;
-  moe_status s = make_tmap(&p->tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
+  // tiled weights: a [*, 64] matrix whose 128-row boxes are the tiles
+  moe_status s = w->tiled ? make_tmap(&p->tmA, w->w13, false, 64, static_cast<uint64_t>(w->groups) * 2 * I * (H / 64), 128)
+                          : make_tmap(&p->tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
   if (s != MOE_OK) return s;
   if ((s = make_token_tmaps(&p->tmB, a, fp8, H, rows)) != MOE_OK) return s;
   GemmArgs& g = p->g;
@@ -281,6 +285,7 @@ moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const
   g.groups = w->groups;
   g.offsets = offsets;
   g.a_rows_per_group = 2 * I;            // w13[e]: gate rows [0, I), up rows [I, 2I)
+  g.a_tiled = w->tiled;
   g.n_mblk = I / 128;
   g.mblk_stride = 128;
   g.sub1_off = I;                        // sub-tile 1: the up rows of the same 128 features
@@ -303,7 +308,8 @@ moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
   const bool fp8 = w->dtype == MOE_E4M3;
   const int I = w->I;
   // bf16: a tile's 256 contiguous w2 rows are one TMA box
-  moe_status s = make_tmap(&p->tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H, fp8 ? 128 : 256);
+  moe_status s = w->tiled ? make_tmap(&p->tmA, w->w2, false, 64, static_cast<uint64_t>(w->groups) * H * (I / 64), 256)
+                          : make_tmap(&p->tmA, w->w2, fp8, I, static_cast<uint64_t>(w->groups) * H, fp8 ? 128 : 256);
   if (s != MOE_OK) return s;
   if ((s = make_token_tmaps(&p->tmB, h, fp8, I, rows)) != MOE_OK) return s;
   GemmArgs& g = p->g;
@@ -313,6 +319,7 @@ moe_status plan_down(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
   g.groups = w->groups;
   g.offsets = offsets;
   g.a_rows_per_group = H;
+  g.a_tiled = w->tiled;
   g.n_mblk = H / 256;
   g.mblk_stride = 256;
   g.sub1_off = 128;                      // sub-tiles: w2 rows [mb*256, +128) and [mb*256 + 128, +128)
@@ -394,7 +401,8 @@ moe_status moe_gate_up_swiglu_gather(int32_t rows, int32_t H, const moe_ffn_weig
   const int I = w->I;
   CUtensorMap tmA;
   TokenMaps tmB;
-  s = make_tmap(&tmA, w->w13, false, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
+  s = w->tiled ? make_tmap(&tmA, w->w13, false, 64, static_cast<uint64_t>(w->groups) * 2 * I * (H / 64), 128)
+               : make_tmap(&tmA, w->w13, false, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
   if (s != MOE_OK) return s;
   s = make_token_tmaps(&tmB, x, false, H, T);      // not read: token rows are gathered
   if (s != MOE_OK) return s;
@@ -404,6 +412,7 @@ moe_status moe_gate_up_swiglu_gather(int32_t rows, int32_t H, const moe_ffn_weig
   g1.groups = w->groups;
   g1.offsets = offsets;
   g1.a_rows_per_group = 2 * I;
+  g1.a_tiled = w->tiled;
   g1.n_mblk = I / 128;
   g1.mblk_stride = 128;
   g1.sub1_off = I;
@@ -485,6 +494,21 @@ moe_status moe_down_proj_with_shared(int32_t rows, int32_t H, const moe_ffn_weig
   if ((s = plan_down(sh_rows, H, sw, sh_h, sh_h_scale, nullptr, nullptr, sh_out, dev_status, &q)) != MOE_OK)
     return s;
   return launch_plan(p, EPI_WEIGHTED, st, nsm, &q);
+}
+
+moe_status moe_tile_ffn_weights(int32_t H, const moe_ffn_weights* src, void* w13_t, void* w2_t, void* stream) {
+  if (!src || H < 1 || src->groups < 1 || src->I < 1 || src->tiled != 0) return MOE_ERR_INVALID_ARG;
+  if (src->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (H % 256 != 0 || src->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if ((w13_t && !src->w13) || (w2_t && !src->w2)) return MOE_ERR_INVALID_ARG;
+  if (any_misaligned(src->w13, src->w2, w13_t, w2_t)) return MOE_ERR_ALIGNMENT;
+  cudaStream_t st = as_stream(stream);
+  if (w13_t) {
+    moe_status s = check_launch(launch_tile_weights(src->w13, w13_t, src->groups, 2 * src->I, H, 128, st));
+    if (s != MOE_OK) return s;
+  }
+  if (w2_t) return check_launch(launch_tile_weights(src->w2, w2_t, src->groups, H, src->I, 256, st));
+  return MOE_OK;
 }
 
 moe_status moe_swiglu_ffn_sync_size(int32_t rows, int32_t groups, int32_t sh_rows, size_t* bytes) {

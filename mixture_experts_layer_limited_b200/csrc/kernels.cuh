@@ -18,6 +18,7 @@ struct GemmArgs {
   int32_t feat_sub1 = 0;           // output-feature offset of sub-tile 1 (0 / 128)
   int32_t bn_max = 256;            // max tokens per tile (multiple of 32, <= 256)
   int32_t a_one_box = 0;           // a tile's 256 weight rows are contiguous: one TMA box
+  int32_t a_tiled = 0;             // weights in moe_tile_ffn_weights' layout (tile (rb, kb) at row (rb*nk+kb)*box)
   void* out = nullptr;             // [rows, out_ld] bf16, or e4m3 codes (GEMM1 FP8)
   int32_t out_ld = 0;
   const float* row_w = nullptr;    // [rows] or nullptr
@@ -90,6 +91,9 @@ static_assert(sizeof(FfnArgs) <= 4096, "FfnArgs must fit the kernel parameter sp
 constexpr int kFfnEpiWarps = 12;
 constexpr int kGuQ = 1;       // epilogue warps per TMEM lane quarter on the gate/up tiles
 cudaError_t launch_ffn_bf16(const FfnArgs& f, int grid, cudaStream_t stream);
+// w [G, M, K] bf16 row-major -> tiles of R rows x 64 K, tile (g*(M/R) + rb, kb)
+// at rows ((g*(M/R) + rb)*(K/64) + kb)*R of a [*, 64] matrix
+cudaError_t launch_tile_weights(const void* src, void* dst, int G, int M, int K, int R, cudaStream_t stream);
 // route: also route the tokens in the same launch where the shape allows
 // (route8_experts_per_thread(r) > 0); counts must be zeroed beforehand. The
 // split of the hidden size over a cluster's CTAs depends on T and num_sms only,

@@ -40,7 +40,8 @@ class MoELayer:
     def __init__(self, spec: LayerSpec, gate: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor,
                  sw13: Optional[torch.Tensor], sw2: Optional[torch.Tensor],
                  bias: Optional[torch.Tensor], T_max: int, gather: bool = False,
-                 fuse_shared: bool = True, fuse_combine: bool = False, fuse_ffn: Optional[bool] = None):
+                 fuse_shared: bool = True, fuse_combine: bool = False, fuse_ffn: Optional[bool] = None,
+                 tiled_weights: bool = True):
         self.spec = spec
         # gather=True: bf16 layers read the routed experts' token rows straight
         # from x (the permutation fused into the first GEMM; no x_perm). At the
@@ -81,6 +82,14 @@ class MoELayer:
             self.sw13 = sw13.contiguous() if sw13 is not None else None
             self.sw2 = sw2.contiguous() if sw2 is not None else None
             self.sw13_s = self.sw2_s = None
+            if tiled_weights:
+                # the layer's own copies in the tiled layout (each weight tile
+                # the GEMMs load in one step is contiguous in HBM)
+                self.w13, self.w2 = self._tiled(self.w13, self.w2, E, I)
+                if self.sw13 is not None:
+                    self.sw13, self.sw2 = self._tiled(self.sw13, self.sw2, 1, I_s)
+        # bf16 weights held tiled (moe_tile_ffn_weights); E4M3 ones row-major
+        self.tiled = tiled_weights and not self.fp8
         self.T_max = T_max
         R = T_max * k
         i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
@@ -121,6 +130,11 @@ class MoELayer:
             self.ffn_ws = z((n + 15) // 16 * 16, dt=torch.uint8)
         else:
             self.ffn_ws = None
+
+    def _tiled(self, w13, w2, groups, I):
+        t13, t2 = torch.empty_like(w13), torch.empty_like(w2)
+        N.moe_tile_ffn_weights(self.spec.H, w13, w2, groups, I, t13, t2)
+        return t13, t2
 
     def _quant_blocks(self, w):
         B, Nr, K = w.shape
@@ -167,19 +181,22 @@ class MoELayer:
         R = T * s.k
         if self.gather:
             N.moe_gate_up_swiglu_gather(R, s.H, self.w13, s.E, s.I, x, T, self.src_token[:R],
-                                        self.offsets, self.h[:R], dev_status=self.status)
+                                        self.offsets, self.h[:R], dev_status=self.status,
+                                        tiled=self.tiled)
             return
         N.moe_gate_up_swiglu(R, s.H, self.w13, self._dt(), s.E, s.I, self.x_perm[:R], self.offsets,
                              self.h[:R], w13_scale=self.w13_s,
                              a_scale=self.x_perm_s[:R] if self.fp8 else None,
-                             h_scale_ws=self.h_s[:R] if self.fp8 else None, dev_status=self.status)
+                             h_scale_ws=self.h_s[:R] if self.fp8 else None, dev_status=self.status,
+                             tiled=self.tiled)
 
     def experts_down(self, T: int):
         s = self.spec
         R = T * s.k
         N.moe_down_proj(R, s.H, self.w2, self._dt(), s.E, s.I, self.h[:R], self.offsets,
                         self.row_w[:R], self.o[:R], w2_scale=self.w2_s,
-                        h_scale=self.h_s[:R] if self.fp8 else None, dev_status=self.status)
+                        h_scale=self.h_s[:R] if self.fp8 else None, dev_status=self.status,
+                        tiled=self.tiled)
 
     def shared_gate_up(self, x: torch.Tensor, T: int):
         s = self.spec
@@ -187,13 +204,14 @@ class MoELayer:
         N.moe_gate_up_swiglu(T, s.H, self.sw13, self._dt(), 1, s.I_s, a, None, self.sh_h[:T],
                              w13_scale=self.sw13_s, a_scale=self.xs[:T] if self.fp8 else None,
                              h_scale_ws=self.sh_h_s[:T] if self.fp8 else None,
-                             dev_status=self.status)
+                             dev_status=self.status, tiled=self.tiled)
 
     def shared_down(self, T: int):
         s = self.spec
         N.moe_down_proj(T, s.H, self.sw2, self._dt(), 1, s.I_s, self.sh_h[:T], None, None,
                         self.sh_o[:T], w2_scale=self.sw2_s,
-                        h_scale=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status)
+                        h_scale=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status,
+                        tiled=self.tiled)
 
     def gate_up_with_shared(self, x: torch.Tensor, T: int):
         """Routed experts' and shared expert's first GEMM in one launch."""
@@ -205,7 +223,8 @@ class MoELayer:
             w13_scale=self.w13_s, a_scale=self.x_perm_s[:R] if self.fp8 else None,
             h_scale_ws=self.h_s[:R] if self.fp8 else None, sw13_scale=self.sw13_s,
             sh_a_scale=self.xs[:T] if self.fp8 else None,
-            sh_h_scale_ws=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status)
+            sh_h_scale_ws=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status,
+            tiled=self.tiled)
 
     def down_with_shared(self, T: int):
         """Routed experts' and shared expert's second GEMM in one launch."""
@@ -215,7 +234,8 @@ class MoELayer:
             R, s.H, self.w2, self._dt(), s.E, s.I, self.h[:R], self.offsets, self.row_w[:R], self.o[:R],
             T, self.sw2, s.I_s, self.sh_h[:T], self.sh_o[:T], w2_scale=self.w2_s,
             h_scale=self.h_s[:R] if self.fp8 else None, sw2_scale=self.sw2_s,
-            sh_h_scale=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status)
+            sh_h_scale=self.sh_h_s[:T] if self.fp8 else None, dev_status=self.status,
+            tiled=self.tiled)
 
     def ffn_with_shared(self, x: torch.Tensor, T: int):
         """Both GEMMs of the routed experts and of the shared expert in one launch."""
@@ -224,7 +244,7 @@ class MoELayer:
         N.moe_swiglu_ffn_with_shared(
             R, s.H, self.w13, self.w2, s.E, s.I, self.x_perm[:R], self.offsets, self.row_w[:R], self.h[:R],
             self.o[:R], T, self.sw13, self.sw2, s.I_s, x, self.sh_h[:T], self.sh_o[:T], self.ffn_ws,
-            dev_status=self.status)
+            dev_status=self.status, tiled=self.tiled)
 
     def down_with_combine(self, T: int):
         """The routed and shared down GEMMs with the combine in their epilogue."""
@@ -233,7 +253,8 @@ class MoELayer:
         N.moe_down_proj_combine(R, T, s.H, self.w2, s.E, s.I, self.h[:R], self.offsets, self.row_w[:R],
                                 self.src_token[:R], self.sw2, s.I_s,
                                 self.sh_h[:T] if self.sh_h is not None else None,
-                                self.y_acc[:T], self.y[:T], dev_status=self.status)
+                                self.y_acc[:T], self.y[:T], dev_status=self.status,
+                                tiled=self.tiled)
 
     def combine(self, T: int):
         s = self.spec

@@ -30,7 +30,7 @@ EXPORTED = [
     "moe_grouped_swiglu",
     "moe_gate_up_swiglu", "moe_gate_up_swiglu_gather", "moe_down_proj",
     "moe_gate_up_swiglu_with_shared", "moe_down_proj_with_shared", "moe_down_proj_combine",
-    "moe_swiglu_ffn_sync_size", "moe_swiglu_ffn_with_shared",
+    "moe_swiglu_ffn_sync_size", "moe_swiglu_ffn_with_shared", "moe_tile_ffn_weights",
     "moe_combine", "moe_bias_update", "moe_aux_loss_workspace_size", "moe_aux_loss",
     "moe_quantize_blocks", "moe_quantize_rows",
     "moe_read_device_status", "moe_last_cuda_error", "moe_status_string", "moe_abi_version",
@@ -54,7 +54,8 @@ class RouteParams(ctypes.Structure):
 class FFNWeights(ctypes.Structure):
     _fields_ = [("w13", ctypes.c_void_p), ("w2", ctypes.c_void_p),
                 ("w13_scale", ctypes.c_void_p), ("w2_scale", ctypes.c_void_p),
-                ("dtype", ctypes.c_int32), ("groups", ctypes.c_int32), ("I", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("groups", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("tiled", ctypes.c_int32)]
 
 
 _LIB = None
@@ -88,6 +89,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_down_proj_with_shared": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P,
                                       _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P],
         "moe_swiglu_ffn_sync_size": [_I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
+        "moe_tile_ffn_weights": [_I, ctypes.POINTER(FFNWeights), _P, _P, _P],
         "moe_swiglu_ffn_with_shared": [_I, _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, _P,
                                        _I, ctypes.POINTER(FFNWeights), _P, _P, _P, _P, ctypes.c_size_t,
                                        _P, _P],
@@ -177,32 +179,36 @@ def moe_permute(T, k, E, H, topk_ids, topk_w, x, x_dtype, x_scale, x_perm, x_per
 
 def moe_grouped_swiglu(rows, H, w13, w2, dtype, groups, I, a, offsets, row_w, h_ws, out,
                        w13_scale=None, w2_scale=None, a_scale=None, h_scale_ws=None,
-                       dev_status=None, stream=None):
+                       dev_status=None, stream=None, tiled=False):
     w = FFNWeights(_ptr(w13), _ptr(w2), _ptr(w13_scale), _ptr(w2_scale), dtype, groups, I)
+    w.tiled = int(tiled)
     _check("moe_grouped_swiglu", load_library().moe_grouped_swiglu(
         rows, H, ctypes.byref(w), _ptr(a), _ptr(a_scale), _ptr(offsets), _ptr(row_w), _ptr(h_ws),
         _ptr(h_scale_ws), _ptr(out), _ptr(dev_status), _stream(stream)))
 
 
 def moe_gate_up_swiglu(rows, H, w13, dtype, groups, I, a, offsets, h_ws, w13_scale=None,
-                       a_scale=None, h_scale_ws=None, dev_status=None, stream=None):
+                       a_scale=None, h_scale_ws=None, dev_status=None, stream=None, tiled=False):
     w = FFNWeights(_ptr(w13), None, _ptr(w13_scale), None, dtype, groups, I)
+    w.tiled = int(tiled)
     _check("moe_gate_up_swiglu", load_library().moe_gate_up_swiglu(
         rows, H, ctypes.byref(w), _ptr(a), _ptr(a_scale), _ptr(offsets), _ptr(h_ws),
         _ptr(h_scale_ws), _ptr(dev_status), _stream(stream)))
 
 
 def moe_gate_up_swiglu_gather(rows, H, w13, groups, I, x, T, src_token, offsets, h_ws,
-                              dev_status=None, stream=None):
+                              dev_status=None, stream=None, tiled=False):
     w = FFNWeights(_ptr(w13), None, None, None, MOE_BF16, groups, I)
+    w.tiled = int(tiled)
     _check("moe_gate_up_swiglu_gather", load_library().moe_gate_up_swiglu_gather(
         rows, H, ctypes.byref(w), _ptr(x), T, _ptr(src_token), _ptr(offsets), _ptr(h_ws),
         _ptr(dev_status), _stream(stream)))
 
 
 def moe_down_proj(rows, H, w2, dtype, groups, I, h, offsets, row_w, out, w2_scale=None,
-                  h_scale=None, dev_status=None, stream=None):
+                  h_scale=None, dev_status=None, stream=None, tiled=False):
     w = FFNWeights(None, _ptr(w2), None, _ptr(w2_scale), dtype, groups, I)
+    w.tiled = int(tiled)
     _check("moe_down_proj", load_library().moe_down_proj(
         rows, H, ctypes.byref(w), _ptr(h), _ptr(h_scale), _ptr(offsets), _ptr(row_w), _ptr(out),
         _ptr(dev_status), _stream(stream)))
@@ -211,9 +217,11 @@ def moe_down_proj(rows, H, w2, dtype, groups, I, h, offsets, row_w, out, w2_scal
 def moe_gate_up_swiglu_with_shared(rows, H, w13, dtype, groups, I, a, offsets, h_ws,
                                    sh_rows, sw13, I_s, sh_a, sh_h_ws, w13_scale=None, a_scale=None,
                                    h_scale_ws=None, sw13_scale=None, sh_a_scale=None, sh_h_scale_ws=None,
-                                   dev_status=None, stream=None):
+                                   dev_status=None, stream=None, tiled=False):
     w = FFNWeights(_ptr(w13), None, _ptr(w13_scale), None, dtype, groups, I)
+    w.tiled = int(tiled)
     sw = FFNWeights(_ptr(sw13), None, _ptr(sw13_scale), None, dtype, 1, I_s)
+    sw.tiled = int(tiled)
     _check("moe_gate_up_swiglu_with_shared", load_library().moe_gate_up_swiglu_with_shared(
         rows, H, ctypes.byref(w), _ptr(a), _ptr(a_scale), _ptr(offsets), _ptr(h_ws), _ptr(h_scale_ws),
         sh_rows, ctypes.byref(sw), _ptr(sh_a), _ptr(sh_a_scale), _ptr(sh_h_ws), _ptr(sh_h_scale_ws),
@@ -222,9 +230,11 @@ def moe_gate_up_swiglu_with_shared(rows, H, w13, dtype, groups, I, a, offsets, h
 
 def moe_down_proj_with_shared(rows, H, w2, dtype, groups, I, h, offsets, row_w, out,
                               sh_rows, sw2, I_s, sh_h, sh_out, w2_scale=None, h_scale=None,
-                              sw2_scale=None, sh_h_scale=None, dev_status=None, stream=None):
+                              sw2_scale=None, sh_h_scale=None, dev_status=None, stream=None, tiled=False):
     w = FFNWeights(None, _ptr(w2), None, _ptr(w2_scale), dtype, groups, I)
+    w.tiled = int(tiled)
     sw = FFNWeights(None, _ptr(sw2), None, _ptr(sw2_scale), dtype, 1, I_s)
+    sw.tiled = int(tiled)
     _check("moe_down_proj_with_shared", load_library().moe_down_proj_with_shared(
         rows, H, ctypes.byref(w), _ptr(h), _ptr(h_scale), _ptr(offsets), _ptr(row_w), _ptr(out),
         sh_rows, ctypes.byref(sw), _ptr(sh_h), _ptr(sh_h_scale), _ptr(sh_out),
@@ -240,19 +250,35 @@ def moe_swiglu_ffn_sync_size(rows, groups, sh_rows):
 
 def moe_swiglu_ffn_with_shared(rows, H, w13, w2, groups, I, a, offsets, row_w, h_ws, out,
                                sh_rows, sw13, sw2, I_s, sh_a, sh_h_ws, sh_out, sync_ws,
-                               dev_status=None, stream=None):
+                               dev_status=None, stream=None, tiled=False):
     w = FFNWeights(_ptr(w13), _ptr(w2), None, None, MOE_BF16, groups, I)
+    w.tiled = int(tiled)
     sw = FFNWeights(_ptr(sw13), _ptr(sw2), None, None, MOE_BF16, 1, I_s)
+    sw.tiled = int(tiled)
     _check("moe_swiglu_ffn_with_shared", load_library().moe_swiglu_ffn_with_shared(
         rows, H, ctypes.byref(w), _ptr(a), _ptr(offsets), _ptr(row_w), _ptr(h_ws), _ptr(out),
         sh_rows, ctypes.byref(sw), _ptr(sh_a), _ptr(sh_h_ws), _ptr(sh_out),
         _ptr(sync_ws), sync_ws.numel() * sync_ws.element_size(), _ptr(dev_status), _stream(stream)))
 
 
+def moe_tile_ffn_weights(H, w13, w2, groups, I, w13_t, w2_t, stream=None):
+    """bf16 w13 [groups, 2I, H] / w2 [groups, H, I] -> the tiled copies w13_t /
+    w2_t (same sizes; either pair may be None)."""
+    for src, dst, n in ((w13, w13_t, groups * 2 * I * H), (w2, w2_t, groups * H * I)):
+        if dst is not None and (src.numel() != n or dst.numel() != n):
+            raise ValueError(f"moe_tile_ffn_weights: expected {n} elements, got {src.numel()} / {dst.numel()}")
+    w = FFNWeights(_ptr(w13), _ptr(w2), None, None, MOE_BF16, groups, I)
+    _check("moe_tile_ffn_weights", load_library().moe_tile_ffn_weights(
+        H, ctypes.byref(w), _ptr(w13_t), _ptr(w2_t), _stream(stream)))
+
+
 def moe_down_proj_combine(rows, T, H, w2, groups, I, h, offsets, row_w, src_token, sw2, I_s, sh_h,
-                          acc_ws, y, dev_status=None, stream=None):
+                          acc_ws, y, dev_status=None, stream=None, tiled=False):
     w = FFNWeights(None, _ptr(w2), None, None, MOE_BF16, groups, I)
+    w.tiled = int(tiled)
     sw = FFNWeights(None, _ptr(sw2), None, None, MOE_BF16, 1, I_s) if sw2 is not None else None
+    if sw is not None:
+        sw.tiled = int(tiled)
     _check("moe_down_proj_combine", load_library().moe_down_proj_combine(
         rows, T, H, ctypes.byref(w), _ptr(h), _ptr(offsets), _ptr(row_w), _ptr(src_token),
         ctypes.byref(sw) if sw is not None else None, _ptr(sh_h), _ptr(acc_ws), _ptr(y),

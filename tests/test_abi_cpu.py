@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     lib = N.load_library()
-    assert lib.moe_abi_version() == 2
+    assert lib.moe_abi_version() == 3
     assert lib.moe_status_string(0) == b"ok"
     assert b"invalid" in lib.moe_status_string(N.MOE_ERR_INVALID_ARG)
     assert lib.moe_status_string(99) == b"unknown status"

@@ -51,7 +51,7 @@ def test_every_layer_stage_has_a_launch_count_and_a_cost_model():
                    {"fuse_ffn": False}):
             # shapes only: stages() builds the launch closures without running them
             lay = MoELayer(spec, z(E, 8), z(1, 1), z(1, 1), z(1, 1) if Is else None,
-                           z(1, 1) if Is else None, None, T, **kw)
+                           z(1, 1) if Is else None, None, T, tiled_weights=False, **kw)
             names = [n for n, _ in lay.stages(z(T, H))] + ["bias_update"]
             for n in names:
                 assert n in bench.LAUNCHES and n in model, (name, kw, n)
@@ -73,7 +73,8 @@ def test_one_launch_ffn_is_chosen_from_512_routed_rows_per_expert():
     T_max = 512 * E // k                                  # exactly two token blocks per expert
     for fuse, T, want in ((None, T_max, "ffn"), (None, T_max - 1, "gate_up"), (True, 8, "ffn"),
                           (False, T_max, "gate_up")):
-        lay = MoELayer(spec, z(E, 8), z(1, 1), z(1, 1), z(1, 1), z(1, 1), None, T_max, fuse_ffn=fuse)
+        lay = MoELayer(spec, z(E, 8), z(1, 1), z(1, 1), z(1, 1), z(1, 1), None, T_max, fuse_ffn=fuse,
+                       tiled_weights=False)
         names = [n for n, _ in lay.stages(z(T, H))]
         assert want in names, (fuse, T, names)
 

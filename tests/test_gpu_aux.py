@@ -93,7 +93,7 @@ def test_layer_aux_loss_after_routing(name):
     gate = (torch.randn(cfg.E, cfg.H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
     tiny = torch.zeros(1, 1, 1, dtype=torch.bfloat16, device=DEV)     # experts unused here
     bias = uniform_bias(cfg.E, cfg.seed + 5) if cfg.scoring == "sigmoid" else None
-    layer = MoELayer(spec, gate, tiny, tiny, None, None, bias, T_max=T)
+    layer = MoELayer(spec, gate, tiny, tiny, None, None, bias, T_max=T, tiled_weights=False)
     L = make_logits(cfg, device=DEV, T=T)
     x = torch.zeros(T, cfg.H, dtype=torch.bfloat16, device=DEV)
     layer.logits[:T].copy_(L)                    # the logits the layer keeps for the aux loss

@@ -552,6 +552,61 @@ def test_swiglu_ffn_one_launch_equals_two_launches(H, I, I_s, sizes, T):
     assert rel_err(np64(o2), ref) < BF16_TOL
 
 
+@pytest.mark.parametrize("H,I,I_s,sizes,T", [
+    (512, 256, 384, [0, 17, 300, 5, 256, 0, 129], 300),
+    (7168, 2048, 2048, [2100, 0, 17, 260, 513], 1000),
+])
+def test_tiled_weights_match_row_major(H, I, I_s, sizes, T):
+    """moe_tile_ffn_weights lays each weight tile the GEMMs load in one step
+    out contiguously (checked against a reshape of the row-major tensor), and
+    the grouped GEMMs read the tiled copies to the same h and outputs, bit for
+    bit, as the row-major weights: two launches, the one-launch FFN and the
+    gathering gate/up GEMM."""
+    G = len(sizes)
+    off = _segments(sizes)
+    R = int(off[-1])
+    g = _gen(H + I + 3 * T)
+    x = torch.randn(T, H, generator=g, device=DEV).to(torch.bfloat16)
+    src = torch.randint(0, T, (R,), generator=g, device=DEV, dtype=torch.int32)
+    xp = x[src.long()].contiguous()
+    w13 = (torch.randn(G, 2 * I, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    w2 = (torch.randn(G, H, I, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    sw13 = (torch.randn(1, 2 * I_s, H, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    sw2 = (torch.randn(1, H, I_s, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    row_w = torch.rand(R, generator=g, device=DEV) + 0.5
+    offd = torch.from_numpy(off).to(DEV)
+    tiles = lambda w, Rr: w.reshape(w.shape[0], w.shape[1] // Rr, Rr, w.shape[2] // 64, 64).permute(0, 1, 3, 2, 4)
+    t13, t2, ts13, ts2 = (torch.empty_like(w) for w in (w13, w2, sw13, sw2))
+    N.moe_tile_ffn_weights(H, w13, w2, G, I, t13, t2)
+    N.moe_tile_ffn_weights(H, sw13, sw2, 1, I_s, ts13, ts2)
+    assert torch.equal(t13.reshape(-1), tiles(w13, 128).reshape(-1))
+    assert torch.equal(t2.reshape(-1), tiles(w2, 256).reshape(-1))
+    assert torch.equal(ts13.reshape(-1), tiles(sw13, 128).reshape(-1))
+    e = lambda *shape: torch.empty(*shape, dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    outs = []
+    for a13, a2, s13, s2, tl in ((w13, w2, sw13, sw2, False), (t13, t2, ts13, ts2, True)):
+        h, sh_h, o, sh_o = e(R, I), e(T, I_s), e(R, H), e(T, H)
+        N.moe_gate_up_swiglu_with_shared(R, H, a13, N.MOE_BF16, G, I, xp, offd, h, T, s13, I_s, x, sh_h,
+                                         dev_status=status, tiled=tl)
+        N.moe_down_proj_with_shared(R, H, a2, N.MOE_BF16, G, I, h, offd, row_w, o, T, s2, I_s, sh_h, sh_o,
+                                    dev_status=status, tiled=tl)
+        outs.append((h, sh_h, o, sh_o))
+    sync = torch.empty(N.moe_swiglu_ffn_sync_size(R, G, T), dtype=torch.uint8, device=DEV)
+    h, sh_h, o, sh_o = e(R, I), e(T, I_s), e(R, H), e(T, H)
+    N.moe_swiglu_ffn_with_shared(R, H, t13, t2, G, I, xp, offd, row_w, h, o, T, ts13, ts2, I_s, x, sh_h, sh_o,
+                                 sync, dev_status=status, tiled=True)
+    outs.append((h, sh_h, o, sh_o))
+    h_gat = e(R, I)
+    N.moe_gate_up_swiglu_gather(R, H, t13, G, I, x, T, src, offd, h_gat, dev_status=status, tiled=True)
+    torch.cuda.synchronize()
+    assert N.moe_read_device_status(status) == 0
+    assert torch.equal(h_gat, outs[0][0])
+    for got in outs[1:]:
+        for a, b in zip(got, outs[0]):
+            assert torch.equal(a, b)
+
+
 def test_swiglu_ffn_rejects_e4m3_and_short_scratch():
     """The one-launch FFN is bf16 only, and its scratch must hold a counter
     per token block (checked on the host, nothing launched)."""
