@@ -427,11 +427,12 @@ MOE_API moe_status moe_aux_loss(int32_t T, int32_t E, int32_t k, int32_t seq_len
 
 /* ------------------------------------------------------------------------ *
  * moe_tile_ffn_weights -- the bf16 expert weights in the layout the grouped
- * GEMMs stream fastest: each tile the GEMM loads in one step (128 rows of
- * w13 or 256 rows of w2, by 64 K) is one contiguous 16 / 32 KB block, the
- * tiles of a row block in K order:
- *   w13_t[((g*(2I/128) + rb)*(H/64) + kb)*128 + r][c] = w13[g][rb*128 + r][kb*64 + c]
- *   w2_t [((g*(H/256)  + rb)*(I/64) + kb)*256 + r][c] = w2 [g][rb*256 + r][kb*64 + c]
+ * GEMMs stream fastest: the 256 weight rows x 64 K a GEMM tile loads in one
+ * step (w13: 128 gate rows and the same features' 128 up rows; w2: 256 rows)
+ * are one contiguous 32 KB block, the blocks of a tile in K order:
+ *   w13_t[((g*(I/128) + f)*(H/64) + kb)*256 + r][c] = w13[g][f*128 + r][kb*64 + c]        (r < 128)
+ *   w13_t[((g*(I/128) + f)*(H/64) + kb)*256 + r][c] = w13[g][I + f*128 + r-128][kb*64 + c] (r >= 128)
+ *   w2_t [((g*(H/256) + b)*(I/64) + kb)*256 + r][c] = w2 [g][b*256 + r][kb*64 + c]
  * (c < 64). The values are unchanged, so results are bit-identical to the
  * row-major weights; pass the tiled copies with w->tiled = 1. The pages
  * state the weights only as [E, 2I, H] / [E, H, I] matrices; the tiling is

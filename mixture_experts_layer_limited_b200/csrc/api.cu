@@ -246,6 +246,8 @@ moe_status check_ffn(int32_t rows, int32_t H, const moe_ffn_weights* w, const vo
   if (static_cast<long long>(w->groups) * 2 * w->I > 0x7fffffffLL ||
       static_cast<long long>(w->groups) * H > 0x7fffffffLL)
     return MOE_ERR_UNSUPPORTED;
+  // the tiled view's rows are TMA coordinates (int32)
+  if (w->tiled && static_cast<long long>(w->groups) * 2 * w->I * (H / 64) > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
   if (any_misaligned(w->w13, w->w2, w->w13_scale, w->w2_scale, a, a_scale)) return MOE_ERR_ALIGNMENT;
   return MOE_OK;
 }
@@ -273,8 +275,9 @@ moe_status plan_gate_up(int32_t rows, int32_t H, const moe_ffn_weights* w, const
                         const int32_t* offsets, void* h_ws, float* h_scale_ws, int32_t* dev_status, GemmPlan* p) {
   const bool fp8 = w->dtype == MOE_E4M3;
   const int I = w->I;
-  // tiled weights: a [*, 64] matrix whose 128-row boxes are the tiles
-  moe_status s = w->tiled ? make_tmap(&p->tmA, w->w13, false, 64, static_cast<uint64_t>(w->groups) * 2 * I * (H / 64), 128)
+  // tiled weights: a [*, 64] matrix whose 256-row boxes (128 gate rows, then
+  // the same features' 128 up rows) are the tiles
+  moe_status s = w->tiled ? make_tmap(&p->tmA, w->w13, false, 64, static_cast<uint64_t>(w->groups) * 2 * I * (H / 64), 256)
                           : make_tmap(&p->tmA, w->w13, fp8, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
   if (s != MOE_OK) return s;
   if ((s = make_token_tmaps(&p->tmB, a, fp8, H, rows)) != MOE_OK) return s;
@@ -401,7 +404,7 @@ moe_status moe_gate_up_swiglu_gather(int32_t rows, int32_t H, const moe_ffn_weig
   const int I = w->I;
   CUtensorMap tmA;
   TokenMaps tmB;
-  s = w->tiled ? make_tmap(&tmA, w->w13, false, 64, static_cast<uint64_t>(w->groups) * 2 * I * (H / 64), 128)
+  s = w->tiled ? make_tmap(&tmA, w->w13, false, 64, static_cast<uint64_t>(w->groups) * 2 * I * (H / 64), 256)
                : make_tmap(&tmA, w->w13, false, H, static_cast<uint64_t>(w->groups) * 2 * I, 128);
   if (s != MOE_OK) return s;
   s = make_token_tmaps(&tmB, x, false, H, T);      // not read: token rows are gathered
@@ -500,14 +503,15 @@ moe_status moe_tile_ffn_weights(int32_t H, const moe_ffn_weights* src, void* w13
   if (!src || H < 1 || src->groups < 1 || src->I < 1 || src->tiled != 0) return MOE_ERR_INVALID_ARG;
   if (src->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (H % 256 != 0 || src->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(src->groups) * 2 * src->I * (H / 64) > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
   if ((w13_t && !src->w13) || (w2_t && !src->w2)) return MOE_ERR_INVALID_ARG;
   if (any_misaligned(src->w13, src->w2, w13_t, w2_t)) return MOE_ERR_ALIGNMENT;
   cudaStream_t st = as_stream(stream);
-  if (w13_t) {
-    moe_status s = check_launch(launch_tile_weights(src->w13, w13_t, src->groups, 2 * src->I, H, 128, st));
+  if (w13_t) {   // 256-row tiles: 128 gate rows, then the same features' 128 up rows
+    moe_status s = check_launch(launch_tile_weights(src->w13, w13_t, src->groups, 2 * src->I, H, src->I, st));
     if (s != MOE_OK) return s;
   }
-  if (w2_t) return check_launch(launch_tile_weights(src->w2, w2_t, src->groups, H, src->I, 256, st));
+  if (w2_t) return check_launch(launch_tile_weights(src->w2, w2_t, src->groups, H, src->I, 0, st));
   return MOE_OK;
 }
 

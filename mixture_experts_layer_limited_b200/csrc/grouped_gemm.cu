@@ -154,18 +154,17 @@ __device__ __forceinline__ TileInfo decode_tile_nb(const Sched& s, const GemmArg
                            t - s.tb_start[lo] * a.n_mblk);
 }
 
-// The weight rows of K block kb of a tile: sub-tiles at rows a_row0 and a_row1
-// (128 rows each), or one 256-row box at a_row0. Row-major weights are read at
-// (kb * 64, row); tiled ones (moe_tile_ffn_weights) at (0, (row / box * nk +
-// kb) * box), each box one contiguous block.
+// The weight rows of K block kb of a tile. Row-major weights: sub-tiles at
+// rows a_row0 and a_row1 (128 rows each), or one 256-row box at a_row0, read
+// at (kb * 64, row). Tiled weights (moe_tile_ffn_weights, wblk >= 0): the
+// tile's 256 rows of K block kb (gate/up: the 128 gate rows, then the 128 up
+// rows) are one contiguous block at row (wblk * nk + kb) * 256.
 __device__ __forceinline__ void load_weight_rows(void* dst0, void* dst1, const CUtensorMap* mA, uint64_t* bar,
-                                                 int kb, int nk, int a_row0, int a_row1, bool one_box, bool tiled,
+                                                 int kb, int nk, int a_row0, int a_row1, bool one_box, int wblk,
                                                  uint64_t pol) {
   constexpr int KB = 64;
-  const int box = one_box ? 256 : 128;
-  if (tiled) {
-    tma_load_2d(dst0, mA, bar, 0, (a_row0 / box * nk + kb) * box, pol);
-    if (!one_box) tma_load_2d(dst1, mA, bar, 0, (a_row1 / box * nk + kb) * box, pol);
+  if (wblk >= 0) {
+    tma_load_2d(dst0, mA, bar, 0, (wblk * nk + kb) * 256, pol);
   } else {
     tma_load_2d(dst0, mA, bar, kb * KB, a_row0, pol);
     if (!one_box) tma_load_2d(dst1, mA, bar, kb * KB, a_row1, pol);
@@ -303,14 +302,14 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         const int a_row0 = sh ? ti.mb * a2.mblk_stride : ti.g * a.a_rows_per_group + ti.mb * a.mblk_stride;
         const int a_row1 = a_row0 + (sh ? a2.sub1_off : a.sub1_off);
         const bool one_box = sh ? a2.a_one_box != 0 : a.a_one_box != 0;
-        const bool tiled = sh ? a2.a_tiled != 0 : a.a_tiled != 0;
+        const int wblk = !(sh ? a2.a_tiled : a.a_tiled) ? -1 : sh ? ti.mb : ti.g * a.n_mblk + ti.mb;
         const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;   // re-read by sibling token blocks
         const uint32_t bytes = 2 * A_SUB_BYTES + (GATHER ? 0u : static_cast<uint32_t>(ti.N) * 128u);
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, a.status, wait_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
-          load_weight_rows(sA(stage, 0), sA(stage, 1), mA, &full_bar[stage], kb, nk, a_row0, a_row1, one_box, tiled,
+          load_weight_rows(sA(stage, 0), sA(stage, 1), mA, &full_bar[stage], kb, nk, a_row0, a_row1, one_box, wblk,
                            pol_w);
           if (!GATHER) {
             uint8_t* bdst = sB(stage);
@@ -618,7 +617,7 @@ grouped_ffn_bf16_kernel(const __grid_constant__ FfnArgs f) {
         const int a_row0 = ti.g * g.a_rows_per_group + ti.mb * g.mblk_stride;
         const int a_row1 = a_row0 + g.sub1_off;
         const bool one_box = g.a_one_box != 0;
-        const bool tiled = g.a_tiled != 0;
+        const int wblk = g.a_tiled ? ti.g * g.n_mblk + ti.mb : -1;
         const uint64_t pol_w = ti.ntb > 1 ? pol_reuse : pol_once;
         const uint32_t bytes = 2 * A_SUB_BYTES + static_cast<uint32_t>(ti.N) * 128u;
         bool ok = true;
@@ -626,7 +625,7 @@ grouped_ffn_bf16_kernel(const __grid_constant__ FfnArgs f) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, status, wait_ns)) { ok = false; break; }
           stage_tile[stage] = t;
           mbar_arrive_expect_tx(&full_bar[stage], bytes);
-          load_weight_rows(sA(stage, 0), sA(stage, 1), mA, &full_bar[stage], kb, nk, a_row0, a_row1, one_box, tiled,
+          load_weight_rows(sA(stage, 0), sA(stage, 1), mA, &full_bar[stage], kb, nk, a_row0, a_row1, one_box, wblk,
                            pol_w);
           uint8_t* bdst = sB(stage);
           uint64_t* fb = &full_bar[stage];

@@ -93,7 +93,7 @@ constexpr int kGuQ = 1;       // epilogue warps per TMEM lane quarter on the gat
 cudaError_t launch_ffn_bf16(const FfnArgs& f, int grid, cudaStream_t stream);
 // w [G, M, K] bf16 row-major -> tiles of R rows x 64 K, tile (g*(M/R) + rb, kb)
 // at rows ((g*(M/R) + rb)*(K/64) + kb)*R of a [*, 64] matrix
-cudaError_t launch_tile_weights(const void* src, void* dst, int G, int M, int K, int R, cudaStream_t stream);
+cudaError_t launch_tile_weights(const void* src, void* dst, int G, int M, int K, int split, cudaStream_t stream);
 // route: also route the tokens in the same launch where the shape allows
 // (route8_experts_per_thread(r) > 0); counts must be zeroed beforehand. The
 // split of the hidden size over a cluster's CTAs depends on T and num_sms only,

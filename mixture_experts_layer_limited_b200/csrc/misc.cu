@@ -382,28 +382,39 @@ cudaError_t launch_quant_rows(int M, int K, const void* a, void* q, float* scale
 
 // ------------------------------------------------------------------------
 // Weight tiling (moe_tile_ffn_weights): one thread per 16-byte chunk of the
-// output; tile t = (g*(M/R) + rb)*(K/64) + kb holds rows [rb*R, +R) of group g,
-// columns [kb*64, +64), row-major, at rows [t*R, +R) of a [*, 64] matrix.
+// output, each tile 256 rows x 64 columns (32 KB) of one group's weights.
 // ------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
-tile_weights_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t chunks, int K, int R) {
+tile_weights_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t chunks, int M, int K, int split) {
   const int nkb = K / 64;
+  const int nblk = split ? M / 256 : 0;   // 256-row tiles per group when they interleave two halves
   for (size_t d = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; d < chunks;
        d += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const size_t tile = d / (static_cast<size_t>(R) * 8);
-    const int within = static_cast<int>(d - tile * static_cast<size_t>(R) * 8);
+    const size_t tile = d / (256 * 8);
+    const int within = static_cast<int>(d - tile * (256 * 8));
     const int r = within >> 3, c16 = within & 7;
-    const size_t kb = tile % nkb, rbg = tile / nkb;       // rbg = g*(M/R) + rb
-    dst[d] = src[(rbg * R + r) * static_cast<size_t>(K / 8) + kb * 8 + c16];
+    const size_t kb = tile % nkb, blk = tile / nkb;      // blk = g * (M / 256) + row block
+    size_t row;
+    if (split) {   // rows [0, 128): block rows of the first half; [128, 256): the same of the second
+      const size_t g = blk / nblk, f = blk % nblk;
+      row = g * M + f * 128 + (r >= 128 ? split : 0) + (r & 127);
+    } else {
+      row = blk * 256 + r;
+    }
+    dst[d] = src[row * static_cast<size_t>(K / 8) + kb * 8 + c16];
   }
 }
 
-cudaError_t launch_tile_weights(const void* src, void* dst, int G, int M, int K, int R, cudaStream_t stream) {
+// dst tile t = (g * (M / 256) + b) * (K / 64) + kb holds, at rows t * 256 of a
+// [*, 64] matrix, the 64 columns kb of 256 source rows of group g: rows b * 256
+// + [0, 256) (split = 0), or rows b * 128 + [0, 128) followed by split + b * 128
+// + [0, 128) (gate/up weights, split = I).
+cudaError_t launch_tile_weights(const void* src, void* dst, int G, int M, int K, int split, cudaStream_t stream) {
   const size_t chunks = static_cast<size_t>(G) * M * (K / 8);
   const size_t blocks = (chunks + 255) / 256;
   const int grid = static_cast<int>(blocks < 65535 * 16 ? blocks : 65535 * 16);
-  tile_weights_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), chunks, K,
-                                                R);
+  tile_weights_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), chunks, M, K,
+                                                split);
   return cudaGetLastError();
 }
 

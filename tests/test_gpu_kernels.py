@@ -575,13 +575,16 @@ def test_tiled_weights_match_row_major(H, I, I_s, sizes, T):
     sw2 = (torch.randn(1, H, I_s, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
     row_w = torch.rand(R, generator=g, device=DEV) + 0.5
     offd = torch.from_numpy(off).to(DEV)
-    tiles = lambda w, Rr: w.reshape(w.shape[0], w.shape[1] // Rr, Rr, w.shape[2] // 64, 64).permute(0, 1, 3, 2, 4)
+    # w2: [g, b, kb, 256 rows, 64]; w13: [g, f, kb, (gate | up), 128 rows, 64]
+    tiles2 = lambda w: w.reshape(w.shape[0], w.shape[1] // 256, 256, w.shape[2] // 64, 64).permute(0, 1, 3, 2, 4)
+    tiles13 = lambda w: w.reshape(w.shape[0], 2, w.shape[1] // 256, 128, w.shape[2] // 64, 64).permute(0, 2, 4, 1, 3, 5)
     t13, t2, ts13, ts2 = (torch.empty_like(w) for w in (w13, w2, sw13, sw2))
     N.moe_tile_ffn_weights(H, w13, w2, G, I, t13, t2)
     N.moe_tile_ffn_weights(H, sw13, sw2, 1, I_s, ts13, ts2)
-    assert torch.equal(t13.reshape(-1), tiles(w13, 128).reshape(-1))
-    assert torch.equal(t2.reshape(-1), tiles(w2, 256).reshape(-1))
-    assert torch.equal(ts13.reshape(-1), tiles(sw13, 128).reshape(-1))
+    assert torch.equal(t13.reshape(-1), tiles13(w13).reshape(-1))
+    assert torch.equal(t2.reshape(-1), tiles2(w2).reshape(-1))
+    assert torch.equal(ts13.reshape(-1), tiles13(sw13).reshape(-1))
+    assert torch.equal(ts2.reshape(-1), tiles2(sw2).reshape(-1))
     e = lambda *shape: torch.empty(*shape, dtype=torch.bfloat16, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     outs = []
