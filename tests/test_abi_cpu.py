@@ -74,6 +74,40 @@ def test_ffn_sync_size_and_host_validation():
     assert call(fake, need, e4) != N.MOE_OK
 
 
+def test_tiled_weights_host_validation():
+    """moe_tile_ffn_weights and the GEMM calls check the weight layout flag on
+    the host: only bf16 weights tile, a tiled source or a flag other than 0/1
+    is refused, shapes outside the GEMM limits or past int32 tiled rows are
+    unsupported, and misaligned buffers are caught, all before any launch."""
+    lib = N.load_library()
+    P = ctypes.c_void_p
+    fake, odd = P(0x1000), P(0x1004)
+
+    def w(dtype=N.MOE_BF16, groups=4, I=256, tiled=0, w13=fake, scale=None):
+        f = N.FFNWeights(w13, fake, scale, scale, dtype, groups, I)
+        f.tiled = tiled
+        return f
+
+    def tile(H, src, w13_t=fake, w2_t=fake):
+        return lib.moe_tile_ffn_weights(H, ctypes.byref(src) if src is not None else None, w13_t, w2_t, None)
+    assert tile(512, None) == N.MOE_ERR_INVALID_ARG
+    assert tile(512, w(tiled=1)) == N.MOE_ERR_INVALID_ARG                 # already tiled
+    assert tile(512, w(dtype=N.MOE_E4M3, scale=fake)) == N.MOE_ERR_UNSUPPORTED
+    assert tile(384, w()) == N.MOE_ERR_UNSUPPORTED                        # H % 256
+    assert tile(512, w(I=192)) == N.MOE_ERR_UNSUPPORTED                   # I % 128
+    assert tile(65536, w(groups=512, I=8192)) == N.MOE_ERR_UNSUPPORTED    # tiled rows past int32
+    assert tile(512, w(w13=None)) == N.MOE_ERR_INVALID_ARG                # w13_t without w13
+    assert tile(512, w(), w13_t=odd) == N.MOE_ERR_ALIGNMENT
+
+    def gate_up(weights, H=512):
+        return lib.moe_gate_up_swiglu(64, H, ctypes.byref(weights), fake, None, fake, fake, None, None, None)
+    assert gate_up(w(tiled=2)) == N.MOE_ERR_INVALID_ARG
+    assert gate_up(w(tiled=-1)) == N.MOE_ERR_INVALID_ARG
+    assert gate_up(w(dtype=N.MOE_E4M3, scale=fake, tiled=1)) == N.MOE_ERR_UNSUPPORTED
+    assert gate_up(w(groups=512, I=8192, tiled=1), H=65536) == N.MOE_ERR_UNSUPPORTED
+    assert lib.moe_last_cuda_error() == 0      # nothing above reached the CUDA runtime
+
+
 def _raw(lib, fn, *args):
     return getattr(lib, fn)(*args)
 
