@@ -18,7 +18,8 @@ struct GemmArgs {
   int32_t feat_sub1 = 0;           // output-feature offset of sub-tile 1 (0 / 128)
   int32_t bn_max = 256;            // max tokens per tile (multiple of 32, <= 256)
   int32_t a_one_box = 0;           // a tile's 256 weight rows are contiguous: one TMA box
-  int32_t a_tiled = 0;             // weights in moe_tile_ffn_weights' layout (tile (rb, kb) at row (rb*nk+kb)*box)
+  int32_t a_tiled = 0;             // weights in moe_tile_ffn_weights' layout: a tile's 256 rows of K block kb at
+                                   // row ((g * n_mblk + mb) * nk + kb) * 256 of a [*, 64] matrix
   void* out = nullptr;             // [rows, out_ld] bf16, or e4m3 codes (GEMM1 FP8)
   int32_t out_ld = 0;
   const float* row_w = nullptr;    // [rows] or nullptr
