@@ -84,7 +84,10 @@ class MoELayer:
             self.sw13_s = self.sw2_s = None
             if tiled_weights:
                 # the layer's own copies in the tiled layout (each weight tile
-                # the GEMMs load in one step is contiguous in HBM)
+                # the GEMMs load in one step is contiguous in HBM; 3 % faster
+                # GEMMs at the V3 shape on B200). They are new tensors of the
+                # weights' size: the caller may free its row-major ones.
+                # tiled_weights=False reads the caller's tensors as they are.
                 self.w13, self.w2 = self._tiled(self.w13, self.w2, E, I)
                 if self.sw13 is not None:
                     self.sw13, self.sw2 = self._tiled(self.sw13, self.sw2, 1, I_s)
