@@ -278,6 +278,30 @@ def test_layer_one_launch_ffn_matches_two_launches(name):
     assert torch.equal(y1, y2)
 
 
+@pytest.mark.parametrize("name,fuse", [("tiny", None), ("v2lite", None), ("v3", None), ("v3_skewed", True)])
+def test_layer_tiled_weights_match_row_major(name, fuse):
+    """The layer holding its bf16 weights tiled (the default) gives the output
+    of the same layer reading the caller's row-major weights, bit for bit, at
+    the full sizes (both GEMM forms: two launches, and one launch for the
+    skewed layer)."""
+    cfg = get_config(name)
+    inp = make_inputs(cfg, device=DEV)
+    mk = lambda tiled: MoELayer(LayerSpec.from_config(cfg), inp.gate, inp.w13, inp.w2, inp.sw13, inp.sw2,
+                                inp.bias, cfg.T, fuse_ffn=fuse, tiled_weights=tiled)
+    lt = mk(True)
+    assert lt.tiled
+    y1 = lt.forward(inp.x).clone()
+    torch.cuda.synchronize()
+    assert lt.device_status() == 0
+    del lt
+    lr = mk(False)
+    assert not lr.tiled and lr.w13.data_ptr() == inp.w13.data_ptr()
+    y2 = lr.forward(inp.x)
+    torch.cuda.synchronize()
+    assert lr.device_status() == 0
+    assert torch.equal(y1, y2)
+
+
 @pytest.mark.parametrize("name", ["v2lite", "v3"])
 def test_host_pipeline_matches_one_forward_at_a_time(name):
     """HostPipeline overlaps each batch's copies with its neighbours' compute;
