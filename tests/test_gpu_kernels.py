@@ -442,6 +442,10 @@ def _ref_grouped(a, w13, w2, off, row_w):
     # partial chunk of token blocks (5000 rows = 20 blocks = 8 + 8 + 4)
     (512, 256, [2300, 5000, 3]),
     (7168, 2048, [2100, 0, 17]),
+    # segments just past a multiple of 256 rows: balanced token blocks of
+    # 136-144 rows (two for 257-288 rows, three for 513-545)
+    (512, 256, [257, 270, 272, 273, 288, 289, 544, 545, 530, 0, 256]),
+    (7168, 2048, [270, 282, 256, 520, 288]),
 ])
 def test_grouped_swiglu_bf16(H, I, sizes):
     G = len(sizes)
@@ -467,6 +471,7 @@ def test_grouped_swiglu_bf16(H, I, sizes):
 @pytest.mark.parametrize("H,I,I_s,sizes,T", [
     (512, 256, 384, [0, 17, 300, 5, 256, 0, 129], 300),
     (7168, 2048, 2048, [300, 77, 512, 1], 1000),
+    (512, 256, 384, [280, 1, 0, 530, 288], 270),     # routed and shared rows just past a full block
     (2048, 1408, 2816, [384, 0, 5, 513], 129),
 ])
 def test_routed_and_shared_in_one_launch(H, I, I_s, sizes, T):
