@@ -439,7 +439,8 @@ MOE_API moe_status moe_aux_loss(int32_t T, int32_t E, int32_t k, int32_t seq_len
  * a layout of this library.
  *   src   row-major weights (src->tiled must be 0, dtype MOE_BF16).
  *   w13_t / w2_t  device outputs of the same sizes as src->w13 / src->w2 (either
- *         may be NULL to skip it); they may not overlap the inputs.
+ *         may be NULL to skip it); an output overlapping an input or the other
+ *         output is refused (MOE_ERR_INVALID_ARG).
  * Limits: those of moe_grouped_swiglu (I % 128 == 0, H % 256 == 0).
  * ------------------------------------------------------------------------ */
 MOE_API moe_status moe_tile_ffn_weights(int32_t H, const moe_ffn_weights* src, void* w13_t, void* w2_t,

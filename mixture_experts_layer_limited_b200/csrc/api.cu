@@ -506,6 +506,15 @@ moe_status moe_tile_ffn_weights(int32_t H, const moe_ffn_weights* src, void* w13
   if (static_cast<long long>(src->groups) * 2 * src->I * (H / 64) > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
   if ((w13_t && !src->w13) || (w2_t && !src->w2)) return MOE_ERR_INVALID_ARG;
   if (any_misaligned(src->w13, src->w2, w13_t, w2_t)) return MOE_ERR_ALIGNMENT;
+  // the copies are gathers: an output overlapping any input would be read after being written
+  const size_t b13 = static_cast<size_t>(src->groups) * 2 * src->I * H * 2, b2 = static_cast<size_t>(src->groups) * H * src->I * 2;
+  auto overlap = [](const void* p, size_t np, const void* q, size_t nq) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return p && q && a < b + nq && b < a + np;
+  };
+  if (overlap(w13_t, b13, src->w13, b13) || overlap(w13_t, b13, src->w2, b2) || overlap(w2_t, b2, src->w13, b13) ||
+      overlap(w2_t, b2, src->w2, b2) || overlap(w13_t, b13, w2_t, b2))
+    return MOE_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);
   if (w13_t) {   // 256-row tiles: 128 gate rows, then the same features' 128 up rows
     moe_status s = check_launch(launch_tile_weights(src->w13, w13_t, src->groups, 2 * src->I, H, src->I, st));

@@ -98,6 +98,9 @@ def test_tiled_weights_host_validation():
     assert tile(65536, w(groups=512, I=8192)) == N.MOE_ERR_UNSUPPORTED    # tiled rows past int32
     assert tile(512, w(w13=None)) == N.MOE_ERR_INVALID_ARG                # w13_t without w13
     assert tile(512, w(), w13_t=odd) == N.MOE_ERR_ALIGNMENT
+    # outputs may not overlap the inputs or each other (w13 at 0x1000 spans 4*512*512*2 bytes)
+    assert tile(512, w(), w13_t=P(0x1000 + 4096), w2_t=P(0x10000000)) == N.MOE_ERR_INVALID_ARG
+    assert tile(512, w(), w13_t=P(0x10000000), w2_t=P(0x10000000 + 4096)) == N.MOE_ERR_INVALID_ARG
 
     def gate_up(weights, H=512):
         return lib.moe_gate_up_swiglu(64, H, ctypes.byref(weights), fake, None, fake, fake, None, None, None)
