@@ -32,7 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer fwd tokens/s and achieved TFLOP/s vs B200 peak at V3 shape"
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "gate_up_swiglu_v3_traffic.txt")
+PROFILE_DIR = os.path.join(ROOT, "profiles")      # *_traffic.txt: DRAM bytes of one launch per workload
 GEMM_SOURCES = ["grouped_gemm.cu", "common.cuh", "kernels.cuh"]
 
 
@@ -268,23 +268,28 @@ def gemm_source_hash():
 
 
 def profiled_traffic(stage, workload):
-    """DRAM bytes per launch of the gate/up GEMM from the committed ncu
-    summary, only if it was taken of this stage's launch, scaled to this
-    workload, and the GEMM source has not changed since."""
-    if not os.path.exists(PROFILE_TRAFFIC):
+    """DRAM bytes per launch of a stage's GEMM from the committed ncu
+    summaries (profiles/*_traffic.txt), only from one taken of this stage's
+    launch on this workload, and only while the GEMM source is the one
+    captured."""
+    if not os.path.isdir(PROFILE_DIR):
         return None
-    kv = {}
-    for line in open(PROFILE_TRAFFIC):
-        if ":" in line:
-            k, v = line.split(":", 1)
-            kv[k.strip()] = v.strip()
-    if (kv.get("gemm_source_sha256_16") != gemm_source_hash() or kv.get("stage") != stage
-            or kv.get("workload") != workload):
-        return None
-    try:
-        return float(kv["traffic_bytes_per_launch_full_size"])
-    except (KeyError, ValueError):
-        return None
+    for name in sorted(os.listdir(PROFILE_DIR)):
+        if not name.endswith("_traffic.txt"):
+            continue
+        kv = {}
+        for line in open(os.path.join(PROFILE_DIR, name)):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if (kv.get("gemm_source_sha256_16") != gemm_source_hash() or kv.get("stage") != stage
+                or kv.get("workload") != workload):
+            continue
+        try:
+            return float(kv["traffic_bytes_per_launch_full_size"])
+        except (KeyError, ValueError):
+            return None
+    return None
 
 
 LAUNCHES = {"route": 1, "permute": 3, "gate_up_routed": 1, "down_routed": 1,
@@ -440,7 +445,7 @@ def run_ours(args):
         gbs = model[dom]["bytes"] / (avg[dom] * 1e-3) / 1e9
         roofline = {"kernel": f"grouped_gemm_e4m3 (gate/up + SwiGLU, {what})", "bound": "hbm",
                     "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                    "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": profiled_traffic(dom, cfg.name),
                     "sm_mhz": clk.get("sm_mhz"),
                     "peak_note": f"HBM copy, {peaks['source']}",
                     "algorithmic_flops_per_launch": model[dom]["flops"],
