@@ -111,8 +111,9 @@ def test_cpu_sample_holds_every_token_of_the_hottest_and_coldest_expert():
 
 def test_profiled_traffic_matches_workload_stage_and_source(monkeypatch):
     """roofline.traffic comes from the committed one-launch DRAM summaries
-    (profiles/*_traffic.txt): the V3 gate/up launch and the E4M3 decode
-    layer's gate/up stage, each only for its own workload and stage, near
+    (profiles/*_traffic.txt): the V3 gate/up launch, the E4M3 decode layer's
+    gate/up stage and the skewed layer's one-launch FFN, each only for its
+    own workload and stage, near
     the algorithmic bytes, and none once the GEMM source differs from the one
     captured."""
     sys.path.insert(0, ROOT)
@@ -122,6 +123,8 @@ def test_profiled_traffic_matches_workload_stage_and_source(monkeypatch):
     assert v3 is not None and f8 is not None
     assert 1.0 <= v3 / 16450060288 < 1.2          # the split experts re-read part of their weights
     assert 0.85 < f8 / 7566786560 <= 1.0          # experts without tokens are never read
+    sk = bench.profiled_traffic("ffn", "v3_skewed")
+    assert sk is not None and 1.0 <= sk / 33508294656 < 1.2
     assert bench.profiled_traffic("down", "v3") is None
     assert bench.profiled_traffic("gate_up", "v2lite") is None
     monkeypatch.setattr(bench, "gemm_source_hash", lambda: "0" * 16)
