@@ -126,6 +126,8 @@ def test_profiled_traffic_matches_workload_stage_and_source(monkeypatch):
     sk = bench.profiled_traffic("ffn", "v3_skewed")
     assert sk is not None and 1.0 <= sk / 33508294656 < 1.2
     assert bench.profiled_traffic("down", "v3") is None
-    assert bench.profiled_traffic("gate_up", "v2lite") is None
+    v2 = bench.profiled_traffic("gate_up", "v2lite")
+    assert v2 is not None and 0.9 < v2 / 970981376 < 1.1
+    assert bench.profiled_traffic("gate_up", "tiny") is None
     monkeypatch.setattr(bench, "gemm_source_hash", lambda: "0" * 16)
     assert bench.profiled_traffic("gate_up", "v3") is None
